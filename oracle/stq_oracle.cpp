@@ -1,0 +1,717 @@
+/*
+ * stq_oracle.cpp -- plain, single-threaded CPU oracle for the quantized
+ * Delta-rule recurrent-state decode step.
+ *
+ * TEST INFRASTRUCTURE ONLY (see stq_oracle.h).  Built with
+ * -O2 -ffp-contract=off and no fast-math, so every float expression below is
+ * evaluated exactly as written: one IEEE rounding per +, -, *, /, and fmaf
+ * only where it is spelled out.
+ *
+ * Two evaluations of the step live here:
+ *   orc_step_f64  the plain definition in double precision, natural key order;
+ *   orc_step_f32  the canonical fp32 evaluation that the GPU kernel must
+ *                 reproduce bit for bit.  The pages fix no fp32 evaluation
+ *                 order; requiring bit-identical integer codes forces one, so
+ *                 the order is part of the definition here:
+ *                   - the state is handled in column-normalised units
+ *                     T = S / c (so the value-column scale c_j leaves the
+ *                     inner loops);
+ *                   - a column sum sum_s w_s T_sj runs over stored rows in
+ *                     blocks of ORC_SUM_BLOCK consecutive rows, each block a
+ *                     chain p = fmaf(w_s, T_sj, p) from p = 0 in ascending s,
+ *                     and the block partials are added by a balanced pairwise
+ *                     tree in block order;
+ *                   - requantization rounds the exact product T' * inv once
+ *                     (to an integer, ties to even);
+ *                   - inv = qmax / m rounded toward zero, which keeps every
+ *                     scaled value inside [-qmax, qmax].
+ *                 orc_step_f64 pins this evaluation to the mathematics.
+ *
+ * parity pins: every function here is pinned by tests/test_oracle_*.py
+ * (closed forms, brute force at d_k = d_v = 4, invariants, library
+ * routines).  No function is "parity unpinned".
+ */
+#include "stq_oracle.h"
+
+#include <cmath>
+#include <cstring>
+#include <vector>
+#include <algorithm>
+
+static const int ORC_SUM_BLOCK = 32;
+
+extern "C" int orc_sum_block(void) { return ORC_SUM_BLOCK; }
+
+/* ------------------------------------------------------------------------ */
+/* format helpers                                                           */
+/* ------------------------------------------------------------------------ */
+
+static int group_of_row(const orc_format *f, int s)
+{
+    int acc = 0;
+    for (int g = 0; g < f->n_groups; ++g) {
+        acc += f->group_rows[g];
+        if (s < acc) return g;
+    }
+    return -1;
+}
+
+extern "C" int orc_format_check(const orc_format *f)
+{
+    if (!f) return -1;
+    if (f->d_k < 1 || f->d_v < 1 || f->d_k > 4096 || f->d_v > 4096) return -2;
+    if (f->n_groups < 1 || f->n_groups > ORC_MAX_GROUPS) return -3;
+    int total = 0;
+    for (int g = 0; g < f->n_groups; ++g) {
+        if (f->group_rows[g] < 1) return -4;
+        total += f->group_rows[g];
+        int kind = f->group_kind[g];
+        if (kind == ORC_KIND_INT) {
+            if (f->group_bits[g] < 2 || f->group_bits[g] > 8) return -5;
+        } else if (kind != ORC_KIND_FP16 && kind != ORC_KIND_FP32) {
+            return -6;
+        }
+    }
+    if (total != f->d_k) return -7;
+    return 0;
+}
+
+extern "C" int orc_row_kind(const orc_format *f, int s)
+{
+    return f->group_kind[group_of_row(f, s)];
+}
+
+extern "C" int orc_row_qmax(const orc_format *f, int s)
+{
+    int g = group_of_row(f, s);
+    if (f->group_kind[g] != ORC_KIND_INT) return 0;
+    return (1 << (f->group_bits[g] - 1)) - 1;
+}
+
+/* Planes of a b-bit code: the binary decomposition of b, widest plane first,
+ * the widest plane holding the lowest bits.  FP16 rows are one 16-bit plane. */
+static int planes_of(int kind, int bits, int width[3], int low[3])
+{
+    if (kind == ORC_KIND_FP16) { width[0] = 16; low[0] = 0; return 1; }
+    if (bits == 8) { width[0] = 8; low[0] = 0; return 1; }
+    int n = 0, lo = 0;
+    for (int w = 4; w >= 1; w >>= 1) {
+        if (bits & w) { width[n] = w; low[n] = lo; lo += w; ++n; }
+    }
+    return n;
+}
+
+static int packable(const orc_format *f)
+{
+    if (orc_format_check(f) != 0) return 0;
+    if (f->d_k != 128 || f->d_v != 128) return 0;
+    for (int g = 0; g < f->n_groups; ++g) {
+        if (f->group_rows[g] % 16 != 0) return 0;
+        if (f->group_kind[g] == ORC_KIND_FP32) return 0;
+    }
+    return 1;
+}
+
+static int n_int_rows(const orc_format *f)
+{
+    int n = 0;
+    for (int g = 0; g < f->n_groups; ++g)
+        if (f->group_kind[g] == ORC_KIND_INT) n += f->group_rows[g];
+    return n;
+}
+
+extern "C" long orc_page_bytes(const orc_format *f)
+{
+    if (!packable(f)) return -1;
+    long bytes = 0;
+    for (int blk = 0; blk < 8; ++blk) {
+        int g = group_of_row(f, 16 * blk);
+        int width[3], low[3];
+        int np = planes_of(f->group_kind[g], f->group_bits[g], width, low);
+        for (int p = 0; p < np; ++p) bytes += 256L * width[p];
+    }
+    bytes += 4L * n_int_rows(f);
+    if (f->col_scales) bytes += 4L * 128;
+    return bytes;
+}
+
+/* ------------------------------------------------------------------------ */
+/* scalar building blocks                                                   */
+/* ------------------------------------------------------------------------ */
+
+static float bits_to_f32(uint32_t u) { float x; std::memcpy(&x, &u, 4); return x; }
+static uint32_t f32_to_bits(float x) { uint32_t u; std::memcpy(&u, &x, 4); return u; }
+
+/* IEEE 754 binary16, round to nearest, ties to even, with subnormals;
+ * written from the format's definition: value = (-1)^s 2^(e-15) (1 + m/1024)
+ * for 1 <= e <= 30, (-1)^s 2^-14 (m/1024) for e = 0. */
+extern "C" uint16_t orc_f32_to_f16_rn(float x)
+{
+    uint32_t u = f32_to_bits(x);
+    uint16_t sign = (uint16_t)((u >> 16) & 0x8000u);
+    float ax = std::fabs(x);
+    if (std::isnan(x)) return (uint16_t)(sign | 0x7E00u);
+    if (std::isinf(x)) return (uint16_t)(sign | 0x7C00u);
+    /* largest finite half is 65504; the midpoint to the next (virtual) value
+     * 65536 is 65520, which ties to the even significand, i.e. overflows */
+    if (ax >= 65520.0f) return (uint16_t)(sign | 0x7C00u);
+    if (ax < 0x1p-14f) {
+        /* subnormal range: multiples of 2^-24 */
+        double t = (double)ax * 0x1p24;          /* exact */
+        double n = std::nearbyint(t);            /* ties to even */
+        return (uint16_t)(sign | (uint16_t)n);   /* n == 1024 is the smallest normal */
+    }
+    int e = std::ilogb(ax);                      /* -14 .. 15 */
+    double t = std::ldexp((double)ax, 10 - e);   /* in [1024, 2048), exact */
+    double n = std::nearbyint(t);
+    if (n >= 2048.0) { n = 1024.0; e += 1; }
+    if (e > 15) return (uint16_t)(sign | 0x7C00u);
+    return (uint16_t)(sign | (uint16_t)((e + 15) << 10) | (uint16_t)((int)n - 1024));
+}
+
+extern "C" float orc_f16_to_f32(uint16_t h)
+{
+    int s = (h >> 15) & 1, e = (h >> 10) & 0x1F, m = h & 0x3FF;
+    double v;
+    if (e == 0) v = std::ldexp((double)m, -24);
+    else if (e == 31) v = m ? NAN : INFINITY;
+    else v = std::ldexp((double)(1024 + m), e - 25);
+    return (float)(s ? -v : v);
+}
+
+/* a / b rounded toward zero (a, b > 0 finite): the largest float q with
+ * q * b <= a.  Products of two floats are exact in double. */
+extern "C" float orc_div_rz(float a, float b)
+{
+    float q = (float)((double)a / (double)b);
+    while ((double)q * (double)b > (double)a) q = std::nextafter(q, 0.0f);
+    for (;;) {
+        float up = std::nextafter(q, INFINITY);
+        if ((double)up * (double)b <= (double)a) q = up; else break;
+    }
+    return q;
+}
+
+extern "C" void orc_f32_to_f16_rn_n(const float *x, uint16_t *out, long n)
+{
+    for (long i = 0; i < n; ++i) out[i] = orc_f32_to_f16_rn(x[i]);
+}
+
+extern "C" void orc_f16_to_f32_n(const uint16_t *x, float *out, long n)
+{
+    for (long i = 0; i < n; ++i) out[i] = orc_f16_to_f32(x[i]);
+}
+
+extern "C" void orc_div_rz_n(const float *a, const float *b, float *out, long n)
+{
+    for (long i = 0; i < n; ++i) out[i] = orc_div_rz(a[i], b[i]);
+}
+
+/* Philox-4x32-10, the counter-based generator of Salmon, Moraes, Dror and
+ * Shaw, "Parallel random numbers: as easy as 1, 2, 3" (SC'11): ten rounds of
+ * a multiply-xor bijection on a 128-bit counter, the 64-bit key bumped by the
+ * Weyl constants between rounds. */
+extern "C" void orc_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4])
+{
+    uint32_t x0 = ctr[0], x1 = ctr[1], x2 = ctr[2], x3 = ctr[3];
+    uint32_t k0 = key[0], k1 = key[1];
+    for (int round = 0; round < 10; ++round) {
+        if (round > 0) { k0 += 0x9E3779B9u; k1 += 0xBB67AE85u; }
+        uint64_t p0 = (uint64_t)0xD2511F53u * (uint64_t)x0;
+        uint64_t p1 = (uint64_t)0xCD9E8D57u * (uint64_t)x2;
+        uint32_t hi0 = (uint32_t)(p0 >> 32), lo0 = (uint32_t)p0;
+        uint32_t hi1 = (uint32_t)(p1 >> 32), lo1 = (uint32_t)p1;
+        uint32_t y0 = hi1 ^ x1 ^ k0;
+        uint32_t y1 = lo1;
+        uint32_t y2 = hi0 ^ x3 ^ k1;
+        uint32_t y3 = lo0;
+        x0 = y0; x1 = y1; x2 = y2; x3 = y3;
+    }
+    out[0] = x0; out[1] = x1; out[2] = x2; out[3] = x3;
+}
+
+/* Stochastic-rounding offset for element (s, j) of page (b, h) at a step.
+ * One Philox call serves a 2-row x 4-column tile: counter
+ * (tile index, step, request, head), key = the 64-bit seed.  Word
+ * 2*(s & 1) + ((j >> 1) & 1) of the output holds columns j & ~1 (high 16 bits)
+ * and j | 1 (low 16 bits).  delta = (h16 - 32767.5) / 65536, exactly. */
+extern "C" float orc_sr_delta(uint64_t seed, uint32_t step, uint32_t b, uint32_t h,
+                              int s, int j, int d_v)
+{
+    uint32_t quads = (uint32_t)((d_v + 3) / 4);
+    uint32_t ctr[4] = { (uint32_t)(s >> 1) * quads + (uint32_t)(j >> 2), step, b, h };
+    uint32_t key[2] = { (uint32_t)seed, (uint32_t)(seed >> 32) };
+    uint32_t out[4];
+    orc_philox4x32_10(ctr, key, out);
+    uint32_t word = out[((s & 1) << 1) | ((j >> 1) & 1)];
+    uint32_t h16 = (j & 1) ? (word & 0xFFFFu) : (word >> 16);
+    return (float)(2 * (int)h16 - 65535) * 0x1p-17f;
+}
+
+/* ------------------------------------------------------------------------ */
+/* requantization of one stored row (shared by quantize and step)          */
+/* ------------------------------------------------------------------------ */
+
+static double dist_to_half(double x)
+{
+    return std::fabs(x - (std::floor(x) + 0.5));
+}
+
+static double f16_margin(float x)
+{
+    double ax = std::fabs((double)x);
+    double spacing;
+    if (ax < 0x1p-14) spacing = 0x1p-24;
+    else spacing = std::ldexp(1.0, std::ilogb(ax) - 10);
+    return dist_to_half(ax / spacing);
+}
+
+static void requant_row(const orc_format *f, int s, const float *Tp, orc_page *p,
+                        uint64_t seed, uint32_t step, uint32_t b, uint32_t h,
+                        int use_sr, double *margin)
+{
+    const int d_v = f->d_v;
+    const int kind = orc_row_kind(f, s);
+    int32_t *code = p->code + (size_t)s * d_v;
+    if (kind == ORC_KIND_FP32) {
+        for (int j = 0; j < d_v; ++j) {
+            code[j] = (int32_t)f32_to_bits(Tp[j]);
+            if (margin) margin[j] = INFINITY;
+        }
+        p->r[s] = 0.0f;
+        return;
+    }
+    if (kind == ORC_KIND_FP16) {
+        for (int j = 0; j < d_v; ++j) {
+            code[j] = (int32_t)orc_f32_to_f16_rn(Tp[j]);
+            if (margin) margin[j] = f16_margin(Tp[j]);
+        }
+        p->r[s] = 0.0f;
+        return;
+    }
+    const int qmax = orc_row_qmax(f, s);
+    float m = 0.0f;
+    for (int j = 0; j < d_v; ++j) {
+        float a = std::fabs(Tp[j]);
+        if (a > m) m = a;
+    }
+    float r, inv;
+    if (m > 0.0f) {
+        r = m / (float)qmax;
+        inv = orc_div_rz((float)qmax, m);
+    } else {
+        r = 0.0f;
+        inv = 0.0f;
+    }
+    p->r[s] = r;
+    for (int j = 0; j < d_v; ++j) {
+        double x = (double)Tp[j] * (double)inv;    /* exact */
+        double zr;
+        if (!use_sr) {
+            zr = std::nearbyint(x);
+            if (margin) margin[j] = dist_to_half(x);
+        } else {
+            float delta = orc_sr_delta(seed, step, b, h, s, j, d_v);
+            float w = std::fmaf(Tp[j], inv, delta);
+            zr = std::nearbyint((double)w);
+            if (margin) margin[j] = dist_to_half(x + (double)delta);
+        }
+        if (!(zr == zr)) zr = 0.0;                 /* non-finite input */
+        if (zr > qmax) zr = qmax;
+        if (zr < -qmax) zr = -qmax;
+        code[j] = (int32_t)zr;
+    }
+}
+
+/* value held by element (s, j): the integer code, or the float it encodes */
+static float element_value(const orc_format *f, const orc_page *p, int s, int j)
+{
+    int32_t c = p->code[(size_t)s * f->d_v + j];
+    int kind = orc_row_kind(f, s);
+    if (kind == ORC_KIND_INT) return (float)c;
+    if (kind == ORC_KIND_FP16) return orc_f16_to_f32((uint16_t)c);
+    return bits_to_f32((uint32_t)c);
+}
+
+/* ------------------------------------------------------------------------ */
+/* calibration: precision map                                               */
+/* ------------------------------------------------------------------------ */
+
+extern "C" int orc_rank_rows(const orc_format *f, int B, int H, const float *S,
+                             const float *row_weight, int32_t *perm_out)
+{
+    if (orc_format_check(f) != 0 || B < 1 || H < 1 || !S || !perm_out) return -1;
+    const int d_k = f->d_k, d_v = f->d_v;
+    std::vector<double> score(d_k);
+    std::vector<int> order(d_k);
+    for (int h = 0; h < H; ++h) {
+        /* score = row-mean-square summed over the batch, times the optional
+         * retention weight; the constant 1 / (B d_v) is left out (it does
+         * not change the ranking) */
+        for (int kap = 0; kap < d_k; ++kap) {
+            double acc = 0.0;
+            for (int b = 0; b < B; ++b) {
+                const float *row = S + (((size_t)b * H + h) * d_k + kap) * d_v;
+                double rs = 0.0;
+                for (int j = 0; j < d_v; ++j) rs += (double)row[j] * (double)row[j];
+                acc += rs;
+            }
+            if (row_weight) acc *= (double)row_weight[(size_t)h * d_k + kap];
+            score[kap] = acc;
+        }
+        for (int kap = 0; kap < d_k; ++kap) order[kap] = kap;
+        /* descending score; equal scores keep ascending key channel */
+        std::stable_sort(order.begin(), order.end(),
+                         [&](int a, int b2) { return score[a] > score[b2]; });
+        /* the best-ranked rows go to the first (widest) group; inside a group
+         * rows are stored in ascending key channel */
+        int32_t *perm = perm_out + (size_t)h * d_k;
+        int start = 0;
+        for (int g = 0; g < f->n_groups; ++g) {
+            int n = f->group_rows[g];
+            std::vector<int> members(order.begin() + start, order.begin() + start + n);
+            std::sort(members.begin(), members.end());
+            for (int i = 0; i < n; ++i) perm[start + i] = members[i];
+            start += n;
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* quantize / dequantize                                                    */
+/* ------------------------------------------------------------------------ */
+
+extern "C" int orc_quantize_page(const orc_format *f, const float *S_nat,
+                                 const int32_t *perm, orc_page *out)
+{
+    if (orc_format_check(f) != 0 || !S_nat || !perm || !out) return -1;
+    const int d_k = f->d_k, d_v = f->d_v;
+    std::vector<float> ic(d_v);
+    for (int j = 0; j < d_v; ++j) {
+        float c = 1.0f;
+        if (f->col_scales) {
+            float m = 0.0f;
+            for (int kap = 0; kap < d_k; ++kap) {
+                float a = std::fabs(S_nat[(size_t)kap * d_v + j]);
+                if (a > m) m = a;
+            }
+            c = (m > 0.0f) ? m : 1.0f;
+        }
+        out->c[j] = c;
+        ic[j] = f->col_scales ? 1.0f / c : 1.0f;
+    }
+    std::vector<float> T(d_v);
+    for (int s = 0; s < d_k; ++s) {
+        const float *row = S_nat + (size_t)perm[s] * d_v;
+        for (int j = 0; j < d_v; ++j) T[j] = row[j] * ic[j];
+        /* the initial quantization always rounds to nearest */
+        requant_row(f, s, T.data(), out, 0, 0, 0, 0, 0, nullptr);
+    }
+    return 0;
+}
+
+extern "C" int orc_dequantize_page(const orc_format *f, const orc_page *p,
+                                   const int32_t *perm, float *S_nat)
+{
+    if (orc_format_check(f) != 0 || !p || !perm || !S_nat) return -1;
+    const int d_k = f->d_k, d_v = f->d_v;
+    for (int s = 0; s < d_k; ++s) {
+        int kind = orc_row_kind(f, s);
+        float rs = (kind == ORC_KIND_INT) ? p->r[s] : 1.0f;
+        for (int j = 0; j < d_v; ++j) {
+            float x = element_value(f, p, s, j);
+            float c = f->col_scales ? p->c[j] : 1.0f;
+            S_nat[(size_t)perm[s] * d_v + j] = (x * rs) * c;
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* decode step: canonical fp32 evaluation                                   */
+/* ------------------------------------------------------------------------ */
+
+static float tree_sum(const float *P, int n)
+{
+    if (n == 1) return P[0];
+    int m = (n + 1) / 2;
+    return tree_sum(P, m) + tree_sum(P + m, n - m);
+}
+
+/* out_j = sum over stored rows s of w[perm[s]] * X[s][j], in the canonical
+ * blocked order */
+static void column_sum(const orc_format *f, const int32_t *perm, const float *w_nat,
+                       const float *X, float *out)
+{
+    const int d_k = f->d_k, d_v = f->d_v;
+    const int nb = (d_k + ORC_SUM_BLOCK - 1) / ORC_SUM_BLOCK;
+    std::vector<float> P(nb);
+    for (int j = 0; j < d_v; ++j) {
+        for (int blk = 0; blk < nb; ++blk) {
+            float acc = 0.0f;
+            int s_end = std::min(d_k, (blk + 1) * ORC_SUM_BLOCK);
+            for (int s = blk * ORC_SUM_BLOCK; s < s_end; ++s)
+                acc = std::fmaf(w_nat[perm[s]], X[(size_t)s * d_v + j], acc);
+            P[blk] = acc;
+        }
+        out[j] = tree_sum(P.data(), nb);
+    }
+}
+
+extern "C" int orc_step_f32(const orc_format *f, orc_page *page, const int32_t *perm,
+                            const float *q, const float *k, const float *v,
+                            const float *alpha, float beta, float *o_out,
+                            uint64_t seed, uint32_t step, uint32_t b, uint32_t h,
+                            float *Tp_out, double *margin_out)
+{
+    if (orc_format_check(f) != 0 || !page || !perm || !q || !k || !v || !alpha || !o_out)
+        return -1;
+    const int d_k = f->d_k, d_v = f->d_v;
+    std::vector<float> ic(d_v), a(d_k), T((size_t)d_k * d_v), Tp((size_t)d_k * d_v);
+    std::vector<float> u(d_v), e(d_v), ot(d_v);
+
+    for (int j = 0; j < d_v; ++j) ic[j] = f->col_scales ? 1.0f / page->c[j] : 1.0f;
+
+    /* dequantize into column-normalised units and decay: T = z * (alpha r) */
+    for (int s = 0; s < d_k; ++s) {
+        float al = f->gate_vector ? alpha[perm[s]] : alpha[0];
+        a[s] = (orc_row_kind(f, s) == ORC_KIND_INT) ? al * page->r[s] : al;
+        for (int j = 0; j < d_v; ++j)
+            T[(size_t)s * d_v + j] = element_value(f, page, s, j) * a[s];
+    }
+    /* prediction (A S)^T k, then the error e = v - prediction (both / c) */
+    column_sum(f, perm, k, T.data(), u.data());
+    for (int j = 0; j < d_v; ++j) e[j] = v[j] * ic[j] - u[j];
+    /* rank-1 delta update T' = T + (beta k) e^T */
+    for (int s = 0; s < d_k; ++s) {
+        float bk = beta * k[perm[s]];
+        for (int j = 0; j < d_v; ++j) {
+            size_t i = (size_t)s * d_v + j;
+            Tp[i] = std::fmaf(bk, e[j], T[i]);
+        }
+    }
+    /* readout o = S'^T q */
+    column_sum(f, perm, q, Tp.data(), ot.data());
+    for (int j = 0; j < d_v; ++j) o_out[j] = f->col_scales ? page->c[j] * ot[j] : ot[j];
+    if (Tp_out) std::memcpy(Tp_out, Tp.data(), sizeof(float) * Tp.size());
+    /* requantize in place; c is unchanged */
+    for (int s = 0; s < d_k; ++s)
+        requant_row(f, s, Tp.data() + (size_t)s * d_v, page, seed, step, b, h,
+                    f->stochastic, margin_out ? margin_out + (size_t)s * d_v : nullptr);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* decode step: plain definition in fp64                                    */
+/* ------------------------------------------------------------------------ */
+
+extern "C" int orc_step_f64(const orc_format *f, const orc_page *page, const int32_t *perm,
+                            const float *q, const float *k, const float *v,
+                            const float *alpha, float beta, double *o_out, double *Sp_out)
+{
+    if (orc_format_check(f) != 0 || !page || !perm || !q || !k || !v || !alpha || !o_out)
+        return -1;
+    const int d_k = f->d_k, d_v = f->d_v;
+    std::vector<double> AS((size_t)d_k * d_v), Sp((size_t)d_k * d_v), pred(d_v);
+    /* S in natural key order, in double, then A S */
+    for (int s = 0; s < d_k; ++s) {
+        int kap = perm[s];
+        int kind = orc_row_kind(f, s);
+        double rs = (kind == ORC_KIND_INT) ? (double)page->r[s] : 1.0;
+        double al = f->gate_vector ? (double)alpha[kap] : (double)alpha[0];
+        for (int j = 0; j < d_v; ++j) {
+            double c = f->col_scales ? (double)page->c[j] : 1.0;
+            double Sij = (double)element_value(f, page, s, j) * rs * c;
+            AS[(size_t)kap * d_v + j] = al * Sij;
+        }
+    }
+    for (int j = 0; j < d_v; ++j) {
+        double acc = 0.0;
+        for (int kap = 0; kap < d_k; ++kap) acc += (double)k[kap] * AS[(size_t)kap * d_v + j];
+        pred[j] = acc;
+    }
+    for (int kap = 0; kap < d_k; ++kap)
+        for (int j = 0; j < d_v; ++j)
+            Sp[(size_t)kap * d_v + j] = AS[(size_t)kap * d_v + j]
+                                        + (double)beta * (double)k[kap] * ((double)v[j] - pred[j]);
+    for (int j = 0; j < d_v; ++j) {
+        double acc = 0.0;
+        for (int kap = 0; kap < d_k; ++kap) acc += (double)q[kap] * Sp[(size_t)kap * d_v + j];
+        o_out[j] = acc;
+    }
+    if (Sp_out) std::memcpy(Sp_out, Sp.data(), sizeof(double) * Sp.size());
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* packed byte layout                                                       */
+/* ------------------------------------------------------------------------ */
+/*
+ * A page is: the code region, then r (fp32, one per INT row, stored order),
+ * then c (fp32 x 128) when the format has column scales.
+ *
+ * The code region is eight blocks of 16 stored rows in order.  A block is the
+ * planes of its rows' codes, widest plane first (an INT code of b bits is
+ * split into planes of widths given by the binary decomposition of b, the
+ * widest plane holding the low bits; an FP16 row is one 16-bit plane).  INT
+ * codes are stored biased: u = z + 2^(b-1).
+ *
+ * A plane of width w covers 16 rows x 128 columns in 256 w bytes.  Column
+ * quad l (columns 4l .. 4l+3) owns 2w little-endian 32-bit words of it.  For
+ * w <= 8, word n holds rows n*(8/w) + sigma, sigma = 0 .. 8/w - 1: column
+ * 4l + beta sits in byte beta, bits [w sigma, w sigma + w).  For w = 16, word n
+ * holds row n/2, columns 4l + 2(n%2) (low half) and 4l + 2(n%2) + 1 (high
+ * half).  The words of one quad are grouped into chunks of 16 bytes (8 bytes
+ * for w = 1), and chunk t of quad l sits at ((t * 32) + l) * chunk_bytes.
+ */
+
+static size_t lane_word_offset(int w, int lane, int n)
+{
+    int cw = (w == 1) ? 2 : 4;   /* words per chunk */
+    return ((size_t)(n / cw) * 32 + lane) * (size_t)(4 * cw) + (size_t)(n % cw) * 4;
+}
+
+static uint32_t load_u32(const uint8_t *p)
+{
+    return (uint32_t)p[0] | ((uint32_t)p[1] << 8) | ((uint32_t)p[2] << 16) | ((uint32_t)p[3] << 24);
+}
+
+static void store_u32(uint8_t *p, uint32_t x)
+{
+    p[0] = (uint8_t)x; p[1] = (uint8_t)(x >> 8); p[2] = (uint8_t)(x >> 16); p[3] = (uint8_t)(x >> 24);
+}
+
+extern "C" int orc_pack_page(const orc_format *f, const orc_page *p, uint8_t *bytes)
+{
+    if (!packable(f) || !p || !bytes) return -1;
+    size_t off = 0;
+    for (int blk = 0; blk < 8; ++blk) {
+        int s0 = 16 * blk;
+        int g = group_of_row(f, s0);
+        int kind = f->group_kind[g], bits = f->group_bits[g];
+        int width[3], low[3];
+        int np = planes_of(kind, bits, width, low);
+        int bias = (kind == ORC_KIND_INT) ? (1 << (bits - 1)) : 0;
+        for (int pl = 0; pl < np; ++pl) {
+            int w = width[pl];
+            uint8_t *plane = bytes + off;
+            for (int lane = 0; lane < 32; ++lane) {
+                for (int n = 0; n < 2 * w; ++n) {
+                    uint32_t word = 0;
+                    if (w == 16) {
+                        int s = s0 + n / 2;
+                        int j = 4 * lane + 2 * (n % 2);
+                        uint32_t lo = (uint32_t)p->code[(size_t)s * 128 + j] & 0xFFFFu;
+                        uint32_t hi = (uint32_t)p->code[(size_t)s * 128 + j + 1] & 0xFFFFu;
+                        word = lo | (hi << 16);
+                    } else {
+                        int rows_per_word = 8 / w;
+                        for (int sig = 0; sig < rows_per_word; ++sig) {
+                            int s = s0 + n * rows_per_word + sig;
+                            for (int beta = 0; beta < 4; ++beta) {
+                                int j = 4 * lane + beta;
+                                uint32_t u = (uint32_t)(p->code[(size_t)s * 128 + j] + bias);
+                                uint32_t part = (u >> low[pl]) & ((1u << w) - 1u);
+                                word |= part << (8 * beta + w * sig);
+                            }
+                        }
+                    }
+                    store_u32(plane + lane_word_offset(w, lane, n), word);
+                }
+            }
+            off += 256 * (size_t)w;
+        }
+    }
+    for (int s = 0; s < 128; ++s) {
+        if (orc_row_kind(f, s) != ORC_KIND_INT) continue;
+        store_u32(bytes + off, f32_to_bits(p->r[s]));
+        off += 4;
+    }
+    if (f->col_scales) {
+        for (int j = 0; j < 128; ++j) { store_u32(bytes + off, f32_to_bits(p->c[j])); off += 4; }
+    }
+    return 0;
+}
+
+extern "C" int orc_unpack_page(const orc_format *f, const uint8_t *bytes, orc_page *p)
+{
+    if (!packable(f) || !p || !bytes) return -1;
+    size_t off = 0;
+    for (int i = 0; i < 128 * 128; ++i) p->code[i] = 0;
+    for (int blk = 0; blk < 8; ++blk) {
+        int s0 = 16 * blk;
+        int g = group_of_row(f, s0);
+        int kind = f->group_kind[g], bits = f->group_bits[g];
+        int width[3], low[3];
+        int np = planes_of(kind, bits, width, low);
+        for (int pl = 0; pl < np; ++pl) {
+            int w = width[pl];
+            const uint8_t *plane = bytes + off;
+            for (int lane = 0; lane < 32; ++lane) {
+                for (int n = 0; n < 2 * w; ++n) {
+                    uint32_t word = load_u32(plane + lane_word_offset(w, lane, n));
+                    if (w == 16) {
+                        int s = s0 + n / 2;
+                        int j = 4 * lane + 2 * (n % 2);
+                        p->code[(size_t)s * 128 + j] = (int32_t)(word & 0xFFFFu);
+                        p->code[(size_t)s * 128 + j + 1] = (int32_t)(word >> 16);
+                    } else {
+                        int rows_per_word = 8 / w;
+                        for (int sig = 0; sig < rows_per_word; ++sig) {
+                            int s = s0 + n * rows_per_word + sig;
+                            for (int beta = 0; beta < 4; ++beta) {
+                                int j = 4 * lane + beta;
+                                uint32_t part = (word >> (8 * beta + w * sig)) & ((1u << w) - 1u);
+                                p->code[(size_t)s * 128 + j] |= (int32_t)(part << low[pl]);
+                            }
+                        }
+                    }
+                }
+            }
+            off += 256 * (size_t)w;
+        }
+    }
+    /* remove the bias from INT rows */
+    for (int s = 0; s < 128; ++s) {
+        if (orc_row_kind(f, s) != ORC_KIND_INT) continue;
+        int bias = 1 << (f->group_bits[group_of_row(f, s)] - 1);
+        for (int j = 0; j < 128; ++j) p->code[(size_t)s * 128 + j] -= bias;
+    }
+    for (int s = 0; s < 128; ++s) {
+        if (orc_row_kind(f, s) != ORC_KIND_INT) { p->r[s] = 0.0f; continue; }
+        p->r[s] = bits_to_f32(load_u32(bytes + off));
+        off += 4;
+    }
+    for (int j = 0; j < 128; ++j) {
+        if (f->col_scales) { p->c[j] = bits_to_f32(load_u32(bytes + off)); off += 4; }
+        else p->c[j] = 1.0f;
+    }
+    return 0;
+}
+
+extern "C" int orc_decode_step_pages(const orc_format *f, int B, int H, uint8_t *pages,
+                                     const int32_t *perm, const float *q, const float *k,
+                                     const float *v, const float *alpha, const float *beta,
+                                     float *o, uint64_t seed, uint32_t step,
+                                     long page_begin, long page_end)
+{
+    if (!packable(f) || B < 1 || H < 1 || !pages || !perm) return -1;
+    long pb = orc_page_bytes(f);
+    long n_pages = (long)B * H;
+    if (page_begin < 0 || page_end > n_pages || page_begin > page_end) return -2;
+    std::vector<int32_t> code(128 * 128);
+    std::vector<float> r(128), c(128);
+    orc_page pg = { code.data(), r.data(), c.data() };
+    for (long pi = page_begin; pi < page_end; ++pi) {
+        uint32_t b = (uint32_t)(pi / H), h = (uint32_t)(pi % H);
+        uint8_t *bytes = pages + (size_t)pi * pb;
+        orc_unpack_page(f, bytes, &pg);
+        const float *al = f->gate_vector ? alpha + (size_t)pi * 128 : alpha + pi;
+        orc_step_f32(f, &pg, perm + (size_t)h * 128, q + (size_t)pi * 128, k + (size_t)pi * 128,
+                     v + (size_t)pi * 128, al, beta[pi], o + (size_t)pi * 128,
+                     seed, step, b, h, nullptr, nullptr);
+        orc_pack_page(f, &pg, bytes);
+    }
+    return 0;
+}

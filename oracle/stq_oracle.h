@@ -1,0 +1,142 @@
+/*
+ * stq_oracle.h -- plain, single-threaded CPU oracle for the quantized
+ * Delta-rule recurrent-state decode step.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may include, link,
+ * load or execute this code: only tests/, __graft_entry__.smoke() and the
+ * cpu_baseline / reference legs of bench.py use it.  It shares no code,
+ * header, table or constant generator with the CUDA library.
+ *
+ * What it computes, and where the pages say so:
+ *   - the state S in R^{d_k x d_v} per (request, head); fp32, 128 x 128 in the
+ *     serving setting ("STEPQuant" landing page, Fig. 5 / Figure B2 caption:
+ *     128x128 states; freedom251 post, "Memory and speed gains": 144 MiB FP32
+ *     per request = 2,304 heads x 128 x 128 x 4 B);
+ *   - key rows split into groups of different bit widths, dequantized as
+ *     z_ij * r_i * c_j with a key-row scale r and a value-column scale c
+ *     ("DAMP" card page, STEPQuant abstract; freedom251 post, "STEPQuant:
+ *     precision can be allocated selectively");
+ *   - the DAMP-style format: selected key channels in FP16, the rest INT8
+ *     with stochastic rounding (freedom251 post, "DAMP: accuracy depends on
+ *     the task");
+ *   - the delta rule S <- S(I - k k^T) + v k^T in the d_v x d_k convention
+ *     (dev.to post, "The state is a running sum, not a buffer"), here in the
+ *     d_k x d_v convention with a decay gate alpha and a write strength beta:
+ *       S' = A S + beta k (v - (A S)^T k)^T,  A = alpha I (GDN) or diag(alpha) (KDA),
+ *       o  = S'^T q.
+ *
+ * Conventions: stored row s (group order), natural key channel perm[s].
+ * Codes of INT rows are signed integers z in [-qmax, qmax], qmax = 2^(b-1)-1.
+ * Every function returns 0 on success and a negative value on bad arguments.
+ */
+#ifndef STQ_ORACLE_H
+#define STQ_ORACLE_H
+
+#include <stdint.h>
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum { ORC_KIND_INT = 0, ORC_KIND_FP16 = 1, ORC_KIND_FP32 = 2 };
+
+#define ORC_MAX_GROUPS 8
+
+/* Row-group description.  Groups are listed widest first; their row counts
+ * sum to d_k.  FP32 rows are an oracle-only kind (an unquantized state, used
+ * to check the retrieval invariant); the packed byte layout does not hold
+ * them. */
+typedef struct {
+    int d_k, d_v;
+    int n_groups;
+    int group_rows[ORC_MAX_GROUPS];
+    int group_kind[ORC_MAX_GROUPS];
+    int group_bits[ORC_MAX_GROUPS];
+    int col_scales;   /* 1: per-column scale c_j; 0: c_j == 1 */
+    int stochastic;   /* 1: stochastic rounding on INT rows; 0: round to nearest even */
+    int gate_vector;  /* 1: alpha is a vector over key channels (KDA); 0: scalar (GDN) */
+} orc_format;
+
+/* An unpacked page.  code[s*d_v + j] holds, for an INT row, the signed code;
+ * for an FP16 row, the 16 raw bits; for an FP32 row, the 32 raw bits.
+ * r[s] is the row scale (INT rows only; 0 elsewhere), c[j] the column scale
+ * (1 when the format has none). */
+typedef struct {
+    int32_t *code;
+    float *r;
+    float *c;
+} orc_page;
+
+/* Sum-block size of the canonical fp32 column reductions (see stq_oracle.cpp). */
+int orc_sum_block(void);
+
+int orc_format_check(const orc_format *f);
+int orc_row_qmax(const orc_format *f, int s);     /* qmax of stored row s, 0 for float rows */
+int orc_row_kind(const orc_format *f, int s);
+long orc_page_bytes(const orc_format *f);          /* packed bytes per page (d = 128 formats) */
+
+/* ---- calibration: precision map (per head, shared by the batch) ---------- */
+/* S: [B][H][d_k][d_v] natural order; row_weight: [H][d_k] or NULL;
+ * perm_out: [H][d_k], perm_out[h*d_k + s] = natural key channel of stored row s. */
+int orc_rank_rows(const orc_format *f, int B, int H, const float *S,
+                  const float *row_weight, int32_t *perm_out);
+
+/* ---- quantize / dequantize one page ------------------------------------- */
+int orc_quantize_page(const orc_format *f, const float *S_nat, const int32_t *perm,
+                      orc_page *out);
+int orc_dequantize_page(const orc_format *f, const orc_page *p, const int32_t *perm,
+                        float *S_nat);
+
+/* ---- one decode step on one page: canonical fp32 evaluation -------------
+ * page is updated in place.  alpha points to 1 value (GDN) or d_k values in
+ * natural key order (KDA).  q, k, v: d_k, d_k, d_v values.  o_out: d_v.
+ * Tp_out (optional, d_k*d_v, stored order): the updated state in
+ * column-normalised units before requantization.
+ * margin_out (optional, d_k*d_v, stored order): distance of each element's
+ * pre-rounding value from the nearest rounding boundary, in units of the
+ * row's rounding step (code units for INT rows, fp16 spacing for FP16 rows,
+ * +inf for FP32 rows). */
+int orc_step_f32(const orc_format *f, orc_page *page, const int32_t *perm,
+                 const float *q, const float *k, const float *v,
+                 const float *alpha, float beta, float *o_out,
+                 uint64_t seed, uint32_t step, uint32_t b, uint32_t h,
+                 float *Tp_out, double *margin_out);
+
+/* ---- the same step from the plain definition in fp64 -------------------
+ * Dequantizes the page in double, then S' = A S + beta k (v - (A S)^T k)^T,
+ * o = S'^T q.  Sp_out: d_k*d_v natural order (optional); o_out: d_v. */
+int orc_step_f64(const orc_format *f, const orc_page *page, const int32_t *perm,
+                 const float *q, const float *k, const float *v,
+                 const float *alpha, float beta, double *o_out, double *Sp_out);
+
+/* ---- packed byte layout (d_k = d_v = 128, row groups multiples of 16) ---- */
+int orc_pack_page(const orc_format *f, const orc_page *p, uint8_t *bytes);
+int orc_unpack_page(const orc_format *f, const uint8_t *bytes, orc_page *p);
+
+/* Packed-page step over a range of pages of a [B][H] batch (single thread).
+ * pages: B*H*page_bytes; perm: [H][128]; q,k,v,o: [B][H][128];
+ * alpha: [B][H] or [B][H][128]; beta: [B][H]. */
+int orc_decode_step_pages(const orc_format *f, int B, int H, uint8_t *pages,
+                          const int32_t *perm, const float *q, const float *k,
+                          const float *v, const float *alpha, const float *beta,
+                          float *o, uint64_t seed, uint32_t step,
+                          long page_begin, long page_end);
+
+/* ---- scalar building blocks, exported so tests can pin them ------------- */
+uint16_t orc_f32_to_f16_rn(float x);
+float orc_f16_to_f32(uint16_t h);
+float orc_div_rz(float a, float b);
+/* element-wise loops over the three functions above */
+void orc_f32_to_f16_rn_n(const float *x, uint16_t *out, long n);
+void orc_f16_to_f32_n(const uint16_t *x, float *out, long n);
+void orc_div_rz_n(const float *a, const float *b, float *out, long n);
+void orc_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4]);
+/* stochastic-rounding offset delta in (-1/2, 1/2) for element (s, j) */
+float orc_sr_delta(uint64_t seed, uint32_t step, uint32_t b, uint32_t h,
+                   int s, int j, int d_v);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

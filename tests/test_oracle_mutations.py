@@ -1,0 +1,75 @@
+"""The oracle's pins must catch plausible mistakes.
+
+Each case plants one mistake (a dropped term, a wrong sign, a wrong index, a
+transposed operand, a wrong constant) in a temporary copy of the oracle
+source, builds it, and runs the other oracle pin files against it: the run
+must fail.  The planted copies live only in a temporary directory on the CPU.
+"""
+import os
+import shutil
+import subprocess
+import sys
+import tempfile
+from concurrent.futures import ThreadPoolExecutor
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "stq_oracle.cpp")
+HDR = os.path.join(ROOT, "oracle", "stq_oracle.h")
+PIN_FILES = ["tests/test_oracle_scalars.py", "tests/test_oracle_format.py",
+             "tests/test_oracle_quantize.py", "tests/test_oracle_step.py"]
+
+MUTANTS = {
+    "error sign": ("e[j] = v[j] * ic[j] - u[j];", "e[j] = v[j] * ic[j] + u[j];"),
+    "key index not permuted": ("float bk = beta * k[perm[s]];", "float bk = beta * k[s];"),
+    "readout with k": ("column_sum(f, perm, q, Tp.data(), ot.data());",
+                       "column_sum(f, perm, k, Tp.data(), ot.data());"),
+    "f32 decay dropped": ("a[s] = (orc_row_kind(f, s) == ORC_KIND_INT) ? al * page->r[s] : al;",
+                          "a[s] = (orc_row_kind(f, s) == ORC_KIND_INT) ? page->r[s] : 1.0f;"),
+    "f64 decay dropped": ("AS[(size_t)kap * d_v + j] = al * Sij;", "AS[(size_t)kap * d_v + j] = Sij;"),
+    "f64 prediction transposed": ("acc += (double)k[kap] * AS[(size_t)kap * d_v + j];",
+                                  "acc += (double)k[j] * AS[(size_t)j * d_v + kap];"),
+    "f64 beta dropped": ("+ (double)beta * (double)k[kap] * ((double)v[j] - pred[j]);",
+                         "+ (double)k[kap] * ((double)v[j] - pred[j]);"),
+    "row scale off by one": ("r = m / (float)qmax;", "r = m / (float)(qmax + 1);"),
+    "rounding truncates": ("zr = std::nearbyint(x);", "zr = std::trunc(x);"),
+    "bias wrong": ("int bias = (kind == ORC_KIND_INT) ? (1 << (bits - 1)) : 0;",
+                   "int bias = (kind == ORC_KIND_INT) ? (1 << bits) - 1 : 0;"),
+    "philox key bump": ("k1 += 0xBB67AE85u;", "k1 += 0x9E3779B9u;"),
+    "fp16 ties away": ("double n = std::nearbyint(t);\n    if (n >= 2048.0)",
+                       "double n = std::floor(t + 0.5);\n    if (n >= 2048.0)"),
+    "ranking ascending": ("return score[a] > score[b2];", "return score[a] < score[b2];"),
+    "dequantize drops c": ("S_nat[(size_t)perm[s] * d_v + j] = (x * rs) * c;",
+                           "S_nat[(size_t)perm[s] * d_v + j] = x * rs;"),
+    "sr halves swapped": ("uint32_t h16 = (j & 1) ? (word & 0xFFFFu) : (word >> 16);",
+                          "uint32_t h16 = (j & 1) ? (word >> 16) : (word & 0xFFFFu);"),
+    "column absmax over one row": ("float a = std::fabs(S_nat[(size_t)kap * d_v + j]);",
+                                   "float a = std::fabs(S_nat[(size_t)j]);"),
+}
+
+
+def _run_mutant(name, tmp):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, name
+    d = os.path.join(tmp, "m%d" % list(MUTANTS).index(name))
+    os.makedirs(d)
+    shutil.copy(HDR, d)
+    with open(os.path.join(d, "stq_oracle.cpp"), "w") as fh:
+        fh.write(src.replace(old, new))
+    lib = os.path.join(d, "libmut.so")
+    subprocess.run(["g++", "-std=c++17", "-O2", "-ffp-contract=off", "-fPIC", "-shared", "-o", lib,
+                    os.path.join(d, "stq_oracle.cpp")], check=True)
+    env = dict(os.environ, STQ_ORACLE_LIB=lib)
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider"] + PIN_FILES,
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    return name, r.returncode
+
+
+def test_every_planted_mistake_fails_a_pin():
+    with tempfile.TemporaryDirectory() as tmp:
+        with ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
+            results = list(ex.map(lambda n: _run_mutant(n, tmp), MUTANTS))
+    survivors = [n for n, rc in results if rc == 0]
+    assert not survivors, "mutants not caught: %s" % survivors
