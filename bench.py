@@ -1,0 +1,397 @@
+"""Benchmark of the quantized Delta-rule decode step (one JSON line on stdout).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config I] [--impl ours|reference]
+
+A step is one decode step (unpack, dequant + decay, delta rule, readout,
+requant + repack in place) over every page of the workload's batch; the
+default workload is STEPQuant-style 6-bit GDN, 1024 requests x 32 heads.
+Inputs for all steps are generated on the device before timing; the state
+and per-step inputs (~0.9 GB per step) exceed the 126 MB L2, so no flush is
+needed between steps.  Under torchrun each rank runs its own batch (weak
+scaling, no collective on the data path); time is the max over ranks.
+
+--impl reference times the CPU oracle (single thread, as written) on a
+bounded sample of the same workload; only rank 0 runs it.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from linear_attention_recurrent_delta_b200 import workloads as W  # noqa: E402
+
+METRIC = "decode state-update head-steps/s"
+UNIT = "head-steps/s"
+
+
+def algorithmic_bytes_per_page(spec):
+    """Bytes one page-step must move: codes + r read and written, c read,
+    q, k, v, the gate(s) and beta read, o written (the precision map is
+    L2-resident and not counted)."""
+    code = sum(rows * 128 * (16 if kind == "fp16" else bits) // 8 for rows, kind, bits in spec["groups"])
+    n_int = sum(rows for rows, kind, _ in spec["groups"] if kind == "int")
+    b = 2 * code + 2 * 4 * n_int + (512 if spec["col_scales"] else 0)
+    b += 3 * 512 + (512 if spec["gate_vector"] else 4) + 4 + 512
+    return b
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "linear_attention_recurrent_delta_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as fh:
+            h.update(name.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            return float(json.load(fh)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 6650.0, "fallback"
+
+
+def ncu_traffic(workload_name):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    try:
+        with open(path) as fh:
+            d = json.load(fh)
+    except (OSError, ValueError):
+        return None
+    e = d.get(workload_name)
+    if not e or e.get("kernel_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 200 ms."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = str(gpu_index)
+        self.rows = []
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9 and parts[0] == self.gpu:
+                self.rows.append((time.monotonic(), parts))
+
+    def stop(self, t0=None, t1=None):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=5)
+        rows = [r for t, r in self.rows if (t0 is None or t >= t0) and (t1 is None or t <= t1)]
+        if not rows:   # region shorter than one sampling period: keep the nearest samples
+            rows = [r for _, r in self.rows[-2:]]
+        self.rows = rows
+        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in self.rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.rows)}
+
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def run_gpu(w, steps, warmup, rank, world, sample_clocks=True, e2e_steps=64):
+    from linear_attention_recurrent_delta_b200 import binding as B
+    dev = torch.device("cuda", torch.cuda.current_device())
+    wr = W.Workload(w.index, w.name, w.fmt, w.batch, w.heads, w.steps, w.gate_mu, w.gate_sigma,
+                    w.seed + 7919 * rank)
+    qs = B.QuantizedState(wr.format, wr.batch, wr.heads, device=dev)
+    S = W.initial_state(wr, device=dev)
+    qs.calibrate_and_quantize(S)
+    del S
+    torch.cuda.synchronize()
+    n_in = min(wr.steps, max(steps, warmup, 1))
+    inputs = [W.step_inputs(wr, t, device=dev) for t in range(n_in)]
+    o = torch.empty(wr.batch, wr.heads, 128, device=dev)
+    seed = W.sr_seed(wr)
+    stream = torch.cuda.current_stream()
+
+    def step(t):
+        x = inputs[t % n_in]
+        B.stq_decode_step(qs.state, x["q"], x["k"], x["v"], x["alpha"], x["beta"], o, seed, t, stream)
+
+    for t in range(warmup):
+        step(t)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(torch.cuda.current_device()) if sample_clocks else None
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    h0 = time.monotonic()
+    ev0.record(stream)
+    for t in range(steps):
+        step(warmup + t)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    h1 = time.monotonic()
+    barrier(world)
+    torch.cuda.synchronize()
+    ms = ev0.elapsed_time(ev1)
+    clk = clocks.stop(h0, h1) if clocks else None
+    status = B.stq_device_status(qs.state)
+    if status != B.STQ_OK:
+        raise RuntimeError("device status: %s" % B.stq_status_string(status))
+    ms_max = max_over_ranks(ms, world)
+
+    # end to end through the host-buffer entry point: H2D of the step's inputs
+    # from pinned memory, the step, D2H of o, all inside the timed region
+    host = [{k: v.cpu().pin_memory() for k, v in x.items()} for x in inputs[:min(n_in, 8)]]
+    o_host = torch.empty(wr.batch, wr.heads, 128).pin_memory()
+    io_bytes = B.stq_decode_io_bytes(qs.state)
+    io_buf = torch.empty(io_bytes + 256, dtype=torch.uint8, device=dev)
+    off = (-io_buf.data_ptr()) % 256
+    io = io_buf[off:off + io_bytes]
+    h2d = sum(v.numel() * v.element_size() for v in host[0].values())
+    d2h = o_host.numel() * o_host.element_size()
+    for t in range(3):
+        x = host[t % len(host)]
+        B.stq_decode_step_host(qs.state, x["q"], x["k"], x["v"], x["alpha"], x["beta"], o_host, io, seed, t, stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for t in range(e2e_steps):
+        x = host[t % len(host)]
+        B.stq_decode_step_host(qs.state, x["q"], x["k"], x["v"], x["alpha"], x["beta"], o_host, io, seed, t, stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    barrier(world)
+    del qs, inputs, host, io_buf
+    torch.cuda.empty_cache()
+    return {"ms": ms_max, "clocks": clk, "e2e_ms": e2e_ms, "h2d": h2d, "d2h": d2h,
+            "e2e_steps": e2e_steps}
+
+
+class OracleSample:
+    """The CPU oracle (single thread, as written) stepping a sample of the
+    workload's pages: the first ``n_pages`` pages of a batch whose fp32 state
+    comes from the workload generator and is quantized by the oracle."""
+
+    def __init__(self, w, n_pages):
+        import oracle as O
+        self.O = O
+        self.fmt = O.format_from_spec(w.format)
+        n_pages = max(1, min(n_pages, w.pages))
+        b_s = -(-n_pages // w.heads)
+        self.ws = w.resized(batch=b_s)
+        S = W.initial_state(self.ws).numpy()
+        self.perm = O.rank_rows(self.fmt, S)
+        pb = O.page_bytes(self.fmt)
+        self.n = n_pages
+        self.pages = np.zeros(self.ws.pages * pb, np.uint8)
+        for i in range(n_pages):
+            b, h = divmod(i, w.heads)
+            self.pages[i * pb:(i + 1) * pb] = O.pack_page(self.fmt, O.quantize_page(self.fmt, S[b, h], self.perm[h]))
+        m = self.ws.pages
+        x = W.step_inputs(self.ws, 0)
+        self.x = {k: np.ascontiguousarray(v.numpy().reshape(m, -1)) for k, v in x.items()}
+        self.o = np.zeros((m, 128), np.float32)
+        self.seed = W.sr_seed(w)
+        self.t = 0
+        self.desc = "%d of %d pages (%s, %d heads)" % (n_pages, w.pages, w.name, w.heads)
+
+    def step(self):
+        x = self.x
+        self.O.decode_step_pages(self.fmt, self.ws.batch, self.ws.heads, self.pages, self.perm, x["q"], x["k"],
+                                 x["v"], np.ascontiguousarray(x["alpha"].reshape(-1)),
+                                 np.ascontiguousarray(x["beta"].reshape(-1)), self.o, self.seed, self.t,
+                                 0, self.n)
+        self.t += 1
+        return self.n
+
+
+def oracle_rate(w, budget_s, n_pages=64):
+    """CPU-oracle head-steps/s over about budget_s seconds of work."""
+    smp = OracleSample(w, n_pages)
+    smp.step()
+    done, steps = 0, 0
+    t0 = time.perf_counter()
+    while True:
+        done += smp.step()
+        steps += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    return done / el, "%s x %d steps" % (smp.desc, steps), el
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--config", type=int, default=2)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--ref-seconds", type=float, default=60.0)
+    ap.add_argument("--only", action="store_true", help="skip the other workloads")
+    args = ap.parse_args()
+    w = W.WORKLOADS[args.config]
+    spec = w.format
+    dtype = "f32"
+
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        if rank != 0:
+            return
+        # one step = the oracle over a sample of pages sized so that the whole
+        # run (warm-up + timed steps) takes about args.ref_seconds
+        probe = OracleSample(w, 8)
+        t0 = time.perf_counter()
+        for _ in range(3):
+            probe.step()
+        t_page = (time.perf_counter() - t0) / (3 * probe.n)
+        n_pages = int(max(1, min(w.pages, args.ref_seconds / (max(1, args.steps + args.warmup) * t_page))))
+        smp = OracleSample(w, n_pages)
+        for _ in range(args.warmup):
+            smp.step()
+        t0 = time.perf_counter()
+        done = 0
+        for _ in range(args.steps):
+            done += smp.step()
+        el = time.perf_counter() - t0
+        value = done / el
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": 1000.0 * w.pages / value, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": dtype, "data": "synthetic",
+                "impl": "reference",
+                "config": {"workload": w.name, "batch": w.batch, "heads": w.heads, "d_k": 128, "d_v": 128,
+                           "format": w.fmt, "parallelism": "pages per rank"},
+                "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                                 "sample": "%s per step, %d steps" % (smp.desc, args.steps)},
+                "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return
+
+    world, rank, local = dist_setup(args.gpus)
+    from linear_attention_recurrent_delta_b200 import build as build_mod
+    if rank == 0:
+        build_mod.build()
+    barrier(world)
+    res = run_gpu(w, args.steps, args.warmup, rank, world)
+    pages_total = w.pages * world
+    value = pages_total * args.steps / (res["ms"] / 1000.0)
+    per_launch_s = res["ms"] / 1000.0 / args.steps
+    bpp = algorithmic_bytes_per_page(spec)
+    achieved = bpp * w.pages / per_launch_s / 1e9
+    peak, peak_kind = measured_peak()
+    e2e_value = pages_total * res["e2e_steps"] / (res["e2e_ms"] / 1000.0)
+
+    others = {}
+    if not args.only:
+        for i in (1, 3, 4):
+            if i == args.config:
+                continue
+            wi = W.WORKLOADS[i]
+            r = run_gpu(wi, max(200, args.steps // 3), args.warmup, rank, world, sample_clocks=False, e2e_steps=8)
+            v = wi.pages * world * max(200, args.steps // 3) / (r["ms"] / 1000.0)
+            b = algorithmic_bytes_per_page(wi.format)
+            gbs = b * wi.pages * max(200, args.steps // 3) / (r["ms"] / 1000.0) / 1e9
+            others[wi.name] = {"value": v, "unit": UNIT, "hbm_gbs": gbs, "frac_of_%s_peak" % peak_kind: gbs / peak,
+                               "bytes_per_head_step": b, "pages": wi.pages}
+
+    if rank != 0:
+        return
+    cpu_v, cpu_sample, _ = oracle_rate(w, args.cpu_seconds) if world == 1 else (None, None, None)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": res["ms"] / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": dtype, "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "heads": w.heads, "d_k": 128, "d_v": 128,
+                   "format": w.fmt, "groups": spec["groups"], "col_scales": spec["col_scales"],
+                   "stochastic": spec["stochastic"], "gate_vector": spec["gate_vector"],
+                   "parallelism": "pages per rank" if world > 1 else "single GPU",
+                   "l2": "inputs larger than L2 (%.0f MB moved per step)" % (bpp * w.pages / 1e6)},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": ncu_traffic(w.name),
+                     "peak_kind": peak_kind, "bytes_per_head_step": bpp, "kernel": "stq::decode_kernel"},
+        "cpu_baseline": ({"value": cpu_v, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": cpu_sample}
+                         if cpu_v else None),
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"],
+                "steps": res["e2e_steps"], "entry_point": "stq_decode_step_host"},
+        "gpu_launches": args.steps,
+        "clocks": res["clocks"],
+        "other_workloads": others,
+    }
+    print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,183 @@
+/*
+ * stq.h -- C ABI of the quantized Delta-rule recurrent-state decode step
+ * (Gated DeltaNet / Kimi Delta Attention) for NVIDIA B200 (sm_100a).
+ *
+ * The method.  Per (request b, head h) the recurrent state is
+ * S in R^{128 x 128}, rows = key channels, columns = value channels
+ * ("STEPQuant" landing page, Fig. 5 / Figure B2: 128x128 states).  Its key
+ * rows are split into groups of different bit widths and every element is
+ * stored as z_ij * r_i * c_j with a key-row scale r and a value-column scale
+ * c (DAMP card page, STEPQuant abstract; freedom251 post, "STEPQuant:
+ * precision can be allocated selectively"), or, in the DAMP-style format,
+ * selected key rows in FP16 and the rest INT8 with stochastic rounding
+ * (freedom251 post, "DAMP: accuracy depends on the task").  One decode step
+ * applies the gated delta rule (dev.to post, "The state is a running sum, not
+ * a buffer": S <- S(I - k k^T) + v k^T in the d_v x d_k convention; here the
+ * d_k x d_v convention with a decay gate and a write strength):
+ *     S' = A S + beta k (v - (A S)^T k)^T,  A = alpha I (GDN) or diag(alpha) (KDA)
+ *     o  = S'^T q
+ * and requantizes S' in place.
+ *
+ * Conventions for every entry point:
+ *   - All tensors are caller-owned.  Pointers named d_* are device pointers,
+ *     h_* host pointers.  The library allocates only the host descriptor
+ *     (stq_state); it never allocates device memory and never synchronizes,
+ *     except stq_device_status, which says so.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  All device work is enqueued on it in call order.
+ *   - fp32 tensors are row-major and contiguous: q, k, v, o are [B][H][128];
+ *     a scalar (GDN) alpha is [B][H], a vector (KDA) alpha is [B][H][128] in
+ *     natural key order; beta is [B][H].
+ *   - Errors are returned as stq_status; arguments are checked on the host
+ *     before anything is enqueued, so an error return means nothing was
+ *     enqueued.  Launch failures map to STQ_ERR_CUDA.  A device-side wait that
+ *     runs out (it has a bounded limit) sets the state's status word, read by
+ *     stq_device_status.  Non-finite inputs give unspecified values but never
+ *     fault or hang.
+ */
+#ifndef STQ_H
+#define STQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    STQ_OK = 0,
+    STQ_ERR_INVALID_ARG = 1,      /* null pointer, bad size, overlapping buffers */
+    STQ_ERR_UNSUPPORTED = 2,      /* a format the kernels do not handle */
+    STQ_ERR_BUFFER_TOO_SMALL = 3, /* caller buffer smaller than required */
+    STQ_ERR_MISALIGNED = 4,       /* pointer not aligned as documented */
+    STQ_ERR_CUDA = 5,             /* a CUDA runtime call or launch failed */
+    STQ_ERR_DEVICE_TIMEOUT = 6    /* a bounded device-side wait ran out */
+} stq_status;
+
+typedef enum { STQ_INT = 0, STQ_FP16 = 1 } stq_kind;
+
+#define STQ_MAX_GROUPS 8
+
+/* Row-group format of every page of a state.
+ *   d_k = d_v = 128 (other sizes: STQ_ERR_UNSUPPORTED).
+ *   Groups are listed in stored order, conventionally widest first; the rows
+ *   of the widest group are the best-ranked key channels (calibration,
+ *   stq_calibrate).  group_rows: multiples of 16 summing to 128.
+ *   group_kind: STQ_INT (group_bits in 2..8, symmetric codes in
+ *   [-(2^(b-1)-1), 2^(b-1)-1]) or STQ_FP16 (binary16 values, no row scale).
+ *   col_scales: 1 = a per-column scale c_j is stored; 0 = c_j = 1.
+ *   stochastic: 1 = INT rows are requantized with stochastic rounding (FP16
+ *   rows always round to nearest); 0 = round to nearest even.
+ *   gate_vector: 1 = alpha is a vector over key channels (KDA); 0 = scalar. */
+typedef struct {
+    int d_k, d_v;
+    int n_groups;
+    int group_rows[STQ_MAX_GROUPS];
+    int group_kind[STQ_MAX_GROUPS];
+    int group_bits[STQ_MAX_GROUPS];
+    int col_scales;
+    int stochastic;
+    int gate_vector;
+} stq_format;
+
+typedef struct stq_state stq_state;   /* opaque host descriptor */
+
+/* Bytes of one packed page (one request, one head) of format f; 0 if the
+ * format is invalid or unsupported.  Layout: codes, then fp32 r for each INT
+ * row (stored order), then fp32 c[128] if col_scales; a multiple of 16. */
+size_t stq_page_bytes(const stq_format *f);
+
+/* Bytes of device memory a state of B requests x H heads needs: a 256-byte
+ * header (status word), the precision map [H][128] (uint8, stored row ->
+ * key channel) padded to 256 bytes, then B*H pages, page (b, h) at index
+ * b*H + h.  0 on invalid arguments. */
+size_t stq_state_bytes(const stq_format *f, int batch, int heads);
+
+/* Bind a caller-owned device buffer (>= stq_state_bytes, 256-byte aligned)
+ * to a new host descriptor.  Touches no device memory; the state holds
+ * nothing valid until stq_calibrate (or a caller-written map) and
+ * stq_quantize_state.  Errors: INVALID_ARG (nulls, batch/heads < 1),
+ * UNSUPPORTED (format), MISALIGNED, BUFFER_TOO_SMALL. */
+stq_status stq_state_alloc(const stq_format *f, int batch, int heads,
+                           void *d_buf, size_t buf_bytes, stq_state **out);
+
+/* Free the host descriptor only; the device buffer stays the caller's. */
+void stq_state_free(stq_state *s);
+
+/* Byte offsets inside the state buffer (any output may be NULL). */
+stq_status stq_state_layout(const stq_state *s, size_t *page_bytes, size_t *perm_offset,
+                            size_t *pages_offset, size_t *status_offset);
+
+/* Workspace bytes stq_calibrate needs for this state (fp64 partial scores). */
+size_t stq_calibrate_workspace_bytes(const stq_state *s);
+
+/* Precision map (calibration; DAMP's ranking of key channels, freedom251
+ * post, "DAMP: accuracy depends on the task"; STEPQuant's ranking of key
+ * rows, landing page Fig. 2).  Per head h, key channel kappa scores
+ *     sum_b sum_j S[b][h][kappa][j]^2  x  row_weight[h][kappa]
+ * (the batch's row mean square up to a constant, times an optional retention
+ * weight); channels are ranked by descending score (ties: lower channel
+ * first), the best go to group 0, and inside a group rows are stored in
+ * ascending channel.  d_S: [B][H][128][128] fp32, natural key order, 16-byte
+ * aligned.  d_row_weight: [H][128] fp32 or NULL (weight 1).  d_workspace:
+ * >= stq_calibrate_workspace_bytes, 8-byte aligned, contents on entry
+ * ignored.  Writes the state's map. */
+stq_status stq_calibrate(stq_state *s, const float *d_S, const float *d_row_weight,
+                         void *d_workspace, size_t workspace_bytes, void *stream);
+
+/* Quantize an fp32 state into every page using the state's precision map:
+ * c_j = max_i |S_ij| (1 if 0; 1 without column scales); T = S * (1/c);
+ * INT rows: r = max_j |T| / qmax, codes = round-to-nearest-even of
+ * T * (qmax / max_j |T| rounded toward zero); FP16 rows: binary16(T).
+ * Clears the status word.  d_S as in stq_calibrate. */
+stq_status stq_quantize_state(stq_state *s, const float *d_S, void *stream);
+
+/* One decode step on every page, in place (see the header comment).
+ * d_q, d_k, d_v, d_o: [B][H][128], 16-byte aligned.  d_alpha: [B][H]
+ * (4-byte aligned) or [B][H][128] (16-byte aligned, gate_vector).  d_beta:
+ * [B][H].  None may overlap the state buffer, and d_o may overlap no input.
+ * seed and step feed the stochastic-rounding generator only (Philox-4x32-10,
+ * key = seed, counter = (tile, step, request, head)).  q is used as given. */
+stq_status stq_decode_step(stq_state *s, const float *d_q, const float *d_k, const float *d_v,
+                           const float *d_alpha, const float *d_beta, float *d_o,
+                           uint64_t seed, uint32_t step, void *stream);
+
+/* Device staging bytes stq_decode_step_host needs (q, k, v, alpha, beta, o). */
+size_t stq_decode_io_bytes(const stq_state *s);
+
+/* The same step with host-resident inputs and output: enqueues the
+ * host-to-device copies of h_q, h_k, h_v, h_alpha, h_beta into d_io, the
+ * step, and the device-to-host copy of o into h_o, all on `stream`.  Host
+ * buffers should be pinned for the copies to be asynchronous.  d_io:
+ * >= stq_decode_io_bytes, 256-byte aligned, caller-owned scratch.  The
+ * caller synchronizes the stream before reading h_o. */
+stq_status stq_decode_step_host(stq_state *s, const float *h_q, const float *h_k,
+                                const float *h_v, const float *h_alpha, const float *h_beta,
+                                float *h_o, void *d_io, size_t io_bytes,
+                                uint64_t seed, uint32_t step, void *stream);
+
+/* Dequantize every page to fp32 [B][H][128][128] in natural key order:
+ * S_ij = (z_ij * r_i) * c_j (FP16 rows: h_ij * c_j).  d_S 16-byte aligned. */
+stq_status stq_dequantize_state(const stq_state *s, float *d_S, void *stream);
+
+/* Synchronizes `stream`, then reads the state's status word: STQ_OK, or
+ * STQ_ERR_DEVICE_TIMEOUT if a bounded device wait ran out since the last
+ * clear.  clear != 0 resets the word. */
+stq_status stq_device_status(stq_state *s, void *stream, int clear);
+
+/* Limit of every bounded device-side wait, in nanoseconds (default 1e9).
+ * Test hook: stall_first_wait != 0 makes the next stq_decode_step's first
+ * pipeline wait wait on a barrier nothing ever completes, so it runs out
+ * after the limit, sets the status word and the kernel returns. */
+stq_status stq_set_wait_limit(stq_state *s, uint64_t limit_ns, int stall_first_wait);
+
+const char *stq_status_string(stq_status st);
+
+/* Library version, 100 * major + minor. */
+int stq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* STQ_H */

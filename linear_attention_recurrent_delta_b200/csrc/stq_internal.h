@@ -1,0 +1,45 @@
+// stq_internal.h -- host-side internals shared by the library's .cu files.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/stq.h"
+#include "stq_device.cuh"
+
+struct stq_state {
+    stq_format fmt;
+    int batch, heads;
+    uint8_t *base;               // caller's device buffer
+    size_t buf_bytes;
+    size_t page_bytes, perm_offset, pages_offset, status_offset;
+    stq::DevFormat dev;
+    uint64_t wait_limit_ns;
+    int stall_first_wait;
+};
+
+namespace stq {
+
+constexpr size_t kHeaderBytes = 256;
+constexpr int kStages = 3;           // bulk-copy ring depth of the decode kernel
+
+// Validate a format and build its device constants.  Returns STQ_OK,
+// STQ_ERR_INVALID_ARG or STQ_ERR_UNSUPPORTED.
+stq_status build_dev_format(const stq_format *f, DevFormat *out);
+
+// Persistent-grid size for a kernel: SM count x resident CTAs (cached per
+// device and kernel).
+int persistent_grid(const void *kernel, size_t dyn_smem, long n_units);
+
+// Launchers (return cudaError_t of the launch).
+cudaError_t launch_decode(const stq_state *s, const float *q, const float *k, const float *v,
+                          const float *alpha, const float *beta, float *o, uint64_t seed,
+                          uint32_t step, int stall_first_wait, cudaStream_t stream);
+cudaError_t launch_calibrate(const stq_state *s, const float *S, const float *row_weight,
+                             double *workspace, cudaStream_t stream);
+size_t calibrate_workspace_bytes(int batch, int heads);
+cudaError_t launch_quantize(const stq_state *s, const float *S, cudaStream_t stream);
+cudaError_t launch_dequantize(const stq_state *s, float *S, cudaStream_t stream);
+
+}  // namespace stq
