@@ -301,10 +301,11 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
             if (F.col_scales)
                 ic = make_float4(__fdiv_rn(1.f, c4.x), __fdiv_rn(1.f, c4.y), __fdiv_rn(1.f, c4.z),
                                  __fdiv_rn(1.f, c4.w));
-            const float2 vn01 = __fmul2_rn(make_float2(v4.x, v4.y), make_float2(ic.x, ic.y));
-            const float2 vn23 = __fmul2_rn(make_float2(v4.z, v4.w), make_float2(ic.z, ic.w));
-            e01 = __fadd2_rn(vn01, make_float2(-ua.x, -ua.y));
-            e23 = __fadd2_rn(vn23, make_float2(-ub.x, -ub.y));
+            // e = v (1/c) - u with two roundings.  Scalar __fmul_rn/__fsub_rn:
+            // the compiler fuses an f32x2 multiply feeding an f32x2 add into one
+            // f32x2 fma, which would round once.
+            e01 = make_float2(__fsub_rn(__fmul_rn(v4.x, ic.x), ua.x), __fsub_rn(__fmul_rn(v4.y, ic.y), ua.y));
+            e23 = make_float2(__fsub_rn(__fmul_rn(v4.z, ic.z), ub.x), __fsub_rn(__fmul_rn(v4.w, ic.w), ub.y));
         }
 
         // S4 + S5 partial + row absmax partial
