@@ -205,6 +205,10 @@ def run_gpu(w, steps, warmup, rank, world, sample_clocks=True, e2e_steps=64):
         raise RuntimeError("device status: %s" % B.stq_status_string(status))
     ms_max = max_over_ranks(ms, world)
 
+    if e2e_steps == 0:
+        del qs, inputs
+        torch.cuda.empty_cache()
+        return {"ms": ms_max, "clocks": clk}
     # end to end through the host-buffer entry point: H2D of the step's inputs
     # from pinned memory, the step, D2H of o, all inside the timed region
     host = [{k: v.cpu().pin_memory() for k, v in x.items()} for x in inputs[:min(n_in, 8)]]
@@ -298,8 +302,13 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-seconds", type=float, default=60.0)
     ap.add_argument("--only", action="store_true", help="skip the other workloads")
+    ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling)")
+    ap.add_argument("--profile", action="store_true",
+                    help="decode steps only: no clock sampling, e2e, CPU baseline or other workloads")
     args = ap.parse_args()
     w = W.WORKLOADS[args.config]
+    if args.batch:
+        w = w.resized(batch=args.batch)
     spec = w.format
     dtype = "f32"
 
@@ -342,6 +351,11 @@ def main():
     if rank == 0:
         build_mod.build()
     barrier(world)
+    if args.profile:
+        res = run_gpu(w, args.steps, args.warmup, rank, world, sample_clocks=False, e2e_steps=0)
+        if rank == 0:
+            print(json.dumps({"workload": w.name, "batch": w.batch, "ms_per_step": res["ms"] / args.steps}))
+        return
     res = run_gpu(w, args.steps, args.warmup, rank, world)
     pages_total = w.pages * world
     value = pages_total * args.steps / (res["ms"] / 1000.0)

@@ -78,6 +78,13 @@ __device__ __forceinline__ void store_plane(uint8_t *plane, int lane, const uint
 template <int W>
 __host__ __device__ constexpr uint32_t plane_mask() { return 0x01010101u * ((1u << W) - 1u); }
 
+// x moved from bit `from` to bit `to` of every byte (a shift of the word).
+template <int FROM, int TO>
+__device__ __forceinline__ uint32_t move_bits(uint32_t x) {
+    if constexpr (TO >= FROM) return x << (TO - FROM);
+    else return x >> (FROM - TO);
+}
+
 // Biased b-bit codes of a 16-row INT block, as byte vectors: ub[rho] holds the
 // codes of row rho for columns 4l .. 4l+3 in bytes 0..3.  Planes are the
 // binary decomposition of B, widest plane first, holding the low bits.
@@ -94,29 +101,49 @@ __device__ __forceinline__ void unpack_int_block(const uint8_t *blk, int lane, u
         constexpr int lo1 = lo2 + (p2 ? 2 : 0);
         constexpr int off2 = p4 ? 1024 : 0;
         constexpr int off1 = off2 + (p2 ? 512 : 0);
+        uint32_t w4[8], w2[4], w1[2];
+        if constexpr (p4) load_plane<4>(blk, lane, w4);
+        if constexpr (p2) load_plane<2>(blk + off2, lane, w2);
+        if constexpr (p1) load_plane<1>(blk + off1, lane, w1);
 #pragma unroll
-        for (int r = 0; r < 16; ++r) ub[r] = 0;
-        if constexpr (p4) {
-            uint32_t w[8];
-            load_plane<4>(blk, lane, w);
-#pragma unroll
-            for (int r = 0; r < 16; ++r) ub[r] |= (w[r >> 1] >> (4 * (r & 1))) & plane_mask<4>();
-        }
-        if constexpr (p2) {
-            uint32_t w[4];
-            load_plane<2>(blk + off2, lane, w);
-#pragma unroll
-            for (int r = 0; r < 16; ++r) ub[r] |= ((w[r >> 2] >> (2 * (r & 3))) & plane_mask<2>()) << lo2;
-        }
-        if constexpr (p1) {
-            uint32_t w[2];
-            load_plane<1>(blk + off1, lane, w);
-#pragma unroll
-            for (int r = 0; r < 16; ++r) ub[r] |= ((w[r >> 3] >> (r & 7)) & plane_mask<1>()) << lo1;
+        for (int r = 0; r < 16; ++r) {
+            uint32_t x = 0;
+            if constexpr (p4) {
+                // rows 2n (low nibbles) and 2n+1 (high nibbles) of word n
+                x = (r & 1) ? (w4[r >> 1] >> 4) & plane_mask<4>() : w4[r >> 1] & plane_mask<4>();
+            }
+            if constexpr (p2) {
+                const uint32_t src = w2[r >> 2];
+                uint32_t f;
+                switch (r & 3) {
+                    case 0: f = move_bits<0, lo2>(src); break;
+                    case 1: f = move_bits<2, lo2>(src); break;
+                    case 2: f = move_bits<4, lo2>(src); break;
+                    default: f = move_bits<6, lo2>(src); break;
+                }
+                x |= f & (plane_mask<2>() << lo2);
+            }
+            if constexpr (p1) {
+                const uint32_t src = w1[r >> 3];
+                uint32_t f;
+                switch (r & 7) {
+                    case 0: f = move_bits<0, lo1>(src); break;
+                    case 1: f = move_bits<1, lo1>(src); break;
+                    case 2: f = move_bits<2, lo1>(src); break;
+                    case 3: f = move_bits<3, lo1>(src); break;
+                    case 4: f = move_bits<4, lo1>(src); break;
+                    case 5: f = move_bits<5, lo1>(src); break;
+                    case 6: f = move_bits<6, lo1>(src); break;
+                    default: f = move_bits<7, lo1>(src); break;
+                }
+                x |= f & (plane_mask<1>() << lo1);
+            }
+            ub[r] = x;
         }
     }
 }
 
+// Inverse of unpack_int_block; ub bytes hold values < 2^B.
 template <int B>
 __device__ __forceinline__ void pack_int_block(uint8_t *blk, int lane, const uint32_t (&ub)[16]) {
     if constexpr (B == 8) {
@@ -133,17 +160,27 @@ __device__ __forceinline__ void pack_int_block(uint8_t *blk, int lane, const uin
         if constexpr (p4) {
             uint32_t w[8];
 #pragma unroll
-            for (int n = 0; n < 8; ++n)
-                w[n] = (ub[2 * n] & plane_mask<4>()) | ((ub[2 * n + 1] & plane_mask<4>()) << 4);
+            for (int n = 0; n < 8; ++n) {
+                if constexpr (B == 4)   // codes < 16: the nibbles need no mask
+                    w[n] = ub[2 * n] | (ub[2 * n + 1] << 4);
+                else
+                    w[n] = (ub[2 * n] & plane_mask<4>()) | ((ub[2 * n + 1] << 4) & ~plane_mask<4>());
+            }
             store_plane<4>(blk, lane, w);
         }
         if constexpr (p2) {
             uint32_t w[4];
 #pragma unroll
             for (int n = 0; n < 4; ++n) {
-                uint32_t x = 0;
-#pragma unroll
-                for (int s = 0; s < 4; ++s) x |= ((ub[4 * n + s] >> lo2) & plane_mask<2>()) << (2 * s);
+                uint32_t x;
+                if constexpr (B == 2) {   // codes < 4: fields never spill
+                    x = ub[4 * n] | (ub[4 * n + 1] << 2) | (ub[4 * n + 2] << 4) | (ub[4 * n + 3] << 6);
+                } else {
+                    x = move_bits<lo2, 0>(ub[4 * n]) & plane_mask<2>();
+                    x |= move_bits<lo2, 2>(ub[4 * n + 1]) & (plane_mask<2>() << 2);
+                    x |= move_bits<lo2, 4>(ub[4 * n + 2]) & (plane_mask<2>() << 4);
+                    x |= move_bits<lo2, 6>(ub[4 * n + 3]) & (plane_mask<2>() << 6);
+                }
                 w[n] = x;
             }
             store_plane<2>(blk + off2, lane, w);
@@ -152,9 +189,14 @@ __device__ __forceinline__ void pack_int_block(uint8_t *blk, int lane, const uin
             uint32_t w[2];
 #pragma unroll
             for (int n = 0; n < 2; ++n) {
-                uint32_t x = 0;
-#pragma unroll
-                for (int s = 0; s < 8; ++s) x |= ((ub[8 * n + s] >> lo1) & plane_mask<1>()) << s;
+                uint32_t x = move_bits<lo1, 0>(ub[8 * n]) & plane_mask<1>();
+                x |= move_bits<lo1, 1>(ub[8 * n + 1]) & (plane_mask<1>() << 1);
+                x |= move_bits<lo1, 2>(ub[8 * n + 2]) & (plane_mask<1>() << 2);
+                x |= move_bits<lo1, 3>(ub[8 * n + 3]) & (plane_mask<1>() << 3);
+                x |= move_bits<lo1, 4>(ub[8 * n + 4]) & (plane_mask<1>() << 4);
+                x |= move_bits<lo1, 5>(ub[8 * n + 5]) & (plane_mask<1>() << 5);
+                x |= move_bits<lo1, 6>(ub[8 * n + 6]) & (plane_mask<1>() << 6);
+                x |= move_bits<lo1, 7>(ub[8 * n + 7]) & (plane_mask<1>() << 7);
                 w[n] = x;
             }
             store_plane<1>(blk + off1, lane, w);

@@ -17,10 +17,11 @@
  *                     T = S / c (so the value-column scale c_j leaves the
  *                     inner loops);
  *                   - a column sum sum_s w_s T_sj runs over stored rows in
- *                     blocks of ORC_SUM_BLOCK consecutive rows, each block a
- *                     chain p = fmaf(w_s, T_sj, p) from p = 0 in ascending s,
- *                     and the block partials are added by a balanced pairwise
- *                     tree in block order;
+ *                     blocks of ORC_SUM_BLOCK = 16 consecutive rows (one
+ *                     16-row block of the packed layout), each block a chain
+ *                     p = fmaf(w_s, T_sj, p) from p = 0 in ascending s, and
+ *                     the 8 block partials are added by a balanced pairwise
+ *                     tree in block order, ((P0+P1)+(P2+P3))+((P4+P5)+(P6+P7));
  *                   - requantization rounds the exact product T' * inv once
  *                     (to an integer, ties to even);
  *                   - inv = qmax / m rounded toward zero, which keeps every
@@ -38,7 +39,7 @@
 #include <vector>
 #include <algorithm>
 
-static const int ORC_SUM_BLOCK = 32;
+static const int ORC_SUM_BLOCK = 16;
 
 extern "C" int orc_sum_block(void) { return ORC_SUM_BLOCK; }
 
