@@ -53,13 +53,13 @@ stq_status build_dev_format(const stq_format *f, DevFormat *out) {
     return STQ_OK;
 }
 
-int persistent_grid(const void *kernel, size_t dyn_smem, long n_units) {
+int persistent_grid(const void *kernel, int threads, size_t dyn_smem, long n_units) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return -1;
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
     int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, dyn_smem) != cudaSuccess)
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, dyn_smem) != cudaSuccess)
         return -1;
     if (per_sm < 1) return -1;
     long g = (long)sms * per_sm;

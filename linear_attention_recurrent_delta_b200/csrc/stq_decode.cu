@@ -19,6 +19,12 @@
 // run time.  All warps share one copy of the loop: per-warp copies specialised
 // to each warp's widths were measured slower, the larger code overflowing the
 // instruction cache the SM's warps share.
+//
+// One CTA-wide barrier per page: each warp prepares the operands of its own
+// rows (thread 32w + l: stored row 32w + l) and syncs within the warp; the
+// column sums' block partials and 1/c are double-buffered by page parity, so
+// the only cross-warp dependency is u (and o, finished after the next page's
+// barrier).  Warps of a CTA drift apart by up to a page.
 #include "stq_internal.h"
 
 namespace stq {
@@ -42,19 +48,21 @@ constexpr int kMaxStages = 4;
 constexpr int kRmxPitch = 36;     // words per row of the row-max tile
 
 struct SmemFixed {
-    // per stored row, duplicated into pairs for the f32x2 pipes:
-    float2 a2[kD];                          // alpha * r (decay x row scale)
-    float2 kp2[kD];                         // k of the row's key channel
-    float2 bk2[kD];                         // beta * k
-    float2 qp2[kD];                         // q
-    float red_u[kWarps][kD];                // per warp: P_2w + P_2w+1 of u
-    float red_o[kWarps][kD];                // the same for o
+    // per stored row (a 16-byte load serves 4 rows; an f32x2 operation takes
+    // the value duplicated without a move):
+    float a[kD];                            // alpha * r (decay x row scale)
+    float kp[kD];                           // k of the row's key channel
+    float bk[kD];                           // beta * k
+    float qp[kD];                           // q
+    float red_u[2][kWarps][kD];             // per page parity and warp: P_2w + P_2w+1 of u
+    float red_o[2][kWarps][kD];             // the same for o
     // row-partial maxima: row r of a warp at r * kRmxPitch, one word per lane;
     // the pitch keeps both the per-row stores and the 16-byte row reads
     // free of bank conflicts
     float rmx[kWarps][kRowsPerWarp * kRmxPitch];
-    float2 inv2[kWarps][kRowsPerWarp];      // requant multipliers (pairs)
-    float ic[kD];                           // 1 / c per column
+    float inv[kWarps][kRowsPerWarp];        // requant multipliers
+    float ic[2][kD];                        // per page parity: 1 / c per column
+    float c_prev[kD];                       // c of the page whose o is pending
     uint64_t full[kMaxStages];              // stage-full barriers
     uint64_t never;                         // a barrier nothing completes (test hook)
 };
@@ -74,33 +82,34 @@ __device__ __forceinline__ float div_by_qmax(float m, float qmax, float rcp_qmax
     return __fmaf_rn(__fmaf_rn(-q0, qmax, m), rcp_qmax, q0);
 }
 
-// ---- S1 + S2: one 16-row block into T[r0 .. r0+15] (a2: the block's pairs)
+// ---- S1 + S2: one 16-row block into T[r0 .. r0+15] (a: the block's alpha * r)
 template <int B>
-__device__ __forceinline__ void dequant_int(const uint8_t *blk, int lane, const float2 *a2,
+__device__ __forceinline__ void dequant_int(const uint8_t *blk, int lane, const float *a,
                                             float2 (&T)[kRowsPerWarp][2], int r0) {
     uint32_t ub[16];
     unpack_int_block<B>(blk, lane, ub);
     const float bm = 8388608.0f + (float)(1 << (B - 1));
 #pragma unroll
-    for (int r = 0; r < 16; r += 2) {
-        const float4 aa = *reinterpret_cast<const float4 *>(a2 + r);   // rows r, r+1
-        float2 z01, z23;
-        codes_to_float(ub[r], bm, z01, z23);
-        T[r0 + r][0] = __fmul2_rn(z01, make_float2(aa.x, aa.y));
-        T[r0 + r][1] = __fmul2_rn(z23, make_float2(aa.x, aa.y));
-        codes_to_float(ub[r + 1], bm, z01, z23);
-        T[r0 + r + 1][0] = __fmul2_rn(z01, make_float2(aa.z, aa.w));
-        T[r0 + r + 1][1] = __fmul2_rn(z23, make_float2(aa.z, aa.w));
+    for (int r = 0; r < 16; r += 4) {
+        const float4 aa = *reinterpret_cast<const float4 *>(a + r);   // rows r .. r+3
+        const float av[4] = {aa.x, aa.y, aa.z, aa.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float2 z01, z23;
+            codes_to_float(ub[r + i], bm, z01, z23);
+            T[r0 + r + i][0] = __fmul2_rn(z01, make_float2(av[i], av[i]));
+            T[r0 + r + i][1] = __fmul2_rn(z23, make_float2(av[i], av[i]));
+        }
     }
 }
 
-__device__ __forceinline__ void dequant_fp16(const uint8_t *blk, int lane, const float2 *a2,
+__device__ __forceinline__ void dequant_fp16(const uint8_t *blk, int lane, const float *a,
                                              float2 (&T)[kRowsPerWarp][2], int r0) {
     uint32_t w[32];
     unpack_fp16_block(blk, lane, w);
 #pragma unroll
     for (int r = 0; r < 16; ++r) {
-        const float2 as = a2[r];
+        const float2 as = make_float2(a[r], a[r]);
         float2 x01 = __half22float2(*reinterpret_cast<const __half2 *>(&w[2 * r]));
         float2 x23 = __half22float2(*reinterpret_cast<const __half2 *>(&w[2 * r + 1]));
         T[r0 + r][0] = __fmul2_rn(x01, as);
@@ -110,20 +119,20 @@ __device__ __forceinline__ void dequant_fp16(const uint8_t *blk, int lane, const
 
 // BITS: the block's width (16 = FP16), or 0 to read `bits` at run time.
 template <int BITS, int R0>
-__device__ __forceinline__ void dequant_block(int bits, const uint8_t *blk, int lane, const float2 *a2,
+__device__ __forceinline__ void dequant_block(int bits, const uint8_t *blk, int lane, const float *a,
                                               float2 (&T)[kRowsPerWarp][2]) {
-    if constexpr (BITS == 16) dequant_fp16(blk, lane, a2, T, R0);
-    else if constexpr (BITS != 0) dequant_int<BITS>(blk, lane, a2, T, R0);
+    if constexpr (BITS == 16) dequant_fp16(blk, lane, a, T, R0);
+    else if constexpr (BITS != 0) dequant_int<BITS>(blk, lane, a, T, R0);
     else {
         switch (bits) {
-            case 16: dequant_fp16(blk, lane, a2, T, R0); break;
-            case 8: dequant_int<8>(blk, lane, a2, T, R0); break;
-            case 7: dequant_int<7>(blk, lane, a2, T, R0); break;
-            case 6: dequant_int<6>(blk, lane, a2, T, R0); break;
-            case 5: dequant_int<5>(blk, lane, a2, T, R0); break;
-            case 4: dequant_int<4>(blk, lane, a2, T, R0); break;
-            case 3: dequant_int<3>(blk, lane, a2, T, R0); break;
-            default: dequant_int<2>(blk, lane, a2, T, R0); break;
+            case 16: dequant_fp16(blk, lane, a, T, R0); break;
+            case 8: dequant_int<8>(blk, lane, a, T, R0); break;
+            case 7: dequant_int<7>(blk, lane, a, T, R0); break;
+            case 6: dequant_int<6>(blk, lane, a, T, R0); break;
+            case 5: dequant_int<5>(blk, lane, a, T, R0); break;
+            case 4: dequant_int<4>(blk, lane, a, T, R0); break;
+            case 3: dequant_int<3>(blk, lane, a, T, R0); break;
+            default: dequant_int<2>(blk, lane, a, T, R0); break;
         }
     }
 }
@@ -134,7 +143,7 @@ struct SrCtx {
 };
 
 template <int B, bool SR>
-__device__ __forceinline__ void requant_int(uint8_t *blk, int lane, const float2 *inv2,
+__device__ __forceinline__ void requant_int(uint8_t *blk, int lane, const float *inv,
                                             const float2 (&T)[kRowsPerWarp][2], int r0, int s0,
                                             const SrCtx sr) {
     const float M = 12582912.0f + (float)(1 << (B - 1));   // 1.5 * 2^23 + bias
@@ -142,8 +151,9 @@ __device__ __forceinline__ void requant_int(uint8_t *blk, int lane, const float2
     uint32_t ub[16];
 #pragma unroll
     for (int r = 0; r < 16; r += 2) {
-        const float4 ii = *reinterpret_cast<const float4 *>(inv2 + r);   // rows r, r+1
-        const float2 i0 = make_float2(ii.x, ii.y), i1 = make_float2(ii.z, ii.w);
+        const float4 i4 = *reinterpret_cast<const float4 *>(inv + (r & ~3));   // rows r & ~3 .. +3
+        const float ia = (r & 2) ? i4.z : i4.x, ib = (r & 2) ? i4.w : i4.y;
+        const float2 i0 = make_float2(ia, ia), i1 = make_float2(ib, ib);
         float2 y0, y1, y2, y3;
         if constexpr (SR) {
             const int s = s0 + r;   // even
@@ -179,20 +189,20 @@ __device__ __forceinline__ void requant_fp16(uint8_t *blk, int lane, const float
 }
 
 template <int BITS, int R0, bool SR>
-__device__ __forceinline__ void requant_block(int bits, uint8_t *blk, int lane, const float2 *inv2,
+__device__ __forceinline__ void requant_block(int bits, uint8_t *blk, int lane, const float *inv,
                                               const float2 (&T)[kRowsPerWarp][2], int s0, const SrCtx sr) {
     if constexpr (BITS == 16) requant_fp16(blk, lane, T, R0);
-    else if constexpr (BITS != 0) requant_int<BITS, SR>(blk, lane, inv2, T, R0, s0, sr);
+    else if constexpr (BITS != 0) requant_int<BITS, SR>(blk, lane, inv, T, R0, s0, sr);
     else {
         switch (bits) {
             case 16: requant_fp16(blk, lane, T, R0); break;
-            case 8: requant_int<8, SR>(blk, lane, inv2, T, R0, s0, sr); break;
-            case 7: requant_int<7, SR>(blk, lane, inv2, T, R0, s0, sr); break;
-            case 6: requant_int<6, SR>(blk, lane, inv2, T, R0, s0, sr); break;
-            case 5: requant_int<5, SR>(blk, lane, inv2, T, R0, s0, sr); break;
-            case 4: requant_int<4, SR>(blk, lane, inv2, T, R0, s0, sr); break;
-            case 3: requant_int<3, SR>(blk, lane, inv2, T, R0, s0, sr); break;
-            default: requant_int<2, SR>(blk, lane, inv2, T, R0, s0, sr); break;
+            case 8: requant_int<8, SR>(blk, lane, inv, T, R0, s0, sr); break;
+            case 7: requant_int<7, SR>(blk, lane, inv, T, R0, s0, sr); break;
+            case 6: requant_int<6, SR>(blk, lane, inv, T, R0, s0, sr); break;
+            case 5: requant_int<5, SR>(blk, lane, inv, T, R0, s0, sr); break;
+            case 4: requant_int<4, SR>(blk, lane, inv, T, R0, s0, sr); break;
+            case 3: requant_int<3, SR>(blk, lane, inv, T, R0, s0, sr); break;
+            default: requant_int<2, SR>(blk, lane, inv, T, R0, s0, sr); break;
         }
     }
 }
@@ -200,17 +210,19 @@ __device__ __forceinline__ void requant_block(int bits, uint8_t *blk, int lane, 
 // ---- S3 / S5 partial sums of one 16-row block: chains p = fma(w_s, X_s, p)
 // from 0 in ascending row order, two column pairs.
 template <int R0>
-__device__ __forceinline__ void block_chain(const float2 *w2, const float2 (&X)[kRowsPerWarp][2],
+__device__ __forceinline__ void block_chain(const float *w, const float2 (&X)[kRowsPerWarp][2],
                                             float2 &p01, float2 &p23) {
     p01 = make_float2(0.f, 0.f);
     p23 = make_float2(0.f, 0.f);
 #pragma unroll
-    for (int r = 0; r < 16; r += 2) {
-        const float4 ww = *reinterpret_cast<const float4 *>(w2 + r);
-        p01 = __ffma2_rn(make_float2(ww.x, ww.y), X[R0 + r][0], p01);
-        p23 = __ffma2_rn(make_float2(ww.x, ww.y), X[R0 + r][1], p23);
-        p01 = __ffma2_rn(make_float2(ww.z, ww.w), X[R0 + r + 1][0], p01);
-        p23 = __ffma2_rn(make_float2(ww.z, ww.w), X[R0 + r + 1][1], p23);
+    for (int r = 0; r < 16; r += 4) {
+        const float4 ww = *reinterpret_cast<const float4 *>(w + r);
+        const float wv[4] = {ww.x, ww.y, ww.z, ww.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            p01 = __ffma2_rn(make_float2(wv[i], wv[i]), X[R0 + r + i][0], p01);
+            p23 = __ffma2_rn(make_float2(wv[i], wv[i]), X[R0 + r + i][1], p23);
+        }
     }
 }
 
@@ -226,17 +238,18 @@ __device__ __forceinline__ void issue_stage(const DevFormat &F, const DecodeArgs
 }
 
 // o of a finished page: the tree over the warps' block-pair partials, times c.
-__device__ __forceinline__ void write_o(const SmemFixed &S, const DecodeArgs &A, int p, int lane, float4 c,
-                                        int col_scales) {
-    const float4 o0 = *reinterpret_cast<const float4 *>(&S.red_o[0][4 * lane]);
-    const float4 o1 = *reinterpret_cast<const float4 *>(&S.red_o[1][4 * lane]);
-    const float4 o2 = *reinterpret_cast<const float4 *>(&S.red_o[2][4 * lane]);
-    const float4 o3 = *reinterpret_cast<const float4 *>(&S.red_o[3][4 * lane]);
+__device__ __forceinline__ void write_o(const float (*red_o)[kD], const DecodeArgs &A, int p, int lane,
+                                        const float *c_prev, int col_scales) {
+    const float4 o0 = *reinterpret_cast<const float4 *>(&red_o[0][4 * lane]);
+    const float4 o1 = *reinterpret_cast<const float4 *>(&red_o[1][4 * lane]);
+    const float4 o2 = *reinterpret_cast<const float4 *>(&red_o[2][4 * lane]);
+    const float4 o3 = *reinterpret_cast<const float4 *>(&red_o[3][4 * lane]);
     float2 oa = __fadd2_rn(__fadd2_rn(make_float2(o0.x, o0.y), make_float2(o1.x, o1.y)),
                            __fadd2_rn(make_float2(o2.x, o2.y), make_float2(o3.x, o3.y)));
     float2 ob = __fadd2_rn(__fadd2_rn(make_float2(o0.z, o0.w), make_float2(o1.z, o1.w)),
                            __fadd2_rn(make_float2(o2.z, o2.w), make_float2(o3.z, o3.w)));
     if (col_scales) {
+        const float4 c = *reinterpret_cast<const float4 *>(&c_prev[4 * lane]);
         oa = __fmul2_rn(make_float2(c.x, c.y), oa);
         ob = __fmul2_rn(make_float2(c.z, c.w), ob);
     }
@@ -247,6 +260,11 @@ __device__ __forceinline__ void write_o(const SmemFixed &S, const DecodeArgs &A,
 // the stochastic-rounding variant carries the Philox state and gets 2.
 template <bool SR>
 constexpr int decode_ctas_per_sm() { return SR ? 2 : 3; }
+
+// Iteration index at which a CTA processed page p.
+__device__ __forceinline__ int it_last(int p, unsigned first, unsigned stride) {
+    return (p - (int)first) / (int)stride;
+}
 
 __device__ __forceinline__ float absmax4(float2 a, float2 b) {
     return fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(b.x), fabsf(b.y)));
@@ -302,7 +320,6 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
     const int my_r = F.blk_rbase(lane < 16 ? b0 : b1) + (lane & 15);
     float *rmx = S.rmx[warp];
     int p_prev = -1;                  // page whose o is still to be written
-    float4 c_prev = make_float4(1.f, 1.f, 1.f, 1.f);
     int st = 0;
     uint32_t parity = 0;
 
@@ -319,24 +336,12 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
             kap_n = __ldg(A.perm + pnh * kD + tid) & (kD - 1);
         }
 
+        // a wait that runs out is voted on at the page's barrier, before
+        // anything of the page is written
         bool ok;
         if (A.stall_first_wait && it == 0) ok = mbar_wait_bounded(&S.never, 0, A.wait_limit_ns);
         else ok = mbar_wait_bounded(&S.full[st], parity, A.wait_limit_ns);
-        if (__syncthreads_or(!ok)) {
-            if (tid == 0) {
-                atomicOr(A.status, kStatusTimeout);
-                // let the copies already issued into the ring land before exiting
-                for (int i = 0; i < NS; ++i) {
-                    const int pi = p + i * stride;
-                    if (pi < n) {
-                        const int ii = it + i;
-                        mbar_wait_bounded(&S.full[ii % NS], (uint32_t)((ii / NS) & 1), A.wait_limit_ns);
-                    }
-                }
-            }
-            __syncthreads();
-            return;
-        }
+        const int par = it & 1;
         const uint8_t *stg = stages + st * A.stage_bytes;
         const float *q_s = reinterpret_cast<const float *>(stg + F.page_bytes);
         const float *k_s = q_s + kD;
@@ -355,31 +360,44 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
             }
             const float bk = __fmul_rn(beta_s, kk);
             if (F.col_scales)   // thread s also inverts the scale of column s
-                S.ic[s] = __frcp_rn(reinterpret_cast<const float *>(stg + F.c_off)[s]);
-            S.a2[s] = make_float2(a, a);
-            S.kp2[s] = make_float2(kk, kk);
-            S.qp2[s] = make_float2(qq, qq);
-            S.bk2[s] = make_float2(bk, bk);
+                S.ic[par][s] = __frcp_rn(reinterpret_cast<const float *>(stg + F.c_off)[s]);
+            S.a[s] = a;
+            S.kp[s] = kk;
+            S.qp[s] = qq;
+            S.bk[s] = bk;
         }
-        __syncthreads();
-        // o of the previous page (its block partials were stored before this barrier)
-        if (warp == 0 && p_prev >= 0) write_o(S, A, p_prev, lane, c_prev, F.col_scales);
+        __syncwarp();   // the warp's rows' operands come from its own lanes
 
         // S1 + S2, and S3's block chains
         float2 T[kRowsPerWarp][2];
-        dequant_block<BA, 0>(bits0, stg + off0, lane, &S.a2[32 * warp], T);
-        dequant_block<BB, 16>(bits1, stg + off1, lane, &S.a2[32 * warp + 16], T);
+        dequant_block<BA, 0>(bits0, stg + off0, lane, &S.a[32 * warp], T);
+        dequant_block<BB, 16>(bits1, stg + off1, lane, &S.a[32 * warp + 16], T);
         {
             float2 pa01, pa23, pb01, pb23;
-            block_chain<0>(&S.kp2[32 * warp], T, pa01, pa23);
-            block_chain<16>(&S.kp2[32 * warp + 16], T, pb01, pb23);
+            block_chain<0>(&S.kp[32 * warp], T, pa01, pa23);
+            block_chain<16>(&S.kp[32 * warp + 16], T, pb01, pb23);
             const float2 w01 = __fadd2_rn(pa01, pb01), w23 = __fadd2_rn(pa23, pb23);
-            *reinterpret_cast<float4 *>(&S.red_u[warp][4 * lane]) = make_float4(w01.x, w01.y, w23.x, w23.y);
+            *reinterpret_cast<float4 *>(&S.red_u[par][warp][4 * lane]) = make_float4(w01.x, w01.y, w23.x, w23.y);
         }
         const float4 v4 = *reinterpret_cast<const float4 *>(v_s + 4 * lane);
         float4 c4 = make_float4(1.f, 1.f, 1.f, 1.f);
         if (F.col_scales) c4 = *reinterpret_cast<const float4 *>(stg + F.c_off + 16 * lane);
-        __syncthreads();
+        if (__syncthreads_or(!ok)) {
+            // a stage never arrived: record it, let the copies already issued
+            // into the ring land, and leave; nothing of this page was written
+            if (tid == 0) {
+                atomicOr(A.status, kStatusTimeout);
+                for (int i = 0; i < NS; ++i) {
+                    const int pi = p + i * stride;
+                    if (pi < n) {
+                        const int ii = it + i;
+                        mbar_wait_bounded(&S.full[ii % NS], (uint32_t)((ii / NS) & 1), A.wait_limit_ns);
+                    }
+                }
+            }
+            __syncthreads();
+            return;
+        }
 
         // the stage is no longer read: refill it with the page NS iterations ahead
         if (tid == 0) {
@@ -389,20 +407,25 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
                 issue_stage(F, A, stages + st * A.stage_bytes, pr, &S.full[st]);
             }
         }
+        // o of the previous page (its block partials were stored before this barrier)
+        if (warp == 0 && p_prev >= 0) {
+            write_o(S.red_o[par ^ 1], A, p_prev, lane, S.c_prev, F.col_scales);
+            if (F.col_scales) *reinterpret_cast<float4 *>(&S.c_prev[4 * lane]) = c4;
+        }
 
         // u = ((P0+P1)+(P2+P3))+((P4+P5)+(P6+P7)); e = v (1/c) - u
         float2 e01, e23;
         {
-            const float4 u0 = *reinterpret_cast<const float4 *>(&S.red_u[0][4 * lane]);
-            const float4 u1 = *reinterpret_cast<const float4 *>(&S.red_u[1][4 * lane]);
-            const float4 u2 = *reinterpret_cast<const float4 *>(&S.red_u[2][4 * lane]);
-            const float4 u3 = *reinterpret_cast<const float4 *>(&S.red_u[3][4 * lane]);
+            const float4 u0 = *reinterpret_cast<const float4 *>(&S.red_u[par][0][4 * lane]);
+            const float4 u1 = *reinterpret_cast<const float4 *>(&S.red_u[par][1][4 * lane]);
+            const float4 u2 = *reinterpret_cast<const float4 *>(&S.red_u[par][2][4 * lane]);
+            const float4 u3 = *reinterpret_cast<const float4 *>(&S.red_u[par][3][4 * lane]);
             const float2 ua = __fadd2_rn(__fadd2_rn(make_float2(u0.x, u0.y), make_float2(u1.x, u1.y)),
                                          __fadd2_rn(make_float2(u2.x, u2.y), make_float2(u3.x, u3.y)));
             const float2 ub = __fadd2_rn(__fadd2_rn(make_float2(u0.z, u0.w), make_float2(u1.z, u1.w)),
                                          __fadd2_rn(make_float2(u2.z, u2.w), make_float2(u3.z, u3.w)));
             float4 ic = make_float4(1.f, 1.f, 1.f, 1.f);
-            if (F.col_scales) ic = *reinterpret_cast<const float4 *>(&S.ic[4 * lane]);
+            if (F.col_scales) ic = *reinterpret_cast<const float4 *>(&S.ic[par][4 * lane]);
             // two roundings, scalar: an f32x2 multiply feeding an f32x2 add is
             // fused by the compiler into one f32x2 fma
             e01 = make_float2(__fsub_rn(__fmul_rn(v4.x, ic.x), ua.x), __fsub_rn(__fmul_rn(v4.y, ic.y), ua.y));
@@ -411,22 +434,23 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
 
         // S4: T' = T + (beta k) e; row partial maxima into the row-max tile
 #pragma unroll
-        for (int r = 0; r < kRowsPerWarp; r += 2) {
-            const float4 bb = *reinterpret_cast<const float4 *>(&S.bk2[32 * warp + r]);
-            T[r][0] = __ffma2_rn(make_float2(bb.x, bb.y), e01, T[r][0]);
-            T[r][1] = __ffma2_rn(make_float2(bb.x, bb.y), e23, T[r][1]);
-            T[r + 1][0] = __ffma2_rn(make_float2(bb.z, bb.w), e01, T[r + 1][0]);
-            T[r + 1][1] = __ffma2_rn(make_float2(bb.z, bb.w), e23, T[r + 1][1]);
-            rmx[r * kRmxPitch + lane] = absmax4(T[r][0], T[r][1]);
-            rmx[(r + 1) * kRmxPitch + lane] = absmax4(T[r + 1][0], T[r + 1][1]);
+        for (int r = 0; r < kRowsPerWarp; r += 4) {
+            const float4 bb = *reinterpret_cast<const float4 *>(&S.bk[32 * warp + r]);
+            const float bv[4] = {bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                T[r + i][0] = __ffma2_rn(make_float2(bv[i], bv[i]), e01, T[r + i][0]);
+                T[r + i][1] = __ffma2_rn(make_float2(bv[i], bv[i]), e23, T[r + i][1]);
+                rmx[(r + i) * kRmxPitch + lane] = absmax4(T[r + i][0], T[r + i][1]);
+            }
         }
         // S5: block chains of o, finished at the next page's first barrier
         {
             float2 pa01, pa23, pb01, pb23;
-            block_chain<0>(&S.qp2[32 * warp], T, pa01, pa23);
-            block_chain<16>(&S.qp2[32 * warp + 16], T, pb01, pb23);
+            block_chain<0>(&S.qp[32 * warp], T, pa01, pa23);
+            block_chain<16>(&S.qp[32 * warp + 16], T, pb01, pb23);
             const float2 w01 = __fadd2_rn(pa01, pb01), w23 = __fadd2_rn(pa23, pb23);
-            *reinterpret_cast<float4 *>(&S.red_o[warp][4 * lane]) = make_float4(w01.x, w01.y, w23.x, w23.y);
+            *reinterpret_cast<float4 *>(&S.red_o[par][warp][4 * lane]) = make_float4(w01.x, w01.y, w23.x, w23.y);
         }
         __syncwarp();
 
@@ -449,7 +473,7 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
                 }
                 reinterpret_cast<float *>(page + F.r_off)[my_r] = r;
             }
-            S.inv2[warp][lane] = make_float2(inv, inv);
+            S.inv[warp][lane] = inv;
         }
         __syncwarp();
 
@@ -457,11 +481,11 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
         SrCtx sr;
         sr.k0 = A.seed_lo; sr.k1 = A.seed_hi; sr.step = A.step;
         sr.b = (uint32_t)pb; sr.h = (uint32_t)ph;
-        requant_block<BA, 0, SR>(bits0, page + off0, lane, &S.inv2[warp][0], T, 32 * warp, sr);
-        requant_block<BB, 16, SR>(bits1, page + off1, lane, &S.inv2[warp][16], T, 32 * warp + 16, sr);
+        requant_block<BA, 0, SR>(bits0, page + off0, lane, &S.inv[warp][0], T, 32 * warp, sr);
+        requant_block<BB, 16, SR>(bits1, page + off1, lane, &S.inv[warp][16], T, 32 * warp + 16, sr);
 
+        if (warp == 0 && p_prev < 0 && F.col_scales) *reinterpret_cast<float4 *>(&S.c_prev[4 * lane]) = c4;
         p_prev = p;
-        c_prev = c4;
         alpha_s = alpha_n;
         beta_s = beta_n;
         kap = kap_n;
@@ -471,7 +495,8 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
         if (++st == NS) { st = 0; parity ^= 1u; }
     }
     __syncthreads();
-    if (warp == 0 && p_prev >= 0) write_o(S, A, p_prev, lane, c_prev, F.col_scales);
+    if (warp == 0 && p_prev >= 0) write_o(S.red_o[(it_last(p_prev, blockIdx.x, gridDim.x)) & 1], A, p_prev, lane,
+                                          S.c_prev, F.col_scales);
 }
 
 static int decode_stages(size_t stride, int ctas_per_sm) {
@@ -509,7 +534,7 @@ cudaError_t launch_decode(const stq_state *s, const float *q, const float *k, co
     const void *fn = F.stochastic ? (const void *)decode_kernel<true> : (const void *)decode_kernel<false>;
     cudaError_t err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
-    const int grid = persistent_grid(fn, smem, A.n_pages);
+    const int grid = persistent_grid(fn, kThreads, smem, A.n_pages);
     if (grid <= 0) return cudaErrorInvalidConfiguration;
     if (F.stochastic)
         decode_kernel<true><<<grid, kThreads, smem, stream>>>(F, A);

@@ -22,15 +22,14 @@ struct stq_state {
 namespace stq {
 
 constexpr size_t kHeaderBytes = 256;
-constexpr int kStages = 3;           // bulk-copy ring depth of the decode kernel
 
 // Validate a format and build its device constants.  Returns STQ_OK,
 // STQ_ERR_INVALID_ARG or STQ_ERR_UNSUPPORTED.
 stq_status build_dev_format(const stq_format *f, DevFormat *out);
 
-// Persistent-grid size for a kernel: SM count x resident CTAs (cached per
-// device and kernel).
-int persistent_grid(const void *kernel, size_t dyn_smem, long n_units);
+// Persistent-grid size for a kernel: SM count x resident CTAs of `threads`
+// threads with `dyn_smem` dynamic shared memory, at most n_units.
+int persistent_grid(const void *kernel, int threads, size_t dyn_smem, long n_units);
 
 // Launchers (return cudaError_t of the launch).
 cudaError_t launch_decode(const stq_state *s, const float *q, const float *k, const float *v,

@@ -215,7 +215,7 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_kernel(const DevFormat F
 
 cudaError_t launch_quantize(const stq_state *s, const float *S, cudaStream_t stream) {
     const long n = (long)s->batch * s->heads;
-    const int grid = persistent_grid((const void *)quantize_kernel, 0, n);
+    const int grid = persistent_grid((const void *)quantize_kernel, kThreads, 0, n);
     if (grid <= 0) return cudaErrorInvalidConfiguration;
     quantize_kernel<<<grid, kThreads, 0, stream>>>(s->dev, S, s->base + s->perm_offset,
                                                    s->base + s->pages_offset, n, s->heads);
@@ -299,7 +299,7 @@ __global__ void __launch_bounds__(kThreads) dequantize_kernel(const DevFormat F,
 
 cudaError_t launch_dequantize(const stq_state *s, float *S, cudaStream_t stream) {
     const long n = (long)s->batch * s->heads;
-    const int grid = persistent_grid((const void *)dequantize_kernel, 0, n);
+    const int grid = persistent_grid((const void *)dequantize_kernel, kThreads, 0, n);
     if (grid <= 0) return cudaErrorInvalidConfiguration;
     dequantize_kernel<<<grid, kThreads, 0, stream>>>(s->dev, s->base + s->perm_offset, s->base + s->pages_offset,
                                                      S, n, s->heads);
