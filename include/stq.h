@@ -126,6 +126,31 @@ size_t stq_calibrate_workspace_bytes(const stq_state *s);
 stq_status stq_calibrate(stq_state *s, const float *d_S, const float *d_row_weight,
                          void *d_workspace, size_t workspace_bytes, void *stream);
 
+/* Upper bound of the scratch stq_calibrate_noalloc may use (1 MiB): it serves
+ * states with stq_calibrate_workspace_bytes(s) <= this, e.g. up to 1,024
+ * requests of 32 heads. */
+#define STQ_CALIBRATE_NOALLOC_MAX_BYTES ((size_t)1 << 20)
+
+/* stq_calibrate without a workspace argument and without allocating: for
+ * callers that cannot call cudaMalloc or take device memory from anywhere at
+ * that point -- a serving runtime whose device memory is a pool reserved up
+ * front, code that must not add the synchronisation an allocation can bring
+ * to its stream, or a host library handed only its inputs and outputs.  The
+ * pages have no counterpart of this entry point; it computes exactly what
+ * stq_calibrate computes.
+ *   - Its scratch is a fixed 1 MiB array in the library's device image,
+ *     present on every GPU that loads the library until the process exits.
+ *     States needing more (stq_calibrate_workspace_bytes(s) >
+ *     STQ_CALIBRATE_NOALLOC_MAX_BYTES) get STQ_ERR_BUFFER_TOO_SMALL.
+ *   - The first call on a device looks up the array's device address (a
+ *     CUDA runtime query, with that device current); make that first call
+ *     before capturing the stream into a graph.
+ *   - All calls share the array: calls that overlap on the GPU (other streams,
+ *     other threads, other states) race on it and must be serialized by the
+ *     caller.  Nothing in it needs clearing between calls.
+ * Arguments and other errors as stq_calibrate. */
+stq_status stq_calibrate_noalloc(stq_state *s, const float *d_S, const float *d_row_weight, void *stream);
+
 /* Quantize an fp32 state into every page using the state's precision map:
  * c_j = max_i |S_ij| (1 if 0; 1 without column scales); T = S * (1/c);
  * INT rows: r = max_j |T| / qmax, codes = round-to-nearest-even of

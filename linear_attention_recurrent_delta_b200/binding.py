@@ -53,6 +53,7 @@ def lib():
                                      POINTER(c_size_t)]),
         "stq_calibrate_workspace_bytes": (c_size_t, [P]),
         "stq_calibrate": (c_int, [P, P, P, P, c_size_t, P]),
+        "stq_calibrate_noalloc": (c_int, [P, P, P, P]),
         "stq_quantize_state": (c_int, [P, P, P]),
         "stq_decode_step": (c_int, [P, P, P, P, P, P, P, c_uint64, c_uint32, P]),
         "stq_decode_io_bytes": (c_size_t, [P]),
@@ -157,6 +158,12 @@ def stq_calibrate(state, S, row_weight=None, workspace=None, stream=None):
         workspace = torch.empty(max(need, 8), dtype=torch.uint8, device=S.device)
     _check(lib().stq_calibrate(state.handle, _ptr(S), _ptr(row_weight), _ptr(workspace),
                                workspace.numel() * workspace.element_size(), _stream(stream)), "stq_calibrate")
+
+
+def stq_calibrate_noalloc(state, S, row_weight=None, stream=None):
+    """stq_calibrate with the library's fixed scratch (no workspace, no allocation)."""
+    _check(lib().stq_calibrate_noalloc(state.handle, _ptr(S), _ptr(row_weight), _stream(stream)),
+           "stq_calibrate_noalloc")
 
 
 def stq_quantize_state(state, S, stream=None):

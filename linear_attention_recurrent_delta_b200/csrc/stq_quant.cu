@@ -4,6 +4,9 @@
 // page written here is read back bit for bit by the decode step.
 #include "stq_internal.h"
 
+#include <map>
+#include <mutex>
+
 namespace stq {
 
 constexpr int kCalibChunk = 32;   // requests summed per partial score
@@ -87,6 +90,56 @@ cudaError_t launch_calibrate(const stq_state *s, const float *S, const float *ro
                                                           s->base + s->perm_offset);
     return cudaGetLastError();
 }
+
+// ------------------------------------------------ calibration, no allocation --
+// Scratch of stq_calibrate_noalloc: one fixed array in every GPU that loads the
+// library, held until the process exits.  Every call shares it; the partial
+// kernel writes each entry the rank kernel reads, so nothing in it has to
+// start at zero, and two calls that overlap on the GPU would race on it.
+static __device__ __align__(256) double g_calib_scratch[STQ_CALIBRATE_NOALLOC_MAX_BYTES / sizeof(double)];
+
+// Device address of g_calib_scratch on the current device.  Host code must
+// not hand the symbol itself to a kernel (on the host it names a host-side
+// stand-in); the address is looked up once per device, with that device
+// current, and cached.
+static cudaError_t noalloc_scratch(double **out) {
+    static std::mutex mu;
+    static std::map<int, double *> addr;
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = addr.find(dev);
+    if (it == addr.end()) {
+        void *p = nullptr;
+        err = cudaGetSymbolAddress(&p, g_calib_scratch);
+        if (err != cudaSuccess) return err;
+        it = addr.emplace(dev, static_cast<double *>(p)).first;
+    }
+    *out = it->second;
+    return cudaSuccess;
+}
+
+}  // namespace stq
+
+extern "C" stq_status stq_calibrate_noalloc(stq_state *s, const float *d_S, const float *d_row_weight,
+                                            void *stream) {
+    using namespace stq;
+    if (!s || !d_S) return STQ_ERR_INVALID_ARG;
+    if (!((uintptr_t)d_S % 16 == 0) || (d_row_weight && (uintptr_t)d_row_weight % 4 != 0))
+        return STQ_ERR_MISALIGNED;
+    if (calibrate_workspace_bytes(s->batch, s->heads) > STQ_CALIBRATE_NOALLOC_MAX_BYTES)
+        return STQ_ERR_BUFFER_TOO_SMALL;
+    const uintptr_t S0 = (uintptr_t)d_S, S1 = S0 + (size_t)s->batch * s->heads * kD * kD * sizeof(float);
+    const uintptr_t B0 = (uintptr_t)s->base, B1 = B0 + s->buf_bytes;
+    if (S0 < B1 && B0 < S1) return STQ_ERR_INVALID_ARG;
+    double *ws = nullptr;
+    if (noalloc_scratch(&ws) != cudaSuccess) return STQ_ERR_CUDA;
+    return launch_calibrate(s, d_S, d_row_weight, ws, static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? STQ_OK : STQ_ERR_CUDA;
+}
+
+namespace stq {
 
 // ------------------------------------------------------------- quantize --
 template <int B>
