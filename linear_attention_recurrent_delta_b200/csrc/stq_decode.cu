@@ -3,31 +3,69 @@
 // One persistent CTA of 128 threads walks pages p = blockIdx.x + i*gridDim.x.
 // Each page's bytes and its q, k, v (and KDA alpha) rows are brought into a
 // shared-memory ring by one thread with cp.async.bulk (no multicast), counted
-// on an mbarrier; the ring is 2..4 deep so the copies of later pages overlap
-// the math of the current one.  Per page, all in registers / shared memory:
+// on an mbarrier.  Per page, all in registers / shared memory:
 //   S1 unpack planes -> S2 dequant + decay T = z (alpha r)
-//   S3 column sums u = sum_s k_s T_s (one fma chain per 16-row block, then
-//      ((P0+P1)+(P2+P3))+((P4+P5)+(P6+P7))),  e = v (1/c) - u
-//   S4 T' = T + (beta k_s) e      S5 o = c * sum_s q_s T'_s (same order)
+//   S3 column sums u = sum_s k_s T_s        e = v (1/c) - u
+//   S4 T' = T + (beta k_s) e                 S5 o = c * sum_s q_s T'_s
 //   S6 row absmax -> r' = m/qmax, inv = qmax/m rounded toward zero
 //   S7 requant (RNE of the exact product, or Philox stochastic rounding on
-//      INT rows; binary16 on FP16 rows)   S8 repack and store in place.
-// The state crosses HBM once each way per step.  No tensor cores: the work
-// is rank-1 updates and mat-vecs.
+//      INT rows; binary16 on FP16 rows)    S8 repack.
+// The requantized codes and r' are written back into the page's ring stage,
+// and one bulk copy stores the stage to HBM at the next page's barrier, so
+// the state crosses HBM once each way per step in whole 16-byte chunks.  No
+// tensor cores: the work is rank-1 updates and mat-vecs.
 //
-// Warp w owns the 16-row blocks 2w and 2w+1 and dispatches on their widths at
-// run time.  All warps share one copy of the loop: per-warp copies specialised
-// to each warp's widths were measured slower, the larger code overflowing the
-// instruction cache the SM's warps share.
+// Thread mapping: lane l owns value columns 4l .. 4l+3; warp w owns slice w
+// of every 16-row block, i.e. stored rows 16b + 4w + i (b = 0..7, i = 0..3).
+// Every warp therefore meets the blocks' widths in the same order and all
+// warps of the SM run one instruction stream; for the formats known at
+// compile time that stream has no branch on a width.  Column sums follow
+// the canonical order of the oracle: per thread one fma chain over blocks
+// 0-3 and one over blocks 4-7 (16 rows each, ascending), their sum per warp,
+// then (W0 + W1) + (W2 + W3) over the warps.
 //
 // One CTA-wide barrier per page: each warp prepares the operands of its own
-// rows (thread 32w + l: stored row 32w + l) and syncs within the warp; the
-// column sums' block partials and 1/c are double-buffered by page parity, so
-// the only cross-warp dependency is u (and o, finished after the next page's
-// barrier).  Warps of a CTA drift apart by up to a page.
+// rows and syncs within the warp; the warps' column-sum partials and 1/c are
+// double-buffered by page parity, so the only cross-warp dependency is u
+// (and o, finished after the next page's barrier).
+#include <type_traits>
+
 #include "stq_internal.h"
 
 namespace stq {
+
+// ---- formats: widths per 16-row block (16 = FP16) known at compile time,
+// or read from DevFormat at run time (any other valid format)
+template <int W0, int W1, int W2, int W3, int W4, int W5, int W6, int W7, bool COLS, bool GVEC, bool SR>
+struct StaticFmt {
+    static constexpr bool kRuntime = false;
+    static constexpr bool kCols = COLS, kGvec = GVEC, kSr = SR;
+    __host__ __device__ static constexpr int width(int b) {
+        return b == 0 ? W0 : b == 1 ? W1 : b == 2 ? W2 : b == 3 ? W3 : b == 4 ? W4 : b == 5 ? W5 : b == 6 ? W6 : W7;
+    }
+    // offset of block b's codes and index of its first r (INT rows, stored order)
+    __host__ __device__ static constexpr int offset(int b) {
+        int off = 0;
+        for (int i = 0; i < b; ++i) off += 256 * width(i);
+        return off;
+    }
+    __host__ __device__ static constexpr int rbase(int b) {
+        int r = 0;
+        for (int i = 0; i < b; ++i) r += width(i) == 16 ? 0 : 16;
+        return r;
+    }
+};
+
+template <bool SR>
+struct RuntimeFmt {
+    static constexpr bool kRuntime = true;
+    static constexpr bool kSr = SR;
+};
+
+using FmtStepQuant6 = StaticFmt<8, 8, 6, 6, 6, 6, 4, 4, true, false, false>;
+using FmtInt8Row = StaticFmt<8, 8, 8, 8, 8, 8, 8, 8, false, false, false>;
+using FmtStepQuant4Kda = StaticFmt<8, 4, 4, 4, 3, 3, 3, 3, true, true, false>;
+using FmtDamp = StaticFmt<16, 8, 8, 8, 8, 8, 8, 8, false, false, true>;
 
 struct DecodeArgs {
     uint8_t *pages;
@@ -37,32 +75,26 @@ struct DecodeArgs {
     float *o;
     int n_pages;                  // < 2^31 (checked when the state is bound)
     int heads;
-    int n_stages;                 // ring depth, 2 .. kMaxStages
+    int n_stages;                 // ring depth, 3 .. kMaxStages
     uint32_t stage_bytes;
+    uint32_t store_bytes;         // codes + r: the part of a page a step rewrites
     uint32_t seed_lo, seed_hi, step;
     uint64_t wait_limit_ns;
     int stall_first_wait;
 };
 
 constexpr int kMaxStages = 4;
-constexpr int kRmxPitch = 36;     // words per row of the row-max tile
 
 struct SmemFixed {
-    // per stored row (a 16-byte load serves 4 rows; an f32x2 operation takes
-    // the value duplicated without a move):
-    float a[kD];                            // alpha * r (decay x row scale)
-    float kp[kD];                           // k of the row's key channel
-    float bk[kD];                           // beta * k
-    float qp[kD];                           // q
-    float red_u[2][kWarps][kD];             // per page parity and warp: P_2w + P_2w+1 of u
-    float red_o[2][kWarps][kD];             // the same for o
-    // row-partial maxima: row r of a warp at r * kRmxPitch, one word per lane;
-    // the pitch keeps both the per-row stores and the 16-byte row reads
-    // free of bank conflicts
-    float rmx[kWarps][kRowsPerWarp * kRmxPitch];
+    // per warp, its 32 rows in slice order (row 4b + i = block b, row i):
+    float a[kWarps][kRowsPerWarp];          // alpha * r (decay x row scale)
+    float kp[kWarps][kRowsPerWarp];         // k of the row's key channel
+    float bk[kWarps][kRowsPerWarp];         // beta * k
+    float qp[kWarps][kRowsPerWarp];         // q
     float inv[kWarps][kRowsPerWarp];        // requant multipliers
+    float red_u[2][kWarps][kD];             // per page parity and warp: chain sums of u
+    float red_o[2][kWarps][kD];             // the same for o
     float ic[2][kD];                        // per page parity: 1 / c per column
-    float c_prev[kD];                       // c of the page whose o is pending
     uint64_t full[kMaxStages];              // stage-full barriers
     uint64_t never;                         // a barrier nothing completes (test hook)
 };
@@ -82,148 +114,232 @@ __device__ __forceinline__ float div_by_qmax(float m, float qmax, float rcp_qmax
     return __fmaf_rn(__fmaf_rn(-q0, qmax, m), rcp_qmax, q0);
 }
 
-// ---- S1 + S2: one 16-row block into T[r0 .. r0+15] (a: the block's alpha * r)
+// ---- S1 / S8 on one slice: rows 4w .. 4w+3 of a 16-row block.
+// Plane words of a slice (quad l): width 8: the whole chunk w; width 4: the
+// half chunk holding rows (0,1), (2,3); width 2: one word, row i at bits 2i
+// of each byte; width 1: half the bits of one word (bits 4(w&1) + i), shared
+// with the partner slice w ^ 1.
 template <int B>
-__device__ __forceinline__ void dequant_int(const uint8_t *blk, int lane, const float *a,
-                                            float2 (&T)[kRowsPerWarp][2], int r0) {
-    uint32_t ub[16];
-    unpack_int_block<B>(blk, lane, ub);
-    const float bm = 8388608.0f + (float)(1 << (B - 1));
+__device__ __forceinline__ void unpack_int_slice(const uint8_t *blk, int w, int lane, uint32_t (&ub)[4]) {
+    if constexpr (B == 8) {
+        const uint4 c = *reinterpret_cast<const uint4 *>(blk + (32 * w + lane) * 16);
+        ub[0] = c.x; ub[1] = c.y; ub[2] = c.z; ub[3] = c.w;
+    } else {
+        constexpr bool p4 = (B & 4) != 0, p2 = (B & 2) != 0, p1 = (B & 1) != 0;
+        constexpr int lo2 = p4 ? 4 : 0;
+        constexpr int lo1 = lo2 + (p2 ? 2 : 0);
+        constexpr int off2 = p4 ? 1024 : 0;
+        constexpr int off1 = off2 + (p2 ? 512 : 0);
 #pragma unroll
-    for (int r = 0; r < 16; r += 4) {
-        const float4 aa = *reinterpret_cast<const float4 *>(a + r);   // rows r .. r+3
-        const float av[4] = {aa.x, aa.y, aa.z, aa.w};
+        for (int i = 0; i < 4; ++i) ub[i] = 0;
+        if constexpr (p4) {
+            const uint2 c = *reinterpret_cast<const uint2 *>(blk + (32 * (w >> 1) + lane) * 16 + 8 * (w & 1));
+            ub[0] = c.x & plane_mask<4>();
+            ub[1] = (c.x >> 4) & plane_mask<4>();
+            ub[2] = c.y & plane_mask<4>();
+            ub[3] = (c.y >> 4) & plane_mask<4>();
+        }
+        if constexpr (p2) {
+            const uint32_t c = *reinterpret_cast<const uint32_t *>(blk + off2 + lane * 16 + 4 * w);
+            ub[0] |= move_bits<0, lo2>(c) & (plane_mask<2>() << lo2);
+            ub[1] |= move_bits<2, lo2>(c) & (plane_mask<2>() << lo2);
+            ub[2] |= move_bits<4, lo2>(c) & (plane_mask<2>() << lo2);
+            ub[3] |= move_bits<6, lo2>(c) & (plane_mask<2>() << lo2);
+        }
+        if constexpr (p1) {
+            const uint32_t c = *reinterpret_cast<const uint32_t *>(blk + off1 + lane * 8 + 4 * (w >> 1)) >>
+                               (4 * (w & 1));
+            ub[0] |= move_bits<0, lo1>(c) & (plane_mask<1>() << lo1);
+            ub[1] |= move_bits<1, lo1>(c) & (plane_mask<1>() << lo1);
+            ub[2] |= move_bits<2, lo1>(c) & (plane_mask<1>() << lo1);
+            ub[3] |= move_bits<3, lo1>(c) & (plane_mask<1>() << lo1);
+        }
+    }
+}
+
+// Inverse of unpack_int_slice (ub bytes < 2^B), in place in the stage.  The
+// 1-bit plane's word is shared with the partner slice: only this slice's
+// bits are flipped, by an atomic xor, so the two slices may write in any order.
+template <int B>
+__device__ __forceinline__ void pack_int_slice(uint8_t *blk, int w, int lane, const uint32_t (&ub)[4]) {
+    if constexpr (B == 8) {
+        *reinterpret_cast<uint4 *>(blk + (32 * w + lane) * 16) = make_uint4(ub[0], ub[1], ub[2], ub[3]);
+    } else {
+        constexpr bool p4 = (B & 4) != 0, p2 = (B & 2) != 0, p1 = (B & 1) != 0;
+        constexpr int lo2 = p4 ? 4 : 0;
+        constexpr int lo1 = lo2 + (p2 ? 2 : 0);
+        constexpr int off2 = p4 ? 1024 : 0;
+        constexpr int off1 = off2 + (p2 ? 512 : 0);
+        if constexpr (p4) {
+            uint32_t x0, x1;
+            if constexpr (B == 4) {   // codes < 16: the nibbles need no mask
+                x0 = ub[0] | (ub[1] << 4);
+                x1 = ub[2] | (ub[3] << 4);
+            } else {
+                x0 = (ub[0] & plane_mask<4>()) | ((ub[1] << 4) & ~plane_mask<4>());
+                x1 = (ub[2] & plane_mask<4>()) | ((ub[3] << 4) & ~plane_mask<4>());
+            }
+            *reinterpret_cast<uint2 *>(blk + (32 * (w >> 1) + lane) * 16 + 8 * (w & 1)) = make_uint2(x0, x1);
+        }
+        if constexpr (p2) {
+            uint32_t x;
+            if constexpr (B == 2) {   // codes < 4: fields never spill
+                x = ub[0] | (ub[1] << 2) | (ub[2] << 4) | (ub[3] << 6);
+            } else {
+                x = move_bits<lo2, 0>(ub[0]) & plane_mask<2>();
+                x |= move_bits<lo2, 2>(ub[1]) & (plane_mask<2>() << 2);
+                x |= move_bits<lo2, 4>(ub[2]) & (plane_mask<2>() << 4);
+                x |= move_bits<lo2, 6>(ub[3]) & (plane_mask<2>() << 6);
+            }
+            *reinterpret_cast<uint32_t *>(blk + off2 + lane * 16 + 4 * w) = x;
+        }
+        if constexpr (p1) {
+            uint32_t x = move_bits<lo1, 0>(ub[0]) & plane_mask<1>();
+            x |= move_bits<lo1, 1>(ub[1]) & (plane_mask<1>() << 1);
+            x |= move_bits<lo1, 2>(ub[2]) & (plane_mask<1>() << 2);
+            x |= move_bits<lo1, 3>(ub[3]) & (plane_mask<1>() << 3);
+            uint32_t *word = reinterpret_cast<uint32_t *>(blk + off1 + lane * 8 + 4 * (w >> 1));
+            const int sh = 4 * (w & 1);
+            const uint32_t mine = (*word >> sh) & 0x0F0F0F0Fu;   // this slice's bits: no one else writes them
+            atomicXor(word, (mine ^ x) << sh);
+        }
+    }
+}
+
+// FP16 slice: words 8w .. 8w+7 of the quad (chunks 2w, 2w+1); word 2i + h
+// holds row 4w + i, columns 4l + 2h (low half) and 4l + 2h + 1.
+__device__ __forceinline__ void load_fp16_slice(const uint8_t *blk, int w, int lane, uint32_t (&x)[8]) {
+    const uint4 c0 = *reinterpret_cast<const uint4 *>(blk + (32 * (2 * w) + lane) * 16);
+    const uint4 c1 = *reinterpret_cast<const uint4 *>(blk + (32 * (2 * w + 1) + lane) * 16);
+    x[0] = c0.x; x[1] = c0.y; x[2] = c0.z; x[3] = c0.w;
+    x[4] = c1.x; x[5] = c1.y; x[6] = c1.z; x[7] = c1.w;
+}
+
+__device__ __forceinline__ void store_fp16_slice(uint8_t *blk, int w, int lane, const uint32_t (&x)[8]) {
+    *reinterpret_cast<uint4 *>(blk + (32 * (2 * w) + lane) * 16) = make_uint4(x[0], x[1], x[2], x[3]);
+    *reinterpret_cast<uint4 *>(blk + (32 * (2 * w + 1) + lane) * 16) = make_uint4(x[4], x[5], x[6], x[7]);
+}
+
+// ---- per-block dispatch: fn(std::integral_constant<int, width>) for block B
+template <int V>
+using IC = std::integral_constant<int, V>;
+
+template <class FMT, int B, class Fn>
+__device__ __forceinline__ void with_width(const DevFormat &F, Fn &&fn) {
+    if constexpr (!FMT::kRuntime) {
+        fn(IC<FMT::width(B)>{});
+    } else {
+        switch (F.blk_bits(B)) {
+            case 16: fn(IC<16>{}); break;
+            case 8: fn(IC<8>{}); break;
+            case 7: fn(IC<7>{}); break;
+            case 6: fn(IC<6>{}); break;
+            case 5: fn(IC<5>{}); break;
+            case 4: fn(IC<4>{}); break;
+            case 3: fn(IC<3>{}); break;
+            default: fn(IC<2>{}); break;
+        }
+    }
+}
+
+template <int I, int N, class Fn>
+__device__ __forceinline__ void static_for(Fn &&fn) {
+    if constexpr (I < N) {
+        fn(IC<I>{});
+        static_for<I + 1, N>(fn);
+    }
+}
+
+template <class FMT, int B>
+__device__ __forceinline__ int fmt_offset(const DevFormat &F) {
+    if constexpr (FMT::kRuntime) {
+        return F.blk_off(B);
+    } else {
+        constexpr int off = FMT::offset(B);
+        return off;
+    }
+}
+
+using Tile = float2[kBlocks][4][2];   // a thread's T: [block][row of the slice][column pair]
+
+// ---- S1 + S2 on slice w of block B (a4: the four rows' alpha * r)
+template <int W, int B>
+__device__ __forceinline__ void dequant_slice(const uint8_t *blk, int w, int lane, const float4 a4, Tile &T) {
+    const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+    if constexpr (W == 16) {
+        uint32_t x[8];
+        load_fp16_slice(blk, w, lane, x);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 as = make_float2(av[i], av[i]);
+            T[B][i][0] = __fmul2_rn(__half22float2(*reinterpret_cast<const __half2 *>(&x[2 * i])), as);
+            T[B][i][1] = __fmul2_rn(__half22float2(*reinterpret_cast<const __half2 *>(&x[2 * i + 1])), as);
+        }
+    } else {
+        uint32_t ub[4];
+        unpack_int_slice<W>(blk, w, lane, ub);
+        const float bm = 8388608.0f + (float)(1 << (W - 1));
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             float2 z01, z23;
-            codes_to_float(ub[r + i], bm, z01, z23);
-            T[r0 + r + i][0] = __fmul2_rn(z01, make_float2(av[i], av[i]));
-            T[r0 + r + i][1] = __fmul2_rn(z23, make_float2(av[i], av[i]));
+            codes_to_float(ub[i], bm, z01, z23);
+            T[B][i][0] = __fmul2_rn(z01, make_float2(av[i], av[i]));
+            T[B][i][1] = __fmul2_rn(z23, make_float2(av[i], av[i]));
         }
     }
 }
 
-__device__ __forceinline__ void dequant_fp16(const uint8_t *blk, int lane, const float *a,
-                                             float2 (&T)[kRowsPerWarp][2], int r0) {
-    uint32_t w[32];
-    unpack_fp16_block(blk, lane, w);
-#pragma unroll
-    for (int r = 0; r < 16; ++r) {
-        const float2 as = make_float2(a[r], a[r]);
-        float2 x01 = __half22float2(*reinterpret_cast<const __half2 *>(&w[2 * r]));
-        float2 x23 = __half22float2(*reinterpret_cast<const __half2 *>(&w[2 * r + 1]));
-        T[r0 + r][0] = __fmul2_rn(x01, as);
-        T[r0 + r][1] = __fmul2_rn(x23, as);
-    }
-}
-
-// BITS: the block's width (16 = FP16), or 0 to read `bits` at run time.
-template <int BITS, int R0>
-__device__ __forceinline__ void dequant_block(int bits, const uint8_t *blk, int lane, const float *a,
-                                              float2 (&T)[kRowsPerWarp][2]) {
-    if constexpr (BITS == 16) dequant_fp16(blk, lane, a, T, R0);
-    else if constexpr (BITS != 0) dequant_int<BITS>(blk, lane, a, T, R0);
-    else {
-        switch (bits) {
-            case 16: dequant_fp16(blk, lane, a, T, R0); break;
-            case 8: dequant_int<8>(blk, lane, a, T, R0); break;
-            case 7: dequant_int<7>(blk, lane, a, T, R0); break;
-            case 6: dequant_int<6>(blk, lane, a, T, R0); break;
-            case 5: dequant_int<5>(blk, lane, a, T, R0); break;
-            case 4: dequant_int<4>(blk, lane, a, T, R0); break;
-            case 3: dequant_int<3>(blk, lane, a, T, R0); break;
-            default: dequant_int<2>(blk, lane, a, T, R0); break;
-        }
-    }
-}
-
-// ---- S7 + S8: requantize one 16-row block of T' and store its planes.
+// ---- S7 + S8 on slice w of block B, in place in the stage
 struct SrCtx {
     uint32_t k0, k1, step, b, h;
 };
 
-template <int B, bool SR>
-__device__ __forceinline__ void requant_int(uint8_t *blk, int lane, const float *inv,
-                                            const float2 (&T)[kRowsPerWarp][2], int r0, int s0,
-                                            const SrCtx sr) {
-    const float M = 12582912.0f + (float)(1 << (B - 1));   // 1.5 * 2^23 + bias
-    const float2 M2 = make_float2(M, M);
-    uint32_t ub[16];
-#pragma unroll
-    for (int r = 0; r < 16; r += 2) {
-        const float4 i4 = *reinterpret_cast<const float4 *>(inv + (r & ~3));   // rows r & ~3 .. +3
-        const float ia = (r & 2) ? i4.z : i4.x, ib = (r & 2) ? i4.w : i4.y;
-        const float2 i0 = make_float2(ia, ia), i1 = make_float2(ib, ib);
-        float2 y0, y1, y2, y3;
-        if constexpr (SR) {
-            const int s = s0 + r;   // even
-            const uint4 h = philox4x32_10(
-                make_uint4((uint32_t)(s >> 1) * 32u + (uint32_t)lane, sr.step, sr.b, sr.h), sr.k0, sr.k1);
-            y0 = __fadd2_rn(__ffma2_rn(T[r0 + r][0], i0, sr_delta_pair(h.x)), M2);
-            y1 = __fadd2_rn(__ffma2_rn(T[r0 + r][1], i0, sr_delta_pair(h.y)), M2);
-            y2 = __fadd2_rn(__ffma2_rn(T[r0 + r + 1][0], i1, sr_delta_pair(h.z)), M2);
-            y3 = __fadd2_rn(__ffma2_rn(T[r0 + r + 1][1], i1, sr_delta_pair(h.w)), M2);
-        } else {
-            y0 = __ffma2_rn(T[r0 + r][0], i0, M2);
-            y1 = __ffma2_rn(T[r0 + r][1], i0, M2);
-            y2 = __ffma2_rn(T[r0 + r + 1][0], i1, M2);
-            y3 = __ffma2_rn(T[r0 + r + 1][1], i1, M2);
-        }
-        ub[r] = low_bytes(y0.x, y0.y, y1.x, y1.y);
-        ub[r + 1] = low_bytes(y2.x, y2.y, y3.x, y3.y);
-    }
-    pack_int_block<B>(blk, lane, ub);
-}
-
-__device__ __forceinline__ void requant_fp16(uint8_t *blk, int lane, const float2 (&T)[kRowsPerWarp][2],
-                                             int r0) {
-    uint32_t w[32];
-#pragma unroll
-    for (int r = 0; r < 16; ++r) {
-        __half2 h01 = __floats2half2_rn(T[r0 + r][0].x, T[r0 + r][0].y);
-        __half2 h23 = __floats2half2_rn(T[r0 + r][1].x, T[r0 + r][1].y);
-        w[2 * r] = *reinterpret_cast<uint32_t *>(&h01);
-        w[2 * r + 1] = *reinterpret_cast<uint32_t *>(&h23);
-    }
-    pack_fp16_block(blk, lane, w);
-}
-
-template <int BITS, int R0, bool SR>
-__device__ __forceinline__ void requant_block(int bits, uint8_t *blk, int lane, const float *inv,
-                                              const float2 (&T)[kRowsPerWarp][2], int s0, const SrCtx sr) {
-    if constexpr (BITS == 16) requant_fp16(blk, lane, T, R0);
-    else if constexpr (BITS != 0) requant_int<BITS, SR>(blk, lane, inv, T, R0, s0, sr);
-    else {
-        switch (bits) {
-            case 16: requant_fp16(blk, lane, T, R0); break;
-            case 8: requant_int<8, SR>(blk, lane, inv, T, R0, s0, sr); break;
-            case 7: requant_int<7, SR>(blk, lane, inv, T, R0, s0, sr); break;
-            case 6: requant_int<6, SR>(blk, lane, inv, T, R0, s0, sr); break;
-            case 5: requant_int<5, SR>(blk, lane, inv, T, R0, s0, sr); break;
-            case 4: requant_int<4, SR>(blk, lane, inv, T, R0, s0, sr); break;
-            case 3: requant_int<3, SR>(blk, lane, inv, T, R0, s0, sr); break;
-            default: requant_int<2, SR>(blk, lane, inv, T, R0, s0, sr); break;
-        }
-    }
-}
-
-// ---- S3 / S5 partial sums of one 16-row block: chains p = fma(w_s, X_s, p)
-// from 0 in ascending row order, two column pairs.
-template <int R0>
-__device__ __forceinline__ void block_chain(const float *w, const float2 (&X)[kRowsPerWarp][2],
-                                            float2 &p01, float2 &p23) {
-    p01 = make_float2(0.f, 0.f);
-    p23 = make_float2(0.f, 0.f);
-#pragma unroll
-    for (int r = 0; r < 16; r += 4) {
-        const float4 ww = *reinterpret_cast<const float4 *>(w + r);
-        const float wv[4] = {ww.x, ww.y, ww.z, ww.w};
+template <int W, int B, bool SR>
+__device__ __forceinline__ void requant_slice(uint8_t *blk, int w, int lane, const float4 inv4, const Tile &T,
+                                              const SrCtx sr) {
+    if constexpr (W == 16) {
+        uint32_t x[8];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            p01 = __ffma2_rn(make_float2(wv[i], wv[i]), X[R0 + r + i][0], p01);
-            p23 = __ffma2_rn(make_float2(wv[i], wv[i]), X[R0 + r + i][1], p23);
+            __half2 h01 = __floats2half2_rn(T[B][i][0].x, T[B][i][0].y);
+            __half2 h23 = __floats2half2_rn(T[B][i][1].x, T[B][i][1].y);
+            x[2 * i] = *reinterpret_cast<uint32_t *>(&h01);
+            x[2 * i + 1] = *reinterpret_cast<uint32_t *>(&h23);
         }
+        store_fp16_slice(blk, w, lane, x);
+    } else {
+        const float M = 12582912.0f + (float)(1 << (W - 1));   // 1.5 * 2^23 + bias
+        const float2 M2 = make_float2(M, M);
+        const float iv[4] = {inv4.x, inv4.y, inv4.z, inv4.w};
+        uint32_t ub[4];
+#pragma unroll
+        for (int i = 0; i < 4; i += 2) {
+            const float2 i0 = make_float2(iv[i], iv[i]), i1 = make_float2(iv[i + 1], iv[i + 1]);
+            float2 y0, y1, y2, y3;
+            if constexpr (SR) {
+                const uint32_t s = 16u * B + 4u * (uint32_t)w + (uint32_t)i;   // stored row, even
+                const uint4 h = philox4x32_10(make_uint4((s >> 1) * 32u + (uint32_t)lane, sr.step, sr.b, sr.h),
+                                              sr.k0, sr.k1);
+                y0 = __fadd2_rn(__ffma2_rn(T[B][i][0], i0, sr_delta_pair(h.x)), M2);
+                y1 = __fadd2_rn(__ffma2_rn(T[B][i][1], i0, sr_delta_pair(h.y)), M2);
+                y2 = __fadd2_rn(__ffma2_rn(T[B][i + 1][0], i1, sr_delta_pair(h.z)), M2);
+                y3 = __fadd2_rn(__ffma2_rn(T[B][i + 1][1], i1, sr_delta_pair(h.w)), M2);
+            } else {
+                y0 = __ffma2_rn(T[B][i][0], i0, M2);
+                y1 = __ffma2_rn(T[B][i][1], i0, M2);
+                y2 = __ffma2_rn(T[B][i + 1][0], i1, M2);
+                y3 = __ffma2_rn(T[B][i + 1][1], i1, M2);
+            }
+            ub[i] = low_bytes(y0.x, y0.y, y1.x, y1.y);
+            ub[i + 1] = low_bytes(y2.x, y2.y, y3.x, y3.y);
+        }
+        pack_int_slice<W>(blk, w, lane, ub);
     }
+}
+
+// max |x| over a row's four columns held by one lane
+__device__ __forceinline__ float absmax4(float2 a, float2 b) {
+    return fmaxf(max3f(fabsf(a.x), fabsf(a.y), fabsf(b.x)), fabsf(b.y));
 }
 
 __device__ __forceinline__ void issue_stage(const DevFormat &F, const DecodeArgs &A, uint8_t *dst, int p,
@@ -237,9 +353,10 @@ __device__ __forceinline__ void issue_stage(const DevFormat &F, const DecodeArgs
     if (F.gate_vector) bulk_g2s(rows + 1536, A.alpha + (size_t)p * kD, 512, bar);
 }
 
-// o of a finished page: the tree over the warps' block-pair partials, times c.
+// o of a finished page: the tree over the warps' chain sums, times c (read
+// from the page's stage, which is not refilled before the next barrier).
 __device__ __forceinline__ void write_o(const float (*red_o)[kD], const DecodeArgs &A, int p, int lane,
-                                        const float *c_prev, int col_scales) {
+                                        const uint8_t *stage, const DevFormat &F, bool col_scales) {
     const float4 o0 = *reinterpret_cast<const float4 *>(&red_o[0][4 * lane]);
     const float4 o1 = *reinterpret_cast<const float4 *>(&red_o[1][4 * lane]);
     const float4 o2 = *reinterpret_cast<const float4 *>(&red_o[2][4 * lane]);
@@ -249,7 +366,7 @@ __device__ __forceinline__ void write_o(const float (*red_o)[kD], const DecodeAr
     float2 ob = __fadd2_rn(__fadd2_rn(make_float2(o0.z, o0.w), make_float2(o1.z, o1.w)),
                            __fadd2_rn(make_float2(o2.z, o2.w), make_float2(o3.z, o3.w)));
     if (col_scales) {
-        const float4 c = *reinterpret_cast<const float4 *>(&c_prev[4 * lane]);
+        const float4 c = *reinterpret_cast<const float4 *>(stage + F.c_off + 16 * lane);
         oa = __fmul2_rn(make_float2(c.x, c.y), oa);
         ob = __fmul2_rn(make_float2(c.z, c.w), ob);
     }
@@ -261,45 +378,65 @@ __device__ __forceinline__ void write_o(const float (*red_o)[kD], const DecodeAr
 template <bool SR>
 constexpr int decode_ctas_per_sm() { return SR ? 2 : 3; }
 
-// Iteration index at which a CTA processed page p.
-__device__ __forceinline__ int it_last(int p, unsigned first, unsigned stride) {
-    return (p - (int)first) / (int)stride;
-}
-
-__device__ __forceinline__ float absmax4(float2 a, float2 b) {
-    return fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(b.x), fabsf(b.y)));
-}
-
-// The per-page loop (every warp runs this one body; warp w owns blocks 2w, 2w+1).
-template <bool SR>
-__global__ void __launch_bounds__(kThreads, decode_ctas_per_sm<SR>())
+// The per-page loop.
+template <class FMT>
+__global__ void __launch_bounds__(kThreads, decode_ctas_per_sm<FMT::kSr>())
 decode_kernel(const DevFormat F, const DecodeArgs A) {
     extern __shared__ __align__(128) uint8_t smem[];
     SmemFixed &S = *reinterpret_cast<SmemFixed *>(smem);
     uint8_t *stages = smem + kFixedBytes;
-    const int warp = threadIdx.x >> 5;
-    constexpr int BA = 0, BB = 0;   // block widths come from F at run time
+    constexpr bool SR = FMT::kSr;
+    bool col_scales, gate_vector;
+    if constexpr (FMT::kRuntime) {
+        col_scales = F.col_scales != 0;
+        gate_vector = F.gate_vector != 0;
+    } else {
+        col_scales = FMT::kCols;
+        gate_vector = FMT::kGvec;
+    }
 
-    if (threadIdx.x == 0) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (tid == 0) {
         for (int st = 0; st < A.n_stages; ++st) mbar_init(&S.full[st], 1);
         mbar_init(&S.never, 1);
         fence_mbar_init();
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-        for (int i = 0; i < A.n_stages; ++i) {
-            const int p = (int)blockIdx.x + i * (int)gridDim.x;
-            if (p < A.n_pages) issue_stage(F, A, stages + i * A.stage_bytes, p, &S.full[i]);
-        }
-    }
-    const int tid = threadIdx.x, lane = tid & 31;
     const int stride = (int)gridDim.x;
     const int n = A.n_pages;
     const int NS = A.n_stages;
+    if (tid == 0) {
+        for (int i = 0; i < NS; ++i) {
+            const int p = (int)blockIdx.x + i * stride;
+            if (p < n) issue_stage(F, A, stages + i * A.stage_bytes, p, &S.full[i]);
+        }
+    }
     // (request, head) of a page is carried along: p advances by `stride`,
     // i.e. by (stride / H, stride % H) with a carry
     const int H = A.heads;
     const int sb = stride / H, sh = stride % H;
+
+    // this lane's row of the slice (operand preparation and S6): block
+    // my_blk = lane / 4, stored row my_s
+    const int my_blk = lane >> 2;
+    const int my_s = 16 * my_blk + 4 * warp + (lane & 3);
+    int my_bits, my_rbase;
+    if constexpr (FMT::kRuntime) {
+        my_bits = F.blk_bits(my_blk);
+        my_rbase = F.blk_rbase(my_blk);
+    } else {
+        my_bits = 0;
+        my_rbase = 0;
+#pragma unroll
+        for (int b = 0; b < kBlocks; ++b) {   // selects, not a table in local memory
+            if (b == my_blk) my_bits = FMT::width(b);
+            if (b < my_blk && FMT::width(b) != 16) my_rbase += 16;
+        }
+    }
+    const bool my_int = my_bits != 16;
+    const int my_r = my_rbase + 4 * warp + (lane & 3);
+    const float my_qmax = my_int ? (float)((1 << (my_bits - 1)) - 1) : 0.f;
+    const float my_rcp = my_int ? __frcp_rn(my_qmax) : 0.f;
 
     int p = (int)blockIdx.x;
     int pb = p / H, ph = p % H;            // request and head of page p
@@ -307,23 +444,15 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
     int kap = 0;
     if (p < n) {
         beta_s = __ldg(A.beta + p);
-        if (!F.gate_vector) alpha_s = __ldg(A.alpha + p);
-        kap = __ldg(A.perm + ph * kD + tid) & (kD - 1);
+        if (!gate_vector) alpha_s = __ldg(A.alpha + p);
+        kap = __ldg(A.perm + ph * kD + my_s) & (kD - 1);
     }
-    const int b0 = 2 * warp, b1 = 2 * warp + 1;
-    const int bits0 = BA ? BA : F.blk_bits(b0), bits1 = BB ? BB : F.blk_bits(b1);
-    const int off0 = F.blk_off(b0), off1 = F.blk_off(b1);
-    // this lane's row of S6 (row 32w + lane) and its scales' constants
-    const int my_bits = (lane < 16) ? bits0 : bits1;
-    const float my_qmax = (my_bits == 16) ? 0.f : (float)((1 << (my_bits - 1)) - 1);
-    const float my_rcp = (my_bits == 16) ? 0.f : __frcp_rn(my_qmax);
-    const int my_r = F.blk_rbase(lane < 16 ? b0 : b1) + (lane & 15);
-    float *rmx = S.rmx[warp];
-    int p_prev = -1;                  // page whose o is still to be written
-    int st = 0;
+    int p_prev = -1;                  // page whose codes and o are still to be stored
+    int st = 0, st_prev = 0;
     uint32_t parity = 0;
+    int it = 0;
 
-    for (int it = 0; p < n; ++it) {
+    for (; p < n; ++it) {
         // scalars of the next page, loaded early
         const int pn = p + stride;
         int pnb = pb + sb, pnh = ph + sh;
@@ -332,8 +461,8 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
         int kap_n = 0;
         if (pn < n) {
             beta_n = __ldg(A.beta + pn);
-            if (!F.gate_vector) alpha_n = __ldg(A.alpha + pn);
-            kap_n = __ldg(A.perm + pnh * kD + tid) & (kD - 1);
+            if (!gate_vector) alpha_n = __ldg(A.alpha + pn);
+            kap_n = __ldg(A.perm + pnh * kD + my_s) & (kD - 1);
         }
 
         // a wait that runs out is voted on at the page's barrier, before
@@ -342,78 +471,100 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
         if (A.stall_first_wait && it == 0) ok = mbar_wait_bounded(&S.never, 0, A.wait_limit_ns);
         else ok = mbar_wait_bounded(&S.full[st], parity, A.wait_limit_ns);
         const int par = it & 1;
-        const uint8_t *stg = stages + st * A.stage_bytes;
+        uint8_t *stg = stages + st * A.stage_bytes;
         const float *q_s = reinterpret_cast<const float *>(stg + F.page_bytes);
         const float *k_s = q_s + kD;
         const float *v_s = q_s + 2 * kD;
         const float *al_s = q_s + 3 * kD;
+        float *r_s = reinterpret_cast<float *>(stg + F.r_off);
 
-        // per stored row s = tid: decay x row scale, permuted k and q, beta k
+        // operands of this lane's row: decay x row scale, permuted k and q, beta k
         {
-            const int s = tid, blk = s >> 4;
             const float kk = k_s[kap], qq = q_s[kap];
-            const float al = F.gate_vector ? al_s[kap] : alpha_s;
-            float a = al;
-            if (F.blk_kind(blk) == kKindInt) {
-                const float r = reinterpret_cast<const float *>(stg + F.r_off)[F.blk_rbase(blk) + (s & 15)];
-                a = __fmul_rn(al, r);
-            }
-            const float bk = __fmul_rn(beta_s, kk);
-            if (F.col_scales)   // thread s also inverts the scale of column s
-                S.ic[par][s] = __frcp_rn(reinterpret_cast<const float *>(stg + F.c_off)[s]);
-            S.a[s] = a;
-            S.kp[s] = kk;
-            S.qp[s] = qq;
-            S.bk[s] = bk;
+            const float al = gate_vector ? al_s[kap] : alpha_s;
+            const float a = my_int ? __fmul_rn(al, r_s[my_r]) : al;
+            if (col_scales)   // thread t also inverts the scale of column t
+                S.ic[par][tid] = __frcp_rn(reinterpret_cast<const float *>(stg + F.c_off)[tid]);
+            S.a[warp][lane] = a;
+            S.kp[warp][lane] = kk;
+            S.qp[warp][lane] = qq;
+            S.bk[warp][lane] = __fmul_rn(beta_s, kk);
         }
         __syncwarp();   // the warp's rows' operands come from its own lanes
 
-        // S1 + S2, and S3's block chains
-        float2 T[kRowsPerWarp][2];
-        dequant_block<BA, 0>(bits0, stg + off0, lane, &S.a[32 * warp], T);
-        dequant_block<BB, 16>(bits1, stg + off1, lane, &S.a[32 * warp + 16], T);
+        // S1 + S2 and S3's chains: blocks 0-3 feed chain 0, blocks 4-7 chain 1
+        Tile T;
+        float2 cu[2][2];   // chains from +0, as p = fma(w, x, p) from 0
+#pragma unroll
+        for (int h = 0; h < 2; ++h) cu[h][0] = cu[h][1] = make_float2(0.f, 0.f);
+        static_for<0, kBlocks>([&](auto bc) {
+            constexpr int b = decltype(bc)::value;
+            const float4 a4 = *reinterpret_cast<const float4 *>(&S.a[warp][4 * b]);
+            const uint8_t *blk = stg + fmt_offset<FMT, b>(F);
+            with_width<FMT, b>(F, [&](auto wc) {
+                constexpr int W = decltype(wc)::value;
+                dequant_slice<W, b>(blk, warp, lane, a4, T);
+            });
+            const float4 k4 = *reinterpret_cast<const float4 *>(&S.kp[warp][4 * b]);
+            const float kv[4] = {k4.x, k4.y, k4.z, k4.w};
+            constexpr int h = b >> 2;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                cu[h][0] = __ffma2_rn(make_float2(kv[i], kv[i]), T[b][i][0], cu[h][0]);
+                cu[h][1] = __ffma2_rn(make_float2(kv[i], kv[i]), T[b][i][1], cu[h][1]);
+            }
+        });
         {
-            float2 pa01, pa23, pb01, pb23;
-            block_chain<0>(&S.kp[32 * warp], T, pa01, pa23);
-            block_chain<16>(&S.kp[32 * warp + 16], T, pb01, pb23);
-            const float2 w01 = __fadd2_rn(pa01, pb01), w23 = __fadd2_rn(pa23, pb23);
+            const float2 w01 = __fadd2_rn(cu[0][0], cu[1][0]), w23 = __fadd2_rn(cu[0][1], cu[1][1]);
             *reinterpret_cast<float4 *>(&S.red_u[par][warp][4 * lane]) = make_float4(w01.x, w01.y, w23.x, w23.y);
         }
         const float4 v4 = *reinterpret_cast<const float4 *>(v_s + 4 * lane);
-        float4 c4 = make_float4(1.f, 1.f, 1.f, 1.f);
-        if (F.col_scales) c4 = *reinterpret_cast<const float4 *>(stg + F.c_off + 16 * lane);
         if (__syncthreads_or(!ok)) {
-            // a stage never arrived: record it, let the copies already issued
-            // into the ring land, and leave; nothing of this page was written
+            // a stage never arrived: record it, finish the previous page, let
+            // the copies in flight land and leave; nothing of this page (or
+            // a later one) is written
+            if (warp == 0 && p_prev >= 0)
+                write_o(S.red_o[par ^ 1], A, p_prev, lane, stages + st_prev * A.stage_bytes, F, col_scales);
             if (tid == 0) {
                 atomicOr(A.status, kStatusTimeout);
-                for (int i = 0; i < NS; ++i) {
-                    const int pi = p + i * stride;
-                    if (pi < n) {
-                        const int ii = it + i;
-                        mbar_wait_bounded(&S.full[ii % NS], (uint32_t)((ii / NS) & 1), A.wait_limit_ns);
-                    }
+                if (p_prev >= 0) {
+                    bulk_s2g(A.pages + (size_t)p_prev * F.page_bytes, stages + st_prev * A.stage_bytes,
+                             A.store_bytes);
+                    bulk_commit();
                 }
+                const int last = (it < 2 ? NS - 1 : it - 3 + NS);   // last ring slot whose load was issued
+                for (int j = it; j <= last; ++j) {
+                    if ((int)blockIdx.x + j * stride < n)
+                        mbar_wait_bounded(&S.full[j % NS], (uint32_t)((j / NS) & 1), A.wait_limit_ns);
+                }
+                bulk_wait<0>();
             }
             __syncthreads();
             return;
         }
 
-        // the stage is no longer read: refill it with the page NS iterations ahead
         if (tid == 0) {
-            const int pr = p + NS * stride;
-            if (pr < n) {
-                fence_proxy_async_smem();
-                issue_stage(F, A, stages + st * A.stage_bytes, pr, &S.full[st]);
+            // the previous page is complete in its stage: store it; then the
+            // stage stored one page earlier is free once its store has read it
+            if (p_prev >= 0) {
+                bulk_s2g(A.pages + (size_t)p_prev * F.page_bytes, stages + st_prev * A.stage_bytes, A.store_bytes);
+                bulk_commit();
+            }
+            if (it >= 2) {
+                bulk_wait_read<1>();
+                const int j = it - 2 + NS;
+                const int pr = (int)blockIdx.x + j * stride;
+                if (pr < n) {
+                    fence_proxy_async_smem();
+                    issue_stage(F, A, stages + (j % NS) * A.stage_bytes, pr, &S.full[j % NS]);
+                }
             }
         }
-        // o of the previous page (its block partials were stored before this barrier)
-        if (warp == 0 && p_prev >= 0) {
-            write_o(S.red_o[par ^ 1], A, p_prev, lane, S.c_prev, F.col_scales);
-            if (F.col_scales) *reinterpret_cast<float4 *>(&S.c_prev[4 * lane]) = c4;
-        }
+        // o of the previous page (its chain sums were stored before this barrier)
+        if (warp == 0 && p_prev >= 0)
+            write_o(S.red_o[par ^ 1], A, p_prev, lane, stages + st_prev * A.stage_bytes, F, col_scales);
 
-        // u = ((P0+P1)+(P2+P3))+((P4+P5)+(P6+P7)); e = v (1/c) - u
+        // u = (W0 + W1) + (W2 + W3); e = v (1/c) - u
         float2 e01, e23;
         {
             const float4 u0 = *reinterpret_cast<const float4 *>(&S.red_u[par][0][4 * lane]);
@@ -425,67 +576,73 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
             const float2 ub = __fadd2_rn(__fadd2_rn(make_float2(u0.z, u0.w), make_float2(u1.z, u1.w)),
                                          __fadd2_rn(make_float2(u2.z, u2.w), make_float2(u3.z, u3.w)));
             float4 ic = make_float4(1.f, 1.f, 1.f, 1.f);
-            if (F.col_scales) ic = *reinterpret_cast<const float4 *>(&S.ic[par][4 * lane]);
+            if (col_scales) ic = *reinterpret_cast<const float4 *>(&S.ic[par][4 * lane]);
             // two roundings, scalar: an f32x2 multiply feeding an f32x2 add is
             // fused by the compiler into one f32x2 fma
             e01 = make_float2(__fsub_rn(__fmul_rn(v4.x, ic.x), ua.x), __fsub_rn(__fmul_rn(v4.y, ic.y), ua.y));
             e23 = make_float2(__fsub_rn(__fmul_rn(v4.z, ic.z), ub.x), __fsub_rn(__fmul_rn(v4.w, ic.w), ub.y));
         }
 
-        // S4: T' = T + (beta k) e; row partial maxima into the row-max tile
+        // S4: T' = T + (beta k) e; S6's row maxima (one warp reduction per
+        // row, kept in the row's inv slot); S5's chains
+        float2 co[2][2];
 #pragma unroll
-        for (int r = 0; r < kRowsPerWarp; r += 4) {
-            const float4 bb = *reinterpret_cast<const float4 *>(&S.bk[32 * warp + r]);
-            const float bv[4] = {bb.x, bb.y, bb.z, bb.w};
+        for (int h = 0; h < 2; ++h) co[h][0] = co[h][1] = make_float2(0.f, 0.f);
+        static_for<0, kBlocks>([&](auto bc) {
+            constexpr int b = decltype(bc)::value;
+            constexpr int h = b >> 2;
+            const float4 b4 = *reinterpret_cast<const float4 *>(&S.bk[warp][4 * b]);
+            const float4 q4 = *reinterpret_cast<const float4 *>(&S.qp[warp][4 * b]);
+            const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
+            const float qv[4] = {q4.x, q4.y, q4.z, q4.w};
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                T[r + i][0] = __ffma2_rn(make_float2(bv[i], bv[i]), e01, T[r + i][0]);
-                T[r + i][1] = __ffma2_rn(make_float2(bv[i], bv[i]), e23, T[r + i][1]);
-                rmx[(r + i) * kRmxPitch + lane] = absmax4(T[r + i][0], T[r + i][1]);
+                T[b][i][0] = __ffma2_rn(make_float2(bv[i], bv[i]), e01, T[b][i][0]);
+                T[b][i][1] = __ffma2_rn(make_float2(bv[i], bv[i]), e23, T[b][i][1]);
+                S.inv[warp][4 * b + i] = warp_absmax(absmax4(T[b][i][0], T[b][i][1]));
+                co[h][0] = __ffma2_rn(make_float2(qv[i], qv[i]), T[b][i][0], co[h][0]);
+                co[h][1] = __ffma2_rn(make_float2(qv[i], qv[i]), T[b][i][1], co[h][1]);
             }
-        }
-        // S5: block chains of o, finished at the next page's first barrier
+        });
         {
-            float2 pa01, pa23, pb01, pb23;
-            block_chain<0>(&S.qp[32 * warp], T, pa01, pa23);
-            block_chain<16>(&S.qp[32 * warp + 16], T, pb01, pb23);
-            const float2 w01 = __fadd2_rn(pa01, pb01), w23 = __fadd2_rn(pa23, pb23);
+            const float2 w01 = __fadd2_rn(co[0][0], co[1][0]), w23 = __fadd2_rn(co[0][1], co[1][1]);
             *reinterpret_cast<float4 *>(&S.red_o[par][warp][4 * lane]) = make_float4(w01.x, w01.y, w23.x, w23.y);
         }
         __syncwarp();
 
-        // S6: lane l reduces row l of its warp: r' = m / qmax, inv = qmax / m (toward zero)
-        uint8_t *page = A.pages + (size_t)p * (size_t)F.page_bytes;
+        // S6: lane l finishes row l of the slice: r' = m / qmax, inv = qmax / m (toward zero)
         {
-            const float4 *row = reinterpret_cast<const float4 *>(rmx + lane * kRmxPitch);
-            float m = 0.f;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const float4 x = row[c];
-                m = fmaxf(m, fmaxf(fmaxf(x.x, x.y), fmaxf(x.z, x.w)));
-            }
+            const float m = S.inv[warp][lane];
             float inv = 0.f;
-            if (my_bits != 16) {
+            if (my_int) {
                 float r = 0.f;
                 if (m > 0.f) {
                     r = div_by_qmax(m, my_qmax, my_rcp);
                     inv = __fdiv_rz(my_qmax, m);
                 }
-                reinterpret_cast<float *>(page + F.r_off)[my_r] = r;
+                r_s[my_r] = r;
             }
             S.inv[warp][lane] = inv;
         }
         __syncwarp();
 
-        // S7 + S8
+        // S7 + S8, into the stage
         SrCtx sr;
         sr.k0 = A.seed_lo; sr.k1 = A.seed_hi; sr.step = A.step;
         sr.b = (uint32_t)pb; sr.h = (uint32_t)ph;
-        requant_block<BA, 0, SR>(bits0, page + off0, lane, &S.inv[warp][0], T, 32 * warp, sr);
-        requant_block<BB, 16, SR>(bits1, page + off1, lane, &S.inv[warp][16], T, 32 * warp + 16, sr);
+        static_for<0, kBlocks>([&](auto bc) {
+            constexpr int b = decltype(bc)::value;
+            const float4 i4 = *reinterpret_cast<const float4 *>(&S.inv[warp][4 * b]);
+            uint8_t *blk = stg + fmt_offset<FMT, b>(F);
+            with_width<FMT, b>(F, [&](auto wc) {
+                constexpr int W = decltype(wc)::value;
+                requant_slice<W, b, SR>(blk, warp, lane, i4, T, sr);
+            });
+        });
+        fence_proxy_async_smem();   // the stage's new bytes are read by the bulk store
 
-        if (warp == 0 && p_prev < 0 && F.col_scales) *reinterpret_cast<float4 *>(&S.c_prev[4 * lane]) = c4;
         p_prev = p;
+        st_prev = st;
         alpha_s = alpha_n;
         beta_s = beta_n;
         kap = kap_n;
@@ -495,12 +652,28 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
         if (++st == NS) { st = 0; parity ^= 1u; }
     }
     __syncthreads();
-    if (warp == 0 && p_prev >= 0) write_o(S.red_o[(it_last(p_prev, blockIdx.x, gridDim.x)) & 1], A, p_prev, lane,
-                                          S.c_prev, F.col_scales);
+    if (p_prev >= 0) {
+        if (tid == 0) {
+            bulk_s2g(A.pages + (size_t)p_prev * F.page_bytes, stages + st_prev * A.stage_bytes, A.store_bytes);
+            bulk_commit();
+        }
+        if (warp == 0)
+            write_o(S.red_o[(it - 1) & 1], A, p_prev, lane, stages + st_prev * A.stage_bytes, F, col_scales);
+    }
+    if (tid == 0) bulk_wait<0>();
+}
+
+template <class FMT>
+static bool format_is(const DevFormat &F) {
+    for (int b = 0; b < kBlocks; ++b)
+        if (F.blk_bits(b) != FMT::width(b)) return false;
+    return (F.col_scales != 0) == FMT::kCols && (F.gate_vector != 0) == FMT::kGvec &&
+           (F.stochastic != 0) == FMT::kSr;
 }
 
 static int decode_stages(size_t stride, int ctas_per_sm) {
-    // as many ring stages as fit next to the fixed part at the target occupancy
+    // as many ring stages as fit next to the fixed part at the target
+    // occupancy, at least 3 (a stage is refilled two pages after its use)
     int dev = 0, smem_sm = 0, reserved = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
@@ -508,8 +681,22 @@ static int decode_stages(size_t stride, int ctas_per_sm) {
     const long budget = (long)smem_sm / ctas_per_sm - reserved - (long)kFixedBytes;
     long ns = budget / (long)stride;
     if (ns > kMaxStages) ns = kMaxStages;
-    if (ns < 2) ns = 2;
+    if (ns < 3) ns = 3;
     return (int)ns;
+}
+
+template <class FMT>
+static cudaError_t launch_with(const DevFormat &F, const DecodeArgs &A0, cudaStream_t stream) {
+    DecodeArgs A = A0;
+    A.n_stages = decode_stages(A.stage_bytes, decode_ctas_per_sm<FMT::kSr>());
+    const size_t smem = kFixedBytes + (size_t)A.n_stages * A.stage_bytes;
+    const void *fn = (const void *)decode_kernel<FMT>;
+    cudaError_t err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    const int grid = persistent_grid(fn, kThreads, smem, A.n_pages);
+    if (grid <= 0) return cudaErrorInvalidConfiguration;
+    decode_kernel<FMT><<<grid, kThreads, smem, stream>>>(F, A);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_decode(const stq_state *s, const float *q, const float *k, const float *v,
@@ -524,23 +711,19 @@ cudaError_t launch_decode(const stq_state *s, const float *q, const float *k, co
     A.n_pages = s->batch * s->heads;
     A.heads = s->heads;
     A.stage_bytes = (decode_stage_bytes(F) + 127) / 128 * 128;
-    A.n_stages = decode_stages(A.stage_bytes, F.stochastic ? decode_ctas_per_sm<true>() : decode_ctas_per_sm<false>());
+    A.store_bytes = (uint32_t)(F.col_scales ? F.c_off : F.page_bytes);
+    A.n_stages = 0;
     A.seed_lo = (uint32_t)seed;
     A.seed_hi = (uint32_t)(seed >> 32);
     A.step = step;
     A.wait_limit_ns = s->wait_limit_ns;
     A.stall_first_wait = stall_first_wait;
-    const size_t smem = kFixedBytes + (size_t)A.n_stages * A.stage_bytes;
-    const void *fn = F.stochastic ? (const void *)decode_kernel<true> : (const void *)decode_kernel<false>;
-    cudaError_t err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (err != cudaSuccess) return err;
-    const int grid = persistent_grid(fn, kThreads, smem, A.n_pages);
-    if (grid <= 0) return cudaErrorInvalidConfiguration;
-    if (F.stochastic)
-        decode_kernel<true><<<grid, kThreads, smem, stream>>>(F, A);
-    else
-        decode_kernel<false><<<grid, kThreads, smem, stream>>>(F, A);
-    return cudaGetLastError();
+    if (format_is<FmtStepQuant6>(F)) return launch_with<FmtStepQuant6>(F, A, stream);
+    if (format_is<FmtInt8Row>(F)) return launch_with<FmtInt8Row>(F, A, stream);
+    if (format_is<FmtStepQuant4Kda>(F)) return launch_with<FmtStepQuant4Kda>(F, A, stream);
+    if (format_is<FmtDamp>(F)) return launch_with<FmtDamp>(F, A, stream);
+    if (F.stochastic) return launch_with<RuntimeFmt<true>>(F, A, stream);
+    return launch_with<RuntimeFmt<false>>(F, A, stream);
 }
 
 }  // namespace stq

@@ -2,11 +2,12 @@
 // decode step for sm_100a: page format, plane unpack/pack, dequant/requant,
 // Philox-4x32-10, bulk-copy staging with bounded mbarrier waits.
 //
-// Thread mapping used by every page kernel: a CTA of 128 threads (4 warps)
-// owns one page at a time; warp w owns stored rows 32w .. 32w+31 (16-row
-// blocks 2w and 2w+1), lane l owns columns 4l .. 4l+3.  The packed layout
-// (see stq_format.cu) is built so that a lane reads and writes its columns
-// as whole 16-byte chunks and one mask + shift yields four columns of a row.
+// In every page kernel lane l of a warp owns value columns 4l .. 4l+3.  The
+// packed layout is built so that a lane reads and writes its columns as
+// whole 16-byte chunks (or aligned parts of one) and one mask + shift yields
+// the four columns of a row.  The quantize and dequantize kernels give warp w
+// the 16-row blocks 2w and 2w+1; the decode kernel gives warp w slice w
+// (rows 4w .. 4w+3) of every block.
 #pragma once
 
 #include <cstdint>
@@ -293,6 +294,45 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
 __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
     asm volatile("cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
                  :: "r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
+}
+
+// Shared -> global bulk copy, tracked as a bulk async-group of the issuing
+// thread; bytes and both addresses are multiples of 16.
+__device__ __forceinline__ void bulk_s2g(void *dst, const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+                 :: "l"(dst), "r"(smem_u32(src)), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() {
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// Wait until at most N of this thread's bulk groups still read shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" :: "n"(N) : "memory");
+}
+
+// Wait until at most N of this thread's bulk groups are incomplete.
+template <int N>
+__device__ __forceinline__ void bulk_wait() {
+    asm volatile("cp.async.bulk.wait_group %0;" :: "n"(N) : "memory");
+}
+
+// ------------------------------------------------------- small reductions --
+// max(|x|) over the 32 lanes of a full warp, in every lane (sm_100a).
+__device__ __forceinline__ float warp_absmax(float x) {
+    float r;
+    asm volatile("redux.sync.max.abs.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+// max of three floats (one instruction on sm_100a); the result for NaN
+// inputs is left unspecified.
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
 }
 
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {

@@ -45,7 +45,6 @@ def lib():
         _lib = ctypes.CDLL(path)
         L = _lib
         P = ctypes.c_void_p
-        L.orc_sum_block.restype = c_int
         L.orc_format_check.argtypes = [P]
         L.orc_row_qmax.argtypes = [P, c_int]
         L.orc_row_kind.argtypes = [P, c_int]
@@ -121,10 +120,6 @@ class Page:
         return _OrcPage(self.code.ctypes.data_as(POINTER(ctypes.c_int32)),
                         self.r.ctypes.data_as(POINTER(c_float)),
                         self.c.ctypes.data_as(POINTER(c_float)))
-
-
-def sum_block():
-    return lib().orc_sum_block()
 
 
 def row_qmax(fmt, s):

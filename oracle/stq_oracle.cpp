@@ -16,12 +16,14 @@
  *                   - the state is handled in column-normalised units
  *                     T = S / c (so the value-column scale c_j leaves the
  *                     inner loops);
- *                   - a column sum sum_s w_s T_sj runs over stored rows in
- *                     blocks of ORC_SUM_BLOCK = 16 consecutive rows (one
- *                     16-row block of the packed layout), each block a chain
- *                     p = fmaf(w_s, T_sj, p) from p = 0 in ascending s, and
- *                     the 8 block partials are added by a balanced pairwise
- *                     tree in block order, ((P0+P1)+(P2+P3))+((P4+P5)+(P6+P7));
+ *                   - a column sum sum_s w_s T_sj deals the stored rows
+ *                     of every 16-row block into four slices of 4
+ *                     consecutive rows (slice (s mod 16) / 4); the rows of
+ *                     one slice in one half of the page (s / 64) form a
+ *                     chain p = fmaf(w_s, T_sj, p) from p = 0 in ascending
+ *                     s; per slice the two half partials are added, and the
+ *                     four slice sums by a pairwise tree in slice order,
+ *                     (R0 + R1) + (R2 + R3);
  *                   - requantization rounds the exact product T' * inv once
  *                     (to an integer, ties to even);
  *                   - inv = qmax / m rounded toward zero, which keeps every
@@ -39,9 +41,10 @@
 #include <vector>
 #include <algorithm>
 
-static const int ORC_SUM_BLOCK = 16;
-
-extern "C" int orc_sum_block(void) { return ORC_SUM_BLOCK; }
+/* the canonical column-sum partition (see the header comment) */
+static const int ORC_BLOCK_ROWS = 16;   /* rows of a block */
+static const int ORC_SLICE_ROWS = 4;    /* consecutive rows of a block in one slice */
+static const int ORC_HALF_ROWS = 64;    /* rows whose slice rows form one chain */
 
 /* ------------------------------------------------------------------------ */
 /* format helpers                                                           */
@@ -440,23 +443,34 @@ static float tree_sum(const float *P, int n)
     return tree_sum(P, m) + tree_sum(P + m, n - m);
 }
 
-/* out_j = sum over stored rows s of w[perm[s]] * X[s][j], in the canonical
- * blocked order */
+/* out_j = sum over stored rows s of w[perm[s]] * X[s][j] in the canonical
+ * order: chain (slice, half) over the rows s with (s mod 16) / 4 == slice and
+ * s / 64 == half, ascending; per slice a tree over its non-empty half
+ * chains, then a tree over the non-empty slices in slice order. */
 static void column_sum(const orc_format *f, const int32_t *perm, const float *w_nat,
                        const float *X, float *out)
 {
     const int d_k = f->d_k, d_v = f->d_v;
-    const int nb = (d_k + ORC_SUM_BLOCK - 1) / ORC_SUM_BLOCK;
-    std::vector<float> P(nb);
+    const int n_slice = ORC_BLOCK_ROWS / ORC_SLICE_ROWS;
+    const int n_half = (d_k + ORC_HALF_ROWS - 1) / ORC_HALF_ROWS;
+    std::vector<float> P(n_half), R(n_slice);
     for (int j = 0; j < d_v; ++j) {
-        for (int blk = 0; blk < nb; ++blk) {
-            float acc = 0.0f;
-            int s_end = std::min(d_k, (blk + 1) * ORC_SUM_BLOCK);
-            for (int s = blk * ORC_SUM_BLOCK; s < s_end; ++s)
-                acc = std::fmaf(w_nat[perm[s]], X[(size_t)s * d_v + j], acc);
-            P[blk] = acc;
+        int nr = 0;
+        for (int w = 0; w < n_slice; ++w) {
+            int np = 0;
+            for (int h = 0; h < n_half; ++h) {
+                float acc = 0.0f;
+                bool any = false;
+                for (int s = h * ORC_HALF_ROWS; s < std::min(d_k, (h + 1) * ORC_HALF_ROWS); ++s) {
+                    if ((s % ORC_BLOCK_ROWS) / ORC_SLICE_ROWS != w) continue;
+                    acc = std::fmaf(w_nat[perm[s]], X[(size_t)s * d_v + j], acc);
+                    any = true;
+                }
+                if (any) P[np++] = acc;
+            }
+            if (np > 0) R[nr++] = tree_sum(P.data(), np);
         }
-        out[j] = tree_sum(P.data(), nb);
+        out[j] = tree_sum(R.data(), nr);
     }
 }
 

@@ -68,9 +68,6 @@ typedef struct {
     float *c;
 } orc_page;
 
-/* Sum-block size of the canonical fp32 column reductions (see stq_oracle.cpp). */
-int orc_sum_block(void);
-
 int orc_format_check(const orc_format *f);
 int orc_row_qmax(const orc_format *f, int s);     /* qmax of stored row s, 0 for float rows */
 int orc_row_kind(const orc_format *f, int s);

@@ -1,0 +1,105 @@
+"""GPU parity at the full workload sizes, in the launch configuration the
+benchmark times: one stq_decode_step over every page of the batch (256 to
+4,096 requests x 32 heads), checked on sampled pages the oracle steps one by
+one.
+
+The state is the GPU's own quantization of a device-generated fp32 state,
+except at the sampled positions, which hold oracle-made pages (from a small
+CPU-generated batch of the same workload) and get CPU-generated step inputs;
+the precision map is the oracle's calibration of that small batch.  So every
+oracle input and expected value comes from the generators and the oracle, and
+the kernel runs the full-size grid with its wrap-around and ragged tail.
+Samples: the first and last pages, both sides of the grid-wrap boundaries
+for 2 and 3 resident CTAs per SM, and seeded random positions.  Two chained
+steps (each side continues from its own result).  Bar: o, row scales and
+packed pages bit-identical, code mismatches only inside the rounding band.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from linear_attention_recurrent_delta_b200 import binding as B
+from linear_attention_recurrent_delta_b200 import workloads as W
+
+from parity_util import BAND, make_state
+
+pytestmark = pytest.mark.gpu
+
+SMALL_BATCH = 4   # CPU-generated requests the sampled pages are drawn from
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from linear_attention_recurrent_delta_b200 import build
+    build.build()
+    B.lib()
+    assert torch.cuda.is_available()
+
+
+def _sample_positions(n, seed):
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    pos = {0, 1, n - 2, n - 1}
+    for ctas in (2, 3):
+        g = sms * ctas
+        for m in (1, 2, n // g):
+            for d in (-1, 0):
+                if 0 <= m * g + d < n:
+                    pos.add(m * g + d)
+    rng = np.random.default_rng(seed)
+    pos.update(int(x) for x in rng.integers(0, n, 12))
+    return sorted(pos)
+
+
+@pytest.mark.parametrize("index", [1, 2, 3, 4])
+def test_full_size_step_on_sampled_pages(index):
+    w = W.WORKLOADS[index]
+    H, n = w.heads, w.pages
+    fmt = O.format_from_spec(w.format)
+
+    # oracle side: map and pages of a small CPU-generated batch
+    S_small = W.initial_state(w, batch=SMALL_BATCH).numpy()
+    perm = O.rank_rows(fmt, S_small)
+    pos = _sample_positions(n, w.seed)
+    src = [(i % SMALL_BATCH, p % H) for i, p in enumerate(pos)]   # (request, head) of S_small per sample
+    pages = [O.quantize_page(fmt, S_small[b, h], perm[h]) for b, h in src]
+
+    # full-size GPU state: device-generated, quantized on the GPU with the oracle's map
+    qs = make_state(w)
+    qs.perm().copy_(torch.from_numpy(np.ascontiguousarray(perm, np.uint8)))
+    S_dev = W.initial_state(w, device="cuda")
+    B.stq_quantize_state(qs.state, S_dev)
+    del S_dev
+    torch.cuda.synchronize()
+    dev_pages = qs.pages()
+    idx = torch.tensor(pos, dtype=torch.long, device="cuda")
+    dev_pages[idx] = torch.from_numpy(np.stack([O.pack_page(fmt, pg) for pg in pages])).cuda()
+
+    seed = W.sr_seed(w)
+    o = torch.empty(w.batch, H, 128, device="cuda")
+    for step in range(2):
+        xd = W.step_inputs(w, step, device="cuda")
+        xc = W.step_inputs(w, step, batch=SMALL_BATCH)
+        for k in xd:
+            flat = xd[k].view(n, -1)
+            flat[idx] = torch.stack([xc[k][b, h].reshape(-1) for b, h in src]).cuda()
+        qs.step(xd["q"], xd["k"], xd["v"], xd["alpha"], xd["beta"], o=o, seed=seed, step=step)
+        assert B.stq_device_status(qs.state) == B.STQ_OK
+        got_o = o.view(n, 128)[idx].cpu().numpy()
+        torch.cuda.synchronize()
+        got_pages = qs.pages()[idx].cpu().numpy()
+        band = 0
+        for i, (p, (b, h)) in enumerate(zip(pos, src)):
+            # the oracle steps its own page in place (each side continues from its own result)
+            o_ref, _, margin = O.step_f32(fmt, pages[i], perm[h], xc["q"][b, h].numpy(), xc["k"][b, h].numpy(),
+                                          xc["v"][b, h].numpy(), xc["alpha"][b, h].numpy(),
+                                          float(xc["beta"][b, h]), seed=seed, step=step, b=p // H, h=p % H,
+                                          want_margin=True)
+            assert np.array_equal(got_o[i], o_ref), "o of page %d (step %d)" % (p, step)
+            if not np.array_equal(got_pages[i], O.pack_page(fmt, pages[i])):
+                pg = O.unpack_page(fmt, got_pages[i])
+                assert np.array_equal(pg.r.view(np.uint32), pages[i].r.view(np.uint32)), "r of page %d" % p
+                bad = pg.code != pages[i].code
+                assert np.all(margin[bad] < BAND), "codes of page %d outside the rounding band" % p
+                band += int(bad.sum())
+        assert band == 0, "%d codes inside the rounding band differ (step %d)" % (band, step)
