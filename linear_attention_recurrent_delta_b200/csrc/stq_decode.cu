@@ -114,6 +114,21 @@ __device__ __forceinline__ float div_by_qmax(float m, float qmax, float rcp_qmax
     return __fmaf_rn(__fmaf_rn(-q0, qmax, m), rcp_qmax, q0);
 }
 
+// qmax / m rounded toward zero, for finite m > 0 and qmax = 2^(b-1) - 1:
+// a Markstein step on qmax * RN(1/m) gives q1 within half an ulp of the
+// quotient, and the exact residual qmax - q1 m says whether q1 lies above it
+// (then the next float below is the result).  Below 2^-100 (1/m near
+// overflow) the library division is used.  Equal to __fdiv_rz for every m
+// >= 2^-100 and every qmax of 2..8-bit codes (checked exhaustively on the GPU).
+__device__ __forceinline__ float div_rz_qmax(float qmax, float m) {
+    if (m < 0x1p-100f) return __fdiv_rz(qmax, m);
+    const float y = __frcp_rn(m);
+    const float q0 = __fmul_rn(qmax, y);
+    const float q1 = __fmaf_rn(__fmaf_rn(-q0, m, qmax), y, q0);
+    const float r1 = __fmaf_rn(-q1, m, qmax);
+    return r1 < 0.f ? __int_as_float(__float_as_int(q1) - 1) : q1;
+}
+
 // ---- S1 / S8 on one slice: rows 4w .. 4w+3 of a 16-row block.
 // Plane words of a slice (quad l): width 8: the whole chunk w; width 4: the
 // half chunk holding rows (0,1), (2,3); width 2: one word, row i at bits 2i
@@ -434,6 +449,11 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
         }
     }
     const bool my_int = my_bits != 16;
+    bool all_int = false;   // every row INT: the S6 test on my_int folds away
+    if constexpr (!FMT::kRuntime) {
+        all_int = true;
+        for (int b = 0; b < kBlocks; ++b) all_int = all_int && FMT::width(b) != 16;
+    }
     const int my_r = my_rbase + 4 * warp + (lane & 3);
     const float my_qmax = my_int ? (float)((1 << (my_bits - 1)) - 1) : 0.f;
     const float my_rcp = my_int ? __frcp_rn(my_qmax) : 0.f;
@@ -482,7 +502,7 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
         {
             const float kk = k_s[kap], qq = q_s[kap];
             const float al = gate_vector ? al_s[kap] : alpha_s;
-            const float a = my_int ? __fmul_rn(al, r_s[my_r]) : al;
+            const float a = (all_int || my_int) ? __fmul_rn(al, r_s[my_r]) : al;
             if (col_scales)   // thread t also inverts the scale of column t
                 S.ic[par][tid] = __frcp_rn(reinterpret_cast<const float *>(stg + F.c_off)[tid]);
             S.a[warp][lane] = a;
@@ -523,7 +543,7 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
             // a stage never arrived: record it, finish the previous page, let
             // the copies in flight land and leave; nothing of this page (or
             // a later one) is written
-            if (warp == 0 && p_prev >= 0)
+            if (warp == kWarps - 1 && p_prev >= 0)
                 write_o(S.red_o[par ^ 1], A, p_prev, lane, stages + st_prev * A.stage_bytes, F, col_scales);
             if (tid == 0) {
                 atomicOr(A.status, kStatusTimeout);
@@ -560,8 +580,9 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
                 }
             }
         }
-        // o of the previous page (its chain sums were stored before this barrier)
-        if (warp == 0 && p_prev >= 0)
+        // o of the previous page (its chain sums were stored before this
+        // barrier), by the last warp: warp 0's first thread handles the copies
+        if (warp == kWarps - 1 && p_prev >= 0)
             write_o(S.red_o[par ^ 1], A, p_prev, lane, stages + st_prev * A.stage_bytes, F, col_scales);
 
         // u = (W0 + W1) + (W2 + W3); e = v (1/c) - u
@@ -614,12 +635,10 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
         {
             const float m = S.inv[warp][lane];
             float inv = 0.f;
-            if (my_int) {
-                float r = 0.f;
-                if (m > 0.f) {
-                    r = div_by_qmax(m, my_qmax, my_rcp);
-                    inv = __fdiv_rz(my_qmax, m);
-                }
+            if (all_int || my_int) {
+                // m = 0 (a zero row): r' = 0 and inv = 0, codes 0
+                const float r = div_by_qmax(m, my_qmax, my_rcp);
+                inv = m > 0.f ? div_rz_qmax(my_qmax, m) : 0.f;
                 r_s[my_r] = r;
             }
             S.inv[warp][lane] = inv;
@@ -657,7 +676,7 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
             bulk_s2g(A.pages + (size_t)p_prev * F.page_bytes, stages + st_prev * A.stage_bytes, A.store_bytes);
             bulk_commit();
         }
-        if (warp == 0)
+        if (warp == kWarps - 1)
             write_o(S.red_o[(it - 1) & 1], A, p_prev, lane, stages + st_prev * A.stage_bytes, F, col_scales);
     }
     if (tid == 0) bulk_wait<0>();
