@@ -45,6 +45,7 @@
 static const int ORC_BLOCK_ROWS = 16;   /* rows of a block */
 static const int ORC_SLICE_ROWS = 4;    /* consecutive rows of a block in one slice */
 static const int ORC_HALF_ROWS = 64;    /* rows whose slice rows form one chain */
+static const int ORC_CALIB_CHUNK = 32;  /* requests per partial sum of a calibration score */
 
 /* ------------------------------------------------------------------------ */
 /* format helpers                                                           */
@@ -351,14 +352,21 @@ extern "C" int orc_rank_rows(const orc_format *f, int B, int H, const float *S,
     for (int h = 0; h < H; ++h) {
         /* score = row-mean-square summed over the batch, times the optional
          * retention weight; the constant 1 / (B d_v) is left out (it does
-         * not change the ranking) */
+         * not change the ranking).  The batch sum is taken in chunks of
+         * ORC_CALIB_CHUNK requests (each chunk from 0, requests ascending),
+         * and the chunk sums are added in chunk order: a fixed double
+         * evaluation order, so that equal inputs give one ranking. */
         for (int kap = 0; kap < d_k; ++kap) {
             double acc = 0.0;
-            for (int b = 0; b < B; ++b) {
-                const float *row = S + (((size_t)b * H + h) * d_k + kap) * d_v;
-                double rs = 0.0;
-                for (int j = 0; j < d_v; ++j) rs += (double)row[j] * (double)row[j];
-                acc += rs;
+            for (int b0 = 0; b0 < B; b0 += ORC_CALIB_CHUNK) {
+                double part = 0.0;
+                for (int b = b0; b < std::min(B, b0 + ORC_CALIB_CHUNK); ++b) {
+                    const float *row = S + (((size_t)b * H + h) * d_k + kap) * d_v;
+                    double rs = 0.0;
+                    for (int j = 0; j < d_v; ++j) rs += (double)row[j] * (double)row[j];
+                    part += rs;
+                }
+                acc += part;
             }
             if (row_weight) acc *= (double)row_weight[(size_t)h * d_k + kap];
             score[kap] = acc;

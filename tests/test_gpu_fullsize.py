@@ -103,3 +103,16 @@ def test_full_size_step_on_sampled_pages(index):
                 assert np.all(margin[bad] < BAND), "codes of page %d outside the rounding band" % p
                 band += int(bad.sum())
         assert band == 0, "%d codes inside the rounding band differ (step %d)" % (band, step)
+
+
+def test_full_size_calibration_map():
+    """The precision map of the full int8row batch (256 requests = 8 chunks of
+    the calibration sum) from the CUDA path equals the oracle's, bit for bit."""
+    w = W.WORKLOADS[1]
+    S = W.initial_state(w)
+    fmt = O.format_from_spec(w.format)
+    perm = O.rank_rows(fmt, S.numpy())
+    qs = make_state(w)
+    B.stq_calibrate(qs.state, S.cuda())
+    torch.cuda.synchronize()
+    assert np.array_equal(qs.perm().cpu().numpy(), perm)
