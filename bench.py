@@ -29,6 +29,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+from linear_attention_recurrent_delta_b200 import ranks as R  # noqa: E402
 from linear_attention_recurrent_delta_b200 import workloads as W  # noqa: E402
 
 METRIC = "decode state-update head-steps/s"
@@ -130,40 +131,27 @@ class ClockSampler:
 
 
 def dist_setup(n_gpus):
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = R.rank_env()
     if world > 1:
-        import datetime
-        import torch.distributed as dist
         torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        R.init("nccl", timeout_s=120, device_id=torch.device("cuda", local))
     elif torch.cuda.is_available():
         torch.cuda.set_device(0)
     return world, rank, local
 
 
 def barrier(world):
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
+    R.barrier(world)
 
 
 def max_over_ranks(x, world):
-    if world == 1:
-        return x
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    return R.max_over_ranks(x, world, device="cuda")
 
 
 def run_gpu(w, steps, warmup, rank, world, sample_clocks=True, e2e_steps=64):
     from linear_attention_recurrent_delta_b200 import binding as B
     dev = torch.device("cuda", torch.cuda.current_device())
-    wr = W.Workload(w.index, w.name, w.fmt, w.batch, w.heads, w.steps, w.gate_mu, w.gate_sigma,
-                    w.seed + 7919 * rank)
+    wr = R.rank_workload(w, rank)   # this rank's own requests: no exchange on the data path
     qs = B.QuantizedState(wr.format, wr.batch, wr.heads, device=dev)
     S = W.initial_state(wr, device=dev)
     qs.calibrate_and_quantize(S)
@@ -355,15 +343,15 @@ def main():
         res = run_gpu(w, args.steps, args.warmup, rank, world, sample_clocks=False, e2e_steps=0)
         if rank == 0:
             print(json.dumps({"workload": w.name, "batch": w.batch, "ms_per_step": res["ms"] / args.steps}))
+        R.finish(world)
         return
     res = run_gpu(w, args.steps, args.warmup, rank, world)
-    pages_total = w.pages * world
-    value = pages_total * args.steps / (res["ms"] / 1000.0)
+    value = R.aggregate_rate(w.pages, world, args.steps, res["ms"])
     per_launch_s = res["ms"] / 1000.0 / args.steps
     bpp = algorithmic_bytes_per_page(spec)
     achieved = bpp * w.pages / per_launch_s / 1e9
     peak, peak_kind = measured_peak()
-    e2e_value = pages_total * res["e2e_steps"] / (res["e2e_ms"] / 1000.0)
+    e2e_value = R.aggregate_rate(w.pages, world, res["e2e_steps"], res["e2e_ms"])
 
     others = {}
     if not args.only:
@@ -372,13 +360,14 @@ def main():
                 continue
             wi = W.WORKLOADS[i]
             r = run_gpu(wi, max(200, args.steps // 3), args.warmup, rank, world, sample_clocks=False, e2e_steps=8)
-            v = wi.pages * world * max(200, args.steps // 3) / (r["ms"] / 1000.0)
+            v = R.aggregate_rate(wi.pages, world, max(200, args.steps // 3), r["ms"])
             b = algorithmic_bytes_per_page(wi.format)
             gbs = b * wi.pages * max(200, args.steps // 3) / (r["ms"] / 1000.0) / 1e9
             others[wi.name] = {"value": v, "unit": UNIT, "hbm_gbs": gbs, "frac_of_%s_peak" % peak_kind: gbs / peak,
                                "bytes_per_head_step": b, "pages": wi.pages}
 
     if rank != 0:
+        R.finish(world)
         return
     cpu_v, cpu_sample, _ = oracle_rate(w, args.cpu_seconds) if world == 1 else (None, None, None)
     line = {
@@ -397,14 +386,12 @@ def main():
                          if cpu_v else None),
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"],
                 "steps": res["e2e_steps"], "entry_point": "stq_decode_step_host"},
-        "gpu_launches": args.steps,
+        "gpu_launches": args.steps * world,   # one decode_kernel launch per step and rank
         "clocks": res["clocks"],
         "other_workloads": others,
     }
     print(json.dumps(line))
-    if world > 1:
-        import torch.distributed as dist
-        dist.destroy_process_group()
+    R.finish(world)
 
 
 if __name__ == "__main__":
