@@ -258,13 +258,15 @@ __device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1
 }
 
 // Stochastic-rounding offsets of the two columns held by one 32-bit word:
-// delta = (h16 - 32767.5) / 65536, built exactly: the float 2^23 + 2 h16 + 1,
-// scaled by 2^-17, minus 64.5 (one exact fma).
+// delta = (h16 - 32767.5) / 65536 for the high and the low 16-bit half,
+// built exactly: a byte permute makes the float 2^23 + h16, one f32x2 fma
+// scales it by 2^-16 and removes 128 (exact: h16 / 65536), one f32x2 add
+// subtracts 32767.5 / 65536 (exact: a multiple of 2^-17 below 1/2).
 __device__ __forceinline__ float2 sr_delta_pair(uint32_t word) {
-    const float hi = __int_as_float(0x4B000000u | ((word >> 15) | 1u));
-    const float lo = __int_as_float(0x4B000000u | ((word << 1) & 0x1FFFEu) | 1u);
-    return __ffma2_rn(make_float2(hi, lo), make_float2(0x1p-17f, 0x1p-17f),
-                      make_float2(-64.5f, -64.5f));
+    const float hi = __int_as_float(__byte_perm(word, 0x4B000000u, 0x7632u));   // 2^23 + high half
+    const float lo = __int_as_float(__byte_perm(word, 0x4B000000u, 0x7610u));   // 2^23 + low half
+    const float2 d = __ffma2_rn(make_float2(hi, lo), make_float2(0x1p-16f, 0x1p-16f), make_float2(-128.f, -128.f));
+    return __fadd2_rn(d, make_float2(-32767.5f / 65536.f, -32767.5f / 65536.f));
 }
 
 // ------------------------------------------------------- bulk-copy staging --
