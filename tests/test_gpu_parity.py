@@ -212,3 +212,37 @@ def test_host_entry_point_matches_device_entry_point():
     torch.cuda.synchronize()
     assert torch.equal(o_host, o_dev.cpu())
     assert torch.equal(qa.pages(), qb.pages())
+
+
+DEGENERATE = {
+    "full_decay": lambda x: x["alpha"].zero_(),            # A S = 0: T' = beta k (v/c)^T, a rank-1 state
+    "decay_only": lambda x: x["beta"].zero_(),             # no delta write: S' = A S
+    "zero_key": lambda x: x["k"].zero_(),                  # u = 0 and beta k = 0: S' = A S
+    "zero_query": lambda x: x["q"].zero_(),                # o = 0 exactly (+0)
+    "zero_value": lambda x: x["v"].zero_(),                # e = -u: pure erasure along k
+    "no_decay_full_write": lambda x: (x["alpha"].fill_(1.0), x["beta"].fill_(1.0)),
+}
+
+
+@pytest.mark.parametrize("case", list(DEGENERATE))
+@pytest.mark.parametrize("name", ["stepquant6", "stepquant4_kda", "damp"])
+def test_degenerate_inputs_match_oracle(name, case):
+    """The method's degenerate inputs, GPU against oracle from the same packed
+    state: every page and o bit-identical."""
+    w = _small(name, batch=3, heads=5, steps=1)
+    S = W.initial_state(w).numpy()
+    fmt, perm, pages = oracle_quantize(w, S)
+    qs = make_state(w)
+    upload(qs, perm, pages)
+    x = W.step_inputs(w, 0)
+    DEGENERATE[case](x)
+    xd = {k: v.cuda() for k, v in x.items()}
+    seed = W.sr_seed(w)
+    o = qs.step(xd["q"], xd["k"], xd["v"], xd["alpha"], xd["beta"], seed=seed, step=0)
+    expect, o_ref = oracle_step(fmt, w, w.batch, w.heads, pages, perm, x, seed, 0)
+    got_o = o.cpu().numpy().reshape(w.pages, 128)
+    assert np.array_equal(got_o.view(np.uint32), o_ref.view(np.uint32)), case   # signs of zeros too
+    res = compare_pages(fmt, download(qs), expect)
+    assert res["pages_equal"] == res["pages"], (case, res)
+    if case == "zero_query":
+        assert not np.any(got_o.view(np.uint32))
