@@ -54,12 +54,21 @@ struct StaticFmt {
         for (int i = 0; i < b; ++i) r += width(i) == 16 ? 0 : 16;
         return r;
     }
+    // Readout chains placed beside S6's division (independent work for its
+    // latency): faster where registers allow it (every block INT8, round to
+    // nearest); with sub-byte or FP16 blocks it spills and is slower.
+    __host__ __device__ static constexpr bool o_late() {
+        bool all8 = !SR;
+        for (int i = 0; i < 8; ++i) all8 = all8 && width(i) == 8;
+        return all8;
+    }
 };
 
 template <bool SR>
 struct RuntimeFmt {
     static constexpr bool kRuntime = true;
     static constexpr bool kSr = SR;
+    __host__ __device__ static constexpr bool o_late() { return false; }
 };
 
 using FmtStepQuant6 = StaticFmt<8, 8, 6, 6, 6, 6, 4, 4, true, false, false>;
@@ -352,6 +361,24 @@ __device__ __forceinline__ void requant_slice(uint8_t *blk, int w, int lane, con
     }
 }
 
+// S5's chains over block B of the slice (q of the slice's rows in qp)
+template <int B>
+__device__ __forceinline__ void readout_block(const float *qp, const Tile &T, float2 (&co)[2]) {
+    const float4 q4 = *reinterpret_cast<const float4 *>(&qp[4 * B]);
+    const float qv[4] = {q4.x, q4.y, q4.z, q4.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        co[0] = __ffma2_rn(make_float2(qv[i], qv[i]), T[B][i][0], co[0]);
+        co[1] = __ffma2_rn(make_float2(qv[i], qv[i]), T[B][i][1], co[1]);
+    }
+}
+
+// the warp's readout partial: chain over blocks 0-3 plus chain over 4-7
+__device__ __forceinline__ void store_readout(float *red, int lane, const float2 (&co)[2][2]) {
+    const float2 w01 = __fadd2_rn(co[0][0], co[1][0]), w23 = __fadd2_rn(co[0][1], co[1][1]);
+    *reinterpret_cast<float4 *>(&red[4 * lane]) = make_float4(w01.x, w01.y, w23.x, w23.y);
+}
+
 // max |x| over a row's four columns held by one lane
 __device__ __forceinline__ float absmax4(float2 a, float2 b) {
     return fmaxf(max3f(fabsf(a.x), fabsf(a.y), fabsf(b.x)), fabsf(b.y));
@@ -611,24 +638,17 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
         for (int h = 0; h < 2; ++h) co[h][0] = co[h][1] = make_float2(0.f, 0.f);
         static_for<0, kBlocks>([&](auto bc) {
             constexpr int b = decltype(bc)::value;
-            constexpr int h = b >> 2;
             const float4 b4 = *reinterpret_cast<const float4 *>(&S.bk[warp][4 * b]);
-            const float4 q4 = *reinterpret_cast<const float4 *>(&S.qp[warp][4 * b]);
             const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
-            const float qv[4] = {q4.x, q4.y, q4.z, q4.w};
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 T[b][i][0] = __ffma2_rn(make_float2(bv[i], bv[i]), e01, T[b][i][0]);
                 T[b][i][1] = __ffma2_rn(make_float2(bv[i], bv[i]), e23, T[b][i][1]);
                 S.inv[warp][4 * b + i] = warp_absmax(absmax4(T[b][i][0], T[b][i][1]));
-                co[h][0] = __ffma2_rn(make_float2(qv[i], qv[i]), T[b][i][0], co[h][0]);
-                co[h][1] = __ffma2_rn(make_float2(qv[i], qv[i]), T[b][i][1], co[h][1]);
             }
+            if constexpr (!FMT::o_late()) readout_block<b>(S.qp[warp], T, co[b >> 2]);
         });
-        {
-            const float2 w01 = __fadd2_rn(co[0][0], co[1][0]), w23 = __fadd2_rn(co[0][1], co[1][1]);
-            *reinterpret_cast<float4 *>(&S.red_o[par][warp][4 * lane]) = make_float4(w01.x, w01.y, w23.x, w23.y);
-        }
+        if constexpr (!FMT::o_late()) store_readout(S.red_o[par][warp], lane, co);
         __syncwarp();
 
         // S6: lane l finishes row l of the slice: r' = m / qmax, inv = qmax / m (toward zero)
@@ -640,6 +660,13 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
                 const float r = div_by_qmax(m, my_qmax, my_rcp);
                 inv = m > 0.f ? div_rz_qmax(my_qmax, m) : 0.f;
                 r_s[my_r] = r;
+            }
+            if constexpr (FMT::o_late()) {
+                static_for<0, kBlocks>([&](auto bc) {
+                    constexpr int b = decltype(bc)::value;
+                    readout_block<b>(S.qp[warp], T, co[b >> 2]);
+                });
+                store_readout(S.red_o[par][warp], lane, co);
             }
             S.inv[warp][lane] = inv;
         }

@@ -246,3 +246,38 @@ def test_degenerate_inputs_match_oracle(name, case):
     assert res["pages_equal"] == res["pages"], (case, res)
     if case == "zero_query":
         assert not np.any(got_o.view(np.uint32))
+
+
+CUSTOM_FORMATS = {
+    # widths 7 and 5 (4+2+1 and 4+1 planes), column scales, GDN: the run-time-width kernel
+    "custom_int7_int5": {"groups": [(48, "int", 7), (80, "int", 5)],
+                         "col_scales": True, "stochastic": False, "gate_vector": False},
+    # FP16 rows in the middle of the page, widths 3 and 2, KDA gate, stochastic rounding
+    "custom_fp16_int3_int2_sr": {"groups": [(16, "int", 8), (32, "fp16", 0), (48, "int", 3), (32, "int", 2)],
+                                 "col_scales": True, "stochastic": True, "gate_vector": True},
+}
+
+
+@pytest.mark.parametrize("fmt_name", list(CUSTOM_FORMATS))
+def test_custom_formats_match_oracle(fmt_name, monkeypatch):
+    """Formats outside the four compiled-in ones run the kernel whose block
+    widths are read at run time; same bar as the named formats."""
+    monkeypatch.setitem(W.FORMATS, fmt_name, CUSTOM_FORMATS[fmt_name])
+    base = W.WORKLOADS[3] if CUSTOM_FORMATS[fmt_name]["gate_vector"] else W.WORKLOADS[2]
+    w = W.Workload(base.index, fmt_name, fmt_name, 7, 11, 2, base.gate_mu, base.gate_sigma, base.seed + 99)
+    S = W.initial_state(w)
+    fmt, perm, pages = oracle_quantize(w, S.numpy())
+    qs = make_state(w)
+    qs.calibrate_and_quantize(S.cuda())
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(qs.perm().cpu().numpy(), perm)
+    assert np.array_equal(download(qs), pages)
+    seed = W.sr_seed(w)
+    for step in range(w.steps):
+        x, xd = step_inputs_gpu(w, step)
+        o = qs.step(xd["q"], xd["k"], xd["v"], xd["alpha"], xd["beta"], seed=seed, step=step)
+        expect, o_ref = oracle_step(fmt, w, w.batch, w.heads, pages, perm, x, seed, step)
+        assert np.array_equal(o.cpu().numpy().reshape(w.pages, 128), o_ref), step
+        res = compare_pages(fmt, download(qs), expect, perm, (pages, x, seed, step, w.heads))
+        assert res["pages_equal"] == res["pages"], (step, res)
+        pages = expect
