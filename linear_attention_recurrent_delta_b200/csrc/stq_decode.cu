@@ -36,10 +36,18 @@ namespace stq {
 
 // ---- formats: widths per 16-row block (16 = FP16) known at compile time,
 // or read from DevFormat at run time (any other valid format)
-template <int W0, int W1, int W2, int W3, int W4, int W5, int W6, int W7, bool COLS, bool GVEC, bool SR>
+// Per-format code-placement choices (measured per format on a B200; each
+// changes only where independent work sits, never the arithmetic):
+//   kOLate   all readout chains beside S6's division (gives its latency work)
+//   kOSplit  the second readout chain (blocks 4-7) beside S6
+//   kFastRcp S6's division starts from the approximate hardware reciprocal
+enum Tune : int { kTuneNone = 0, kOLate = 1, kOSplit = 2, kFastRcp = 4 };
+
+template <int W0, int W1, int W2, int W3, int W4, int W5, int W6, int W7, bool COLS, bool GVEC, bool SR, int TUNE>
 struct StaticFmt {
     static constexpr bool kRuntime = false;
     static constexpr bool kCols = COLS, kGvec = GVEC, kSr = SR;
+    static constexpr int kTune = TUNE;
     __host__ __device__ static constexpr int width(int b) {
         return b == 0 ? W0 : b == 1 ? W1 : b == 2 ? W2 : b == 3 ? W3 : b == 4 ? W4 : b == 5 ? W5 : b == 6 ? W6 : W7;
     }
@@ -54,27 +62,21 @@ struct StaticFmt {
         for (int i = 0; i < b; ++i) r += width(i) == 16 ? 0 : 16;
         return r;
     }
-    // Readout chains placed beside S6's division (independent work for its
-    // latency): faster where registers allow it (every block INT8, round to
-    // nearest); with sub-byte or FP16 blocks it spills and is slower.
-    __host__ __device__ static constexpr bool o_late() {
-        bool all8 = !SR;
-        for (int i = 0; i < 8; ++i) all8 = all8 && width(i) == 8;
-        return all8;
-    }
 };
 
 template <bool SR>
 struct RuntimeFmt {
     static constexpr bool kRuntime = true;
     static constexpr bool kSr = SR;
-    __host__ __device__ static constexpr bool o_late() { return false; }
+    static constexpr int kTune = kTuneNone;
 };
 
-using FmtStepQuant6 = StaticFmt<8, 8, 6, 6, 6, 6, 4, 4, true, false, false>;
-using FmtInt8Row = StaticFmt<8, 8, 8, 8, 8, 8, 8, 8, false, false, false>;
-using FmtStepQuant4Kda = StaticFmt<8, 4, 4, 4, 3, 3, 3, 3, true, true, false>;
-using FmtDamp = StaticFmt<16, 8, 8, 8, 8, 8, 8, 8, false, false, true>;
+// (the stepquant6 instantiation sits at the register limit: either move
+// made it spill and run 6 % slower)
+using FmtStepQuant6 = StaticFmt<8, 8, 6, 6, 6, 6, 4, 4, true, false, false, kTuneNone>;
+using FmtInt8Row = StaticFmt<8, 8, 8, 8, 8, 8, 8, 8, false, false, false, kOLate | kFastRcp>;
+using FmtStepQuant4Kda = StaticFmt<8, 4, 4, 4, 3, 3, 3, 3, true, true, false, kOSplit>;
+using FmtDamp = StaticFmt<16, 8, 8, 8, 8, 8, 8, 8, false, false, true, kFastRcp>;
 
 struct DecodeArgs {
     uint8_t *pages;
@@ -124,14 +126,20 @@ __device__ __forceinline__ float div_by_qmax(float m, float qmax, float rcp_qmax
 }
 
 // qmax / m rounded toward zero, for finite m > 0 and qmax = 2^(b-1) - 1:
-// a Markstein step on qmax * RN(1/m) gives q1 within half an ulp of the
-// quotient, and the exact residual qmax - q1 m says whether q1 lies above it
-// (then the next float below is the result).  Below 2^-100 (1/m near
-// overflow) the library division is used.  Equal to __fdiv_rz for every m
-// >= 2^-100 and every qmax of 2..8-bit codes (checked exhaustively on the GPU).
+// a Markstein step on qmax * y, y a reciprocal of m, gives q1 within half an
+// ulp of the quotient, and the exact residual qmax - q1 m says whether q1
+// lies above it (then the next float below is the result).  y is RN(1/m),
+// or with FAST the hardware approximation (within an ulp: the step still
+// lands within half an ulp).  Outside [2^-100, 2^126] (1/m near overflow, or
+// an approximate 1/m flushed to zero) the library division is used.  Equal
+// to __fdiv_rz for every m >= 2^-100 and every qmax of 2..8-bit codes, both
+// ways (checked exhaustively on the GPU).
+template <bool FAST>
 __device__ __forceinline__ float div_rz_qmax(float qmax, float m) {
-    if (m < 0x1p-100f) return __fdiv_rz(qmax, m);
-    const float y = __frcp_rn(m);
+    if (m < 0x1p-100f || (FAST && m > 0x1p126f)) return __fdiv_rz(qmax, m);
+    float y;
+    if constexpr (FAST) asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(m));
+    else y = __frcp_rn(m);
     const float q0 = __fmul_rn(qmax, y);
     const float q1 = __fmaf_rn(__fmaf_rn(-q0, m, qmax), y, q0);
     const float r1 = __fmaf_rn(-q1, m, qmax);
@@ -646,9 +654,10 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
                 T[b][i][1] = __ffma2_rn(make_float2(bv[i], bv[i]), e23, T[b][i][1]);
                 S.inv[warp][4 * b + i] = warp_absmax(absmax4(T[b][i][0], T[b][i][1]));
             }
-            if constexpr (!FMT::o_late()) readout_block<b>(S.qp[warp], T, co[b >> 2]);
+            if constexpr (!(FMT::kTune & kOLate) && !((FMT::kTune & kOSplit) && b >= 4))
+                readout_block<b>(S.qp[warp], T, co[b >> 2]);
         });
-        if constexpr (!FMT::o_late()) store_readout(S.red_o[par][warp], lane, co);
+        if constexpr (!(FMT::kTune & (kOLate | kOSplit))) store_readout(S.red_o[par][warp], lane, co);
         __syncwarp();
 
         // S6: lane l finishes row l of the slice: r' = m / qmax, inv = qmax / m (toward zero)
@@ -658,11 +667,11 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
             if (all_int || my_int) {
                 // m = 0 (a zero row): r' = 0 and inv = 0, codes 0
                 const float r = div_by_qmax(m, my_qmax, my_rcp);
-                inv = m > 0.f ? div_rz_qmax(my_qmax, m) : 0.f;
+                inv = m > 0.f ? div_rz_qmax<(FMT::kTune & kFastRcp) != 0>(my_qmax, m) : 0.f;
                 r_s[my_r] = r;
             }
-            if constexpr (FMT::o_late()) {
-                static_for<0, kBlocks>([&](auto bc) {
+            if constexpr ((FMT::kTune & (kOLate | kOSplit)) != 0) {
+                static_for<((FMT::kTune & kOLate) ? 0 : 4), kBlocks>([&](auto bc) {
                     constexpr int b = decltype(bc)::value;
                     readout_block<b>(S.qp[warp], T, co[b >> 2]);
                 });

@@ -1,7 +1,8 @@
 // stq_quant.cu -- cold-path kernels: precision map (calibration), quantize,
-// dequantize.  Same thread mapping as the decode kernel (warp w: stored rows
-// 32w .. 32w+31, lane l: columns 4l .. 4l+3) and the same plane packers, so a
-// page written here is read back bit for bit by the decode step.
+// dequantize.  One CTA of 128 threads per page: warp w owns the 16-row blocks
+// 2w and 2w+1, lane l columns 4l .. 4l+3, and the whole-block plane packers of
+// stq_device.cuh write the same byte layout the decode kernel reads and writes
+// slice by slice.
 #include "stq_internal.h"
 
 #include <map>
