@@ -41,7 +41,10 @@ namespace stq {
 //   kOLate   all readout chains beside S6's division (gives its latency work)
 //   kOSplit  the second readout chain (blocks 4-7) beside S6
 //   kFastRcp S6's division starts from the approximate hardware reciprocal
-enum Tune : int { kTuneNone = 0, kOLate = 1, kOSplit = 2, kFastRcp = 4 };
+//   kEarlyRefill a stage is refilled during the page after its own, after
+//            the update (its bulk store has read it by then); otherwise at
+//            the barrier of the page after that (one page less of look-ahead)
+enum Tune : int { kTuneNone = 0, kOLate = 1, kOSplit = 2, kFastRcp = 4, kEarlyRefill = 8 };
 
 template <int W0, int W1, int W2, int W3, int W4, int W5, int W6, int W7, bool COLS, bool GVEC, bool SR, int TUNE>
 struct StaticFmt {
@@ -71,12 +74,12 @@ struct RuntimeFmt {
     static constexpr int kTune = kTuneNone;
 };
 
-// (the stepquant6 instantiation sits at the register limit: either move
-// made it spill and run 6 % slower)
+// (the stepquant6 instantiation sits at the register limit: each move made
+// it spill and run 3-6 % slower; kda likewise with kFastRcp or kEarlyRefill)
 using FmtStepQuant6 = StaticFmt<8, 8, 6, 6, 6, 6, 4, 4, true, false, false, kTuneNone>;
-using FmtInt8Row = StaticFmt<8, 8, 8, 8, 8, 8, 8, 8, false, false, false, kOLate | kFastRcp>;
+using FmtInt8Row = StaticFmt<8, 8, 8, 8, 8, 8, 8, 8, false, false, false, kOLate | kFastRcp | kEarlyRefill>;
 using FmtStepQuant4Kda = StaticFmt<8, 4, 4, 4, 3, 3, 3, 3, true, true, false, kOSplit>;
-using FmtDamp = StaticFmt<16, 8, 8, 8, 8, 8, 8, 8, false, false, true, kFastRcp>;
+using FmtDamp = StaticFmt<16, 8, 8, 8, 8, 8, 8, 8, false, false, true, kFastRcp | kEarlyRefill>;
 
 struct DecodeArgs {
     uint8_t *pages;
@@ -106,6 +109,7 @@ struct SmemFixed {
     float red_u[2][kWarps][kD];             // per page parity and warp: chain sums of u
     float red_o[2][kWarps][kD];             // the same for o
     float ic[2][kD];                        // per page parity: 1 / c per column
+    float cpg[2][kD];                       // per page parity: c (o of a page is finished a page later)
     uint64_t full[kMaxStages];              // stage-full barriers
     uint64_t never;                         // a barrier nothing completes (test hook)
 };
@@ -403,10 +407,9 @@ __device__ __forceinline__ void issue_stage(const DevFormat &F, const DecodeArgs
     if (F.gate_vector) bulk_g2s(rows + 1536, A.alpha + (size_t)p * kD, 512, bar);
 }
 
-// o of a finished page: the tree over the warps' chain sums, times c (read
-// from the page's stage, which is not refilled before the next barrier).
+// o of a finished page: the tree over the warps' chain sums, times c.
 __device__ __forceinline__ void write_o(const float (*red_o)[kD], const DecodeArgs &A, int p, int lane,
-                                        const uint8_t *stage, const DevFormat &F, bool col_scales) {
+                                        const float *cpg, bool col_scales) {
     const float4 o0 = *reinterpret_cast<const float4 *>(&red_o[0][4 * lane]);
     const float4 o1 = *reinterpret_cast<const float4 *>(&red_o[1][4 * lane]);
     const float4 o2 = *reinterpret_cast<const float4 *>(&red_o[2][4 * lane]);
@@ -416,7 +419,7 @@ __device__ __forceinline__ void write_o(const float (*red_o)[kD], const DecodeAr
     float2 ob = __fadd2_rn(__fadd2_rn(make_float2(o0.z, o0.w), make_float2(o1.z, o1.w)),
                            __fadd2_rn(make_float2(o2.z, o2.w), make_float2(o3.z, o3.w)));
     if (col_scales) {
-        const float4 c = *reinterpret_cast<const float4 *>(stage + F.c_off + 16 * lane);
+        const float4 c = *reinterpret_cast<const float4 *>(cpg + 4 * lane);
         oa = __fmul2_rn(make_float2(c.x, c.y), oa);
         ob = __fmul2_rn(make_float2(c.z, c.w), ob);
     }
@@ -538,8 +541,11 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
             const float kk = k_s[kap], qq = q_s[kap];
             const float al = gate_vector ? al_s[kap] : alpha_s;
             const float a = (all_int || my_int) ? __fmul_rn(al, r_s[my_r]) : al;
-            if (col_scales)   // thread t also inverts the scale of column t
-                S.ic[par][tid] = __frcp_rn(reinterpret_cast<const float *>(stg + F.c_off)[tid]);
+            if (col_scales) {   // thread t also keeps and inverts the scale of column t
+                const float c = reinterpret_cast<const float *>(stg + F.c_off)[tid];
+                S.cpg[par][tid] = c;
+                S.ic[par][tid] = __frcp_rn(c);
+            }
             S.a[warp][lane] = a;
             S.kp[warp][lane] = kk;
             S.qp[warp][lane] = qq;
@@ -579,7 +585,7 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
             // the copies in flight land and leave; nothing of this page (or
             // a later one) is written
             if (warp == kWarps - 1 && p_prev >= 0)
-                write_o(S.red_o[par ^ 1], A, p_prev, lane, stages + st_prev * A.stage_bytes, F, col_scales);
+                write_o(S.red_o[par ^ 1], A, p_prev, lane, S.cpg[par ^ 1], col_scales);
             if (tid == 0) {
                 atomicOr(A.status, kStatusTimeout);
                 if (p_prev >= 0) {
@@ -587,7 +593,8 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
                              A.store_bytes);
                     bulk_commit();
                 }
-                const int last = (it < 2 ? NS - 1 : it - 3 + NS);   // last ring slot whose load was issued
+                // last ring slot whose load was issued
+                const int last = it < 2 ? NS - 1 : ((FMT::kTune & kEarlyRefill) ? it - 2 + NS : it - 3 + NS);
                 for (int j = it; j <= last; ++j) {
                     if ((int)blockIdx.x + j * stride < n)
                         mbar_wait_bounded(&S.full[j % NS], (uint32_t)((j / NS) & 1), A.wait_limit_ns);
@@ -598,14 +605,16 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
             return;
         }
 
+        constexpr bool kEarly = (FMT::kTune & kEarlyRefill) != 0;
         if (tid == 0) {
-            // the previous page is complete in its stage: store it; then the
-            // stage stored one page earlier is free once its store has read it
+            // the previous page is complete in its stage: store it; its stage
+            // is refilled once the store has read it (see kEarlyRefill)
             if (p_prev >= 0) {
-                bulk_s2g(A.pages + (size_t)p_prev * F.page_bytes, stages + st_prev * A.stage_bytes, A.store_bytes);
+                bulk_s2g(A.pages + (size_t)p_prev * F.page_bytes, stages + st_prev * A.stage_bytes,
+                         A.store_bytes);
                 bulk_commit();
             }
-            if (it >= 2) {
+            if (!kEarly && it >= 2) {
                 bulk_wait_read<1>();
                 const int j = it - 2 + NS;
                 const int pr = (int)blockIdx.x + j * stride;
@@ -618,7 +627,7 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
         // o of the previous page (its chain sums were stored before this
         // barrier), by the last warp: warp 0's first thread handles the copies
         if (warp == kWarps - 1 && p_prev >= 0)
-            write_o(S.red_o[par ^ 1], A, p_prev, lane, stages + st_prev * A.stage_bytes, F, col_scales);
+            write_o(S.red_o[par ^ 1], A, p_prev, lane, S.cpg[par ^ 1], col_scales);
 
         // u = (W0 + W1) + (W2 + W3); e = v (1/c) - u
         float2 e01, e23;
@@ -658,6 +667,16 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
                 readout_block<b>(S.qp[warp], T, co[b >> 2]);
         });
         if constexpr (!(FMT::kTune & (kOLate | kOSplit))) store_readout(S.red_o[par][warp], lane, co);
+        if (kEarly && tid == 0 && p_prev >= 0) {
+            // refill the previous page's stage with the page NS - 1 ahead of this one
+            bulk_wait_read<0>();
+            const int j = it - 1 + NS;
+            const int pr = (int)blockIdx.x + j * stride;
+            if (pr < n) {
+                fence_proxy_async_smem();
+                issue_stage(F, A, stages + (j % NS) * A.stage_bytes, pr, &S.full[j % NS]);
+            }
+        }
         __syncwarp();
 
         // S6: lane l finishes row l of the slice: r' = m / qmax, inv = qmax / m (toward zero)
@@ -713,7 +732,7 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
             bulk_commit();
         }
         if (warp == kWarps - 1)
-            write_o(S.red_o[(it - 1) & 1], A, p_prev, lane, stages + st_prev * A.stage_bytes, F, col_scales);
+            write_o(S.red_o[(it - 1) & 1], A, p_prev, lane, S.cpg[(it - 1) & 1], col_scales);
     }
     if (tid == 0) bulk_wait<0>();
 }
@@ -728,7 +747,8 @@ static bool format_is(const DevFormat &F) {
 
 static int decode_stages(size_t stride, int ctas_per_sm) {
     // as many ring stages as fit next to the fixed part at the target
-    // occupancy, at least 3 (a stage is refilled two pages after its use)
+    // occupancy, at least 3 (a stage is written back during the page after
+    // its own and refilled then or one page later)
     int dev = 0, smem_sm = 0, reserved = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
