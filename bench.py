@@ -282,6 +282,54 @@ def oracle_rate(w, budget_s, n_pages=64):
     return done / el, "%s x %d steps" % (smp.desc, steps), el
 
 
+def _oracle_worker(args):
+    """One host process of the all-cores baseline: its own 64-page sample of the
+    workload (pages differ per process through the batch offset), stepped for
+    about budget_s seconds.  Returns (pages stepped, seconds)."""
+    index, batch, proc, budget_s = args
+    w = W.WORKLOADS[index]
+    if batch:
+        w = w.resized(batch=batch)
+    w = R.rank_workload(w, 1000 + proc)          # a distinct sample per process
+    smp = OracleSample(w, 64)
+    smp.step()
+    done = 0
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < budget_s:
+        done += smp.step()
+    return done, time.perf_counter() - t0
+
+
+def oracle_rate_all_cores(w, budget_s):
+    """The same oracle on the host cores: one spawned process per core this
+    process may use (at most 32: each process imports torch), each stepping
+    its own sample; head-steps/s = all pages / the slowest process."""
+    import multiprocessing as mp
+    n = max(1, min(32, len(os.sched_getaffinity(0))))
+    ctx = mp.get_context("spawn")   # never fork after the GPU is in use
+    jobs = [(w.index, w.batch if w.batch != W.WORKLOADS[w.index].batch else 0, i, budget_s) for i in range(n)]
+    with ctx.Pool(n) as pool:
+        try:   # bounded: a worker that dies must not hold the bench
+            res = pool.map_async(_oracle_worker, jobs).get(timeout=4 * budget_s + 180)
+        except Exception:
+            pool.terminate()
+            return None, n
+    done = sum(r[0] for r in res)
+    el = max(r[1] for r in res)
+    return done / el, n
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as fh:
+            for line in fh:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -290,6 +338,8 @@ def main():
     ap.add_argument("--config", type=int, default=1)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--cpu-all-seconds", type=float, default=8.0,
+                    help="the oracle on every host core (0: skip)")
     ap.add_argument("--ref-seconds", type=float, default=60.0)
     ap.add_argument("--only", action="store_true", help="skip the other workloads")
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling)")
@@ -372,6 +422,13 @@ def main():
         R.finish(world)
         return
     cpu_v, cpu_sample, _ = oracle_rate(w, args.cpu_seconds) if world == 1 else (None, None, None)
+    cpu_all = None
+    if world == 1 and args.cpu_all_seconds > 0:
+        v_all, n_all = oracle_rate_all_cores(w, args.cpu_all_seconds)
+        if v_all:
+            cpu_all = {"value": v_all, "unit": UNIT, "cores": n_all, "cpu": cpu_model(),
+                       "gbs": v_all * bpp / 1e9, "sample": "64 pages per process (own requests), %.0f s" %
+                       args.cpu_all_seconds}
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": res["ms"] / args.steps, "higher_is_better": True,
@@ -384,7 +441,8 @@ def main():
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": ncu_traffic(w.name),
                      "peak_kind": peak_kind, "bytes_per_head_step": bpp, "kernel": "stq::decode_kernel"},
-        "cpu_baseline": ({"value": cpu_v, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": cpu_sample}
+        "cpu_baseline": ({"value": cpu_v, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": cpu_sample,
+                          "gbs": cpu_v * bpp / 1e9, "cpu": cpu_model(), "all_cores": cpu_all}
                          if cpu_v else None),
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"],
                 "steps": res["e2e_steps"], "entry_point": "stq_decode_step_host"},
