@@ -163,7 +163,11 @@ stq_status stq_quantize_state(stq_state *s, const float *d_S, void *stream);
  * (4-byte aligned) or [B][H][128] (16-byte aligned, gate_vector).  d_beta:
  * [B][H].  None may overlap the state buffer, and d_o may overlap no input.
  * seed and step feed the stochastic-rounding generator only (Philox-4x32-10,
- * key = seed, counter = (tile, step, request, head)).  q is used as given. */
+ * key = seed, counter = (tile, step, request, head)).  q is used as given.
+ * The kernel is launched as a programmatic dependent launch: it may become
+ * resident while the previous kernel on `stream` finishes, and reads nothing
+ * from global memory until that kernel has completed and its writes are
+ * visible, so stream order holds as for a plain launch. */
 stq_status stq_decode_step(stq_state *s, const float *d_q, const float *d_k, const float *d_v,
                            const float *d_alpha, const float *d_beta, float *d_o,
                            uint64_t seed, uint32_t step, void *stream);

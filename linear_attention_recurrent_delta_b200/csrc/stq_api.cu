@@ -210,16 +210,26 @@ static stq_status check_step_args(const stq_state *s, const float *q, const floa
     return STQ_OK;
 }
 
-stq_status stq_decode_step(stq_state *s, const float *d_q, const float *d_k, const float *d_v,
-                           const float *d_alpha, const float *d_beta, float *d_o, uint64_t seed, uint32_t step,
-                           void *stream) {
+// The step behind both entry points.  early_launch: the launch may start while
+// a preceding kernel on the stream finishes (the kernel waits for it before
+// its first global read); the host entry point, whose step follows copies,
+// launches plainly.
+static stq_status decode_step(stq_state *s, const float *d_q, const float *d_k, const float *d_v,
+                              const float *d_alpha, const float *d_beta, float *d_o, uint64_t seed,
+                              uint32_t step, void *stream, bool early_launch) {
     stq_status st = check_step_args(s, d_q, d_k, d_v, d_alpha, d_beta, d_o);
     if (st != STQ_OK) return st;
     const int stall = s->stall_first_wait;
     s->stall_first_wait = 0;
-    cudaError_t err = launch_decode(s, d_q, d_k, d_v, d_alpha, d_beta, d_o, seed, step, stall,
+    cudaError_t err = launch_decode(s, d_q, d_k, d_v, d_alpha, d_beta, d_o, seed, step, stall, early_launch,
                                     static_cast<cudaStream_t>(stream));
     return err == cudaSuccess ? STQ_OK : STQ_ERR_CUDA;
+}
+
+stq_status stq_decode_step(stq_state *s, const float *d_q, const float *d_k, const float *d_v,
+                           const float *d_alpha, const float *d_beta, float *d_o, uint64_t seed, uint32_t step,
+                           void *stream) {
+    return decode_step(s, d_q, d_k, d_v, d_alpha, d_beta, d_o, seed, step, stream, true);
 }
 
 struct IoLayout {
@@ -259,10 +269,10 @@ stq_status stq_decode_step_host(stq_state *s, const float *h_q, const float *h_k
     for (int i = 0; i < 5; ++i)
         if (cudaMemcpyAsync(io + in[i].off, in[i].src, in[i].n, cudaMemcpyHostToDevice, cs) != cudaSuccess)
             return STQ_ERR_CUDA;
-    stq_status st = stq_decode_step(s, reinterpret_cast<float *>(io + L.q), reinterpret_cast<float *>(io + L.k),
-                                    reinterpret_cast<float *>(io + L.v), reinterpret_cast<float *>(io + L.alpha),
-                                    reinterpret_cast<float *>(io + L.beta), reinterpret_cast<float *>(io + L.o),
-                                    seed, step, stream);
+    stq_status st = decode_step(s, reinterpret_cast<float *>(io + L.q), reinterpret_cast<float *>(io + L.k),
+                                reinterpret_cast<float *>(io + L.v), reinterpret_cast<float *>(io + L.alpha),
+                                reinterpret_cast<float *>(io + L.beta), reinterpret_cast<float *>(io + L.o),
+                                seed, step, stream, false);
     if (st != STQ_OK) return st;
     if (cudaMemcpyAsync(h_o, io + L.o, L.vec, cudaMemcpyDeviceToHost, cs) != cudaSuccess) return STQ_ERR_CUDA;
     return STQ_OK;

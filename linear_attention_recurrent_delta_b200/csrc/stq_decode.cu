@@ -455,6 +455,11 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
         fence_mbar_init();
     }
     __syncthreads();
+    // Launched early (programmatic dependent launch), the CTA may start
+    // while the previous kernel on the stream finishes; nothing in global
+    // memory is read before that kernel is complete and its writes visible
+    // (a no-op for a plain launch).
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int stride = (int)gridDim.x;
     const int n = A.n_pages;
     const int NS = A.n_stages;
@@ -725,6 +730,8 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
         ph = pnh;
         if (++st == NS) { st = 0; parity ^= 1u; }
     }
+    // the next kernel on the stream may start its own set-up now
+    asm volatile("griddepcontrol.launch_dependents;");
     __syncthreads();
     if (p_prev >= 0) {
         if (tid == 0) {
@@ -761,7 +768,7 @@ static int decode_stages(size_t stride, int ctas_per_sm) {
 }
 
 template <class FMT>
-static cudaError_t launch_with(const DevFormat &F, const DecodeArgs &A0, cudaStream_t stream) {
+static cudaError_t launch_with(const DevFormat &F, const DecodeArgs &A0, bool early_launch, cudaStream_t stream) {
     DecodeArgs A = A0;
     A.n_stages = decode_stages(A.stage_bytes, decode_ctas_per_sm<FMT::kSr>());
     const size_t smem = kFixedBytes + (size_t)A.n_stages * A.stage_bytes;
@@ -770,13 +777,22 @@ static cudaError_t launch_with(const DevFormat &F, const DecodeArgs &A0, cudaStr
     if (err != cudaSuccess) return err;
     const int grid = persistent_grid(fn, kThreads, smem, A.n_pages);
     if (grid <= 0) return cudaErrorInvalidConfiguration;
-    decode_kernel<FMT><<<grid, kThreads, smem, stream>>>(F, A);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = early_launch ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, decode_kernel<FMT>, F, A);
 }
 
 cudaError_t launch_decode(const stq_state *s, const float *q, const float *k, const float *v,
                           const float *alpha, const float *beta, float *o, uint64_t seed, uint32_t step,
-                          int stall_first_wait, cudaStream_t stream) {
+                          int stall_first_wait, bool early_launch, cudaStream_t stream) {
     const DevFormat &F = s->dev;
     DecodeArgs A;
     A.pages = s->base + s->pages_offset;
@@ -793,12 +809,12 @@ cudaError_t launch_decode(const stq_state *s, const float *q, const float *k, co
     A.step = step;
     A.wait_limit_ns = s->wait_limit_ns;
     A.stall_first_wait = stall_first_wait;
-    if (format_is<FmtStepQuant6>(F)) return launch_with<FmtStepQuant6>(F, A, stream);
-    if (format_is<FmtInt8Row>(F)) return launch_with<FmtInt8Row>(F, A, stream);
-    if (format_is<FmtStepQuant4Kda>(F)) return launch_with<FmtStepQuant4Kda>(F, A, stream);
-    if (format_is<FmtDamp>(F)) return launch_with<FmtDamp>(F, A, stream);
-    if (F.stochastic) return launch_with<RuntimeFmt<true>>(F, A, stream);
-    return launch_with<RuntimeFmt<false>>(F, A, stream);
+    if (format_is<FmtStepQuant6>(F)) return launch_with<FmtStepQuant6>(F, A, early_launch, stream);
+    if (format_is<FmtInt8Row>(F)) return launch_with<FmtInt8Row>(F, A, early_launch, stream);
+    if (format_is<FmtStepQuant4Kda>(F)) return launch_with<FmtStepQuant4Kda>(F, A, early_launch, stream);
+    if (format_is<FmtDamp>(F)) return launch_with<FmtDamp>(F, A, early_launch, stream);
+    if (F.stochastic) return launch_with<RuntimeFmt<true>>(F, A, early_launch, stream);
+    return launch_with<RuntimeFmt<false>>(F, A, early_launch, stream);
 }
 
 }  // namespace stq
