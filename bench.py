@@ -150,7 +150,7 @@ def max_over_ranks(x, world):
     return R.max_over_ranks(x, world, device="cuda")
 
 
-def run_gpu(w, steps, warmup, rank, world, sample_clocks=True, e2e_steps=64):
+def run_gpu(w, steps, warmup, rank, world, sample_clocks=True, e2e_steps=64, paged=False):
     from linear_attention_recurrent_delta_b200 import binding as B
     dev = torch.device("cuda", torch.cuda.current_device())
     wr = R.rank_workload(w, rank)   # this rank's own requests: no exchange on the data path
@@ -165,9 +165,17 @@ def run_gpu(w, steps, warmup, rank, world, sample_clocks=True, e2e_steps=64):
     seed = W.sr_seed(wr)
     stream = torch.cuda.current_stream()
 
+    # paged: every request through the slot table, in a random order of slots
+    table = torch.randperm(wr.batch, generator=torch.Generator().manual_seed(wr.seed)).to(
+        device=dev, dtype=torch.int32) if paged else None
+
     def step(t):
         x = inputs[t % n_in]
-        B.stq_decode_step(qs.state, x["q"], x["k"], x["v"], x["alpha"], x["beta"], o, seed, t, stream)
+        if paged:
+            B.stq_decode_step_slots(qs.state, table, x["q"], x["k"], x["v"], x["alpha"], x["beta"], o, seed, t,
+                                    stream)
+        else:
+            B.stq_decode_step(qs.state, x["q"], x["k"], x["v"], x["alpha"], x["beta"], o, seed, t, stream)
 
     for t in range(warmup):
         step(t)
@@ -343,6 +351,8 @@ def main():
     ap.add_argument("--ref-seconds", type=float, default=60.0)
     ap.add_argument("--only", action="store_true", help="skip the other workloads")
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling)")
+    ap.add_argument("--paged", action="store_true",
+                    help="with --profile: step through the slot table (stq_decode_step_slots)")
     ap.add_argument("--profile", action="store_true",
                     help="decode steps only: no clock sampling, e2e, CPU baseline or other workloads")
     args = ap.parse_args()
@@ -392,7 +402,7 @@ def main():
         build_mod.build()
     barrier(world)
     if args.profile:
-        res = run_gpu(w, args.steps, args.warmup, rank, world, sample_clocks=False, e2e_steps=0)
+        res = run_gpu(w, args.steps, args.warmup, rank, world, sample_clocks=False, e2e_steps=0, paged=args.paged)
         if rank == 0:
             print(json.dumps({"workload": w.name, "batch": w.batch, "ms_per_step": res["ms"] / args.steps}))
         R.finish(world)
@@ -404,6 +414,13 @@ def main():
     achieved = bpp * w.pages / per_launch_s / 1e9
     peak, peak_kind = measured_peak()
     e2e_value = R.aggregate_rate(w.pages, world, res["e2e_steps"], res["e2e_ms"])
+
+    paged = None
+    if not args.only:
+        r = run_gpu(w, args.steps, args.warmup, rank, world, sample_clocks=False, e2e_steps=0, paged=True)
+        paged = {"value": R.aggregate_rate(w.pages, world, args.steps, r["ms"]), "unit": UNIT,
+                 "entry_point": "stq_decode_step_slots", "table": "random permutation of all %d slots" % w.batch,
+                 "frac_of_%s_peak" % peak_kind: bpp * w.pages * args.steps / (r["ms"] / 1000.0) / 1e9 / peak}
 
     others = {}
     if not args.only:
@@ -449,6 +466,7 @@ def main():
         "gpu_launches": args.steps * world,   # one decode_kernel launch per step and rank
         "clocks": res["clocks"],
         "other_workloads": others,
+        "paged_step": paged,
     }
     print(json.dumps(line))
     R.finish(world)

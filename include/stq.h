@@ -172,6 +172,32 @@ stq_status stq_decode_step(stq_state *s, const float *d_q, const float *d_k, con
                            const float *d_alpha, const float *d_beta, float *d_o,
                            uint64_t seed, uint32_t step, void *stream);
 
+/* The decode step on a subset of the state's requests, found through a slot
+ * table: the shape a serving engine with a pool of state slots uses (packed
+ * pages per request in an SGLang integration: freedom251 post, "Memory and
+ * speed gains are implementation-specific").  Input row i (q, k, v, alpha, beta and o
+ * row i, layouts as stq_decode_step with B = n_rows) belongs to the request in
+ * state slot d_slots[i]; the pages (d_slots[i], h) are stepped in place and
+ * no other page is touched.
+ *   d_slots: device, [n_rows] int32, 4-byte aligned, caller-owned; slots must
+ *   be distinct (two rows on one slot race on its pages: unspecified codes,
+ *   never a fault).  1 <= n_rows <= the state's batch.
+ *   Stochastic rounding counts by the slot (counter = (tile, step, slot,
+ *   head)), so a request's rounding does not depend on its row.
+ *   A slot outside [0, batch) is caught on the device before any access: its
+ *   pages are not read or written, its o row is NaN, and stq_device_status
+ *   reports STQ_ERR_INVALID_ARG.  Other errors as stq_decode_step. */
+stq_status stq_decode_step_slots(stq_state *s, const int32_t *d_slots, int n_rows, const float *d_q,
+                                 const float *d_k, const float *d_v, const float *d_alpha,
+                                 const float *d_beta, float *d_o, uint64_t seed, uint32_t step,
+                                 void *stream);
+
+/* Byte offset (from the state buffer's start) and length of the pages of the
+ * request in `slot` -- its H pages are contiguous -- so that a caller can copy
+ * a request's state out (a checkpoint, a preemption) and back in with a
+ * plain device copy.  Errors: INVALID_ARG (null state, slot out of range). */
+stq_status stq_request_pages(const stq_state *s, int slot, size_t *offset, size_t *bytes);
+
 /* Device staging bytes stq_decode_step_host needs (q, k, v, alpha, beta, o). */
 size_t stq_decode_io_bytes(const stq_state *s);
 

@@ -56,6 +56,8 @@ def lib():
         "stq_calibrate_noalloc": (c_int, [P, P, P, P]),
         "stq_quantize_state": (c_int, [P, P, P]),
         "stq_decode_step": (c_int, [P, P, P, P, P, P, P, c_uint64, c_uint32, P]),
+        "stq_decode_step_slots": (c_int, [P, P, c_int, P, P, P, P, P, P, c_uint64, c_uint32, P]),
+        "stq_request_pages": (c_int, [P, c_int, POINTER(c_size_t), POINTER(c_size_t)]),
         "stq_decode_io_bytes": (c_size_t, [P]),
         "stq_decode_step_host": (c_int, [P, P, P, P, P, P, P, P, c_size_t, c_uint64, c_uint32, P]),
         "stq_dequantize_state": (c_int, [P, P, P]),
@@ -173,6 +175,20 @@ def stq_quantize_state(state, S, stream=None):
 def stq_decode_step(state, q, k, v, alpha, beta, o, seed=0, step=0, stream=None):
     _check(lib().stq_decode_step(state.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(o),
                                  int(seed), int(step), _stream(stream)), "stq_decode_step")
+
+
+def stq_decode_step_slots(state, slots, q, k, v, alpha, beta, o, seed=0, step=0, stream=None):
+    """Step the requests in state slots ``slots`` (int32 device tensor, one per input row)."""
+    _check(lib().stq_decode_step_slots(state.handle, _ptr(slots), int(slots.numel()), _ptr(q), _ptr(k), _ptr(v),
+                                       _ptr(alpha), _ptr(beta), _ptr(o), int(seed), int(step), _stream(stream)),
+           "stq_decode_step_slots")
+
+
+def stq_request_pages(state, slot):
+    """(byte offset, bytes) of the pages of the request in ``slot`` inside the state buffer."""
+    off, n = c_size_t(), c_size_t()
+    _check(lib().stq_request_pages(state.handle, int(slot), ctypes.byref(off), ctypes.byref(n)), "stq_request_pages")
+    return off.value, n.value
 
 
 def stq_decode_io_bytes(state):

@@ -190,13 +190,15 @@ stq_status stq_quantize_state(stq_state *s, const float *d_S, void *stream) {
     return err == cudaSuccess ? STQ_OK : STQ_ERR_CUDA;
 }
 
-static stq_status check_step_args(const stq_state *s, const float *q, const float *k, const float *v,
-                                  const float *alpha, const float *beta, const float *o) {
+// n_rows: request rows of the inputs and of o (the state's batch, or the
+// length of a slot table)
+static stq_status check_step_args(const stq_state *s, int n_rows, const float *q, const float *k,
+                                  const float *v, const float *alpha, const float *beta, const float *o) {
     if (!s || !q || !k || !v || !alpha || !beta || !o) return STQ_ERR_INVALID_ARG;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(beta, 4) ||
         !aligned(alpha, s->fmt.gate_vector ? 16 : 4))
         return STQ_ERR_MISALIGNED;
-    const size_t n = (size_t)s->batch * s->heads;
+    const size_t n = (size_t)n_rows * s->heads;
     const size_t vec = n * kD * sizeof(float), sc = n * sizeof(float);
     const size_t na = s->fmt.gate_vector ? vec : sc;
     const size_t span = state_span(s);
@@ -214,22 +216,40 @@ static stq_status check_step_args(const stq_state *s, const float *q, const floa
 // a preceding kernel on the stream finishes (the kernel waits for it before
 // its first global read); the host entry point, whose step follows copies,
 // launches plainly.
-static stq_status decode_step(stq_state *s, const float *d_q, const float *d_k, const float *d_v,
-                              const float *d_alpha, const float *d_beta, float *d_o, uint64_t seed,
-                              uint32_t step, void *stream, bool early_launch) {
-    stq_status st = check_step_args(s, d_q, d_k, d_v, d_alpha, d_beta, d_o);
+static stq_status decode_step(stq_state *s, const int32_t *d_slots, int n_rows, const float *d_q,
+                              const float *d_k, const float *d_v, const float *d_alpha, const float *d_beta,
+                              float *d_o, uint64_t seed, uint32_t step, void *stream, bool early_launch) {
+    stq_status st = check_step_args(s, n_rows, d_q, d_k, d_v, d_alpha, d_beta, d_o);
     if (st != STQ_OK) return st;
     const int stall = s->stall_first_wait;
     s->stall_first_wait = 0;
     cudaError_t err = launch_decode(s, d_q, d_k, d_v, d_alpha, d_beta, d_o, seed, step, stall, early_launch,
-                                    static_cast<cudaStream_t>(stream));
+                                    d_slots, n_rows, static_cast<cudaStream_t>(stream));
     return err == cudaSuccess ? STQ_OK : STQ_ERR_CUDA;
 }
 
 stq_status stq_decode_step(stq_state *s, const float *d_q, const float *d_k, const float *d_v,
                            const float *d_alpha, const float *d_beta, float *d_o, uint64_t seed, uint32_t step,
                            void *stream) {
-    return decode_step(s, d_q, d_k, d_v, d_alpha, d_beta, d_o, seed, step, stream, true);
+    if (!s) return STQ_ERR_INVALID_ARG;
+    return decode_step(s, nullptr, s->batch, d_q, d_k, d_v, d_alpha, d_beta, d_o, seed, step, stream, true);
+}
+
+stq_status stq_decode_step_slots(stq_state *s, const int32_t *d_slots, int n_rows, const float *d_q,
+                                 const float *d_k, const float *d_v, const float *d_alpha, const float *d_beta,
+                                 float *d_o, uint64_t seed, uint32_t step, void *stream) {
+    if (!s || !d_slots) return STQ_ERR_INVALID_ARG;
+    if (n_rows < 1 || n_rows > s->batch) return STQ_ERR_INVALID_ARG;
+    if (!aligned(d_slots, 4)) return STQ_ERR_MISALIGNED;
+    if (overlaps(d_slots, (size_t)n_rows * sizeof(int32_t), s->base, state_span(s))) return STQ_ERR_INVALID_ARG;
+    return decode_step(s, d_slots, n_rows, d_q, d_k, d_v, d_alpha, d_beta, d_o, seed, step, stream, true);
+}
+
+stq_status stq_request_pages(const stq_state *s, int slot, size_t *offset, size_t *bytes) {
+    if (!s || slot < 0 || slot >= s->batch) return STQ_ERR_INVALID_ARG;
+    if (offset) *offset = s->pages_offset + (size_t)slot * s->heads * s->page_bytes;
+    if (bytes) *bytes = (size_t)s->heads * s->page_bytes;
+    return STQ_OK;
 }
 
 struct IoLayout {
@@ -269,7 +289,8 @@ stq_status stq_decode_step_host(stq_state *s, const float *h_q, const float *h_k
     for (int i = 0; i < 5; ++i)
         if (cudaMemcpyAsync(io + in[i].off, in[i].src, in[i].n, cudaMemcpyHostToDevice, cs) != cudaSuccess)
             return STQ_ERR_CUDA;
-    stq_status st = decode_step(s, reinterpret_cast<float *>(io + L.q), reinterpret_cast<float *>(io + L.k),
+    stq_status st = decode_step(s, nullptr, s->batch, reinterpret_cast<float *>(io + L.q),
+                                reinterpret_cast<float *>(io + L.k),
                                 reinterpret_cast<float *>(io + L.v), reinterpret_cast<float *>(io + L.alpha),
                                 reinterpret_cast<float *>(io + L.beta), reinterpret_cast<float *>(io + L.o),
                                 seed, step, stream, false);
@@ -295,7 +316,8 @@ stq_status stq_device_status(stq_state *s, void *stream, int clear) {
     if (cudaMemcpy(&word, s->base + s->status_offset, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
         return STQ_ERR_CUDA;
     if (clear && cudaMemset(s->base + s->status_offset, 0, sizeof(uint32_t)) != cudaSuccess) return STQ_ERR_CUDA;
-    return (word & kStatusTimeout) ? STQ_ERR_DEVICE_TIMEOUT : STQ_OK;
+    if (word & kStatusTimeout) return STQ_ERR_DEVICE_TIMEOUT;
+    return (word & kStatusBadSlot) ? STQ_ERR_INVALID_ARG : STQ_OK;
 }
 
 stq_status stq_set_wait_limit(stq_state *s, uint64_t limit_ns, int stall_first_wait) {

@@ -87,7 +87,7 @@ struct DecodeArgs {
     uint32_t *status;
     const float *q, *k, *v, *alpha, *beta;
     float *o;
-    int n_pages;                  // < 2^31 (checked when the state is bound)
+    int n_pages;                  // work items = input rows x heads, < 2^31
     int heads;
     int n_stages;                 // ring depth, 3 .. kMaxStages
     uint32_t stage_bytes;
@@ -95,6 +95,8 @@ struct DecodeArgs {
     uint32_t seed_lo, seed_hi, step;
     uint64_t wait_limit_ns;
     int stall_first_wait;
+    int n_slots;                  // requests in the state (valid slots: 0 .. n_slots-1)
+    const int32_t *slots;         // slot table of a paged step (else null)
 };
 
 constexpr int kMaxStages = 4;
@@ -112,6 +114,7 @@ struct SmemFixed {
     float cpg[2][kD];                       // per page parity: c (o of a page is finished a page later)
     uint64_t full[kMaxStages];              // stage-full barriers
     uint64_t never;                         // a barrier nothing completes (test hook)
+    int pg[kMaxStages];                     // paged step: page in each stage (-1: bad slot)
 };
 
 constexpr size_t kFixedBytes = (sizeof(SmemFixed) + 127) / 128 * 128;
@@ -396,10 +399,18 @@ __device__ __forceinline__ float absmax4(float2 a, float2 b) {
     return fmaxf(max3f(fabsf(a.x), fabsf(a.y), fabsf(b.x)), fabsf(b.y));
 }
 
+// Stage the page `pg` (paged step: none if pg < 0; else pg == p) and the
+// input rows of work item p.
+template <bool SLOTS>
 __device__ __forceinline__ void issue_stage(const DevFormat &F, const DecodeArgs &A, uint8_t *dst, int p,
-                                            uint64_t *bar) {
-    mbar_expect_tx(bar, decode_stage_bytes(F));
-    bulk_g2s(dst, A.pages + (size_t)p * F.page_bytes, (uint32_t)F.page_bytes, bar);
+                                            uint64_t *bar, int pg) {
+    if constexpr (SLOTS) {
+        mbar_expect_tx(bar, decode_stage_bytes(F) - (pg < 0 ? (uint32_t)F.page_bytes : 0u));
+        if (pg >= 0) bulk_g2s(dst, A.pages + (size_t)pg * F.page_bytes, (uint32_t)F.page_bytes, bar);
+    } else {
+        mbar_expect_tx(bar, decode_stage_bytes(F));
+        bulk_g2s(dst, A.pages + (size_t)p * F.page_bytes, (uint32_t)F.page_bytes, bar);
+    }
     uint8_t *rows = dst + F.page_bytes;
     bulk_g2s(rows, A.q + (size_t)p * kD, 512, bar);
     bulk_g2s(rows + 512, A.k + (size_t)p * kD, 512, bar);
@@ -407,9 +418,19 @@ __device__ __forceinline__ void issue_stage(const DevFormat &F, const DecodeArgs
     if (F.gate_vector) bulk_g2s(rows + 1536, A.alpha + (size_t)p * kD, 512, bar);
 }
 
+// Paged step: the page of work item p (input row p / H, head p % H) is
+// slot(row) * H + head, or -1 when the row's slot is out of range.
+__device__ __forceinline__ int slot_page(const DecodeArgs &A, int p, int slot) {
+    return (slot >= 0 && slot < A.n_slots) ? slot * A.heads + p % A.heads : -1;
+}
+
+__device__ __forceinline__ int item_slot(const DecodeArgs &A, int p) {
+    return __ldg(A.slots + p / A.heads);
+}
+
 // o of a finished page: the tree over the warps' chain sums, times c.
 __device__ __forceinline__ void write_o(const float (*red_o)[kD], const DecodeArgs &A, int p, int lane,
-                                        const float *cpg, bool col_scales) {
+                                        const float *cpg, bool col_scales, bool bad = false) {
     const float4 o0 = *reinterpret_cast<const float4 *>(&red_o[0][4 * lane]);
     const float4 o1 = *reinterpret_cast<const float4 *>(&red_o[1][4 * lane]);
     const float4 o2 = *reinterpret_cast<const float4 *>(&red_o[2][4 * lane]);
@@ -423,6 +444,7 @@ __device__ __forceinline__ void write_o(const float (*red_o)[kD], const DecodeAr
         oa = __fmul2_rn(make_float2(c.x, c.y), oa);
         ob = __fmul2_rn(make_float2(c.z, c.w), ob);
     }
+    if (bad) oa = ob = make_float2(__int_as_float(0x7FC00000), __int_as_float(0x7FC00000));   // NaN
     *reinterpret_cast<float4 *>(A.o + (size_t)p * kD + 4 * lane) = make_float4(oa.x, oa.y, ob.x, ob.y);
 }
 
@@ -432,7 +454,9 @@ template <bool SR>
 constexpr int decode_ctas_per_sm() { return SR ? 2 : 3; }
 
 // The per-page loop.
-template <class FMT>
+// SLOTS: the paged step (pages found through the slot table); otherwise
+// page index = work item.
+template <class FMT, bool SLOTS>
 __global__ void __launch_bounds__(kThreads, decode_ctas_per_sm<FMT::kSr>())
 decode_kernel(const DevFormat F, const DecodeArgs A) {
     extern __shared__ __align__(128) uint8_t smem[];
@@ -463,10 +487,23 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
     const int stride = (int)gridDim.x;
     const int n = A.n_pages;
     const int NS = A.n_stages;
+    int pf_slot = 0;   // paged step, thread 0: slot of the next refill's item, loaded a page ahead
     if (tid == 0) {
         for (int i = 0; i < NS; ++i) {
             const int p = (int)blockIdx.x + i * stride;
-            if (p < n) issue_stage(F, A, stages + i * A.stage_bytes, p, &S.full[i]);
+            if (p < n) {
+                int pg = p;
+                if constexpr (SLOTS) {
+                    pg = slot_page(A, p, item_slot(A, p));
+                    S.pg[i] = pg;
+                    if (pg < 0) atomicOr(A.status, kStatusBadSlot);
+                }
+                issue_stage<SLOTS>(F, A, stages + i * A.stage_bytes, p, &S.full[i], pg);
+            }
+        }
+        if constexpr (SLOTS) {
+            const int p = (int)blockIdx.x + NS * stride;
+            if (p < n) pf_slot = item_slot(A, p);
         }
     }
     // (request, head) of a page is carried along: p advances by `stride`,
@@ -510,7 +547,8 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
         if (!gate_vector) alpha_s = __ldg(A.alpha + p);
         kap = __ldg(A.perm + ph * kD + my_s) & (kD - 1);
     }
-    int p_prev = -1;                  // page whose codes and o are still to be stored
+    int p_prev = -1;                  // work item whose codes and o are still to be stored
+    int pg_prev = -1;                 // its page (paged step: -1 for a bad slot)
     int st = 0, st_prev = 0;
     uint32_t parity = 0;
     int it = 0;
@@ -535,6 +573,8 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
         else ok = mbar_wait_bounded(&S.full[st], parity, A.wait_limit_ns);
         const int par = it & 1;
         uint8_t *stg = stages + st * A.stage_bytes;
+        int pg_cur = p;   // page in this stage (recorded before the stage's barrier was armed)
+        if constexpr (SLOTS) pg_cur = S.pg[st];
         const float *q_s = reinterpret_cast<const float *>(stg + F.page_bytes);
         const float *k_s = q_s + kD;
         const float *v_s = q_s + 2 * kD;
@@ -590,11 +630,11 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
             // the copies in flight land and leave; nothing of this page (or
             // a later one) is written
             if (warp == kWarps - 1 && p_prev >= 0)
-                write_o(S.red_o[par ^ 1], A, p_prev, lane, S.cpg[par ^ 1], col_scales);
+                write_o(S.red_o[par ^ 1], A, p_prev, lane, S.cpg[par ^ 1], col_scales, SLOTS && pg_prev < 0);
             if (tid == 0) {
                 atomicOr(A.status, kStatusTimeout);
-                if (p_prev >= 0) {
-                    bulk_s2g(A.pages + (size_t)p_prev * F.page_bytes, stages + st_prev * A.stage_bytes,
+                if (SLOTS ? pg_prev >= 0 : p_prev >= 0) {
+                    bulk_s2g(A.pages + (size_t)(SLOTS ? pg_prev : p_prev) * F.page_bytes, stages + st_prev * A.stage_bytes,
                              A.store_bytes);
                     bulk_commit();
                 }
@@ -614,8 +654,8 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
         if (tid == 0) {
             // the previous page is complete in its stage: store it; its stage
             // is refilled once the store has read it (see kEarlyRefill)
-            if (p_prev >= 0) {
-                bulk_s2g(A.pages + (size_t)p_prev * F.page_bytes, stages + st_prev * A.stage_bytes,
+            if (SLOTS ? pg_prev >= 0 : p_prev >= 0) {
+                bulk_s2g(A.pages + (size_t)(SLOTS ? pg_prev : p_prev) * F.page_bytes, stages + st_prev * A.stage_bytes,
                          A.store_bytes);
                 bulk_commit();
             }
@@ -624,15 +664,22 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
                 const int j = it - 2 + NS;
                 const int pr = (int)blockIdx.x + j * stride;
                 if (pr < n) {
+                    int pg = pr;
+                    if constexpr (SLOTS) {   // the slot of item pr was loaded a page ago
+                        pg = slot_page(A, pr, pf_slot);
+                        S.pg[j % NS] = pg;
+                        if (pg < 0) atomicOr(A.status, kStatusBadSlot);
+                        if (pr + stride < n) pf_slot = item_slot(A, pr + stride);
+                    }
                     fence_proxy_async_smem();
-                    issue_stage(F, A, stages + (j % NS) * A.stage_bytes, pr, &S.full[j % NS]);
+                    issue_stage<SLOTS>(F, A, stages + (j % NS) * A.stage_bytes, pr, &S.full[j % NS], pg);
                 }
             }
         }
         // o of the previous page (its chain sums were stored before this
         // barrier), by the last warp: warp 0's first thread handles the copies
         if (warp == kWarps - 1 && p_prev >= 0)
-            write_o(S.red_o[par ^ 1], A, p_prev, lane, S.cpg[par ^ 1], col_scales);
+            write_o(S.red_o[par ^ 1], A, p_prev, lane, S.cpg[par ^ 1], col_scales, SLOTS && pg_prev < 0);
 
         // u = (W0 + W1) + (W2 + W3); e = v (1/c) - u
         float2 e01, e23;
@@ -675,11 +722,20 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
         if (kEarly && tid == 0 && p_prev >= 0) {
             // refill the previous page's stage with the page NS - 1 ahead of this one
             bulk_wait_read<0>();
-            const int j = it - 1 + NS;
-            const int pr = (int)blockIdx.x + j * stride;
+            {
+                const int j = it - 1 + NS;
+                const int pr = (int)blockIdx.x + j * stride;
             if (pr < n) {
+                int pg = pr;
+                if constexpr (SLOTS) {   // the slot of item pr was loaded a page ago
+                    pg = slot_page(A, pr, pf_slot);
+                    S.pg[j % NS] = pg;
+                    if (pg < 0) atomicOr(A.status, kStatusBadSlot);
+                    if (pr + stride < n) pf_slot = item_slot(A, pr + stride);
+                }
                 fence_proxy_async_smem();
-                issue_stage(F, A, stages + (j % NS) * A.stage_bytes, pr, &S.full[j % NS]);
+                issue_stage<SLOTS>(F, A, stages + (j % NS) * A.stage_bytes, pr, &S.full[j % NS], pg);
+            }
             }
         }
         __syncwarp();
@@ -708,7 +764,8 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
         // S7 + S8, into the stage
         SrCtx sr;
         sr.k0 = A.seed_lo; sr.k1 = A.seed_hi; sr.step = A.step;
-        sr.b = (uint32_t)pb; sr.h = (uint32_t)ph;
+        sr.b = SLOTS ? (uint32_t)(pg_cur / H) : (uint32_t)pb;   // the request's slot in the state
+        sr.h = (uint32_t)ph;
         static_for<0, kBlocks>([&](auto bc) {
             constexpr int b = decltype(bc)::value;
             const float4 i4 = *reinterpret_cast<const float4 *>(&S.inv[warp][4 * b]);
@@ -721,6 +778,7 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
         fence_proxy_async_smem();   // the stage's new bytes are read by the bulk store
 
         p_prev = p;
+        if constexpr (SLOTS) pg_prev = pg_cur;
         st_prev = st;
         alpha_s = alpha_n;
         beta_s = beta_n;
@@ -734,12 +792,12 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
     asm volatile("griddepcontrol.launch_dependents;");
     __syncthreads();
     if (p_prev >= 0) {
-        if (tid == 0) {
-            bulk_s2g(A.pages + (size_t)p_prev * F.page_bytes, stages + st_prev * A.stage_bytes, A.store_bytes);
+        if (tid == 0 && (SLOTS ? pg_prev >= 0 : true)) {
+            bulk_s2g(A.pages + (size_t)(SLOTS ? pg_prev : p_prev) * F.page_bytes, stages + st_prev * A.stage_bytes, A.store_bytes);
             bulk_commit();
         }
         if (warp == kWarps - 1)
-            write_o(S.red_o[(it - 1) & 1], A, p_prev, lane, S.cpg[(it - 1) & 1], col_scales);
+            write_o(S.red_o[(it - 1) & 1], A, p_prev, lane, S.cpg[(it - 1) & 1], col_scales, SLOTS && pg_prev < 0);
     }
     if (tid == 0) bulk_wait<0>();
 }
@@ -767,12 +825,12 @@ static int decode_stages(size_t stride, int ctas_per_sm) {
     return (int)ns;
 }
 
-template <class FMT>
+template <class FMT, bool SLOTS>
 static cudaError_t launch_with(const DevFormat &F, const DecodeArgs &A0, bool early_launch, cudaStream_t stream) {
     DecodeArgs A = A0;
     A.n_stages = decode_stages(A.stage_bytes, decode_ctas_per_sm<FMT::kSr>());
     const size_t smem = kFixedBytes + (size_t)A.n_stages * A.stage_bytes;
-    const void *fn = (const void *)decode_kernel<FMT>;
+    const void *fn = (const void *)decode_kernel<FMT, SLOTS>;
     cudaError_t err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     const int grid = persistent_grid(fn, kThreads, smem, A.n_pages);
@@ -787,19 +845,32 @@ static cudaError_t launch_with(const DevFormat &F, const DecodeArgs &A0, bool ea
     attr[0].val.programmaticStreamSerializationAllowed = early_launch ? 1 : 0;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_kernel<FMT>, F, A);
+    return cudaLaunchKernelEx(&cfg, decode_kernel<FMT, SLOTS>, F, A);
+}
+
+template <bool SLOTS>
+static cudaError_t launch_fmt(const DevFormat &F, const DecodeArgs &A, bool early_launch, cudaStream_t stream) {
+    if (format_is<FmtStepQuant6>(F)) return launch_with<FmtStepQuant6, SLOTS>(F, A, early_launch, stream);
+    if (format_is<FmtInt8Row>(F)) return launch_with<FmtInt8Row, SLOTS>(F, A, early_launch, stream);
+    if (format_is<FmtStepQuant4Kda>(F)) return launch_with<FmtStepQuant4Kda, SLOTS>(F, A, early_launch, stream);
+    if (format_is<FmtDamp>(F)) return launch_with<FmtDamp, SLOTS>(F, A, early_launch, stream);
+    if (F.stochastic) return launch_with<RuntimeFmt<true>, SLOTS>(F, A, early_launch, stream);
+    return launch_with<RuntimeFmt<false>, SLOTS>(F, A, early_launch, stream);
 }
 
 cudaError_t launch_decode(const stq_state *s, const float *q, const float *k, const float *v,
                           const float *alpha, const float *beta, float *o, uint64_t seed, uint32_t step,
-                          int stall_first_wait, bool early_launch, cudaStream_t stream) {
+                          int stall_first_wait, bool early_launch, const int32_t *slots, int n_rows,
+                          cudaStream_t stream) {
     const DevFormat &F = s->dev;
     DecodeArgs A;
     A.pages = s->base + s->pages_offset;
     A.perm = s->base + s->perm_offset;
     A.status = reinterpret_cast<uint32_t *>(s->base + s->status_offset);
     A.q = q; A.k = k; A.v = v; A.alpha = alpha; A.beta = beta; A.o = o;
-    A.n_pages = s->batch * s->heads;
+    A.slots = slots;
+    A.n_slots = s->batch;
+    A.n_pages = (slots ? n_rows : s->batch) * s->heads;
     A.heads = s->heads;
     A.stage_bytes = (decode_stage_bytes(F) + 127) / 128 * 128;
     A.store_bytes = (uint32_t)(F.col_scales ? F.c_off : F.page_bytes);
@@ -809,12 +880,8 @@ cudaError_t launch_decode(const stq_state *s, const float *q, const float *k, co
     A.step = step;
     A.wait_limit_ns = s->wait_limit_ns;
     A.stall_first_wait = stall_first_wait;
-    if (format_is<FmtStepQuant6>(F)) return launch_with<FmtStepQuant6>(F, A, early_launch, stream);
-    if (format_is<FmtInt8Row>(F)) return launch_with<FmtInt8Row>(F, A, early_launch, stream);
-    if (format_is<FmtStepQuant4Kda>(F)) return launch_with<FmtStepQuant4Kda>(F, A, early_launch, stream);
-    if (format_is<FmtDamp>(F)) return launch_with<FmtDamp>(F, A, early_launch, stream);
-    if (F.stochastic) return launch_with<RuntimeFmt<true>>(F, A, early_launch, stream);
-    return launch_with<RuntimeFmt<false>>(F, A, early_launch, stream);
+    if (slots) return launch_fmt<true>(F, A, early_launch, stream);
+    return launch_fmt<false>(F, A, early_launch, stream);
 }
 
 }  // namespace stq

@@ -24,7 +24,7 @@ constexpr int kBlocks = 8;          // 16-row blocks per page
 enum : int { kKindInt = 0, kKindFp16 = 1 };
 
 // Status word bits (state header).
-enum : uint32_t { kStatusTimeout = 1u };
+enum : uint32_t { kStatusTimeout = 1u, kStatusBadSlot = 2u };
 
 // Per-format constants, passed by value to every kernel.
 struct DevFormat {

@@ -34,7 +34,8 @@ int persistent_grid(const void *kernel, int threads, size_t dyn_smem, long n_uni
 // Launchers (return cudaError_t of the launch).
 cudaError_t launch_decode(const stq_state *s, const float *q, const float *k, const float *v,
                           const float *alpha, const float *beta, float *o, uint64_t seed,
-                          uint32_t step, int stall_first_wait, bool early_launch, cudaStream_t stream);
+                          uint32_t step, int stall_first_wait, bool early_launch, const int32_t *slots,
+                          int n_rows, cudaStream_t stream);
 cudaError_t launch_calibrate(const stq_state *s, const float *S, const float *row_weight,
                              double *workspace, cudaStream_t stream);
 size_t calibrate_workspace_bytes(int batch, int heads);

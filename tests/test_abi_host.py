@@ -148,3 +148,32 @@ def test_other_entry_points_check_arguments(lib):
     assert lib.stq_set_wait_limit(None, 0, 0) == B.STQ_ERR_INVALID_ARG
     assert lib.stq_device_status(None, None, 0) == B.STQ_ERR_INVALID_ARG
     lib.stq_state_free(h)
+
+
+def test_slot_step_and_request_pages_check_arguments(lib):
+    fmt = B.format_from_spec(W.FORMATS["int8row"])
+    st, h = _alloc(lib, fmt, 4, 3)
+    assert st == B.STQ_OK
+    P = ctypes.c_void_p
+    base = 1 << 41
+    q, k, v, a, b, o = (P(base + i * (1 << 24)) for i in range(6))
+    table = 1 << 46
+
+    def call(sl=table, n=2):
+        return lib.stq_decode_step_slots(h, P(sl) if sl else None, n, q, k, v, a, b, o, 0, 0, None)
+
+    assert call(sl=0) == B.STQ_ERR_INVALID_ARG
+    assert call(n=0) == B.STQ_ERR_INVALID_ARG
+    assert call(n=5) == B.STQ_ERR_INVALID_ARG          # more rows than the state has requests
+    assert call(sl=table + 2) == B.STQ_ERR_MISALIGNED
+    assert call(sl=FAKE + 256) == B.STQ_ERR_INVALID_ARG  # the table overlaps the state
+    off, nb = ctypes.c_size_t(), ctypes.c_size_t()
+    for bad in (-1, 4):
+        assert lib.stq_request_pages(h, bad, ctypes.byref(off), ctypes.byref(nb)) == B.STQ_ERR_INVALID_ARG
+    assert lib.stq_request_pages(None, 0, None, None) == B.STQ_ERR_INVALID_ARG
+    assert lib.stq_request_pages(h, 2, ctypes.byref(off), ctypes.byref(nb)) == B.STQ_OK
+    pb, pages_off = ctypes.c_size_t(), ctypes.c_size_t()
+    assert lib.stq_state_layout(h, ctypes.byref(pb), None, ctypes.byref(pages_off), None) == B.STQ_OK
+    assert off.value == pages_off.value + 2 * 3 * pb.value
+    assert nb.value == 3 * pb.value
+    lib.stq_state_free(h)
