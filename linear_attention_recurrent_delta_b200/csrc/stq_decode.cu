@@ -115,6 +115,8 @@ struct SmemFixed {
     uint64_t full[kMaxStages];              // stage-full barriers
     uint64_t never;                         // a barrier nothing completes (test hook)
     int pg[kMaxStages];                     // paged step: page in each stage (-1: bad slot)
+    int bad[2];                             // paged step, per page parity: the page's slot was bad
+    int pf_slot;                            // paged step: slot of the next refill's item (async copy)
 };
 
 constexpr size_t kFixedBytes = (sizeof(SmemFixed) + 127) / 128 * 128;
@@ -428,6 +430,17 @@ __device__ __forceinline__ int item_slot(const DecodeArgs &A, int p) {
     return __ldg(A.slots + p / A.heads);
 }
 
+// Start copying the slot of work item p into *dst (4-byte async copy; no
+// register holds it while it is in flight); cp_async_wait() before reading.
+__device__ __forceinline__ void prefetch_slot(const DecodeArgs &A, int p, int *dst) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n\tcp.async.commit_group;"
+                 :: "r"(smem_u32(dst)), "l"(A.slots + p / A.heads) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
 // o of a finished page: the tree over the warps' chain sums, times c.
 __device__ __forceinline__ void write_o(const float (*red_o)[kD], const DecodeArgs &A, int p, int lane,
                                         const float *cpg, bool col_scales, bool bad = false) {
@@ -487,23 +500,30 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
     const int stride = (int)gridDim.x;
     const int n = A.n_pages;
     const int NS = A.n_stages;
-    int pf_slot = 0;   // paged step, thread 0: slot of the next refill's item, loaded a page ahead
+    if constexpr (SLOTS) {
+        // lanes of warp 0 look up the first stages' pages in parallel
+        if (tid < NS) {
+            const int p = (int)blockIdx.x + tid * stride;
+            if (p < n) {
+                const int pg = slot_page(A, p, item_slot(A, p));
+                S.pg[tid] = pg;
+                if (pg < 0) atomicOr(A.status, kStatusBadSlot);
+            }
+        }
+        __syncwarp();
+    }
     if (tid == 0) {
         for (int i = 0; i < NS; ++i) {
             const int p = (int)blockIdx.x + i * stride;
             if (p < n) {
                 int pg = p;
-                if constexpr (SLOTS) {
-                    pg = slot_page(A, p, item_slot(A, p));
-                    S.pg[i] = pg;
-                    if (pg < 0) atomicOr(A.status, kStatusBadSlot);
-                }
+                if constexpr (SLOTS) pg = S.pg[i];
                 issue_stage<SLOTS>(F, A, stages + i * A.stage_bytes, p, &S.full[i], pg);
             }
         }
         if constexpr (SLOTS) {
             const int p = (int)blockIdx.x + NS * stride;
-            if (p < n) pf_slot = item_slot(A, p);
+            if (p < n) prefetch_slot(A, p, &S.pf_slot);
         }
     }
     // (request, head) of a page is carried along: p advances by `stride`,
@@ -548,7 +568,6 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
         kap = __ldg(A.perm + ph * kD + my_s) & (kD - 1);
     }
     int p_prev = -1;                  // work item whose codes and o are still to be stored
-    int pg_prev = -1;                 // its page (paged step: -1 for a bad slot)
     int st = 0, st_prev = 0;
     uint32_t parity = 0;
     int it = 0;
@@ -573,8 +592,10 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
         else ok = mbar_wait_bounded(&S.full[st], parity, A.wait_limit_ns);
         const int par = it & 1;
         uint8_t *stg = stages + st * A.stage_bytes;
-        int pg_cur = p;   // page in this stage (recorded before the stage's barrier was armed)
-        if constexpr (SLOTS) pg_cur = S.pg[st];
+        if constexpr (SLOTS) {
+            // the stage's page was recorded before its barrier was armed
+            if (tid == 0) S.bad[par] = S.pg[st] < 0;
+        }
         const float *q_s = reinterpret_cast<const float *>(stg + F.page_bytes);
         const float *k_s = q_s + kD;
         const float *v_s = q_s + 2 * kD;
@@ -630,11 +651,11 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
             // the copies in flight land and leave; nothing of this page (or
             // a later one) is written
             if (warp == kWarps - 1 && p_prev >= 0)
-                write_o(S.red_o[par ^ 1], A, p_prev, lane, S.cpg[par ^ 1], col_scales, SLOTS && pg_prev < 0);
+                write_o(S.red_o[par ^ 1], A, p_prev, lane, S.cpg[par ^ 1], col_scales, SLOTS && S.bad[par ^ 1]);
             if (tid == 0) {
                 atomicOr(A.status, kStatusTimeout);
-                if (SLOTS ? pg_prev >= 0 : p_prev >= 0) {
-                    bulk_s2g(A.pages + (size_t)(SLOTS ? pg_prev : p_prev) * F.page_bytes, stages + st_prev * A.stage_bytes,
+                if (SLOTS ? S.pg[st_prev] >= 0 : p_prev >= 0) {
+                    bulk_s2g(A.pages + (size_t)(SLOTS ? S.pg[st_prev] : p_prev) * F.page_bytes, stages + st_prev * A.stage_bytes,
                              A.store_bytes);
                     bulk_commit();
                 }
@@ -645,6 +666,7 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
                         mbar_wait_bounded(&S.full[j % NS], (uint32_t)((j / NS) & 1), A.wait_limit_ns);
                 }
                 bulk_wait<0>();
+                if constexpr (SLOTS) cp_async_wait();   // no copy outlives the CTA
             }
             __syncthreads();
             return;
@@ -654,8 +676,8 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
         if (tid == 0) {
             // the previous page is complete in its stage: store it; its stage
             // is refilled once the store has read it (see kEarlyRefill)
-            if (SLOTS ? pg_prev >= 0 : p_prev >= 0) {
-                bulk_s2g(A.pages + (size_t)(SLOTS ? pg_prev : p_prev) * F.page_bytes, stages + st_prev * A.stage_bytes,
+            if (SLOTS ? p_prev >= 0 && S.pg[st_prev] >= 0 : p_prev >= 0) {
+                bulk_s2g(A.pages + (size_t)(SLOTS ? S.pg[st_prev] : p_prev) * F.page_bytes, stages + st_prev * A.stage_bytes,
                          A.store_bytes);
                 bulk_commit();
             }
@@ -666,10 +688,11 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
                 if (pr < n) {
                     int pg = pr;
                     if constexpr (SLOTS) {   // the slot of item pr was loaded a page ago
-                        pg = slot_page(A, pr, pf_slot);
+                        cp_async_wait();
+                        pg = slot_page(A, pr, S.pf_slot);
                         S.pg[j % NS] = pg;
                         if (pg < 0) atomicOr(A.status, kStatusBadSlot);
-                        if (pr + stride < n) pf_slot = item_slot(A, pr + stride);
+                        if (pr + stride < n) prefetch_slot(A, pr + stride, &S.pf_slot);
                     }
                     fence_proxy_async_smem();
                     issue_stage<SLOTS>(F, A, stages + (j % NS) * A.stage_bytes, pr, &S.full[j % NS], pg);
@@ -679,7 +702,7 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
         // o of the previous page (its chain sums were stored before this
         // barrier), by the last warp: warp 0's first thread handles the copies
         if (warp == kWarps - 1 && p_prev >= 0)
-            write_o(S.red_o[par ^ 1], A, p_prev, lane, S.cpg[par ^ 1], col_scales, SLOTS && pg_prev < 0);
+            write_o(S.red_o[par ^ 1], A, p_prev, lane, S.cpg[par ^ 1], col_scales, SLOTS && S.bad[par ^ 1]);
 
         // u = (W0 + W1) + (W2 + W3); e = v (1/c) - u
         float2 e01, e23;
@@ -728,10 +751,11 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
             if (pr < n) {
                 int pg = pr;
                 if constexpr (SLOTS) {   // the slot of item pr was loaded a page ago
-                    pg = slot_page(A, pr, pf_slot);
+                    cp_async_wait();
+                    pg = slot_page(A, pr, S.pf_slot);
                     S.pg[j % NS] = pg;
                     if (pg < 0) atomicOr(A.status, kStatusBadSlot);
-                    if (pr + stride < n) pf_slot = item_slot(A, pr + stride);
+                    if (pr + stride < n) prefetch_slot(A, pr + stride, &S.pf_slot);
                 }
                 fence_proxy_async_smem();
                 issue_stage<SLOTS>(F, A, stages + (j % NS) * A.stage_bytes, pr, &S.full[j % NS], pg);
@@ -764,7 +788,8 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
         // S7 + S8, into the stage
         SrCtx sr;
         sr.k0 = A.seed_lo; sr.k1 = A.seed_hi; sr.step = A.step;
-        sr.b = SLOTS ? (uint32_t)(pg_cur / H) : (uint32_t)pb;   // the request's slot in the state
+        if constexpr (SLOTS) sr.b = (uint32_t)(S.pg[st] / H);   // the request's slot in the state
+        else sr.b = (uint32_t)pb;
         sr.h = (uint32_t)ph;
         static_for<0, kBlocks>([&](auto bc) {
             constexpr int b = decltype(bc)::value;
@@ -778,7 +803,6 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
         fence_proxy_async_smem();   // the stage's new bytes are read by the bulk store
 
         p_prev = p;
-        if constexpr (SLOTS) pg_prev = pg_cur;
         st_prev = st;
         alpha_s = alpha_n;
         beta_s = beta_n;
@@ -792,14 +816,17 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
     asm volatile("griddepcontrol.launch_dependents;");
     __syncthreads();
     if (p_prev >= 0) {
-        if (tid == 0 && (SLOTS ? pg_prev >= 0 : true)) {
-            bulk_s2g(A.pages + (size_t)(SLOTS ? pg_prev : p_prev) * F.page_bytes, stages + st_prev * A.stage_bytes, A.store_bytes);
+        if (tid == 0 && (SLOTS ? S.pg[st_prev] >= 0 : true)) {
+            bulk_s2g(A.pages + (size_t)(SLOTS ? S.pg[st_prev] : p_prev) * F.page_bytes, stages + st_prev * A.stage_bytes, A.store_bytes);
             bulk_commit();
         }
         if (warp == kWarps - 1)
-            write_o(S.red_o[(it - 1) & 1], A, p_prev, lane, S.cpg[(it - 1) & 1], col_scales, SLOTS && pg_prev < 0);
+            write_o(S.red_o[(it - 1) & 1], A, p_prev, lane, S.cpg[(it - 1) & 1], col_scales, SLOTS && S.bad[(it - 1) & 1]);
     }
-    if (tid == 0) bulk_wait<0>();
+    if (tid == 0) {
+        bulk_wait<0>();
+        if constexpr (SLOTS) cp_async_wait();   // no copy outlives the CTA
+    }
 }
 
 template <class FMT>
