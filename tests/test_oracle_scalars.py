@@ -1,6 +1,6 @@
 """Pins of the oracle's scalar building blocks against things other than itself:
 library routines (numpy's IEEE binary16 conversion), exact rational arithmetic
-(fractions.Fraction), and the published known-answer vectors of Philox-4x32-10.
+(fractions.Fraction), and Philox-4x32-10 against cuRAND's implementation.
 """
 from fractions import Fraction
 
@@ -81,21 +81,71 @@ def test_div_rz_exact_quotients_are_kept():
 
 
 # --------------------------------------------------------------- Philox ----
-# Known-answer vectors published with the Random123 library (Salmon et al.,
-# SC'11), file kat_vectors, generator philox4x32 with 10 rounds.
-PHILOX_KAT = [
-    ((0x00000000, 0x00000000, 0x00000000, 0x00000000), (0x00000000, 0x00000000),
-     (0x6627e8d5, 0xe169c58d, 0xbc57ac4c, 0x9b00dbd8)),
-    ((0xffffffff, 0xffffffff, 0xffffffff, 0xffffffff), (0xffffffff, 0xffffffff),
-     (0x408f276d, 0x41c83b0e, 0xa20bc7c6, 0x6d5451fd)),
-    ((0x243f6a88, 0x85a308d3, 0x13198a2e, 0x03707344), (0xa4093822, 0x299f31d0),
-     (0xd16cfe09, 0x94fdcceb, 0x5001e420, 0x24126ea1)),
-]
+# Philox-4x32-10 (Salmon, Moraes, Dror, Shaw, SC'11) pinned to an independent
+# implementation: cuRAND's host generator CURAND_RNG_PSEUDO_PHILOX4_32_10
+# (NVIDIA's CUDA library, run on the CPU).  With seed s it emits block m
+# (4 words) = Philox(counter = (x, y, z, 0), key = (s mod 2^32, s >> 32))
+# where m = (y * 2^32 + x) * 65536 + z: 65,536 interleaved subsequences.  A
+# generator offset of 4m starts the stream at block m, which reaches the
+# first three counter words; the fourth is pinned on the GPU
+# (tests/test_gpu_philox.py, cuRAND's device API).
+_CURAND = None
 
 
-@pytest.mark.parametrize("ctr,key,expect", PHILOX_KAT)
-def test_philox_known_answers(ctr, key, expect):
-    assert tuple(int(x) for x in O.philox4x32_10(ctr, key)) == expect
+def _curand():
+    global _CURAND
+    if _CURAND is None:
+        import ctypes
+        import glob
+        import os
+        import torch
+        paths = glob.glob(os.path.join(os.path.dirname(torch.__file__), "..", "nvidia", "curand", "lib",
+                                       "libcurand.so*")) + glob.glob("/usr/local/cuda/lib64/libcurand.so*")
+        for path in paths:
+            try:
+                _CURAND = ctypes.CDLL(path)
+                break
+            except OSError:
+                continue
+        if _CURAND is None:
+            pytest.skip("libcurand not found")
+    return _CURAND
+
+
+def _curand_block(seed, x, y, z):
+    import ctypes
+    lib = _curand()
+    gen = ctypes.c_void_p()
+    assert lib.curandCreateGeneratorHost(ctypes.byref(gen), 161) == 0   # PHILOX4_32_10
+    try:
+        assert lib.curandSetPseudoRandomGeneratorSeed(gen, ctypes.c_ulonglong(seed)) == 0
+        block = ((y << 32) + x) * 65536 + z
+        assert lib.curandSetGeneratorOffset(gen, ctypes.c_ulonglong(4 * block)) == 0
+        out = (ctypes.c_uint32 * 4)()
+        assert lib.curandGenerate(gen, out, ctypes.c_size_t(4)) == 0
+        return tuple(int(v) for v in out)
+    finally:
+        lib.curandDestroyGenerator(gen)
+
+
+def test_philox_matches_curand():
+    rng = np.random.default_rng(20260511)
+    for _ in range(48):
+        seed = int(rng.integers(0, 2**63)) * 2 + int(rng.integers(0, 2))
+        x = int(rng.integers(0, 2**32))
+        y = int(rng.integers(0, 2**13))
+        z = int(rng.integers(0, 65536))
+        key = np.array([seed & 0xFFFFFFFF, seed >> 32], np.uint32)
+        got = tuple(int(v) for v in O.philox4x32_10(np.array([x, y, z, 0], np.uint32), key))
+        assert got == _curand_block(seed, x, y, z), (seed, x, y, z)
+
+
+def test_philox_edges_match_curand():
+    for seed in (0, 2**64 - 1):
+        for x, y, z in ((0, 0, 0), (2**32 - 1, 0, 65535), (1, 1, 1)):
+            key = np.array([seed & 0xFFFFFFFF, seed >> 32], np.uint32)
+            got = tuple(int(v) for v in O.philox4x32_10(np.array([x, y, z, 0], np.uint32), key))
+            assert got == _curand_block(seed, x, y, z)
 
 
 # ------------------------------------------------- stochastic-rounding offsets
