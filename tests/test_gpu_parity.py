@@ -3,7 +3,7 @@ by element, on the same seeded inputs.
 
 Sizes: every format at B x H = 37 x 9 = 333 pages (more pages than resident
 CTAs, so the persistent grid wraps with a ragged tail), and the tiny GDN
-workload (1 x 4 pages) over its full 64-step trajectory.  The bar (the benchmark spec):
+workload (1 x 4 pages) over its full 64-step trajectory.  The bar:
 o and the dequantized state within rel-L2 1e-5, integer codes and packed words
 bit-identical except elements whose pre-rounding value lies within 1e-5 of a
 rounding boundary (counted), row scales bit-identical; the free-running

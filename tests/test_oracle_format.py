@@ -52,7 +52,7 @@ def test_state_memory_matches_the_pages_arithmetic():
     assert round(g["fp32_mib_per_request"] / g["packed_mib_per_request"], 2) == g["compression"]
     # DAMP's storage reduction is effective bits over 32: 1 - 9.9/32 = 69.1 %
     assert round(100 * (1 - g["damp_effective_bits"] / 32), 1) == g["damp_storage_reduction_pct"]
-    # this build's formats: bits per element including fp32 scales
+    # the library's formats: bits per element including fp32 scales
     for name, bits in (("stepquant6", 6.5), ("int8row", 8.25), ("stepquant4_kda", 4.5), ("damp", 9.21875)):
         assert O.page_bytes(_fmt(name)) * 8 / (128 * 128) == bits
 

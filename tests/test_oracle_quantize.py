@@ -3,7 +3,7 @@
 * brute force at d_k = d_v = 4: every code is the nearest point of the row's
   grid {z r : |z| <= qmax} (exhaustive search, exact rationals);
 * the absmax element of a row maps to +-qmax; zero rows and columns;
-* values already on the grid round-trip exactly (north_star invariant);
+* values already on the grid round-trip exactly (an invariant of the method);
 * reconstruction error within half a grid step;
 * the precision map on states whose ranking is known by construction.
 """
@@ -84,7 +84,7 @@ def test_quantizer_error_bound_and_dequantizer(name):
 
 @pytest.mark.parametrize("name", ["int8row", "damp"])
 def test_values_on_the_grid_round_trip_exactly(name):
-    """The benchmark spec: values already on the grid round-trip exactly through
+    """Values already on the grid round-trip exactly through
     quantize/dequantize (per-row formats; power-of-two row scales)."""
     fmt = O.format_from_spec(W.FORMATS[name])
     rng = np.random.default_rng(5)

@@ -5,7 +5,7 @@
   state is a running sum, not a buffer"), at d = 4 and d = 128, GDN and KDA;
 * canonical fp32 mode against fp64 mode (rel-L2 <= 1e-5 on o and on the
   pre-rounding state, every format, workload distributions);
-* invariants (north_star): alpha = 1, beta = 0 leaves the state unchanged;
+* invariants of the method: alpha = 1, beta = 0 leaves the state unchanged;
   unquantized fp32 state, alpha = beta = 1, |k| = 1, q = k reads out v;
 * closed forms: beta = 0 is pure decay, alpha = 0 leaves beta k v^T;
 * special cases: KDA with equal alphas == GDN, bit for bit; column scales
@@ -84,7 +84,7 @@ def test_f64_step_is_the_matrix_form_d4(groups, col, gate_vector, seed):
 
 def test_f64_step_is_the_pages_transposed_formula():
     """dev.to post: S <- S(I - k k^T) + v k^T with the state d_v x d_k
-    (alpha = beta = 1); this build's state is its transpose."""
+    (alpha = beta = 1); the library's state is its transpose."""
     fmt = O.make_format([(128, "int", 8)], col_scales=True)
     rng = np.random.default_rng(11)
     page, perm, q, k, v, _, _ = _random_case(fmt, rng, False)
@@ -140,7 +140,7 @@ def test_canonical_f32_matches_f64_d4(gate_vector):
 
 @pytest.mark.parametrize("name", ["stepquant6", "int8row", "stepquant4_kda"])
 def test_identity_step_leaves_the_state_unchanged(name):
-    """The benchmark spec invariant: alpha = 1, beta = 0 leaves the dequantized state
+    """Invariant: alpha = 1, beta = 0 leaves the dequantized state
     unchanged.  The row scale is re-derived from the row's absmax, so codes
     stay bit-identical and r moves by at most one ulp."""
     rng = np.random.default_rng(4)
@@ -172,7 +172,7 @@ def test_identity_step_damp_format():
 
 
 def test_unquantized_state_retrieves_v():
-    """The benchmark spec invariant: unquantized fp32 state, alpha = beta = 1,
+    """Invariant: unquantized fp32 state, alpha = beta = 1,
     |k| = 1: reading out at q = k returns v (exact in the fp64 definition;
     within the fp32 rounding bound in the canonical evaluation)."""
     fmt = O.make_format([(128, "fp32", 0)])
