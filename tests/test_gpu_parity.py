@@ -281,3 +281,34 @@ def test_custom_formats_match_oracle(fmt_name, monkeypatch):
         res = compare_pages(fmt, download(qs), expect, perm, (pages, x, seed, step, w.heads))
         assert res["pages_equal"] == res["pages"], (step, res)
         pages = expect
+
+
+def test_steps_captured_in_a_cuda_graph_match_eager_steps():
+    """Four decode steps captured into one CUDA graph (programmatic launches
+    become graph edges) and replayed give the pages and o of eager steps."""
+    w = _small("stepquant6", batch=6, heads=7, steps=4)
+    S = W.initial_state(w).numpy()
+    fmt, perm, pages = oracle_quantize(w, S)
+    qa, qb = make_state(w), make_state(w)
+    upload(qa, perm, pages)
+    upload(qb, perm, pages)
+    xs = [{k: v.cuda() for k, v in W.step_inputs(w, t).items()} for t in range(4)]
+    o_eager = [qa.step(x["q"], x["k"], x["v"], x["alpha"], x["beta"], seed=3, step=t) for t, x in enumerate(xs)]
+    torch.cuda.synchronize()
+    o_graph = [torch.empty_like(o_eager[0]) for _ in range(4)]
+    stream = torch.cuda.Stream()
+    B.stq_decode_step(qb.state, xs[0]["q"], xs[0]["k"], xs[0]["v"], xs[0]["alpha"], xs[0]["beta"],
+                      torch.empty_like(o_eager[0]), 0, 0, stream)   # first launch outside the capture
+    torch.cuda.synchronize()
+    upload(qb, perm, pages)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for t, x in enumerate(xs):
+            B.stq_decode_step(qb.state, x["q"], x["k"], x["v"], x["alpha"], x["beta"], o_graph[t], 3, t,
+                              torch.cuda.current_stream())
+    upload(qb, perm, pages)          # the capture ran nothing: start the replay from the same pages
+    g.replay()
+    torch.cuda.synchronize()
+    for t in range(4):
+        assert torch.equal(o_graph[t], o_eager[t]), t
+    assert torch.equal(qb.pages(), qa.pages())
