@@ -56,6 +56,8 @@ def lib():
         L.orc_step_f32.argtypes = [P, P, P, P, P, P, P, c_float, P, c_uint64, c_uint32,
                                    c_uint32, c_uint32, P, P]
         L.orc_step_f64.argtypes = [P, P, P, P, P, P, P, c_float, P, P]
+        L.orc_window_step_f32.argtypes = [P, P, P, P, P, P, c_int, c_int, P, P, P, P, c_float, P, c_uint64,
+                                          c_uint32, c_uint32, c_uint32, P]
         L.orc_pack_page.argtypes = [P, P, P]
         L.orc_unpack_page.argtypes = [P, P, P]
         L.orc_decode_step_pages.argtypes = [P, c_int, c_int, P, P, P, P, P, P, P, P,
@@ -184,6 +186,24 @@ def step_f32(fmt, page, perm, q, k, v, alpha, beta, seed=0, step=0, b=0, h=0,
                            _p(a), float(beta), _p(o), int(seed), int(step), int(b), int(h),
                            _p(tp), _p(mg)), "step_f32")
     return o, tp, mg
+
+
+def window_step_f32(fmt, page, perm, P, K, D, t, commit, q, k, v, alpha, beta, seed=0, step=0, b=0, h=0,
+                    want_margin=False):
+    """Per-window decode step t (0-based) on one page; P [d_k], K [W, d_k], D [W, d_v]
+    (float32, updated in place; page updated in place when commit).  Returns (o, margin)."""
+    perm = np.ascontiguousarray(perm, np.int32)
+    q, k, v = (np.ascontiguousarray(x, np.float32) for x in (q, k, v))
+    for arr in (P, K, D):
+        assert arr.dtype == np.float32 and arr.flags["C_CONTIGUOUS"]
+    a = _gate(fmt, alpha)
+    o = np.zeros(fmt.d_v, np.float32)
+    mg = np.zeros((fmt.d_k, fmt.d_v), np.float64) if (want_margin and commit) else None
+    st = page._struct()
+    _ok(lib().orc_window_step_f32(ctypes.byref(fmt), ctypes.byref(st), _p(perm), _p(P), _p(K), _p(D), int(t),
+                                  int(commit), _p(q), _p(k), _p(v), _p(a), float(beta), _p(o), int(seed),
+                                  int(step), int(b), int(h), _p(mg)), "window_step_f32")
+    return o, mg
 
 
 def step_f64(fmt, page, perm, q, k, v, alpha, beta):

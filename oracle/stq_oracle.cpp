@@ -529,6 +529,98 @@ extern "C" int orc_step_f32(const orc_format *f, orc_page *page, const int32_t *
 /* decode step: plain definition in fp64                                    */
 /* ------------------------------------------------------------------------ */
 
+/* ------------------------------------------------------------------------ */
+/* per-window decode                                                        */
+/* ------------------------------------------------------------------------ */
+
+/* x . y over n channels (natural order) in the canonical order: lane l holds
+ * the fma chain over channels 4l .. 4l+3 from +0; the n / 4 lane partials
+ * (a power of two) are combined by an xor butterfly, offsets n/8 .. 1 */
+static float lane_dot(const float *x, const float *y, int n)
+{
+    const int lanes = n / 4;
+    std::vector<float> p(lanes), nx(lanes);
+    for (int l = 0; l < lanes; ++l) {
+        float acc = 0.0f;
+        for (int i = 0; i < 4; ++i) acc = std::fmaf(x[4 * l + i], y[4 * l + i], acc);
+        p[l] = acc;
+    }
+    for (int off = lanes / 2; off >= 1; off /= 2) {
+        for (int l = 0; l < lanes; ++l) nx[l] = p[l] + p[l ^ off];
+        p.swap(nx);
+    }
+    return p[0];
+}
+
+extern "C" int orc_window_step_f32(const orc_format *f, orc_page *page, const int32_t *perm,
+                                   float *P, float *K, float *D, int t, int commit,
+                                   const float *q, const float *k, const float *v,
+                                   const float *alpha, float beta, float *o_out,
+                                   uint64_t seed, uint32_t step, uint32_t b, uint32_t h,
+                                   double *margin_out)
+{
+    if (orc_format_check(f) != 0 || !page || !perm || !P || !K || !D || t < 0 || !q || !k || !v ||
+        !alpha || !o_out)
+        return -1;
+    const int d_k = f->d_k, d_v = f->d_v;
+    if (d_k % 4 != 0) return -1;
+    std::vector<float> ic(d_v), T0((size_t)d_k * d_v), wk(d_k), wq(d_k), u(d_v), ot(d_v);
+    for (int j = 0; j < d_v; ++j) ic[j] = f->col_scales ? 1.0f / page->c[j] : 1.0f;
+
+    /* decay: the window's cumulative product and the earlier entries' keys */
+    for (int kap = 0; kap < d_k; ++kap) {
+        const float al = f->gate_vector ? alpha[kap] : alpha[0];
+        P[kap] = P[kap] * al;
+        for (int tau = 0; tau < t; ++tau) K[(size_t)tau * d_k + kap] = K[(size_t)tau * d_k + kap] * al;
+    }
+    /* the fixed page in column-normalised units, undecayed: T0 = z r (FP16: h) */
+    for (int s = 0; s < d_k; ++s) {
+        const float rs = (orc_row_kind(f, s) == ORC_KIND_INT) ? page->r[s] : 1.0f;
+        for (int j = 0; j < d_v; ++j) T0[(size_t)s * d_v + j] = element_value(f, page, s, j) * rs;
+    }
+    for (int kap = 0; kap < d_k; ++kap) {
+        wk[kap] = P[kap] * k[kap];
+        wq[kap] = P[kap] * q[kap];
+    }
+    /* prediction from the page and the earlier entries */
+    column_sum(f, perm, wk.data(), T0.data(), u.data());
+    for (int tau = 0; tau < t; ++tau) {
+        const float a = lane_dot(K + (size_t)tau * d_k, k, d_k);
+        for (int j = 0; j < d_v; ++j) u[j] = std::fmaf(a, D[(size_t)tau * d_v + j], u[j]);
+    }
+    /* this step's entry */
+    for (int j = 0; j < d_v; ++j) {
+        const float e = v[j] * ic[j] - u[j];
+        D[(size_t)t * d_v + j] = beta * e;
+    }
+    for (int kap = 0; kap < d_k; ++kap) K[(size_t)t * d_k + kap] = k[kap];
+    /* readout from the page and every entry */
+    column_sum(f, perm, wq.data(), T0.data(), ot.data());
+    for (int tau = 0; tau <= t; ++tau) {
+        const float bq = lane_dot(K + (size_t)tau * d_k, q, d_k);
+        for (int j = 0; j < d_v; ++j) ot[j] = std::fmaf(bq, D[(size_t)tau * d_v + j], ot[j]);
+    }
+    for (int j = 0; j < d_v; ++j) o_out[j] = f->col_scales ? page->c[j] * ot[j] : ot[j];
+
+    if (commit) {
+        /* T = P T0 + sum_tau K[tau] D[tau]^T, requantized once */
+        std::vector<float> row(d_v);
+        for (int s = 0; s < d_k; ++s) {
+            const int kap = perm[s];
+            for (int j = 0; j < d_v; ++j) {
+                float x = P[kap] * T0[(size_t)s * d_v + j];
+                for (int tau = 0; tau <= t; ++tau)
+                    x = std::fmaf(K[(size_t)tau * d_k + kap], D[(size_t)tau * d_v + j], x);
+                row[j] = x;
+            }
+            requant_row(f, s, row.data(), page, seed, step, b, h, f->stochastic,
+                        margin_out ? margin_out + (size_t)s * d_v : nullptr);
+        }
+        for (int kap = 0; kap < d_k; ++kap) P[kap] = 1.0f;
+    }
+    return 0;
+}
+
 extern "C" int orc_step_f64(const orc_format *f, const orc_page *page, const int32_t *perm,
                             const float *q, const float *k, const float *v,
                             const float *alpha, float beta, double *o_out, double *Sp_out)

@@ -107,6 +107,35 @@ int orc_step_f64(const orc_format *f, const orc_page *page, const int32_t *perm,
                  const float *q, const float *k, const float *v,
                  const float *alpha, float beta, double *o_out, double *Sp_out);
 
+/* ---- per-window decode (LeapQuant's per-window quantization) ------------
+ * Within a window of steps the packed page stays fixed; each step's output
+ * comes from it together with a buffer of high-precision updates, and the
+ * state is requantized once, at the window's last step (the LeapQuant
+ * abstract on the paper-cards page: per-window quantization).  Buffer of one page (caller-owned, fp32):
+ *   P[d_k]       cumulative decay per key channel (natural order), 1 at the
+ *                window's start;
+ *   K[W][d_k]    entry tau's key, decayed to the current step (natural order);
+ *   D[W][d_v]    entry tau's delta beta_tau e_tau (column-normalised units).
+ * Step t (0-based position in the window) decays P and K[0..t-1] by alpha,
+ * predicts u = S0^T (P k) + sum_{tau<t} (K[tau] . k) D[tau], sets
+ * D[t] = beta (v / c - u), K[t] = k, and reads out
+ * o = c (S0^T (P q) + sum_{tau<=t} (K[tau] . q) D[tau]), where S0 is the page
+ * (column-normalised, undecayed).  With commit != 0 the state
+ * T = P S0 + sum_tau K[tau] D[tau]^T is then requantized into the page
+ * (as orc_step_f32 requantizes) and P is reset to 1.  The canonical fp32
+ * order: the S0 products are the column sums of orc_step_f32 with row
+ * weights RN(P k) and RN(P q) on T0 = z r (FP16 rows: h); a buffer dot
+ * product is 4-channel fma chains per lane (d_k / 4 lanes) combined by an
+ * xor butterfly; the buffer terms are added by fmaf in entry order; the
+ * committed element is an fma chain from RN(P T0) over the entries in
+ * order.  margin_out as orc_step_f32 (commit only). */
+int orc_window_step_f32(const orc_format *f, orc_page *page, const int32_t *perm,
+                        float *P, float *K, float *D, int t, int commit,
+                        const float *q, const float *k, const float *v,
+                        const float *alpha, float beta, float *o_out,
+                        uint64_t seed, uint32_t step, uint32_t b, uint32_t h,
+                        double *margin_out);
+
 /* ---- packed byte layout (d_k = d_v = 128, row groups multiples of 16) ---- */
 int orc_pack_page(const orc_format *f, const orc_page *p, uint8_t *bytes);
 int orc_unpack_page(const orc_format *f, const uint8_t *bytes, orc_page *p);

@@ -18,7 +18,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "stq_oracle.cpp")
 HDR = os.path.join(ROOT, "oracle", "stq_oracle.h")
 PIN_FILES = ["tests/test_oracle_scalars.py", "tests/test_oracle_format.py",
-             "tests/test_oracle_quantize.py", "tests/test_oracle_step.py"]
+             "tests/test_oracle_quantize.py", "tests/test_oracle_step.py", "tests/test_oracle_window.py"]
 
 MUTANTS = {
     "error sign": ("e[j] = v[j] * ic[j] - u[j];", "e[j] = v[j] * ic[j] + u[j];"),
@@ -46,6 +46,19 @@ MUTANTS = {
                           "uint32_t h16 = (j & 1) ? (word >> 16) : (word & 0xFFFFu);"),
     "column absmax over one row": ("float a = std::fabs(S_nat[(size_t)kap * d_v + j]);",
                                    "float a = std::fabs(S_nat[(size_t)j]);"),
+    "window key decay dropped": ("K[(size_t)tau * d_k + kap] = K[(size_t)tau * d_k + kap] * al;",
+                                 "K[(size_t)tau * d_k + kap] = K[(size_t)tau * d_k + kap];"),
+    "window prediction with q": ("const float a = lane_dot(K + (size_t)tau * d_k, k, d_k);",
+                                 "const float a = lane_dot(K + (size_t)tau * d_k, q, d_k);"),
+    "window delta without beta": ("D[(size_t)t * d_v + j] = beta * e;", "D[(size_t)t * d_v + j] = e;"),
+    "window readout skips this step": ("for (int tau = 0; tau <= t; ++tau) {\n        const float bq",
+                                       "for (int tau = 0; tau < t; ++tau) {\n        const float bq"),
+    "window commit drops the decay": ("float x = P[kap] * T0[(size_t)s * d_v + j];",
+                                      "float x = T0[(size_t)s * d_v + j];"),
+    "window decay not reset": ("for (int kap = 0; kap < d_k; ++kap) P[kap] = 1.0f;",
+                               "for (int kap = 0; kap < d_k; ++kap) P[kap] = P[kap];"),
+    "window butterfly half": ("for (int off = lanes / 2; off >= 1; off /= 2) {",
+                              "for (int off = lanes / 2; off >= 2; off /= 2) {"),
 }
 
 
