@@ -570,7 +570,8 @@ extern "C" int orc_window_step_f32(const orc_format *f, orc_page *page, const in
     /* decay: the window's cumulative product and the earlier entries' keys */
     for (int kap = 0; kap < d_k; ++kap) {
         const float al = f->gate_vector ? alpha[kap] : alpha[0];
-        P[kap] = P[kap] * al;
+        const float p0 = (t == 0) ? 1.0f : P[kap];   /* a window starts from no decay */
+        P[kap] = p0 * al;
         for (int tau = 0; tau < t; ++tau) K[(size_t)tau * d_k + kap] = K[(size_t)tau * d_k + kap] * al;
     }
     /* the fixed page in column-normalised units, undecayed: T0 = z r (FP16: h) */

@@ -112,8 +112,8 @@ int orc_step_f64(const orc_format *f, const orc_page *page, const int32_t *perm,
  * comes from it together with a buffer of high-precision updates, and the
  * state is requantized once, at the window's last step (the LeapQuant
  * abstract on the paper-cards page: per-window quantization).  Buffer of one page (caller-owned, fp32):
- *   P[d_k]       cumulative decay per key channel (natural order), 1 at the
- *                window's start;
+ *   P[d_k]       cumulative decay per key channel (natural order); taken as
+ *                1 at the window's first step (t = 0), whatever it holds;
  *   K[W][d_k]    entry tau's key, decayed to the current step (natural order);
  *   D[W][d_v]    entry tau's delta beta_tau e_tau (column-normalised units).
  * Step t (0-based position in the window) decays P and K[0..t-1] by alpha,

@@ -57,6 +57,8 @@ MUTANTS = {
                                       "float x = T0[(size_t)s * d_v + j];"),
     "window decay not reset": ("for (int kap = 0; kap < d_k; ++kap) P[kap] = 1.0f;",
                                "for (int kap = 0; kap < d_k; ++kap) P[kap] = P[kap];"),
+    "window start keeps the old decay": ("const float p0 = (t == 0) ? 1.0f : P[kap];",
+                                         "const float p0 = P[kap];"),
     "window butterfly half": ("for (int off = lanes / 2; off >= 1; off /= 2) {",
                               "for (int off = lanes / 2; off >= 2; off /= 2) {"),
 }

@@ -244,3 +244,18 @@ def test_zero_gate_forgets_the_window_so_far():
     assert not rec[2][1].any() and not rec[2][2][:2].any()
     S_ref = _evolve64(S2, steps[3:])
     assert _rel_l2(rec[3][0], S_ref[0][0]) <= 1e-5
+
+
+def test_first_step_of_a_window_reads_no_decay():
+    """At t = 0 the cumulative decay starts from one whatever the buffer holds."""
+    w, fmt, perm, page = _workload("stepquant4_kda")
+    (q, k, v, alpha, beta), = _inputs(w, 5, 1)
+    outs = []
+    for P0 in (np.ones(fmt.d_k, np.float32), np.full(fmt.d_k, 7.5, np.float32)):
+        P = P0.copy()
+        K = np.zeros((2, fmt.d_k), np.float32)
+        D = np.zeros((2, fmt.d_v), np.float32)
+        o, _ = O.window_step_f32(fmt, page.copy(), perm, P, K, D, 0, False, q, k, v, alpha, beta)
+        outs.append((o, P))
+    np.testing.assert_array_equal(outs[0][0], outs[1][0])
+    np.testing.assert_array_equal(outs[1][1], np.atleast_1d(alpha).astype(np.float32) * np.ones(fmt.d_k, np.float32))
