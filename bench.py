@@ -49,6 +49,24 @@ def algorithmic_bytes_per_page(spec):
     return b
 
 
+def window_bytes_per_page(spec, window):
+    """Bytes one page-step of the per-window path must move, averaged over a
+    window of ``window`` steps (the last one commits).  Every step reads the
+    page (codes, r, c), q, k, v, the gate(s), beta and (t > 0) the buffer's P,
+    K[0..t-1], D[0..t-1]; it writes o and, unless it commits, P', K[0..t] and
+    D[t]; the committing step writes the requantized codes and r instead."""
+    code = sum(rows * 128 * (16 if kind == "fp16" else bits) // 8 for rows, kind, bits in spec["groups"])
+    n_int = sum(rows for rows, kind, _ in spec["groups"] if kind == "int")
+    page_read = code + 4 * n_int + (512 if spec["col_scales"] else 0)
+    inputs = 3 * 512 + (512 if spec["gate_vector"] else 4) + 4
+    total = 0
+    for t in range(window):
+        read = page_read + inputs + (512 + 1024 * t if t > 0 else 0)
+        write = 512 + (code + 4 * n_int if t == window - 1 else 512 + 512 * (t + 1) + 512)
+        total += read + write
+    return total / window
+
+
 def kernel_source_hash():
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "linear_attention_recurrent_delta_b200", "csrc")
@@ -237,6 +255,68 @@ def run_gpu(w, steps, warmup, rank, world, sample_clocks=True, e2e_steps=64, pag
             "e2e_steps": e2e_steps}
 
 
+def run_window(w, window, steps, warmup, rank, world):
+    """Per-window decode steps (stq_window_step), t cycling 0 .. window-1 with
+    a commit at window-1; steps and warmup are rounded up to whole windows.
+    Returns the device time of the timed steps (max over ranks) and the mean
+    time of each window position from a second, per-launch-timed pass."""
+    from linear_attention_recurrent_delta_b200 import binding as B
+    dev = torch.device("cuda", torch.cuda.current_device())
+    wr = R.rank_workload(w, rank)
+    qs = B.QuantizedState(wr.format, wr.batch, wr.heads, device=dev)
+    S = W.initial_state(wr, device=dev)
+    qs.calibrate_and_quantize(S)
+    del S
+    nbuf = B.stq_window_buffer_bytes(qs.state, window)
+    buf_raw = torch.empty(nbuf + 256, dtype=torch.uint8, device=dev)
+    off = (-buf_raw.data_ptr()) % 256
+    buf = buf_raw[off:off + nbuf]
+    n_in = min(wr.steps, 16)
+    inputs = [W.step_inputs(wr, t, device=dev) for t in range(n_in)]
+    o = torch.empty(wr.batch, wr.heads, 128, device=dev)
+    seed = W.sr_seed(wr)
+    stream = torch.cuda.current_stream()
+    steps = -(-steps // window) * window
+    warmup = -(-max(warmup, 3) // window) * window
+
+    def step(i):
+        x = inputs[i % n_in]
+        t = i % window
+        B.stq_window_step(qs.state, buf, window, t, t == window - 1, x["q"], x["k"], x["v"], x["alpha"], x["beta"],
+                          o, seed, i, stream)
+
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for i in range(steps):
+        step(warmup + i)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(ev0.elapsed_time(ev1), world)
+    # per position: an event pair around each launch (this pass only)
+    reps = max(1, min(50, steps // window))
+    per_t = [0.0] * window
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(reps * window)]
+    for i in range(reps * window):
+        evs[i][0].record(stream)
+        step(warmup + steps + i)
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    for i in range(reps * window):
+        per_t[i % window] += evs[i][0].elapsed_time(evs[i][1]) / reps
+    status = B.stq_device_status(qs.state)
+    if status != B.STQ_OK:
+        raise RuntimeError("device status: %s" % B.stq_status_string(status))
+    barrier(world)
+    del qs, inputs, buf_raw
+    torch.cuda.empty_cache()
+    return {"ms": ms, "steps": steps, "per_t_ms": per_t}
+
+
 class OracleSample:
     """The CPU oracle (single thread, as written) stepping a sample of the
     workload's pages: the first ``n_pages`` pages of a batch whose fp32 state
@@ -353,6 +433,8 @@ def main():
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling)")
     ap.add_argument("--paged", action="store_true",
                     help="with --profile: step through the slot table (stq_decode_step_slots)")
+    ap.add_argument("--window", type=int, default=0,
+                    help="with --profile: per-window steps (stq_window_step) of this window length")
     ap.add_argument("--profile", action="store_true",
                     help="decode steps only: no clock sampling, e2e, CPU baseline or other workloads")
     args = ap.parse_args()
@@ -401,6 +483,13 @@ def main():
     if rank == 0:
         build_mod.build()
     barrier(world)
+    if args.profile and args.window:
+        r = run_window(w, args.window, args.steps, args.warmup, rank, world)
+        if rank == 0:
+            print(json.dumps({"workload": w.name, "batch": w.batch, "window": args.window,
+                              "ms_per_step": r["ms"] / r["steps"], "per_t_ms": r["per_t_ms"]}))
+        R.finish(world)
+        return
     if args.profile:
         res = run_gpu(w, args.steps, args.warmup, rank, world, sample_clocks=False, e2e_steps=0, paged=args.paged)
         if rank == 0:
@@ -421,6 +510,16 @@ def main():
         paged = {"value": R.aggregate_rate(w.pages, world, args.steps, r["ms"]), "unit": UNIT,
                  "entry_point": "stq_decode_step_slots", "table": "random permutation of all %d slots" % w.batch,
                  "frac_of_%s_peak" % peak_kind: bpp * w.pages * args.steps / (r["ms"] / 1000.0) / 1e9 / peak}
+
+    windows = {}
+    if not args.only:
+        for wl in (4, 8, 16):
+            r = run_window(w, wl, max(400, args.steps // 5), args.warmup, rank, world)
+            b = window_bytes_per_page(spec, wl)
+            gbs = b * w.pages * r["steps"] / (r["ms"] / 1000.0) / 1e9
+            windows["W%d" % wl] = {"value": R.aggregate_rate(w.pages, world, r["steps"], r["ms"]), "unit": UNIT,
+                                   "hbm_gbs": gbs, "frac_of_%s_peak" % peak_kind: gbs / peak,
+                                   "bytes_per_head_step": b, "ms_per_position": r["per_t_ms"]}
 
     others = {}
     if not args.only:
@@ -463,10 +562,12 @@ def main():
                          if cpu_v else None),
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"],
                 "steps": res["e2e_steps"], "entry_point": "stq_decode_step_host"},
-        "gpu_launches": args.steps * world,   # one decode_kernel launch per step and rank
+        "gpu_launches": args.steps * world,   # one decode_kernel launch per step and rank (timed region)
         "clocks": res["clocks"],
         "other_workloads": others,
         "paged_step": paged,
+        "window_decode": ({"entry_point": "stq_window_step", "kernel": "stq::window_kernel",
+                           "windows": windows} if windows else None),
     }
     print(json.dumps(line))
     R.finish(world)

@@ -97,7 +97,9 @@ size_t stq_state_bytes(const stq_format *f, int batch, int heads);
 /* Bind a caller-owned device buffer (>= stq_state_bytes, 256-byte aligned)
  * to a new host descriptor.  Touches no device memory; the state holds
  * nothing valid until stq_calibrate (or a caller-written map) and
- * stq_quantize_state.  Errors: INVALID_ARG (nulls, batch/heads < 1),
+ * stq_quantize_state.  stq_quantize_state clears the status word; a caller
+ * that writes the map and pages itself zeroes the 256-byte header first (or
+ * calls stq_device_status with clear).  Errors: INVALID_ARG (nulls, batch/heads < 1),
  * UNSUPPORTED (format), MISALIGNED, BUFFER_TOO_SMALL. */
 stq_status stq_state_alloc(const stq_format *f, int batch, int heads,
                            void *d_buf, size_t buf_bytes, stq_state **out);
@@ -197,6 +199,47 @@ stq_status stq_decode_step_slots(stq_state *s, const int32_t *d_slots, int n_row
  * a request's state out (a checkpoint, a preemption) and back in with a
  * plain device copy.  Errors: INVALID_ARG (null state, slot out of range). */
 stq_status stq_request_pages(const stq_state *s, int slot, size_t *offset, size_t *bytes);
+
+/* ---- per-window decode ---------------------------------------------------
+ * Per-window quantization (LeapQuant abstract, paper-cards page): within a
+ * window of W steps (1 <= W <= STQ_WINDOW_MAX) the packed pages stay fixed;
+ * each step's output comes from them together with a caller-owned fp32
+ * buffer of the window's updates, and the window's committing step
+ * requantizes every page once.
+ * Buffer: device, stq_window_buffer_bytes(s, W) bytes, 256-byte aligned,
+ * caller-owned, no initialisation needed; page (b, h) owns the
+ * 512 (1 + 2W) bytes at (b H + h) 512 (1 + 2W):
+ *   P[128]     cumulative decay of the window per key channel (natural order)
+ *   K[W][128]  entry tau's key, decayed to the latest step (natural order)
+ *   D[W][128]  entry tau's delta beta_tau (v_tau (1/c) - u_tau), divided by c
+ * Step t (0-based position in the window) of every page, with S0 the page
+ * (column-normalised, undecayed, stored row s = key channel perm[s]):
+ *   P' = (t > 0 ? P : 1) alpha;   K[tau] <- K[tau] alpha   (tau < t)
+ *   u = S0^T (P' k) + sum_{tau<t} (K[tau] . k) D[tau]
+ *   D[t] = beta (v / c - u);   K[t] = k
+ *   o = c (S0^T (P' q) + sum_{tau<=t} (K[tau] . q) D[tau])
+ * i.e. the gated delta rule run exactly from the page for t + 1 steps.  A
+ * step that does not commit writes P', K[0 .. t] and D[t] to the buffer and
+ * leaves the pages unchanged.  A committing step (commit != 0; required at
+ * t = W - 1, allowed at any t to end a window early) writes no buffer row;
+ * it requantizes T = P' S0 + sum_{tau<=t} K[tau] D[tau]^T into every page as
+ * stq_decode_step requantizes its updated state (same row scales, rounding
+ * and stochastic-rounding counter, with `step`), and the next step is a new
+ * window's t = 0, which reads nothing from the buffer.
+ * Inputs, layouts and alignment as stq_decode_step; the buffer may overlap
+ * neither the state nor an input or o.  Programmatic dependent launch as
+ * stq_decode_step.  Errors: INVALID_ARG (null pointer, W outside
+ * [1, STQ_WINDOW_MAX], t outside [0, W), t = W - 1 without commit, overlap),
+ * MISALIGNED, BUFFER_TOO_SMALL (buf_bytes below stq_window_buffer_bytes),
+ * CUDA; a bounded wait that ran out is reported by stq_device_status. */
+#define STQ_WINDOW_MAX 16
+
+/* Bytes of a window buffer for windows of W steps (0 on bad arguments). */
+size_t stq_window_buffer_bytes(const stq_state *s, int window);
+
+stq_status stq_window_step(stq_state *s, void *d_buf, size_t buf_bytes, int window, int t, int commit,
+                           const float *d_q, const float *d_k, const float *d_v, const float *d_alpha,
+                           const float *d_beta, float *d_o, uint64_t seed, uint32_t step, void *stream);
 
 /* Device staging bytes stq_decode_step_host needs (q, k, v, alpha, beta, o). */
 size_t stq_decode_io_bytes(const stq_state *s);

@@ -15,6 +15,7 @@ MAX_GROUPS = 8
 
 STQ_OK, STQ_ERR_INVALID_ARG, STQ_ERR_UNSUPPORTED, STQ_ERR_BUFFER_TOO_SMALL, \
     STQ_ERR_MISALIGNED, STQ_ERR_CUDA, STQ_ERR_DEVICE_TIMEOUT = range(7)
+STQ_WINDOW_MAX = 16   # steps in a window at most (include/stq.h)
 STQ_INT, STQ_FP16 = 0, 1
 
 
@@ -58,6 +59,8 @@ def lib():
         "stq_decode_step": (c_int, [P, P, P, P, P, P, P, c_uint64, c_uint32, P]),
         "stq_decode_step_slots": (c_int, [P, P, c_int, P, P, P, P, P, P, c_uint64, c_uint32, P]),
         "stq_request_pages": (c_int, [P, c_int, POINTER(c_size_t), POINTER(c_size_t)]),
+        "stq_window_buffer_bytes": (c_size_t, [P, c_int]),
+        "stq_window_step": (c_int, [P, P, c_size_t, c_int, c_int, c_int, P, P, P, P, P, P, c_uint64, c_uint32, P]),
         "stq_decode_io_bytes": (c_size_t, [P]),
         "stq_decode_step_host": (c_int, [P, P, P, P, P, P, P, P, c_size_t, c_uint64, c_uint32, P]),
         "stq_dequantize_state": (c_int, [P, P, P]),
@@ -191,6 +194,18 @@ def stq_request_pages(state, slot):
     return off.value, n.value
 
 
+def stq_window_buffer_bytes(state, window):
+    return lib().stq_window_buffer_bytes(state.handle, int(window))
+
+
+def stq_window_step(state, buf, window, t, commit, q, k, v, alpha, beta, o, seed=0, step=0, stream=None):
+    """Step t of a window of ``window`` steps (``buf``: uint8 device tensor of
+    stq_window_buffer_bytes); ``commit`` requantizes the pages."""
+    _check(lib().stq_window_step(state.handle, _ptr(buf), buf.numel() * buf.element_size(), int(window), int(t),
+                                 int(bool(commit)), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(o),
+                                 int(seed), int(step), _stream(stream)), "stq_window_step")
+
+
 def stq_decode_io_bytes(state):
     return lib().stq_decode_io_bytes(state.handle)
 
@@ -234,6 +249,9 @@ class QuantizedState:
         self.state = stq_state_alloc(self.fmt, batch, heads, self.view, nbytes)
         self.batch, self.heads = batch, heads
         self.layout = stq_state_layout(self.state)
+        # a fresh buffer holds whatever the allocator left there: clear the
+        # header (status word) and the precision map
+        self.view[:self.layout["pages_offset"]].zero_()
 
     def calibrate_and_quantize(self, S, row_weight=None, stream=None):
         stq_calibrate(self.state, S, row_weight, stream=stream)

@@ -252,6 +252,34 @@ stq_status stq_request_pages(const stq_state *s, int slot, size_t *offset, size_
     return STQ_OK;
 }
 
+size_t stq_window_buffer_bytes(const stq_state *s, int window) {
+    if (!s || window < 1 || window > STQ_WINDOW_MAX) return 0;
+    return (size_t)s->batch * s->heads * window_buffer_stride(window);
+}
+
+stq_status stq_window_step(stq_state *s, void *d_buf, size_t buf_bytes, int window, int t, int commit,
+                           const float *d_q, const float *d_k, const float *d_v, const float *d_alpha,
+                           const float *d_beta, float *d_o, uint64_t seed, uint32_t step, void *stream) {
+    if (!s || !d_buf) return STQ_ERR_INVALID_ARG;
+    if (window < 1 || window > STQ_WINDOW_MAX || t < 0 || t >= window || (t == window - 1 && !commit))
+        return STQ_ERR_INVALID_ARG;
+    stq_status st = check_step_args(s, s->batch, d_q, d_k, d_v, d_alpha, d_beta, d_o);
+    if (st != STQ_OK) return st;
+    if (!aligned(d_buf, 256)) return STQ_ERR_MISALIGNED;
+    const size_t need = stq_window_buffer_bytes(s, window);
+    if (buf_bytes < need) return STQ_ERR_BUFFER_TOO_SMALL;
+    const size_t n = (size_t)s->batch * s->heads;
+    const size_t vec = n * kD * sizeof(float), sc = n * sizeof(float);
+    const void *io[6] = {d_q, d_k, d_v, d_alpha, d_beta, d_o};
+    const size_t len[6] = {vec, vec, vec, s->fmt.gate_vector ? vec : sc, sc, vec};
+    if (overlaps(d_buf, need, s->base, state_span(s))) return STQ_ERR_INVALID_ARG;
+    for (int i = 0; i < 6; ++i)
+        if (overlaps(d_buf, need, io[i], len[i])) return STQ_ERR_INVALID_ARG;
+    cudaError_t err = launch_window(s, static_cast<uint8_t *>(d_buf), window, t, commit != 0, d_q, d_k, d_v,
+                                    d_alpha, d_beta, d_o, seed, step, true, static_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? STQ_OK : STQ_ERR_CUDA;
+}
+
 struct IoLayout {
     size_t q, k, v, alpha, beta, o, total, vec, na, sc;
 };

@@ -36,6 +36,12 @@ cudaError_t launch_decode(const stq_state *s, const float *q, const float *k, co
                           const float *alpha, const float *beta, float *o, uint64_t seed,
                           uint32_t step, int stall_first_wait, bool early_launch, const int32_t *slots,
                           int n_rows, cudaStream_t stream);
+// Per-window decode: step t of a window of `window` steps (commit: requantize
+// and store the pages); buf holds window_buffer_stride(window) bytes per page.
+size_t window_buffer_stride(int window);
+cudaError_t launch_window(const stq_state *s, uint8_t *buf, int window, int t, bool commit, const float *q,
+                          const float *k, const float *v, const float *alpha, const float *beta, float *o,
+                          uint64_t seed, uint32_t step, bool early_launch, cudaStream_t stream);
 cudaError_t launch_calibrate(const stq_state *s, const float *S, const float *row_weight,
                              double *workspace, cudaStream_t stream);
 size_t calibrate_workspace_bytes(int batch, int heads);

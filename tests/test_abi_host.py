@@ -177,3 +177,37 @@ def test_slot_step_and_request_pages_check_arguments(lib):
     assert off.value == pages_off.value + 2 * 3 * pb.value
     assert nb.value == 3 * pb.value
     lib.stq_state_free(h)
+
+
+def test_window_step_checks_arguments(lib):
+    fmt = B.format_from_spec(W.FORMATS["stepquant6"])
+    st, h = _alloc(lib, fmt, 2, 3)
+    assert st == B.STQ_OK
+    P = ctypes.c_void_p
+    base = 1 << 41
+    q, k, v, a, b, o = (P(base + i * (1 << 24)) for i in range(6))
+    for bad in (0, B.STQ_WINDOW_MAX + 1, -3):
+        assert lib.stq_window_buffer_bytes(h, bad) == 0
+    assert lib.stq_window_buffer_bytes(None, 4) == 0
+    assert lib.stq_window_buffer_bytes(h, 4) == 2 * 3 * 512 * 9
+    assert lib.stq_window_buffer_bytes(h, B.STQ_WINDOW_MAX) == 2 * 3 * 512 * (1 + 2 * B.STQ_WINDOW_MAX)
+    buf = 1 << 46
+    need = lib.stq_window_buffer_bytes(h, 4)
+
+    def call(window=4, t=0, commit=0, buf=buf, nbytes=need, q=q, o=o):
+        return lib.stq_window_step(h, P(buf) if buf else None, nbytes, window, t, commit, q, k, v, a, b, o, 0, 0,
+                                   None)
+
+    assert call(buf=0) == B.STQ_ERR_INVALID_ARG
+    assert call(window=0) == B.STQ_ERR_INVALID_ARG
+    assert call(window=B.STQ_WINDOW_MAX + 1) == B.STQ_ERR_INVALID_ARG
+    assert call(t=-1) == B.STQ_ERR_INVALID_ARG
+    assert call(t=4) == B.STQ_ERR_INVALID_ARG
+    assert call(t=3, commit=0) == B.STQ_ERR_INVALID_ARG      # a window's last step must commit
+    assert call(q=P(base + 4)) == B.STQ_ERR_MISALIGNED
+    assert call(buf=buf + 16) == B.STQ_ERR_MISALIGNED
+    assert call(nbytes=need - 1) == B.STQ_ERR_BUFFER_TOO_SMALL
+    assert call(buf=FAKE) == B.STQ_ERR_INVALID_ARG           # the buffer overlaps the state
+    assert call(buf=base) == B.STQ_ERR_INVALID_ARG           # the buffer overlaps q
+    assert lib.stq_window_step(None, P(buf), need, 4, 0, 0, q, k, v, a, b, o, 0, 0, None) == B.STQ_ERR_INVALID_ARG
+    lib.stq_state_free(h)
