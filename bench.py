@@ -566,7 +566,8 @@ def main():
         "clocks": res["clocks"],
         "other_workloads": others,
         "paged_step": paged,
-        "window_decode": ({"entry_point": "stq_window_step", "kernel": "stq::window_kernel",
+        "window_decode": ({"entry_point": "stq_window_step",
+                           "kernels": ["stq::window_step_kernel", "stq::window_commit_kernel"],
                            "windows": windows} if windows else None),
     }
     print(json.dumps(line))

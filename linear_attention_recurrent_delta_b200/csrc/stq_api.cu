@@ -275,8 +275,10 @@ stq_status stq_window_step(stq_state *s, void *d_buf, size_t buf_bytes, int wind
     if (overlaps(d_buf, need, s->base, state_span(s))) return STQ_ERR_INVALID_ARG;
     for (int i = 0; i < 6; ++i)
         if (overlaps(d_buf, need, io[i], len[i])) return STQ_ERR_INVALID_ARG;
+    const int stall = s->stall_first_wait;
+    s->stall_first_wait = 0;
     cudaError_t err = launch_window(s, static_cast<uint8_t *>(d_buf), window, t, commit != 0, d_q, d_k, d_v,
-                                    d_alpha, d_beta, d_o, seed, step, true, static_cast<cudaStream_t>(stream));
+                                    d_alpha, d_beta, d_o, seed, step, stall, true, static_cast<cudaStream_t>(stream));
     return err == cudaSuccess ? STQ_OK : STQ_ERR_CUDA;
 }
 

@@ -41,7 +41,8 @@ cudaError_t launch_decode(const stq_state *s, const float *q, const float *k, co
 size_t window_buffer_stride(int window);
 cudaError_t launch_window(const stq_state *s, uint8_t *buf, int window, int t, bool commit, const float *q,
                           const float *k, const float *v, const float *alpha, const float *beta, float *o,
-                          uint64_t seed, uint32_t step, bool early_launch, cudaStream_t stream);
+                          uint64_t seed, uint32_t step, int stall_first_wait, bool early_launch,
+                          cudaStream_t stream);
 cudaError_t launch_calibrate(const stq_state *s, const float *S, const float *row_weight,
                              double *workspace, cudaStream_t stream);
 size_t calibrate_workspace_bytes(int batch, int heads);

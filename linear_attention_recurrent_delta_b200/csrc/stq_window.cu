@@ -23,9 +23,9 @@
 // and requantizes it exactly as the decode step requantizes T'; it writes
 // nothing to the buffer (a window's first step reads none of it).
 //
-// Staging is the decode kernel's: one thread copies the page, the input rows
-// and the buffer rows a step reads into a shared-memory ring with
-// cp.async.bulk (no multicast), counted on an mbarrier with a bounded wait.
+// Staging is the decode kernel's: the page, the input rows and the buffer rows
+// a step reads are copied into a shared-memory ring with cp.async.bulk (no
+// multicast), counted on an mbarrier with a bounded wait.
 #include "stq_slices.cuh"
 
 namespace stq {
@@ -41,16 +41,18 @@ struct WindowArgs {
     float *o;
     uint8_t *buf;                 // window buffer, stride bytes per page
     uint32_t stride;
+    uint32_t buf_d_off;           // D inside a page's buffer: 512 (1 + W)
     int t;                        // position of this step in its window
     int n_pages, heads, n_stages;
     uint32_t stage_bytes;         // ring stride (a multiple of 128)
     uint32_t tx_bytes;            // bytes a stage receives
     uint32_t store_bytes;         // codes + r: the part of a page a commit rewrites
     uint32_t p_off, k_off, d_off; // buffer rows inside a stage
-    uint32_t buf_d_off;           // D inside a page's buffer: 512 (1 + W)
+    uint32_t scr_off;             // the stage's scratch (the warps' sums)
     uint32_t kd_bytes;            // per-warp key table of a commit (0 otherwise)
     uint32_t seed_lo, seed_hi, step;
     uint64_t wait_limit_ns;
+    int stall_first_wait;
 };
 
 struct WindowSmem {
@@ -60,16 +62,26 @@ struct WindowSmem {
     float qp[kWarps][kRowsPerWarp];         // RN(P' q)
     float pk[kWarps][kRowsPerWarp];         // P' (commit)
     float inv[kWarps][kRowsPerWarp];        // commit: row maxima, then requant multipliers
-    float red_u[2][kWarps][kD];             // per page parity and warp: chain sums of u
-    float red_o[2][kWarps][kD];             // the same for o
-    float da[2][kWindowMax];                // per page parity: K[tau] . k
-    float dq[2][kWindowMax];                // K[tau] . q
     uint64_t full[kWindowStages];           // stage-full barriers
+    uint64_t never;                         // a barrier nothing completes (test hook)
+    uint32_t phase[kWindowStages];          // parity of the stage's latest load
+    int issued[kWindowStages];              // the stage has had a load
+};
+
+// A stage's scratch, after the bytes its load brings: the warps' chain sums
+// of the page and the entries' dot products.
+struct WindowScratch {
+    float red_u[kWarps][kD];
+    float red_o[kWarps][kD];
+    float da[kWindowMax];                   // K[tau] . k
+    float dq[kWindowMax];                   // K[tau] . q
 };
 
 constexpr size_t kWindowFixedBytes = (sizeof(WindowSmem) + 127) / 128 * 128;
+constexpr uint32_t kScratchBytes = (uint32_t)((sizeof(WindowScratch) + 127) / 128 * 128);
 
-// Stage layout: page, q, k, v (, alpha), then (t > 0) P, K[0 .. t-1], D[0 .. t-1].
+// Stage layout: page, q, k, v (, alpha), then (t > 0) P, K[0 .. t-1],
+// D[0 .. t-1]; then the scratch.
 __device__ __forceinline__ void issue_window_stage(const DevFormat &F, const WindowArgs &A, uint8_t *dst, int p,
                                                    uint64_t *bar) {
     mbar_expect_tx(bar, A.tx_bytes);
@@ -124,11 +136,11 @@ __device__ __forceinline__ float4 fma4(float s, float4 d, float4 acc) {
 
 // This step's delta for columns 4l .. 4l+3: u from the tree and the earlier
 // entries, e = v (1/c) - u (two roundings), D[t] = RN(beta e).
-__device__ __forceinline__ float4 window_delta(const WindowSmem &S, int par, const float *v_s, const float *d_s,
+__device__ __forceinline__ float4 window_delta(const WindowScratch &X, const float *v_s, const float *d_s,
                                                const float *c_s, int t, float beta, int lane) {
-    float4 u = tree4(S.red_u[par], lane);
+    float4 u = tree4(X.red_u, lane);
     for (int tau = 0; tau < t; ++tau)
-        u = fma4(S.da[par][tau], *reinterpret_cast<const float4 *>(d_s + tau * kD + 4 * lane), u);
+        u = fma4(X.da[tau], *reinterpret_cast<const float4 *>(d_s + tau * kD + 4 * lane), u);
     float4 ic = make_float4(1.f, 1.f, 1.f, 1.f);
     if (c_s) {
         const float4 c = *reinterpret_cast<const float4 *>(c_s + 4 * lane);
@@ -141,34 +153,146 @@ __device__ __forceinline__ float4 window_delta(const WindowSmem &S, int par, con
 }
 
 // o of a page for columns 4l .. 4l+3: the tree, every entry's term, times c
-__device__ __forceinline__ void window_out(const WindowSmem &S, int par, const float *d_s, const float *c_s,
-                                           int t, float4 dt, float *o, int lane) {
-    float4 ot = tree4(S.red_o[par], lane);
+__device__ __forceinline__ float4 window_out(const WindowScratch &X, const float *d_s, const float *c_s, int t,
+                                             float4 dt, int lane) {
+    float4 ot = tree4(X.red_o, lane);
     for (int tau = 0; tau < t; ++tau)
-        ot = fma4(S.dq[par][tau], *reinterpret_cast<const float4 *>(d_s + tau * kD + 4 * lane), ot);
-    ot = fma4(S.dq[par][t], dt, ot);
+        ot = fma4(X.dq[tau], *reinterpret_cast<const float4 *>(d_s + tau * kD + 4 * lane), ot);
+    ot = fma4(X.dq[t], dt, ot);
     if (c_s) ot = mul4(*reinterpret_cast<const float4 *>(c_s + 4 * lane), ot);
-    *reinterpret_cast<float4 *>(o + 4 * lane) = ot;
+    return ot;
 }
 
-// Resident CTAs per SM the register budget is sized for: a step that does
-// not commit keeps no tile of the state in registers (4); a committing step
-// keeps T as the decode step does (2).
-template <bool COMMIT>
-constexpr int window_ctas_per_sm() { return COMMIT ? 2 : 4; }
+// This lane's row of the slice: block lane / 4, stored row s, r index rix.
+struct RowCtx {
+    int s, rix;
+    bool is_int, all_int;
+    float qmax, rcp_qmax;
+};
 
-// The per-page loop (same persistent walk and page -> (request, head) carry
-// as the decode kernel).  One CTA barrier per page, after the column sums;
-// everything of a page that needs the warps' sums happens after it.
+template <class FMT>
+__device__ __forceinline__ RowCtx row_ctx(const DevFormat &F, int warp, int lane) {
+    RowCtx R;
+    const int blk = lane >> 2;
+    R.s = 16 * blk + 4 * warp + (lane & 3);
+    int bits, rbase;
+    if constexpr (FMT::kRuntime) {
+        bits = F.blk_bits(blk);
+        rbase = F.blk_rbase(blk);
+        R.all_int = false;
+    } else {
+        bits = 0;
+        rbase = 0;
+#pragma unroll
+        for (int b = 0; b < kBlocks; ++b) {   // selects, not a table in local memory
+            if (b == blk) bits = FMT::width(b);
+            if (b < blk && FMT::width(b) != 16) rbase += 16;
+        }
+        R.all_int = true;
+        for (int b = 0; b < kBlocks; ++b) R.all_int = R.all_int && FMT::width(b) != 16;
+    }
+    R.is_int = bits != 16;
+    R.rix = rbase + 4 * warp + (lane & 3);
+    R.qmax = R.is_int ? (float)((1 << (bits - 1)) - 1) : 0.f;
+    R.rcp_qmax = R.is_int ? __frcp_rn(R.qmax) : 0.f;
+    return R;
+}
+
+// The page's pointers inside a stage.
+struct StageView {
+    const float *q, *k, *v, *al, *P, *K, *D, *c;
+    float *r;
+    WindowScratch *X;
+};
+
+__device__ __forceinline__ StageView stage_view(const DevFormat &F, const WindowArgs &A, uint8_t *stg,
+                                                bool col_scales) {
+    StageView V;
+    V.q = reinterpret_cast<const float *>(stg + F.page_bytes);
+    V.k = V.q + kD;
+    V.v = V.q + 2 * kD;
+    V.al = V.q + 3 * kD;
+    V.P = reinterpret_cast<const float *>(stg + A.p_off);
+    V.K = reinterpret_cast<const float *>(stg + A.k_off);
+    V.D = reinterpret_cast<const float *>(stg + A.d_off);
+    V.c = col_scales ? reinterpret_cast<const float *>(stg + F.c_off) : nullptr;
+    V.r = reinterpret_cast<float *>(stg + F.r_off);
+    V.X = reinterpret_cast<WindowScratch *>(stg + A.scr_off);
+    return V;
+}
+
+// The first phase of a page, per warp: the operands of this lane's row, the
+// entries' dot products (warp w: entries w, w + 4, ...) and one pass over the
+// warp's slices (dequantize, u's and o's chains), whose sums go to the
+// stage's scratch.  A commit also keeps P' and the row's decayed keys (kd:
+// this warp's [tau][32] table).
 template <class FMT, bool COMMIT>
-__global__ void __launch_bounds__(kThreads, window_ctas_per_sm<COMMIT>())
-window_kernel(const DevFormat F, const WindowArgs A) {
-    extern __shared__ __align__(128) uint8_t smem[];
-    WindowSmem &S = *reinterpret_cast<WindowSmem *>(smem);
-    float *kd_tab = reinterpret_cast<float *>(smem + kWindowFixedBytes);   // commit: [warp][tau][32]
-    uint8_t *stages = smem + kWindowFixedBytes + A.kd_bytes;
-    constexpr bool SR = FMT::kSr;
-    bool col_scales, gate_vector;
+__device__ __forceinline__ void window_first_phase(const DevFormat &F, const WindowArgs &A, WindowSmem &S,
+                                                   const uint8_t *stg, const StageView &V, const RowCtx &R,
+                                                   int kap, float alpha_s, bool gate_vector, int warp, int lane,
+                                                   float *kd) {
+    const int t = A.t;
+    {
+        const float al = gate_vector ? V.al[kap] : alpha_s;
+        const float pp = t > 0 ? __fmul_rn(V.P[kap], al) : al;
+        S.rw[warp][lane] = (R.all_int || R.is_int) ? V.r[R.rix] : 1.f;
+        S.kp[warp][lane] = __fmul_rn(pp, V.k[kap]);
+        S.qp[warp][lane] = __fmul_rn(pp, V.q[kap]);
+        if constexpr (COMMIT) {
+            S.pk[warp][lane] = pp;
+            for (int tau = 0; tau < t; ++tau) kd[tau * kRowsPerWarp + lane] = __fmul_rn(V.K[tau * kD + kap], al);
+            kd[t * kRowsPerWarp + lane] = V.k[kap];
+        }
+    }
+    {
+        const float4 al4 = gate_vector ? *reinterpret_cast<const float4 *>(V.al + 4 * lane)
+                                       : make_float4(alpha_s, alpha_s, alpha_s, alpha_s);
+        const float4 k4 = *reinterpret_cast<const float4 *>(V.k + 4 * lane);
+        const float4 q4 = *reinterpret_cast<const float4 *>(V.q + 4 * lane);
+        for (int tau = warp; tau <= t; tau += kWarps) {
+            float4 kk = k4;
+            if (tau < t) kk = mul4(*reinterpret_cast<const float4 *>(V.K + tau * kD + 4 * lane), al4);
+            const float a = lane_dot(kk, k4);
+            const float b = lane_dot(kk, q4);
+            if (lane == 0) {
+                V.X->da[tau] = a;
+                V.X->dq[tau] = b;
+            }
+        }
+    }
+    __syncwarp();   // the warp's rows' operands come from its own lanes
+
+    float2 cu[2][2], co[2][2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) cu[h][0] = cu[h][1] = co[h][0] = co[h][1] = make_float2(0.f, 0.f);
+    static_for<0, kBlocks>([&](auto bc) {
+        constexpr int b = decltype(bc)::value;
+        const float4 a4 = *reinterpret_cast<const float4 *>(&S.rw[warp][4 * b]);
+        const uint8_t *blk = stg + fmt_offset<FMT, b>(F);
+        Tile T;   // only block b of it is live
+        with_width<FMT, b>(F, [&](auto wc) {
+            constexpr int W = decltype(wc)::value;
+            dequant_slice<W, b>(blk, warp, lane, a4, T);
+        });
+        const float4 k4 = *reinterpret_cast<const float4 *>(&S.kp[warp][4 * b]);
+        const float4 q4 = *reinterpret_cast<const float4 *>(&S.qp[warp][4 * b]);
+        const float kv[4] = {k4.x, k4.y, k4.z, k4.w};
+        const float qv[4] = {q4.x, q4.y, q4.z, q4.w};
+        constexpr int h = b >> 2;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            cu[h][0] = __ffma2_rn(make_float2(kv[i], kv[i]), T[b][i][0], cu[h][0]);
+            cu[h][1] = __ffma2_rn(make_float2(kv[i], kv[i]), T[b][i][1], cu[h][1]);
+            co[h][0] = __ffma2_rn(make_float2(qv[i], qv[i]), T[b][i][0], co[h][0]);
+            co[h][1] = __ffma2_rn(make_float2(qv[i], qv[i]), T[b][i][1], co[h][1]);
+        }
+    });
+    store_readout(V.X->red_u[warp], lane, cu);
+    store_readout(V.X->red_o[warp], lane, co);
+}
+
+template <class FMT>
+__device__ __forceinline__ void format_flags(const DevFormat &F, bool &col_scales, bool &gate_vector) {
     if constexpr (FMT::kRuntime) {
         col_scales = F.col_scales != 0;
         gate_vector = F.gate_vector != 0;
@@ -176,52 +300,173 @@ window_kernel(const DevFormat F, const WindowArgs A) {
         col_scales = FMT::kCols;
         gate_vector = FMT::kGvec;
     }
+}
 
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int t = A.t;
-    if (tid == 0) {
-        for (int st = 0; st < A.n_stages; ++st) mbar_init(&S.full[st], 1);
+// Barriers, counters and the first loads of the ring (thread 0), then the
+// wait for the previous kernel on the stream (see the decode kernel).
+__device__ __forceinline__ void window_start(const DevFormat &F, const WindowArgs &A, WindowSmem &S,
+                                             uint8_t *stages) {
+    const int stride = (int)gridDim.x;
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < A.n_stages; ++st) {
+            mbar_init(&S.full[st], 1);
+            S.phase[st] = 0;
+            S.issued[st] = 0;
+        }
+        mbar_init(&S.never, 1);
         fence_mbar_init();
     }
     __syncthreads();
-    asm volatile("griddepcontrol.wait;" ::: "memory");   // see the decode kernel
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < A.n_stages; ++i) {
+            const int p = (int)blockIdx.x + i * stride;
+            if (p < A.n_pages) {
+                issue_window_stage(F, A, stages + i * A.stage_bytes, p, &S.full[i]);
+                S.issued[i] = 1;
+            }
+        }
+    }
+}
+
+// Loads in flight when the CTA stops early (a wait ran out) land before it
+// exits: thread 0 waits, bounded, for each stage's latest load.
+__device__ __forceinline__ void window_drain(const WindowArgs &A, WindowSmem &S) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < A.n_stages; ++st)
+            if (S.issued[st]) mbar_wait_bounded(&S.full[st], S.phase[st], A.wait_limit_ns);
+    }
+}
+
+// A step that does not commit: one CTA barrier per page, after the first
+// phase.  After it, thread c writes channel c's buffer rows (P', the decayed
+// keys, K[t] = k) and finishes column c: D[t] and o; one warp per page, in
+// turn, refills the previous page's stage.
+template <class FMT>
+__global__ void __launch_bounds__(kThreads, 4) window_step_kernel(const DevFormat F, const WindowArgs A) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    WindowSmem &S = *reinterpret_cast<WindowSmem *>(smem);
+    uint8_t *stages = smem + kWindowFixedBytes;
+    bool col_scales, gate_vector;
+    format_flags<FMT>(F, col_scales, gate_vector);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int t = A.t;
+    window_start(F, A, S, stages);
     const int stride = (int)gridDim.x;
     const int n = A.n_pages;
     const int NS = A.n_stages;
-    if (tid == 0) {
-        for (int i = 0; i < NS; ++i) {
-            const int p = (int)blockIdx.x + i * stride;
-            if (p < n) issue_window_stage(F, A, stages + i * A.stage_bytes, p, &S.full[i]);
-        }
+    const int H = A.heads;
+    const RowCtx R = row_ctx<FMT>(F, warp, lane);
+
+    int p = (int)blockIdx.x;
+    int ph = p % H;
+    float alpha_s = 0.f, beta_s = 0.f;
+    int kap = 0;
+    if (p < n) {
+        beta_s = __ldg(A.beta + p);
+        if (!gate_vector) alpha_s = __ldg(A.alpha + p);
+        kap = __ldg(A.perm + ph * kD + R.s) & (kD - 1);
     }
+    int st = 0, st_prev = 0;
+    uint32_t parity = 0;
+    for (int it = 0; p < n; ++it) {
+        const int pn = p + stride;
+        const int pnh = pn % H;
+        float alpha_n = 0.f, beta_n = 0.f;
+        int kap_n = 0;
+        if (pn < n) {
+            beta_n = __ldg(A.beta + pn);
+            if (!gate_vector) alpha_n = __ldg(A.alpha + pn);
+            kap_n = __ldg(A.perm + pnh * kD + R.s) & (kD - 1);
+        }
+        // a wait that runs out is voted on at the page's barrier, before
+        // anything of the page is written to global memory
+        bool ok;
+        if (A.stall_first_wait && it == 0) ok = mbar_wait_bounded(&S.never, 0, A.wait_limit_ns);
+        else ok = mbar_wait_bounded(&S.full[st], parity, A.wait_limit_ns);
+        uint8_t *stg = stages + st * A.stage_bytes;
+        const StageView V = stage_view(F, A, stg, col_scales);
+        window_first_phase<FMT, false>(F, A, S, stg, V, R, kap, alpha_s, gate_vector, warp, lane, nullptr);
+        if (__syncthreads_or(!ok)) {
+            if (tid == 0) atomicOr(A.status, kStatusTimeout);
+            break;   // the loads in flight land in the drain below
+        }
+        if (it >= 1 && tid == 32 * (it & (kWarps - 1))) {
+            // every warp is done with the previous page: refill its stage
+            const int pr = p + (NS - 1) * stride;
+            if (pr < n) {
+                fence_proxy_async_smem();
+                issue_window_stage(F, A, stages + st_prev * A.stage_bytes, pr, &S.full[st_prev]);
+                S.phase[st_prev] ^= 1u;
+            }
+        }
+        uint8_t *bp = A.buf + (size_t)p * A.stride;
+        {
+            const float al = gate_vector ? V.al[tid] : alpha_s;
+            reinterpret_cast<float *>(bp)[tid] = t > 0 ? __fmul_rn(V.P[tid], al) : al;
+            float *Kg = reinterpret_cast<float *>(bp + 512);
+            for (int tau = 0; tau < t; ++tau) Kg[tau * kD + tid] = __fmul_rn(V.K[tau * kD + tid], al);
+            Kg[t * kD + tid] = V.k[tid];
+        }
+        {
+            // column c = tid: u = (W0 + W1) + (W2 + W3) + the earlier entries,
+            // e = v (1/c) - u, D[t] = RN(beta e); o = c (tree + every entry's term)
+            const WindowScratch &X = *V.X;
+            const int col = tid;
+            float u = __fadd_rn(__fadd_rn(X.red_u[0][col], X.red_u[1][col]),
+                                __fadd_rn(X.red_u[2][col], X.red_u[3][col]));
+            float ot = __fadd_rn(__fadd_rn(X.red_o[0][col], X.red_o[1][col]),
+                                 __fadd_rn(X.red_o[2][col], X.red_o[3][col]));
+            for (int tau = 0; tau < t; ++tau) {
+                const float d = V.D[tau * kD + col];
+                u = __fmaf_rn(X.da[tau], d, u);
+                ot = __fmaf_rn(X.dq[tau], d, ot);
+            }
+            const float c = col_scales ? V.c[col] : 1.f;
+            const float ic = col_scales ? __frcp_rn(c) : 1.f;
+            const float dtc = __fmul_rn(beta_s, __fsub_rn(__fmul_rn(V.v[col], ic), u));
+            ot = __fmaf_rn(X.dq[t], dtc, ot);
+            reinterpret_cast<float *>(bp + A.buf_d_off + (size_t)t * 512)[col] = dtc;
+            A.o[(size_t)p * kD + col] = col_scales ? __fmul_rn(c, ot) : ot;
+        }
+        st_prev = st;
+        alpha_s = alpha_n;
+        beta_s = beta_n;
+        kap = kap_n;
+        p = pn;
+        ph = pnh;
+        if (++st == NS) { st = 0; parity ^= 1u; }
+    }
+    asm volatile("griddepcontrol.launch_dependents;");
+    window_drain(A, S);
+}
+
+// A committing step: one CTA barrier per page, after the first phase, since
+// every warp needs this step's delta D[t] for its own rows.  After it each
+// warp dequantizes its slices again (the page is intact in the stage until
+// the warp requantizes them), rebuilds T = RN(P' T0) and adds the entries in
+// order, takes the row maxima and requantizes in place; the stage is stored
+// at the next page's barrier and refilled once the store has read it.
+template <class FMT>
+__global__ void __launch_bounds__(kThreads, 3) window_commit_kernel(const DevFormat F, const WindowArgs A) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    WindowSmem &S = *reinterpret_cast<WindowSmem *>(smem);
+    float *kd_tab = reinterpret_cast<float *>(smem + kWindowFixedBytes);   // [warp][tau][32]
+    uint8_t *stages = smem + kWindowFixedBytes + A.kd_bytes;
+    constexpr bool SR = FMT::kSr;
+    bool col_scales, gate_vector;
+    format_flags<FMT>(F, col_scales, gate_vector);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int t = A.t;
+    window_start(F, A, S, stages);
+    const int stride = (int)gridDim.x;
+    const int n = A.n_pages;
+    const int NS = A.n_stages;
     const int H = A.heads;
     const int sb = stride / H, sh = stride % H;
-
-    // this lane's row of the slice: block my_blk = lane / 4, stored row my_s
-    const int my_blk = lane >> 2;
-    const int my_s = 16 * my_blk + 4 * warp + (lane & 3);
-    int my_bits, my_rbase;
-    if constexpr (FMT::kRuntime) {
-        my_bits = F.blk_bits(my_blk);
-        my_rbase = F.blk_rbase(my_blk);
-    } else {
-        my_bits = 0;
-        my_rbase = 0;
-#pragma unroll
-        for (int b = 0; b < kBlocks; ++b) {
-            if (b == my_blk) my_bits = FMT::width(b);
-            if (b < my_blk && FMT::width(b) != 16) my_rbase += 16;
-        }
-    }
-    const bool my_int = my_bits != 16;
-    bool all_int = false;
-    if constexpr (!FMT::kRuntime) {
-        all_int = true;
-        for (int b = 0; b < kBlocks; ++b) all_int = all_int && FMT::width(b) != 16;
-    }
-    const int my_r = my_rbase + 4 * warp + (lane & 3);
-    const float my_qmax = my_int ? (float)((1 << (my_bits - 1)) - 1) : 0.f;
-    const float my_rcp = my_int ? __frcp_rn(my_qmax) : 0.f;
+    const RowCtx R = row_ctx<FMT>(F, warp, lane);
+    float *kd = kd_tab + warp * (t + 1) * kRowsPerWarp;
 
     int p = (int)blockIdx.x;
     int pb = p / H, ph = p % H;
@@ -230,13 +475,11 @@ window_kernel(const DevFormat F, const WindowArgs A) {
     if (p < n) {
         beta_s = __ldg(A.beta + p);
         if (!gate_vector) alpha_s = __ldg(A.alpha + p);
-        kap = __ldg(A.perm + ph * kD + my_s) & (kD - 1);
+        kap = __ldg(A.perm + ph * kD + R.s) & (kD - 1);
     }
     int p_prev = -1, st = 0, st_prev = 0;
     uint32_t parity = 0;
-    int it = 0;
-
-    for (; p < n; ++it) {
+    for (int it = 0; p < n; ++it) {
         const int pn = p + stride;
         int pnb = pb + sb, pnh = ph + sh;
         if (pnh >= H) { pnh -= H; ++pnb; }
@@ -245,62 +488,47 @@ window_kernel(const DevFormat F, const WindowArgs A) {
         if (pn < n) {
             beta_n = __ldg(A.beta + pn);
             if (!gate_vector) alpha_n = __ldg(A.alpha + pn);
-            kap_n = __ldg(A.perm + pnh * kD + my_s) & (kD - 1);
+            kap_n = __ldg(A.perm + pnh * kD + R.s) & (kD - 1);
         }
-
         // a wait that runs out is voted on at the page's barrier, before
         // anything of the page is written to global memory
-        const bool ok = mbar_wait_bounded(&S.full[st], parity, A.wait_limit_ns);
-        const int par = it & 1;
+        bool ok;
+        if (A.stall_first_wait && it == 0) ok = mbar_wait_bounded(&S.never, 0, A.wait_limit_ns);
+        else ok = mbar_wait_bounded(&S.full[st], parity, A.wait_limit_ns);
         uint8_t *stg = stages + st * A.stage_bytes;
-        const float *q_s = reinterpret_cast<const float *>(stg + F.page_bytes);
-        const float *k_s = q_s + kD;
-        const float *v_s = q_s + 2 * kD;
-        const float *al_s = q_s + 3 * kD;
-        const float *P_s = reinterpret_cast<const float *>(stg + A.p_off);
-        const float *K_s = reinterpret_cast<const float *>(stg + A.k_off);
-        const float *D_s = reinterpret_cast<const float *>(stg + A.d_off);
-        float *r_s = reinterpret_cast<float *>(stg + F.r_off);
-        const float *c_s = col_scales ? reinterpret_cast<const float *>(stg + F.c_off) : nullptr;
+        const StageView V = stage_view(F, A, stg, col_scales);
+        window_first_phase<FMT, true>(F, A, S, stg, V, R, kap, alpha_s, gate_vector, warp, lane, kd);
 
-        // operands of this lane's row: r, RN(P' k), RN(P' q) (and for a
-        // commit P' and the row's decayed keys)
-        {
-            const float al = gate_vector ? al_s[kap] : alpha_s;
-            const float pp = t > 0 ? __fmul_rn(P_s[kap], al) : al;
-            S.rw[warp][lane] = (all_int || my_int) ? r_s[my_r] : 1.f;
-            S.kp[warp][lane] = __fmul_rn(pp, k_s[kap]);
-            S.qp[warp][lane] = __fmul_rn(pp, q_s[kap]);
-            if constexpr (COMMIT) {
-                float *kd = kd_tab + warp * (t + 1) * kRowsPerWarp;
-                S.pk[warp][lane] = pp;
-                for (int tau = 0; tau < t; ++tau) kd[tau * kRowsPerWarp + lane] = __fmul_rn(K_s[tau * kD + kap], al);
-                kd[t * kRowsPerWarp + lane] = k_s[kap];
-            }
-        }
-        // the entries' dot products: warp w takes entries w, w + 4, ...
-        {
-            const float4 al4 = gate_vector ? *reinterpret_cast<const float4 *>(al_s + 4 * lane)
-                                           : make_float4(alpha_s, alpha_s, alpha_s, alpha_s);
-            const float4 k4 = *reinterpret_cast<const float4 *>(k_s + 4 * lane);
-            const float4 q4 = *reinterpret_cast<const float4 *>(q_s + 4 * lane);
-            for (int tau = warp; tau <= t; tau += kWarps) {
-                const float4 kk = tau < t ? mul4(*reinterpret_cast<const float4 *>(K_s + tau * kD + 4 * lane), al4) : k4;
-                const float a = lane_dot(kk, k4);
-                const float b = lane_dot(kk, q4);
-                if (lane == 0) {
-                    S.da[par][tau] = a;
-                    S.dq[par][tau] = b;
+        if (__syncthreads_or(!ok)) {
+            // record it, store the previous (finished) page and leave; the
+            // loads in flight land in the drain below
+            if (tid == 0) {
+                atomicOr(A.status, kStatusTimeout);
+                if (p_prev >= 0) {
+                    bulk_s2g(A.pages + (size_t)p_prev * F.page_bytes, stages + st_prev * A.stage_bytes,
+                             A.store_bytes);
+                    bulk_commit();
                 }
+                bulk_wait<0>();
             }
+            break;
         }
-        __syncwarp();
+        if (tid == 0 && p_prev >= 0) {
+            // the previous page is complete in its stage: store it
+            bulk_s2g(A.pages + (size_t)p_prev * F.page_bytes, stages + st_prev * A.stage_bytes, A.store_bytes);
+            bulk_commit();
+        }
+        const WindowScratch &X = *V.X;
+        // o of columns 4l .. 4l+3 by one warp (in turn); D[t] of them in every warp
+        const float4 dt = window_delta(X, V.v, V.D, V.c, t, beta_s, lane);
+        if (warp == (it & (kWarps - 1)))
+            *reinterpret_cast<float4 *>(A.o + (size_t)p * kD + 4 * lane) = window_out(X, V.D, V.c, t, dt, lane);
 
-        // one pass over the page: dequantize, u's and o's chains
+        // T = RN(P' T0), then the entries in order (per element one chain;
+        // block by block, so that a block's codes and keys are the only
+        // operands in registers besides T), and the row maxima
+        const float2 dt01 = make_float2(dt.x, dt.y), dt23 = make_float2(dt.z, dt.w);
         Tile T;
-        float2 cu[2][2], co[2][2];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) cu[h][0] = cu[h][1] = co[h][0] = co[h][1] = make_float2(0.f, 0.f);
         static_for<0, kBlocks>([&](auto bc) {
             constexpr int b = decltype(bc)::value;
             const float4 a4 = *reinterpret_cast<const float4 *>(&S.rw[warp][4 * b]);
@@ -309,148 +537,70 @@ window_kernel(const DevFormat F, const WindowArgs A) {
                 constexpr int W = decltype(wc)::value;
                 dequant_slice<W, b>(blk, warp, lane, a4, T);
             });
-            const float4 k4 = *reinterpret_cast<const float4 *>(&S.kp[warp][4 * b]);
-            const float4 q4 = *reinterpret_cast<const float4 *>(&S.qp[warp][4 * b]);
-            const float kv[4] = {k4.x, k4.y, k4.z, k4.w};
-            const float qv[4] = {q4.x, q4.y, q4.z, q4.w};
-            constexpr int h = b >> 2;
+            const float4 p4 = *reinterpret_cast<const float4 *>(&S.pk[warp][4 * b]);
+            const float pv[4] = {p4.x, p4.y, p4.z, p4.w};
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                cu[h][0] = __ffma2_rn(make_float2(kv[i], kv[i]), T[b][i][0], cu[h][0]);
-                cu[h][1] = __ffma2_rn(make_float2(kv[i], kv[i]), T[b][i][1], cu[h][1]);
-                co[h][0] = __ffma2_rn(make_float2(qv[i], qv[i]), T[b][i][0], co[h][0]);
-                co[h][1] = __ffma2_rn(make_float2(qv[i], qv[i]), T[b][i][1], co[h][1]);
+                T[b][i][0] = __fmul2_rn(T[b][i][0], make_float2(pv[i], pv[i]));
+                T[b][i][1] = __fmul2_rn(T[b][i][1], make_float2(pv[i], pv[i]));
+            }
+#pragma unroll 1
+            for (int tau = 0; tau < t; ++tau) {
+                const float4 d = *reinterpret_cast<const float4 *>(V.D + tau * kD + 4 * lane);
+                const float4 k4 = *reinterpret_cast<const float4 *>(kd + tau * kRowsPerWarp + 4 * b);
+                const float kv[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    T[b][i][0] = __ffma2_rn(make_float2(kv[i], kv[i]), make_float2(d.x, d.y), T[b][i][0]);
+                    T[b][i][1] = __ffma2_rn(make_float2(kv[i], kv[i]), make_float2(d.z, d.w), T[b][i][1]);
+                }
+            }
+            const float4 k4 = *reinterpret_cast<const float4 *>(kd + t * kRowsPerWarp + 4 * b);
+            const float kv[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                T[b][i][0] = __ffma2_rn(make_float2(kv[i], kv[i]), dt01, T[b][i][0]);
+                T[b][i][1] = __ffma2_rn(make_float2(kv[i], kv[i]), dt23, T[b][i][1]);
+                S.inv[warp][4 * b + i] = warp_absmax(absmax4(T[b][i][0], T[b][i][1]));
             }
         });
-        store_readout(S.red_u[par][warp], lane, cu);
-        store_readout(S.red_o[par][warp], lane, co);
-
-        if (__syncthreads_or(!ok)) {
-            // a stage never arrived: record it, store the previous page (a
-            // commit), let the copies in flight land and leave
-            if (tid == 0) {
-                atomicOr(A.status, kStatusTimeout);
-                if (COMMIT && p_prev >= 0) {
-                    bulk_s2g(A.pages + (size_t)p_prev * F.page_bytes, stages + st_prev * A.stage_bytes, A.store_bytes);
-                    bulk_commit();
-                }
-                const int last = COMMIT ? (it < 3 ? NS - 1 : it - 3 + NS) : (it < 2 ? NS - 1 : it - 2 + NS);
-                for (int j = it; j <= last; ++j) {
-                    if ((int)blockIdx.x + j * stride < n)
-                        mbar_wait_bounded(&S.full[j % NS], (uint32_t)((j / NS) & 1), A.wait_limit_ns);
-                }
-                bulk_wait<0>();
-            }
-            __syncthreads();
-            return;
-        }
-
-        if (tid == 0) {
-            // a commit stores the previous page and refills the stage of the
-            // one before once its store has read it; otherwise the previous
-            // page's stage is free now
-            int j = -1;
-            if constexpr (COMMIT) {
-                if (p_prev >= 0) {
-                    bulk_s2g(A.pages + (size_t)p_prev * F.page_bytes, stages + st_prev * A.stage_bytes, A.store_bytes);
-                    bulk_commit();
-                }
-                if (it >= 2) {
-                    bulk_wait_read<1>();
-                    j = it - 2 + NS;
-                }
-            } else {
-                if (it >= 1) j = it - 1 + NS;
-            }
-            const int pr = (int)blockIdx.x + j * stride;
-            if (j >= 0 && pr < n) {
+        if (tid == 0 && p_prev >= 0) {
+            // refill the previous page's stage with the page NS - 1 ahead of this one
+            bulk_wait_read<0>();
+            const int pr = p + (NS - 1) * stride;
+            if (pr < n) {
                 fence_proxy_async_smem();
-                issue_window_stage(F, A, stages + (j % NS) * A.stage_bytes, pr, &S.full[j % NS]);
+                issue_window_stage(F, A, stages + st_prev * A.stage_bytes, pr, &S.full[st_prev]);
+                S.phase[st_prev] ^= 1u;
             }
         }
-
-        uint8_t *bp = A.buf + (size_t)p * A.stride;
-        if constexpr (!COMMIT) {
-            // the buffer rows of channel tid: P', the decayed keys, K[t] = k
-            const float al = gate_vector ? al_s[tid] : alpha_s;
-            reinterpret_cast<float *>(bp)[tid] = t > 0 ? __fmul_rn(P_s[tid], al) : al;
-            float *Kg = reinterpret_cast<float *>(bp + 512);
-            for (int tau = 0; tau < t; ++tau) Kg[tau * kD + tid] = __fmul_rn(K_s[tau * kD + tid], al);
-            Kg[t * kD + tid] = k_s[tid];
-        }
-        // D[t] and o by one warp (a commit: D[t] in every warp)
-        const int fw = it & (kWarps - 1);
-        if (COMMIT || warp == fw) {
-            const float4 dt = window_delta(S, par, v_s, D_s, c_s, t, beta_s, lane);
-            if (warp == fw) {
-                if constexpr (!COMMIT)
-                    *reinterpret_cast<float4 *>(bp + A.buf_d_off + (size_t)t * 512 + 16 * lane) = dt;
-                window_out(S, par, D_s, c_s, t, dt, A.o + (size_t)p * kD, lane);
+        __syncwarp();
+        // lane l finishes row l of the slice: r' = m / qmax, inv = qmax / m (toward zero)
+        {
+            const float m = S.inv[warp][lane];
+            float inv = 0.f;
+            if (R.all_int || R.is_int) {
+                const float r = div_by_qmax(m, R.qmax, R.rcp_qmax);
+                inv = m > 0.f ? div_rz_qmax<(FMT::kTune & kFastRcp) != 0>(R.qmax, m) : 0.f;
+                V.r[R.rix] = r;
             }
-            if constexpr (COMMIT) {
-                // T = RN(P' T0), then the entries in order (per element the
-                // same chain; block by block, so that a block's keys are the
-                // only operands in registers), and the row maxima
-                const float *kd = kd_tab + warp * (t + 1) * kRowsPerWarp;
-                const float2 dt01 = make_float2(dt.x, dt.y), dt23 = make_float2(dt.z, dt.w);
-                static_for<0, kBlocks>([&](auto bc) {
-                    constexpr int b = decltype(bc)::value;
-                    const float4 p4 = *reinterpret_cast<const float4 *>(&S.pk[warp][4 * b]);
-                    const float pv[4] = {p4.x, p4.y, p4.z, p4.w};
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        T[b][i][0] = __fmul2_rn(T[b][i][0], make_float2(pv[i], pv[i]));
-                        T[b][i][1] = __fmul2_rn(T[b][i][1], make_float2(pv[i], pv[i]));
-                    }
-#pragma unroll 1
-                    for (int tau = 0; tau < t; ++tau) {
-                        const float4 d = *reinterpret_cast<const float4 *>(D_s + tau * kD + 4 * lane);
-                        const float4 k4 = *reinterpret_cast<const float4 *>(kd + tau * kRowsPerWarp + 4 * b);
-                        const float kv[4] = {k4.x, k4.y, k4.z, k4.w};
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            T[b][i][0] = __ffma2_rn(make_float2(kv[i], kv[i]), make_float2(d.x, d.y), T[b][i][0]);
-                            T[b][i][1] = __ffma2_rn(make_float2(kv[i], kv[i]), make_float2(d.z, d.w), T[b][i][1]);
-                        }
-                    }
-                    const float4 k4 = *reinterpret_cast<const float4 *>(kd + t * kRowsPerWarp + 4 * b);
-                    const float kv[4] = {k4.x, k4.y, k4.z, k4.w};
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        T[b][i][0] = __ffma2_rn(make_float2(kv[i], kv[i]), dt01, T[b][i][0]);
-                        T[b][i][1] = __ffma2_rn(make_float2(kv[i], kv[i]), dt23, T[b][i][1]);
-                        S.inv[warp][4 * b + i] = warp_absmax(absmax4(T[b][i][0], T[b][i][1]));
-                    }
-                });
-                __syncwarp();
-                // lane l finishes row l of the slice: r' = m / qmax, inv = qmax / m (toward zero)
-                {
-                    const float m = S.inv[warp][lane];
-                    float inv = 0.f;
-                    if (all_int || my_int) {
-                        const float r = div_by_qmax(m, my_qmax, my_rcp);
-                        inv = m > 0.f ? div_rz_qmax<(FMT::kTune & kFastRcp) != 0>(my_qmax, m) : 0.f;
-                        r_s[my_r] = r;
-                    }
-                    S.inv[warp][lane] = inv;
-                }
-                __syncwarp();
-                SrCtx sr;
-                sr.k0 = A.seed_lo; sr.k1 = A.seed_hi; sr.step = A.step;
-                sr.b = (uint32_t)pb;
-                sr.h = (uint32_t)ph;
-                static_for<0, kBlocks>([&](auto bc) {
-                    constexpr int b = decltype(bc)::value;
-                    const float4 i4 = *reinterpret_cast<const float4 *>(&S.inv[warp][4 * b]);
-                    uint8_t *blk = stg + fmt_offset<FMT, b>(F);
-                    with_width<FMT, b>(F, [&](auto wc) {
-                        constexpr int W = decltype(wc)::value;
-                        requant_slice<W, b, SR>(blk, warp, lane, i4, T, sr);
-                    });
-                });
-                fence_proxy_async_smem();   // the stage's new bytes are read by the bulk store
-            }
+            S.inv[warp][lane] = inv;
         }
+        __syncwarp();
+        SrCtx sr;
+        sr.k0 = A.seed_lo; sr.k1 = A.seed_hi; sr.step = A.step;
+        sr.b = (uint32_t)pb;
+        sr.h = (uint32_t)ph;
+        static_for<0, kBlocks>([&](auto bc) {
+            constexpr int b = decltype(bc)::value;
+            const float4 i4 = *reinterpret_cast<const float4 *>(&S.inv[warp][4 * b]);
+            uint8_t *blk = stg + fmt_offset<FMT, b>(F);
+            with_width<FMT, b>(F, [&](auto wc) {
+                constexpr int W = decltype(wc)::value;
+                requant_slice<W, b, SR>(blk, warp, lane, i4, T, sr);
+            });
+        });
+        fence_proxy_async_smem();   // the stage's new bytes are read by the bulk store
 
         p_prev = p;
         st_prev = st;
@@ -461,39 +611,33 @@ window_kernel(const DevFormat F, const WindowArgs A) {
         pb = pnb;
         ph = pnh;
         if (++st == NS) { st = 0; parity ^= 1u; }
-    }
-    asm volatile("griddepcontrol.launch_dependents;");
-    __syncthreads();
-    if (tid == 0) {
-        if (COMMIT && p_prev >= 0) {
-            bulk_s2g(A.pages + (size_t)p_prev * F.page_bytes, stages + st_prev * A.stage_bytes, A.store_bytes);
-            bulk_commit();
+        if (p >= n) {
+            // the last page: store it once every warp has requantized its slices
+            asm volatile("griddepcontrol.launch_dependents;");
+            __syncthreads();
+            if (tid == 0) {
+                bulk_s2g(A.pages + (size_t)p_prev * F.page_bytes, stages + st_prev * A.stage_bytes, A.store_bytes);
+                bulk_commit();
+                bulk_wait<0>();
+            }
         }
-        bulk_wait<0>();
     }
+    window_drain(A, S);
 }
 
-// Ring depth and residency: the most pages in flight per SM (resident CTAs x
-// pages of look-ahead: NS - 1, a commit NS - 2 since a stage is refilled only
-// after its page's store has read it), at most `ctas` CTAs.
-static void window_ring(size_t fixed, size_t stage, int ctas, bool commit, int *ns_out) {
+// Ring depth and residency: the most resident CTAs (up to `ctas`) whose ring
+// holds at least two stages, then the deepest ring at that residency (at most
+// kWindowStages).  Measured on a B200: residency beats look-ahead here.
+static int window_ring(size_t fixed, size_t stage, int ctas) {
     int dev = 0, smem_sm = 0, reserved = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
     cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
-    const int min_ns = commit ? 3 : 2;
-    int best_ns = min_ns, best_score = -1;
     for (int c = ctas; c >= 1; --c) {
         long ns = ((long)smem_sm / c - reserved - (long)fixed) / (long)stage;
-        if (ns > kWindowStages) ns = kWindowStages;
-        if (ns < min_ns) continue;
-        const int score = c * (int)(ns - (commit ? 2 : 1));
-        if (score > best_score) {
-            best_score = score;
-            best_ns = (int)ns;
-        }
+        if (ns >= 2) return ns > kWindowStages ? kWindowStages : (int)ns;
     }
-    *ns_out = best_ns;
+    return 2;
 }
 
 template <class FMT, bool COMMIT>
@@ -501,9 +645,9 @@ static cudaError_t launch_window_with(const DevFormat &F, const WindowArgs &A0, 
                                       cudaStream_t stream) {
     WindowArgs A = A0;
     const size_t fixed = kWindowFixedBytes + A.kd_bytes;
-    window_ring(fixed, A.stage_bytes, window_ctas_per_sm<COMMIT>(), COMMIT, &A.n_stages);
+    A.n_stages = window_ring(fixed, A.stage_bytes, COMMIT ? 3 : 4);
     const size_t smem = fixed + (size_t)A.n_stages * A.stage_bytes;
-    const void *fn = (const void *)window_kernel<FMT, COMMIT>;
+    const void *fn = COMMIT ? (const void *)window_commit_kernel<FMT> : (const void *)window_step_kernel<FMT>;
     cudaError_t err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     const int grid = persistent_grid(fn, kThreads, smem, A.n_pages);
@@ -518,7 +662,8 @@ static cudaError_t launch_window_with(const DevFormat &F, const WindowArgs &A0, 
     attr[0].val.programmaticStreamSerializationAllowed = early_launch ? 1 : 0;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, window_kernel<FMT, COMMIT>, F, A);
+    if constexpr (COMMIT) return cudaLaunchKernelEx(&cfg, window_commit_kernel<FMT>, F, A);
+    else return cudaLaunchKernelEx(&cfg, window_step_kernel<FMT>, F, A);
 }
 
 template <bool COMMIT>
@@ -535,7 +680,8 @@ size_t window_buffer_stride(int window) { return 512u * (1u + 2u * (size_t)windo
 
 cudaError_t launch_window(const stq_state *s, uint8_t *buf, int window, int t, bool commit, const float *q,
                           const float *k, const float *v, const float *alpha, const float *beta, float *o,
-                          uint64_t seed, uint32_t step, bool early_launch, cudaStream_t stream) {
+                          uint64_t seed, uint32_t step, int stall_first_wait, bool early_launch,
+                          cudaStream_t stream) {
     const DevFormat &F = s->dev;
     WindowArgs A;
     A.pages = s->base + s->pages_offset;
@@ -554,13 +700,15 @@ cudaError_t launch_window(const stq_state *s, uint8_t *buf, int window, int t, b
     A.k_off = rows + 512u;
     A.d_off = A.k_off + 512u * (uint32_t)t;
     A.tx_bytes = rows + (t > 0 ? 512u + 1024u * (uint32_t)t : 0u);
-    A.stage_bytes = (A.tx_bytes + 127u) / 128u * 128u;
+    A.scr_off = (A.tx_bytes + 127u) / 128u * 128u;
+    A.stage_bytes = A.scr_off + kScratchBytes;
     A.store_bytes = (uint32_t)(F.col_scales ? F.c_off : F.page_bytes);
     A.kd_bytes = commit ? 512u * (uint32_t)(t + 1) : 0u;
     A.seed_lo = (uint32_t)seed;
     A.seed_hi = (uint32_t)(seed >> 32);
     A.step = step;
     A.wait_limit_ns = s->wait_limit_ns;
+    A.stall_first_wait = stall_first_wait;
     if (commit) return launch_window_fmt<true>(F, A, early_launch, stream);
     return launch_window_fmt<false>(F, A, early_launch, stream);
 }

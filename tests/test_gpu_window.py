@@ -179,3 +179,44 @@ def test_window_against_plain_steps_from_the_same_page():
         o_p = qb.step(xd["q"], xd["k"], xd["v"], xd["alpha"], xd["beta"], step=t)
         rel = float(torch.linalg.norm(o_w - o_p) / torch.linalg.norm(o_p))
         assert rel < 5e-2, (t, rel)
+
+
+@pytest.mark.parametrize("commit", [False, True])
+def test_bounded_wait_times_out_and_writes_nothing(commit):
+    """The test hook makes every CTA's first wait run out (20 ms): the status
+    word reports it, no page, buffer row or o is written, and the next step
+    runs normally and matches the oracle."""
+    w, fmt, perm, pages, qs = _setup("stepquant6", 6, 5)
+    n = w.batch * w.heads
+    window, t = 4, (3 if commit else 0)
+    buf = _gpu_buffer(qs, window)
+    x = W.step_inputs(w, 0)
+    xd = {k: v.cuda() for k, v in x.items()}
+    o = torch.full((w.batch, w.heads, 128), 7.0, device="cuda")
+    if commit:   # a committing step needs a window so far: steps 0 .. 2 first
+        orc = OracleWindow(fmt, perm, pages, w.heads, window)
+        for s in range(3):
+            xs = W.step_inputs(w, 10 + s)
+            xsd = {k: v.cuda() for k, v in xs.items()}
+            B.stq_window_step(qs.state, buf, window, s, False, xsd["q"], xsd["k"], xsd["v"], xsd["alpha"],
+                              xsd["beta"], o, step=s)
+            orc.step(xs, s, False, 0, s)
+        o.fill_(7.0)
+    before = buf.clone()
+    B.stq_set_wait_limit(qs.state, 20_000_000, stall_first_wait=True)
+    B.stq_window_step(qs.state, buf, window, t, commit, xd["q"], xd["k"], xd["v"], xd["alpha"], xd["beta"], o,
+                      step=t)
+    assert B.stq_device_status(qs.state, clear=True) == B.STQ_ERR_DEVICE_TIMEOUT
+    assert np.array_equal(download(qs), pages)
+    assert torch.equal(buf, before)
+    assert bool((o == 7.0).all())
+    B.stq_set_wait_limit(qs.state, 0, stall_first_wait=False)
+    B.stq_window_step(qs.state, buf, window, t, commit, xd["q"], xd["k"], xd["v"], xd["alpha"], xd["beta"], o,
+                      step=t)
+    assert B.stq_device_status(qs.state) == B.STQ_OK
+    if not commit:
+        orc = OracleWindow(fmt, perm, pages, w.heads, window)
+    o_ref, margins = orc.step(x, t, commit, 0, t)
+    assert np.array_equal(o.cpu().numpy().reshape(n, 128), o_ref)
+    if commit:
+        _check_commit(fmt, download(qs), orc.packed(), margins)
