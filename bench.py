@@ -67,10 +67,14 @@ def window_bytes_per_page(spec, window):
     return total / window
 
 
-def kernel_source_hash():
+DECODE_SOURCES = ("stq_decode.cu", "stq_device.cuh", "stq_internal.h", "stq_slices.cuh")
+
+
+def kernel_source_hash(names=DECODE_SOURCES):
+    """Hash of the sources the decode kernel is compiled from."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "linear_attention_recurrent_delta_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in sorted(names):
         with open(os.path.join(csrc, name), "rb") as fh:
             h.update(name.encode() + fh.read())
     return h.hexdigest()[:16]
