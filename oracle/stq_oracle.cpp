@@ -564,7 +564,7 @@ extern "C" int orc_window_step_f32(const orc_format *f, orc_page *page, const in
         return -1;
     const int d_k = f->d_k, d_v = f->d_v;
     if (d_k % 4 != 0) return -1;
-    std::vector<float> ic(d_v), T0((size_t)d_k * d_v), wk(d_k), wq(d_k), u(d_v), ot(d_v);
+    std::vector<float> ic(d_v), Z((size_t)d_k * d_v), af(d_k), wk(d_k), wq(d_k), u(d_v), ot(d_v);
     for (int j = 0; j < d_v; ++j) ic[j] = f->col_scales ? 1.0f / page->c[j] : 1.0f;
 
     /* decay: the window's cumulative product and the earlier entries' keys */
@@ -574,17 +574,23 @@ extern "C" int orc_window_step_f32(const orc_format *f, orc_page *page, const in
         P[kap] = p0 * al;
         for (int tau = 0; tau < t; ++tau) K[(size_t)tau * d_k + kap] = K[(size_t)tau * d_k + kap] * al;
     }
-    /* the fixed page in column-normalised units, undecayed: T0 = z r (FP16: h) */
+    /* the fixed page as exact values Z (INT rows: z, FP16 rows: h) and one
+     * factor per stored row, the window's decay times the row scale:
+     * a'_s = P'_kappa r_s (FP16 rows: P'_kappa) */
     for (int s = 0; s < d_k; ++s) {
+        const int kap = perm[s];
         const float rs = (orc_row_kind(f, s) == ORC_KIND_INT) ? page->r[s] : 1.0f;
-        for (int j = 0; j < d_v; ++j) T0[(size_t)s * d_v + j] = element_value(f, page, s, j) * rs;
+        af[s] = P[kap] * rs;
+        for (int j = 0; j < d_v; ++j) Z[(size_t)s * d_v + j] = element_value(f, page, s, j);
     }
-    for (int kap = 0; kap < d_k; ++kap) {
-        wk[kap] = P[kap] * k[kap];
-        wq[kap] = P[kap] * q[kap];
+    /* row weights by key channel: k a', q a' */
+    for (int s = 0; s < d_k; ++s) {
+        const int kap = perm[s];
+        wk[kap] = k[kap] * af[s];
+        wq[kap] = q[kap] * af[s];
     }
     /* prediction from the page and the earlier entries */
-    column_sum(f, perm, wk.data(), T0.data(), u.data());
+    column_sum(f, perm, wk.data(), Z.data(), u.data());
     for (int tau = 0; tau < t; ++tau) {
         const float a = lane_dot(K + (size_t)tau * d_k, k, d_k);
         for (int j = 0; j < d_v; ++j) u[j] = std::fmaf(a, D[(size_t)tau * d_v + j], u[j]);
@@ -596,7 +602,7 @@ extern "C" int orc_window_step_f32(const orc_format *f, orc_page *page, const in
     }
     for (int kap = 0; kap < d_k; ++kap) K[(size_t)t * d_k + kap] = k[kap];
     /* readout from the page and every entry */
-    column_sum(f, perm, wq.data(), T0.data(), ot.data());
+    column_sum(f, perm, wq.data(), Z.data(), ot.data());
     for (int tau = 0; tau <= t; ++tau) {
         const float bq = lane_dot(K + (size_t)tau * d_k, q, d_k);
         for (int j = 0; j < d_v; ++j) ot[j] = std::fmaf(bq, D[(size_t)tau * d_v + j], ot[j]);
@@ -604,12 +610,12 @@ extern "C" int orc_window_step_f32(const orc_format *f, orc_page *page, const in
     for (int j = 0; j < d_v; ++j) o_out[j] = f->col_scales ? page->c[j] * ot[j] : ot[j];
 
     if (commit) {
-        /* T = P T0 + sum_tau K[tau] D[tau]^T, requantized once */
+        /* T = Z a' + sum_tau K[tau] D[tau]^T, requantized once */
         std::vector<float> row(d_v);
         for (int s = 0; s < d_k; ++s) {
             const int kap = perm[s];
             for (int j = 0; j < d_v; ++j) {
-                float x = P[kap] * T0[(size_t)s * d_v + j];
+                float x = Z[(size_t)s * d_v + j] * af[s];
                 for (int tau = 0; tau <= t; ++tau)
                     x = std::fmaf(K[(size_t)tau * d_k + kap], D[(size_t)tau * d_v + j], x);
                 row[j] = x;

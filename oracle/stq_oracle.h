@@ -123,12 +123,14 @@ int orc_step_f64(const orc_format *f, const orc_page *page, const int32_t *perm,
  * (column-normalised, undecayed).  With commit != 0 the state
  * T = P S0 + sum_tau K[tau] D[tau]^T is then requantized into the page
  * (as orc_step_f32 requantizes) and P is reset to 1.  The canonical fp32
- * order: the S0 products are the column sums of orc_step_f32 with row
- * weights RN(P k) and RN(P q) on T0 = z r (FP16 rows: h); a buffer dot
- * product is 4-channel fma chains per lane (d_k / 4 lanes) combined by an
- * xor butterfly; the buffer terms are added by fmaf in entry order; the
- * committed element is an fma chain from RN(P T0) over the entries in
- * order.  margin_out as orc_step_f32 (commit only). */
+ * order: the page's stored row s gets one factor a'_s = RN(P'_kappa r_s)
+ * (FP16 rows: P'_kappa), as the decode step folds the decay into the row
+ * scale; the S0 products are the column sums of orc_step_f32 with row
+ * weights RN(k a') and RN(q a') on the exact codes z (FP16 rows: h); a
+ * buffer dot product is 4-channel fma chains per lane (d_k / 4 lanes)
+ * combined by an xor butterfly; the buffer terms are added by fmaf in entry
+ * order; the committed element is an fma chain from RN(z a') over the
+ * entries in order.  margin_out as orc_step_f32 (commit only). */
 int orc_window_step_f32(const orc_format *f, orc_page *page, const int32_t *perm,
                         float *P, float *K, float *D, int t, int commit,
                         const float *q, const float *k, const float *v,

@@ -53,8 +53,9 @@ MUTANTS = {
     "window delta without beta": ("D[(size_t)t * d_v + j] = beta * e;", "D[(size_t)t * d_v + j] = e;"),
     "window readout skips this step": ("for (int tau = 0; tau <= t; ++tau) {\n        const float bq",
                                        "for (int tau = 0; tau < t; ++tau) {\n        const float bq"),
-    "window commit drops the decay": ("float x = P[kap] * T0[(size_t)s * d_v + j];",
-                                      "float x = T0[(size_t)s * d_v + j];"),
+    "window commit drops the row factor": ("float x = Z[(size_t)s * d_v + j] * af[s];",
+                                           "float x = Z[(size_t)s * d_v + j];"),
+    "window row factor without decay": ("af[s] = P[kap] * rs;", "af[s] = rs;"),
     "window decay not reset": ("for (int kap = 0; kap < d_k; ++kap) P[kap] = 1.0f;",
                                "for (int kap = 0; kap < d_k; ++kap) P[kap] = P[kap];"),
     "window start keeps the old decay": ("const float p0 = (t == 0) ? 1.0f : P[kap];",
