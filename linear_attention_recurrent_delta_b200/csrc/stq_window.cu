@@ -8,18 +8,20 @@
 //   P[128]     cumulative decay per key channel (natural order); not read at t = 0
 //   K[W][128]  entry tau's key, decayed to the current step (natural order)
 //   D[W][128]  entry tau's delta beta_tau e_tau, column-normalised units
-// Step t, with T0 = z r the fixed page (FP16 rows: h; stored order, the row
-// of stored index s holding key channel perm[s]):
+// Step t, with z the fixed page's exact codes (FP16 rows: h; stored order,
+// the row of stored index s holding key channel perm[s]) and one factor per
+// stored row, a'_s = RN(P'_kappa r_s) (FP16 rows: P'_kappa), the window's
+// decay folded into the row scale as the decode step folds alpha into r:
 //   P' = P alpha;   K[tau] <- RN(K[tau] alpha)                  (tau < t)
-//   u = T0^T RN(P' k) + sum_{tau<t} (K[tau] . k) D[tau]
+//   u = z^T RN(k a') + sum_{tau<t} (K[tau] . k) D[tau]
 //   D[t] = RN(beta (v (1/c) - u));   K[t] = k
-//   o = c (T0^T RN(P' q) + sum_{tau<=t} (K[tau] . q) D[tau])
-// The column sums over T0 are the decode kernel's (same slices, chains and
-// tree); both run in one pass over the page, since the page does not change
-// within a window.  A buffer dot product is a 4-channel fma chain per lane
-// (lane l: channels 4l .. 4l+3) and an xor butterfly over the warp; buffer
-// terms are added by fma in entry order.  A committing step then rebuilds
-// T = RN(P' T0), T <- fma(K[tau], D[tau], T) for tau = 0 .. t, in registers,
+//   o = c (z^T RN(q a') + sum_{tau<=t} (K[tau] . q) D[tau])
+// The column sums over the page are the decode kernel's (same slices, chains
+// and tree); both run in one pass, since the page does not change within a
+// window.  A buffer dot product is a 4-channel fma chain per lane (lane l:
+// channels 4l .. 4l+3) and an xor butterfly over the warp; buffer terms are
+// added by fma in entry order.  A committing step then rebuilds
+// T = RN(z a'), T <- fma(K[tau], D[tau], T) for tau = 0 .. t, in registers,
 // and requantizes it exactly as the decode step requantizes T'; it writes
 // nothing to the buffer (a window's first step reads none of it).
 //
@@ -57,10 +59,9 @@ struct WindowArgs {
 
 struct WindowSmem {
     // per warp, its 32 rows in slice order (row 4b + i = block b, row i):
-    float rw[kWarps][kRowsPerWarp];         // r (FP16 rows: 1)
-    float kp[kWarps][kRowsPerWarp];         // RN(P' k) of the row's key channel
-    float qp[kWarps][kRowsPerWarp];         // RN(P' q)
-    float pk[kWarps][kRowsPerWarp];         // P' (commit)
+    float kp[kWarps][kRowsPerWarp];         // RN(k a') of the row's key channel
+    float qp[kWarps][kRowsPerWarp];         // RN(q a')
+    float pk[kWarps][kRowsPerWarp];         // a' = RN(P' r), FP16 rows P' (commit)
     float inv[kWarps][kRowsPerWarp];        // commit: row maxima, then requant multipliers
     uint64_t full[kWindowStages];           // stage-full barriers
     uint64_t never;                         // a barrier nothing completes (test hook)
@@ -221,6 +222,26 @@ __device__ __forceinline__ StageView stage_view(const DevFormat &F, const Window
     return V;
 }
 
+// The exact values of slice w of block B: the codes z (FP16 rows: h) as floats.
+template <int W, int B>
+__device__ __forceinline__ void codes_slice(const uint8_t *blk, int w, int lane, Tile &T) {
+    if constexpr (W == 16) {
+        uint32_t x[8];
+        load_fp16_slice(blk, w, lane, x);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            T[B][i][0] = __half22float2(*reinterpret_cast<const __half2 *>(&x[2 * i]));
+            T[B][i][1] = __half22float2(*reinterpret_cast<const __half2 *>(&x[2 * i + 1]));
+        }
+    } else {
+        uint32_t ub[4];
+        unpack_int_slice<W>(blk, w, lane, ub);
+        const float bm = 8388608.0f + (float)(1 << (W - 1));
+#pragma unroll
+        for (int i = 0; i < 4; ++i) codes_to_float(ub[i], bm, T[B][i][0], T[B][i][1]);
+    }
+}
+
 // The first phase of a page, per warp: the operands of this lane's row, the
 // entries' dot products (warp w: entries w, w + 4, ...) and one pass over the
 // warp's slices (dequantize, u's and o's chains), whose sums go to the
@@ -235,11 +256,11 @@ __device__ __forceinline__ void window_first_phase(const DevFormat &F, const Win
     {
         const float al = gate_vector ? V.al[kap] : alpha_s;
         const float pp = t > 0 ? __fmul_rn(V.P[kap], al) : al;
-        S.rw[warp][lane] = (R.all_int || R.is_int) ? V.r[R.rix] : 1.f;
-        S.kp[warp][lane] = __fmul_rn(pp, V.k[kap]);
-        S.qp[warp][lane] = __fmul_rn(pp, V.q[kap]);
+        const float af = (R.all_int || R.is_int) ? __fmul_rn(pp, V.r[R.rix]) : pp;   // a'
+        S.kp[warp][lane] = __fmul_rn(V.k[kap], af);
+        S.qp[warp][lane] = __fmul_rn(V.q[kap], af);
         if constexpr (COMMIT) {
-            S.pk[warp][lane] = pp;
+            S.pk[warp][lane] = af;
             for (int tau = 0; tau < t; ++tau) kd[tau * kRowsPerWarp + lane] = __fmul_rn(V.K[tau * kD + kap], al);
             kd[t * kRowsPerWarp + lane] = V.k[kap];
         }
@@ -267,12 +288,11 @@ __device__ __forceinline__ void window_first_phase(const DevFormat &F, const Win
     for (int h = 0; h < 2; ++h) cu[h][0] = cu[h][1] = co[h][0] = co[h][1] = make_float2(0.f, 0.f);
     static_for<0, kBlocks>([&](auto bc) {
         constexpr int b = decltype(bc)::value;
-        const float4 a4 = *reinterpret_cast<const float4 *>(&S.rw[warp][4 * b]);
         const uint8_t *blk = stg + fmt_offset<FMT, b>(F);
-        Tile T;   // only block b of it is live
+        Tile T;   // only block b of it is live: the exact codes
         with_width<FMT, b>(F, [&](auto wc) {
             constexpr int W = decltype(wc)::value;
-            dequant_slice<W, b>(blk, warp, lane, a4, T);
+            codes_slice<W, b>(blk, warp, lane, T);
         });
         const float4 k4 = *reinterpret_cast<const float4 *>(&S.kp[warp][4 * b]);
         const float4 q4 = *reinterpret_cast<const float4 *>(&S.qp[warp][4 * b]);
@@ -444,9 +464,9 @@ __global__ void __launch_bounds__(kThreads, 4) window_step_kernel(const DevForma
 
 // A committing step: one CTA barrier per page, after the first phase, since
 // every warp needs this step's delta D[t] for its own rows.  After it each
-// warp dequantizes its slices again (the page is intact in the stage until
-// the warp requantizes them), rebuilds T = RN(P' T0) and adds the entries in
-// order, takes the row maxima and requantizes in place; the stage is stored
+// warp dequantizes its slices again with the row factor, T = RN(z a') (the
+// page is intact in the stage until the warp requantizes them), adds the
+// entries in order, takes the row maxima and requantizes in place; the stage is stored
 // at the next page's barrier and refilled once the store has read it.
 template <class FMT>
 __global__ void __launch_bounds__(kThreads, 3) window_commit_kernel(const DevFormat F, const WindowArgs A) {
@@ -524,26 +544,19 @@ __global__ void __launch_bounds__(kThreads, 3) window_commit_kernel(const DevFor
         if (warp == (it & (kWarps - 1)))
             *reinterpret_cast<float4 *>(A.o + (size_t)p * kD + 4 * lane) = window_out(X, V.D, V.c, t, dt, lane);
 
-        // T = RN(P' T0), then the entries in order (per element one chain;
+        // T = RN(z a'), then the entries in order (per element one chain;
         // block by block, so that a block's codes and keys are the only
         // operands in registers besides T), and the row maxima
         const float2 dt01 = make_float2(dt.x, dt.y), dt23 = make_float2(dt.z, dt.w);
         Tile T;
         static_for<0, kBlocks>([&](auto bc) {
             constexpr int b = decltype(bc)::value;
-            const float4 a4 = *reinterpret_cast<const float4 *>(&S.rw[warp][4 * b]);
+            const float4 a4 = *reinterpret_cast<const float4 *>(&S.pk[warp][4 * b]);
             const uint8_t *blk = stg + fmt_offset<FMT, b>(F);
             with_width<FMT, b>(F, [&](auto wc) {
                 constexpr int W = decltype(wc)::value;
-                dequant_slice<W, b>(blk, warp, lane, a4, T);
+                dequant_slice<W, b>(blk, warp, lane, a4, T);   // RN(z a')
             });
-            const float4 p4 = *reinterpret_cast<const float4 *>(&S.pk[warp][4 * b]);
-            const float pv[4] = {p4.x, p4.y, p4.z, p4.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                T[b][i][0] = __fmul2_rn(T[b][i][0], make_float2(pv[i], pv[i]));
-                T[b][i][1] = __fmul2_rn(T[b][i][1], make_float2(pv[i], pv[i]));
-            }
 #pragma unroll 1
             for (int tau = 0; tau < t; ++tau) {
                 const float4 d = *reinterpret_cast<const float4 *>(V.D + tau * kD + 4 * lane);

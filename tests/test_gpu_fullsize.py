@@ -13,6 +13,8 @@ Samples: the first and last pages, both sides of the grid-wrap boundaries
 for 2 and 3 resident CTAs per SM, and seeded random positions.  Two chained
 steps (each side continues from its own result).  Bar: o, row scales and
 packed pages bit-identical, code mismatches only inside the rounding band.
+The per-window path (stq_window_step) is checked the same way over one whole
+window, its buffer rows included.
 """
 import numpy as np
 import pytest
@@ -116,3 +118,66 @@ def test_full_size_calibration_map():
     B.stq_calibrate(qs.state, S.cuda())
     torch.cuda.synchronize()
     assert np.array_equal(qs.perm().cpu().numpy(), perm)
+
+
+@pytest.mark.parametrize("index,window", [(1, 8), (2, 4), (3, 4), (4, 4)])
+def test_full_size_window_on_sampled_pages(index, window):
+    """A whole window of stq_window_step over the full batch (the launch
+    configuration the benchmark times), checked on the same kind of sampled
+    pages: o and the buffer rows bit-identical at every step, the committed
+    pages bit-identical outside the rounding band."""
+    w = W.WORKLOADS[index]
+    H, n = w.heads, w.pages
+    fmt = O.format_from_spec(w.format)
+    S_small = W.initial_state(w, batch=SMALL_BATCH).numpy()
+    perm = O.rank_rows(fmt, S_small)
+    pos = _sample_positions(n, w.seed + 1)
+    src = [(i % SMALL_BATCH, p % H) for i, p in enumerate(pos)]
+    pages = [O.quantize_page(fmt, S_small[b, h], perm[h]) for b, h in src]
+
+    qs = make_state(w)
+    qs.perm().copy_(torch.from_numpy(np.ascontiguousarray(perm, np.uint8)))
+    S_dev = W.initial_state(w, device="cuda")
+    B.stq_quantize_state(qs.state, S_dev)
+    del S_dev
+    torch.cuda.synchronize()
+    idx = torch.tensor(pos, dtype=torch.long, device="cuda")
+    qs.pages()[idx] = torch.from_numpy(np.stack([O.pack_page(fmt, pg) for pg in pages])).cuda()
+    nbuf = B.stq_window_buffer_bytes(qs.state, window)
+    buf = torch.full((nbuf,), 0xFF, dtype=torch.uint8, device="cuda")
+    rows = buf.view(torch.float32).view(n, 1 + 2 * window, 128)
+    Pb = [np.ones(128, np.float32) for _ in pos]
+    Kb = [np.zeros((window, 128), np.float32) for _ in pos]
+    Db = [np.zeros((window, 128), np.float32) for _ in pos]
+
+    seed = W.sr_seed(w)
+    o = torch.empty(w.batch, H, 128, device="cuda")
+    for t in range(window):
+        commit = t == window - 1
+        xd = W.step_inputs(w, 20 + t, device="cuda")
+        xc = W.step_inputs(w, 20 + t, batch=SMALL_BATCH)
+        for k in xd:
+            flat = xd[k].view(n, -1)
+            flat[idx] = torch.stack([xc[k][b, h].reshape(-1) for b, h in src]).cuda()
+        B.stq_window_step(qs.state, buf, window, t, commit, xd["q"], xd["k"], xd["v"], xd["alpha"], xd["beta"], o,
+                          seed=seed, step=t)
+        assert B.stq_device_status(qs.state) == B.STQ_OK
+        got_o = o.view(n, 128)[idx].cpu().numpy()
+        got_rows = rows[idx].cpu().numpy()
+        torch.cuda.synchronize()
+        got_pages = qs.pages()[idx].cpu().numpy()
+        for i, (p, (b, h)) in enumerate(zip(pos, src)):
+            o_ref, margin = O.window_step_f32(fmt, pages[i], perm[h], Pb[i], Kb[i], Db[i], t, commit,
+                                              xc["q"][b, h].numpy(), xc["k"][b, h].numpy(), xc["v"][b, h].numpy(),
+                                              xc["alpha"][b, h].numpy(), float(xc["beta"][b, h]), seed=seed, step=t,
+                                              b=p // H, h=p % H, want_margin=commit)
+            assert np.array_equal(got_o[i], o_ref), "o of page %d (t %d)" % (p, t)
+            if not commit:
+                assert np.array_equal(got_rows[i][0], Pb[i]), "P of page %d (t %d)" % (p, t)
+                assert np.array_equal(got_rows[i][1:2 + t], Kb[i][:t + 1]), "K of page %d (t %d)" % (p, t)
+                assert np.array_equal(got_rows[i][1 + window:2 + window + t], Db[i][:t + 1]), "D of page %d" % p
+            elif not np.array_equal(got_pages[i], O.pack_page(fmt, pages[i])):
+                pg = O.unpack_page(fmt, got_pages[i])
+                assert np.array_equal(pg.r.view(np.uint32), pages[i].r.view(np.uint32)), "r of page %d" % p
+                bad = pg.code != pages[i].code
+                assert np.all(margin[bad] < BAND), "codes of page %d outside the rounding band" % p
