@@ -377,6 +377,7 @@ __global__ void __launch_bounds__(kThreads, 4) window_step_kernel(const DevForma
     const int n = A.n_pages;
     const int NS = A.n_stages;
     const int H = A.heads;
+    const int sh = stride % H;
     const RowCtx R = row_ctx<FMT>(F, warp, lane);
 
     int p = (int)blockIdx.x;
@@ -392,7 +393,8 @@ __global__ void __launch_bounds__(kThreads, 4) window_step_kernel(const DevForma
     uint32_t parity = 0;
     for (int it = 0; p < n; ++it) {
         const int pn = p + stride;
-        const int pnh = pn % H;
+        int pnh = ph + sh;   // the head advances by stride mod H
+        if (pnh >= H) pnh -= H;
         float alpha_n = 0.f, beta_n = 0.f;
         int kap_n = 0;
         if (pn < n) {
