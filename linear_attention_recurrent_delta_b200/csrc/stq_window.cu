@@ -34,6 +34,7 @@ namespace stq {
 
 constexpr int kWindowMax = STQ_WINDOW_MAX;
 constexpr int kWindowStages = 4;          // ring depth at most
+constexpr int kRebuildGroup = 4;          // blocks per pass of a commit's entry loop (measured: 1, 2, 4)
 
 struct WindowArgs {
     uint8_t *pages;
@@ -551,33 +552,44 @@ __global__ void __launch_bounds__(kThreads, 3) window_commit_kernel(const DevFor
         // operands in registers besides T), and the row maxima
         const float2 dt01 = make_float2(dt.x, dt.y), dt23 = make_float2(dt.z, dt.w);
         Tile T;
-        static_for<0, kBlocks>([&](auto bc) {
-            constexpr int b = decltype(bc)::value;
-            const float4 a4 = *reinterpret_cast<const float4 *>(&S.pk[warp][4 * b]);
-            const uint8_t *blk = stg + fmt_offset<FMT, b>(F);
-            with_width<FMT, b>(F, [&](auto wc) {
-                constexpr int W = decltype(wc)::value;
-                dequant_slice<W, b>(blk, warp, lane, a4, T);   // RN(z a')
+        // blocks in groups of kRebuildGroup: each entry's delta row is read
+        // once per group
+        static_for<0, kBlocks / kRebuildGroup>([&](auto gc) {
+            constexpr int g = decltype(gc)::value;
+            static_for<0, kRebuildGroup>([&](auto jc) {
+                constexpr int b = g * kRebuildGroup + decltype(jc)::value;
+                const float4 a4 = *reinterpret_cast<const float4 *>(&S.pk[warp][4 * b]);
+                const uint8_t *blk = stg + fmt_offset<FMT, b>(F);
+                with_width<FMT, b>(F, [&](auto wc) {
+                    constexpr int W = decltype(wc)::value;
+                    dequant_slice<W, b>(blk, warp, lane, a4, T);   // RN(z a')
+                });
             });
 #pragma unroll 1
             for (int tau = 0; tau < t; ++tau) {
                 const float4 d = *reinterpret_cast<const float4 *>(V.D + tau * kD + 4 * lane);
-                const float4 k4 = *reinterpret_cast<const float4 *>(kd + tau * kRowsPerWarp + 4 * b);
+                static_for<0, kRebuildGroup>([&](auto jc) {
+                    constexpr int b = g * kRebuildGroup + decltype(jc)::value;
+                    const float4 k4 = *reinterpret_cast<const float4 *>(kd + tau * kRowsPerWarp + 4 * b);
+                    const float kv[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        T[b][i][0] = __ffma2_rn(make_float2(kv[i], kv[i]), make_float2(d.x, d.y), T[b][i][0]);
+                        T[b][i][1] = __ffma2_rn(make_float2(kv[i], kv[i]), make_float2(d.z, d.w), T[b][i][1]);
+                    }
+                });
+            }
+            static_for<0, kRebuildGroup>([&](auto jc) {
+                constexpr int b = g * kRebuildGroup + decltype(jc)::value;
+                const float4 k4 = *reinterpret_cast<const float4 *>(kd + t * kRowsPerWarp + 4 * b);
                 const float kv[4] = {k4.x, k4.y, k4.z, k4.w};
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    T[b][i][0] = __ffma2_rn(make_float2(kv[i], kv[i]), make_float2(d.x, d.y), T[b][i][0]);
-                    T[b][i][1] = __ffma2_rn(make_float2(kv[i], kv[i]), make_float2(d.z, d.w), T[b][i][1]);
+                    T[b][i][0] = __ffma2_rn(make_float2(kv[i], kv[i]), dt01, T[b][i][0]);
+                    T[b][i][1] = __ffma2_rn(make_float2(kv[i], kv[i]), dt23, T[b][i][1]);
+                    S.inv[warp][4 * b + i] = warp_absmax(absmax4(T[b][i][0], T[b][i][1]));
                 }
-            }
-            const float4 k4 = *reinterpret_cast<const float4 *>(kd + t * kRowsPerWarp + 4 * b);
-            const float kv[4] = {k4.x, k4.y, k4.z, k4.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                T[b][i][0] = __ffma2_rn(make_float2(kv[i], kv[i]), dt01, T[b][i][0]);
-                T[b][i][1] = __ffma2_rn(make_float2(kv[i], kv[i]), dt23, T[b][i][1]);
-                S.inv[warp][4 * b + i] = warp_absmax(absmax4(T[b][i][0], T[b][i][1]));
-            }
+            });
         });
         if (tid == 0 && p_prev >= 0) {
             // refill the previous page's stage with the page NS - 1 ahead of this one
