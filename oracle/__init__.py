@@ -56,6 +56,8 @@ def lib():
         L.orc_step_f32.argtypes = [P, P, P, P, P, P, P, c_float, P, c_uint64, c_uint32,
                                    c_uint32, c_uint32, P, P]
         L.orc_step_f64.argtypes = [P, P, P, P, P, P, P, c_float, P, P]
+        L.orc_prefill_f32.argtypes = [P, P, P, c_int, P, P, P, P, P, P, c_uint64, c_uint32, c_uint32, c_uint32,
+                                      P, P]
         L.orc_window_step_f32.argtypes = [P, P, P, P, P, P, c_int, c_int, P, P, P, P, c_float, P, c_uint64,
                                           c_uint32, c_uint32, c_uint32, P]
         L.orc_pack_page.argtypes = [P, P, P]
@@ -204,6 +206,25 @@ def window_step_f32(fmt, page, perm, P, K, D, t, commit, q, k, v, alpha, beta, s
                                   int(commit), _p(q), _p(k), _p(v), _p(a), float(beta), _p(o), int(seed),
                                   int(step), int(b), int(h), _p(mg)), "window_step_f32")
     return o, mg
+
+
+def prefill_f32(fmt, page, perm, q, k, v, alpha, beta, seed=0, step=0, b=0, h=0, want_tp=False,
+                want_margin=False):
+    """A prompt of L tokens through one page (page requantized in place at
+    the end).  q, k, v: [L, 128]; alpha: [L] or [L, 128]; beta: [L].
+    Returns (o [L, d_v], T before requantization or None, margin or None)."""
+    perm = np.ascontiguousarray(perm, np.int32)
+    q, k, v = (np.ascontiguousarray(x, np.float32) for x in (q, k, v))
+    L = q.shape[0]
+    a = np.ascontiguousarray(np.asarray(alpha, np.float32).reshape(L, -1)[:, :fmt.d_k if fmt.gate_vector else 1])
+    bt = np.ascontiguousarray(np.asarray(beta, np.float32).reshape(L))
+    o = np.zeros((L, fmt.d_v), np.float32)
+    tp = np.zeros((fmt.d_k, fmt.d_v), np.float32) if want_tp else None
+    mg = np.zeros((fmt.d_k, fmt.d_v), np.float64) if want_margin else None
+    st = page._struct()
+    _ok(lib().orc_prefill_f32(ctypes.byref(fmt), ctypes.byref(st), _p(perm), int(L), _p(q), _p(k), _p(v), _p(a),
+                              _p(bt), _p(o), int(seed), int(step), int(b), int(h), _p(tp), _p(mg)), "prefill_f32")
+    return o, tp, mg
 
 
 def step_f64(fmt, page, perm, q, k, v, alpha, beta):

@@ -628,6 +628,58 @@ extern "C" int orc_window_step_f32(const orc_format *f, orc_page *page, const in
     return 0;
 }
 
+/* ------------------------------------------------------------------------ */
+/* prefill: a prompt of L tokens through one page, one requantization       */
+/* ------------------------------------------------------------------------ */
+
+extern "C" int orc_prefill_f32(const orc_format *f, orc_page *page, const int32_t *perm, int L,
+                               const float *q, const float *k, const float *v,
+                               const float *alpha, const float *beta, float *o_out,
+                               uint64_t seed, uint32_t step, uint32_t b, uint32_t h,
+                               float *Tp_out, double *margin_out)
+{
+    if (orc_format_check(f) != 0 || !page || !perm || L < 1 || !q || !k || !v || !alpha || !beta || !o_out)
+        return -1;
+    const int d_k = f->d_k, d_v = f->d_v;
+    const int na = f->gate_vector ? d_k : 1;
+    std::vector<float> ic(d_v), T((size_t)d_k * d_v), u(d_v), e(d_v), ot(d_v);
+    for (int j = 0; j < d_v; ++j) ic[j] = f->col_scales ? 1.0f / page->c[j] : 1.0f;
+
+    for (int l = 0; l < L; ++l) {
+        const float *ql = q + (size_t)l * d_k, *kl = k + (size_t)l * d_k, *vl = v + (size_t)l * d_v;
+        const float *al = alpha + (size_t)l * na;
+        /* decay: the first token dequantizes the page with the gate folded
+         * into the row scale, T = z (alpha r), as the decode step does; later
+         * tokens decay the fp32 state in place, T = alpha T */
+        for (int s = 0; s < d_k; ++s) {
+            const float a_s = f->gate_vector ? al[perm[s]] : al[0];
+            if (l == 0) {
+                const float a = (orc_row_kind(f, s) == ORC_KIND_INT) ? a_s * page->r[s] : a_s;
+                for (int j = 0; j < d_v; ++j) T[(size_t)s * d_v + j] = element_value(f, page, s, j) * a;
+            } else {
+                for (int j = 0; j < d_v; ++j) T[(size_t)s * d_v + j] = a_s * T[(size_t)s * d_v + j];
+            }
+        }
+        /* the decode step's prediction, rank-1 update and readout */
+        column_sum(f, perm, kl, T.data(), u.data());
+        for (int j = 0; j < d_v; ++j) e[j] = vl[j] * ic[j] - u[j];
+        for (int s = 0; s < d_k; ++s) {
+            const float bk = beta[l] * kl[perm[s]];
+            for (int j = 0; j < d_v; ++j) {
+                const size_t i = (size_t)s * d_v + j;
+                T[i] = std::fmaf(bk, e[j], T[i]);
+            }
+        }
+        column_sum(f, perm, ql, T.data(), ot.data());
+        for (int j = 0; j < d_v; ++j) o_out[(size_t)l * d_v + j] = f->col_scales ? page->c[j] * ot[j] : ot[j];
+    }
+    if (Tp_out) std::memcpy(Tp_out, T.data(), sizeof(float) * T.size());
+    for (int s = 0; s < d_k; ++s)
+        requant_row(f, s, T.data() + (size_t)s * d_v, page, seed, step, b, h, f->stochastic,
+                    margin_out ? margin_out + (size_t)s * d_v : nullptr);
+    return 0;
+}
+
 extern "C" int orc_step_f64(const orc_format *f, const orc_page *page, const int32_t *perm,
                             const float *q, const float *k, const float *v,
                             const float *alpha, float beta, double *o_out, double *Sp_out)

@@ -138,6 +138,25 @@ int orc_window_step_f32(const orc_format *f, orc_page *page, const int32_t *perm
                         uint64_t seed, uint32_t step, uint32_t b, uint32_t h,
                         double *margin_out);
 
+/* ---- prefill: a prompt of L tokens through one page --------------------
+ * The page's state runs through L decode steps in fp32 without being
+ * requantized between them, then is requantized once (the step before decode
+ * that builds the state from a prompt; "repeated prefill" on the DASC card
+ * page).  Token 0 dequantizes and decays the page exactly as orc_step_f32
+ * (T = z (alpha r)); token l > 0 decays the fp32 state in place,
+ * T = RN(alpha T); each token then takes orc_step_f32's prediction, update
+ * and readout in its canonical order.  q, k: [L][d_k], v, o_out: [L][d_v],
+ * alpha: [L][d_k] (gate_vector) or [L], beta: [L].  After the last token the
+ * rows are requantized as orc_step_f32 requantizes (seed, step, b, h: the
+ * stochastic-rounding counter).  Tp_out (optional): the final T before the
+ * requantization, stored order, column-normalised.  With L = 1 this is
+ * orc_step_f32. */
+int orc_prefill_f32(const orc_format *f, orc_page *page, const int32_t *perm, int L,
+                    const float *q, const float *k, const float *v,
+                    const float *alpha, const float *beta, float *o_out,
+                    uint64_t seed, uint32_t step, uint32_t b, uint32_t h,
+                    float *Tp_out, double *margin_out);
+
 /* ---- packed byte layout (d_k = d_v = 128, row groups multiples of 16) ---- */
 int orc_pack_page(const orc_format *f, const orc_page *p, uint8_t *bytes);
 int orc_unpack_page(const orc_format *f, const uint8_t *bytes, orc_page *p);

@@ -18,7 +18,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "stq_oracle.cpp")
 HDR = os.path.join(ROOT, "oracle", "stq_oracle.h")
 PIN_FILES = ["tests/test_oracle_scalars.py", "tests/test_oracle_format.py",
-             "tests/test_oracle_quantize.py", "tests/test_oracle_step.py", "tests/test_oracle_window.py"]
+             "tests/test_oracle_quantize.py", "tests/test_oracle_step.py", "tests/test_oracle_window.py",
+             "tests/test_oracle_prefill.py"]
 
 MUTANTS = {
     "error sign": ("e[j] = v[j] * ic[j] - u[j];", "e[j] = v[j] * ic[j] + u[j];"),
@@ -60,6 +61,10 @@ MUTANTS = {
                                "for (int kap = 0; kap < d_k; ++kap) P[kap] = P[kap];"),
     "window start keeps the old decay": ("const float p0 = (t == 0) ? 1.0f : P[kap];",
                                          "const float p0 = P[kap];"),
+    "prefill later tokens not decayed": ("for (int j = 0; j < d_v; ++j) T[(size_t)s * d_v + j] = a_s * T[(size_t)s * d_v + j];",
+                                         "for (int j = 0; j < d_v; ++j) T[(size_t)s * d_v + j] = T[(size_t)s * d_v + j];"),
+    "prefill first beta for every token": ("const float bk = beta[l] * kl[perm[s]];", "const float bk = beta[0] * kl[perm[s]];"),
+    "prefill readout with k": ("column_sum(f, perm, ql, T.data(), ot.data());", "column_sum(f, perm, kl, T.data(), ot.data());"),
     "window butterfly half": ("for (int off = lanes / 2; off >= 1; off /= 2) {",
                               "for (int off = lanes / 2; off >= 2; off /= 2) {"),
 }
