@@ -241,6 +241,32 @@ stq_status stq_window_step(stq_state *s, void *d_buf, size_t buf_bytes, int wind
                            const float *d_q, const float *d_k, const float *d_v, const float *d_alpha,
                            const float *d_beta, float *d_o, uint64_t seed, uint32_t step, void *stream);
 
+/* ---- prefill ------------------------------------------------------------
+ * A prompt of L tokens through every page: the step before decode that
+ * builds the state from a prompt ("repeated prefill", DASC card page).  Each
+ * page's state runs through L decode steps in fp32 -- token 0 dequantizes and
+ * decays the page exactly as stq_decode_step, token l > 0 decays the fp32
+ * state in place (T = alpha T); every token then takes the decode step's
+ * prediction, rank-1 update and readout -- and is requantized once, after
+ * the last token, as stq_decode_step requantizes (row scales re-derived,
+ * column scales kept; stochastic rounding with `step`).  With L = 1 this is
+ * stq_decode_step.  To build a state from nothing, quantize a zero state
+ * first (stq_quantize_state: codes 0, r = 0, c = 1).
+ *   d_q, d_k, d_v, d_o: [L][B][H][128]; d_alpha: [L][B][H] or
+ *   [L][B][H][128] (gate_vector); d_beta: [L][B][H]; alignment as
+ *   stq_decode_step.  L >= 1 and L * B * H <= 2^31 - 16.
+ *   d_S_out (optional, NULL = none): [B][H][128][128] fp32, 16-byte aligned,
+ *   natural key order: the state after the last token before the
+ *   requantization, S = T c; a caller can calibrate and quantize it afresh
+ *   (stq_calibrate, stq_quantize_state) to fit new column scales.
+ * No buffer may overlap the state, an input or another output.  Programmatic
+ * dependent launch as stq_decode_step.  Errors: INVALID_ARG, MISALIGNED,
+ * CUDA; a bounded wait that ran out is reported by stq_device_status, and
+ * then pages that were not finished keep their codes. */
+stq_status stq_prefill(stq_state *s, int L, const float *d_q, const float *d_k, const float *d_v,
+                       const float *d_alpha, const float *d_beta, float *d_o, float *d_S_out, uint64_t seed,
+                       uint32_t step, void *stream);
+
 /* Device staging bytes stq_decode_step_host needs (q, k, v, alpha, beta, o). */
 size_t stq_decode_io_bytes(const stq_state *s);
 

@@ -61,6 +61,7 @@ def lib():
         "stq_request_pages": (c_int, [P, c_int, POINTER(c_size_t), POINTER(c_size_t)]),
         "stq_window_buffer_bytes": (c_size_t, [P, c_int]),
         "stq_window_step": (c_int, [P, P, c_size_t, c_int, c_int, c_int, P, P, P, P, P, P, c_uint64, c_uint32, P]),
+        "stq_prefill": (c_int, [P, c_int, P, P, P, P, P, P, P, c_uint64, c_uint32, P]),
         "stq_decode_io_bytes": (c_size_t, [P]),
         "stq_decode_step_host": (c_int, [P, P, P, P, P, P, P, P, c_size_t, c_uint64, c_uint32, P]),
         "stq_dequantize_state": (c_int, [P, P, P]),
@@ -204,6 +205,12 @@ def stq_window_step(state, buf, window, t, commit, q, k, v, alpha, beta, o, seed
     _check(lib().stq_window_step(state.handle, _ptr(buf), buf.numel() * buf.element_size(), int(window), int(t),
                                  int(bool(commit)), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(o),
                                  int(seed), int(step), _stream(stream)), "stq_window_step")
+
+
+def stq_prefill(state, q, k, v, alpha, beta, o, S_out=None, seed=0, step=0, stream=None):
+    """A prompt of L = q.shape[0] tokens through every page (q, k, v, o: [L, B, H, 128])."""
+    _check(lib().stq_prefill(state.handle, int(q.shape[0]), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),
+                             _ptr(o), _ptr(S_out), int(seed), int(step), _stream(stream)), "stq_prefill")
 
 
 def stq_decode_io_bytes(state):

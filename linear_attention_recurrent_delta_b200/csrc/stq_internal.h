@@ -43,6 +43,10 @@ cudaError_t launch_window(const stq_state *s, uint8_t *buf, int window, int t, b
                           const float *k, const float *v, const float *alpha, const float *beta, float *o,
                           uint64_t seed, uint32_t step, int stall_first_wait, bool early_launch,
                           cudaStream_t stream);
+// Prefill: a prompt of L tokens through every page, one requantization.
+cudaError_t launch_prefill(const stq_state *s, int L, const float *q, const float *k, const float *v,
+                           const float *alpha, const float *beta, float *o, float *S_out, uint64_t seed,
+                           uint32_t step, int stall_first_wait, bool early_launch, cudaStream_t stream);
 cudaError_t launch_calibrate(const stq_state *s, const float *S, const float *row_weight,
                              double *workspace, cudaStream_t stream);
 size_t calibrate_workspace_bytes(int batch, int heads);

@@ -211,3 +211,29 @@ def test_window_step_checks_arguments(lib):
     assert call(buf=base) == B.STQ_ERR_INVALID_ARG           # the buffer overlaps q
     assert lib.stq_window_step(None, P(buf), need, 4, 0, 0, q, k, v, a, b, o, 0, 0, None) == B.STQ_ERR_INVALID_ARG
     lib.stq_state_free(h)
+
+
+def test_prefill_checks_arguments(lib):
+    fmt = B.format_from_spec(W.FORMATS["stepquant4_kda"])
+    st, h = _alloc(lib, fmt, 2, 3)
+    assert st == B.STQ_OK
+    P = ctypes.c_void_p
+    base = 1 << 41
+    q, k, v, a, b, o = (base + i * (1 << 26) for i in range(6))
+    S = 1 << 45
+
+    def call(L=4, q=q, a=a, o=o, S_out=None, state=h):
+        return lib.stq_prefill(state, L, P(q) if q else None, P(k), P(v), P(a), P(b), P(o),
+                               P(S_out) if S_out else None, 0, 0, None)
+
+    assert call(state=None) == B.STQ_ERR_INVALID_ARG
+    assert call(q=0) == B.STQ_ERR_INVALID_ARG
+    assert call(L=0) == B.STQ_ERR_INVALID_ARG
+    assert call(L=2**30) == B.STQ_ERR_INVALID_ARG                # L * pages must stay below 2^31
+    assert call(q=q + 4) == B.STQ_ERR_MISALIGNED
+    assert call(a=a + 4) == B.STQ_ERR_MISALIGNED                  # a vector gate needs 16-byte alignment
+    assert call(S_out=S + 8) == B.STQ_ERR_MISALIGNED
+    assert call(o=q + 256) == B.STQ_ERR_INVALID_ARG               # output overlaps an input
+    assert call(o=FAKE + 512) == B.STQ_ERR_INVALID_ARG            # output overlaps the state
+    assert call(S_out=o) == B.STQ_ERR_INVALID_ARG                 # the state output overlaps o
+    lib.stq_state_free(h)
