@@ -321,6 +321,55 @@ def run_window(w, window, steps, warmup, rank, world):
     return {"ms": ms, "steps": steps, "per_t_ms": per_t}
 
 
+# FP32 peak of the CUDA cores for the prefill's plain arithmetic: 148 SMs x
+# 128 FP32 lanes x 2 flops per fma x 1.965 GHz (clocks.max.sm).
+FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def prefill_flops_per_head_token():
+    """Per page and token: the decay (one multiply per element; the first
+    token's dequantization instead), the prediction, the update and the
+    readout (one fma each per element)."""
+    return 128 * 128 * (1 + 2 + 2 + 2)
+
+
+def run_prefill(w, L, steps, warmup, rank, world):
+    """stq_prefill of an L-token prompt over the whole batch, K times (each
+    from the state the previous left).  Returns the device time (max over ranks)."""
+    from linear_attention_recurrent_delta_b200 import binding as B
+    dev = torch.device("cuda", torch.cuda.current_device())
+    wr = R.rank_workload(w, rank)
+    qs = B.QuantizedState(wr.format, wr.batch, wr.heads, device=dev)
+    S = W.initial_state(wr, device=dev)
+    qs.calibrate_and_quantize(S)
+    del S
+    xs = [W.step_inputs(wr, l, device=dev) for l in range(L)]
+    x = {k: torch.stack([xi[k] for xi in xs]).contiguous() for k in xs[0]}
+    del xs
+    o = torch.empty(L, wr.batch, wr.heads, 128, device=dev)
+    seed = W.sr_seed(wr)
+    stream = torch.cuda.current_stream()
+    for i in range(max(warmup, 3)):
+        B.stq_prefill(qs.state, x["q"], x["k"], x["v"], x["alpha"], x["beta"], o, None, seed, i, stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for i in range(steps):
+        B.stq_prefill(qs.state, x["q"], x["k"], x["v"], x["alpha"], x["beta"], o, None, seed, 100 + i, stream)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    status = B.stq_device_status(qs.state)
+    if status != B.STQ_OK:
+        raise RuntimeError("device status: %s" % B.stq_status_string(status))
+    ms = max_over_ranks(ev0.elapsed_time(ev1), world)
+    barrier(world)
+    del qs, x, o
+    torch.cuda.empty_cache()
+    return {"ms": ms, "steps": steps}
+
+
 class OracleSample:
     """The CPU oracle (single thread, as written) stepping a sample of the
     workload's pages: the first ``n_pages`` pages of a batch whose fp32 state
@@ -439,6 +488,8 @@ def main():
                     help="with --profile: step through the slot table (stq_decode_step_slots)")
     ap.add_argument("--window", type=int, default=0,
                     help="with --profile: per-window steps (stq_window_step) of this window length")
+    ap.add_argument("--prefill", type=int, default=0,
+                    help="with --profile: stq_prefill of a prompt of this many tokens")
     ap.add_argument("--profile", action="store_true",
                     help="decode steps only: no clock sampling, e2e, CPU baseline or other workloads")
     args = ap.parse_args()
@@ -487,6 +538,13 @@ def main():
     if rank == 0:
         build_mod.build()
     barrier(world)
+    if args.profile and args.prefill:
+        r = run_prefill(w, args.prefill, args.steps, args.warmup, rank, world)
+        if rank == 0:
+            print(json.dumps({"workload": w.name, "batch": w.batch, "prompt": args.prefill,
+                              "ms_per_prefill": r["ms"] / r["steps"]}))
+        R.finish(world)
+        return
     if args.profile and args.window:
         r = run_window(w, args.window, args.steps, args.warmup, rank, world)
         if rank == 0:
@@ -524,6 +582,19 @@ def main():
             windows["W%d" % wl] = {"value": R.aggregate_rate(w.pages, world, r["steps"], r["ms"]), "unit": UNIT,
                                    "hbm_gbs": gbs, "frac_of_%s_peak" % peak_kind: gbs / peak,
                                    "bytes_per_head_step": b, "ms_per_position": r["per_t_ms"]}
+
+    prefill = {}
+    if not args.only:
+        fl = prefill_flops_per_head_token()
+        for L in (16, 64):
+            r = run_prefill(w, L, max(20, args.steps // 500), args.warmup, rank, world)
+            rate = R.aggregate_rate(w.pages * L, world, r["steps"], r["ms"])
+            prefill["L%d" % L] = {"value": rate, "unit": "head-tokens/s", "prompt": L,
+                                  "ms_per_prefill": r["ms"] / r["steps"],
+                                  "roofline": {"bound": "alu", "achieved": rate * fl / 1e12,
+                                               "peak": FP32_PEAK_TFLOPS, "unit": "TFLOP/s",
+                                               "frac": rate * fl / 1e12 / FP32_PEAK_TFLOPS,
+                                               "flops_per_head_token": fl}}
 
     others = {}
     if not args.only:
@@ -570,6 +641,9 @@ def main():
         "clocks": res["clocks"],
         "other_workloads": others,
         "paged_step": paged,
+        "prefill": ({"entry_point": "stq_prefill", "kernel": "stq::prefill_kernel",
+                     "peak_kind": "derived: 148 SMs x 128 FP32 lanes x 2 x 1.965 GHz", "prompts": prefill}
+                    if prefill else None),
         "window_decode": ({"entry_point": "stq_window_step",
                            "kernels": ["stq::window_step_kernel", "stq::window_commit_kernel"],
                            "windows": windows} if windows else None),
