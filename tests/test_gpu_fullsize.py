@@ -13,7 +13,8 @@ Samples: the first and last pages, both sides of the grid-wrap boundaries
 for 2 and 3 resident CTAs per SM, and seeded random positions.  Two chained
 steps (each side continues from its own result).  Bar: o, row scales and
 packed pages bit-identical, code mismatches only inside the rounding band.
-The per-window path (stq_window_step) is checked the same way over one whole
+The per-window path (stq_window_step) and the prefill (stq_prefill, a
+64-token prompt) are checked the same way, the window over one whole
 window, its buffer rows included.
 """
 import numpy as np
@@ -181,3 +182,58 @@ def test_full_size_window_on_sampled_pages(index, window):
                 assert np.array_equal(pg.r.view(np.uint32), pages[i].r.view(np.uint32)), "r of page %d" % p
                 bad = pg.code != pages[i].code
                 assert np.all(margin[bad] < BAND), "codes of page %d outside the rounding band" % p
+
+
+def test_full_size_prefill_on_sampled_pages():
+    """stq_prefill of a 64-token prompt over the full default batch (the
+    benchmark's launch configuration), checked on sampled pages: o of every
+    token and the fp32 state bit-identical, pages bit-identical outside the
+    rounding band."""
+    w = W.WORKLOADS[1]
+    H, n, L = w.heads, w.pages, 64
+    fmt = O.format_from_spec(w.format)
+    S_small = W.initial_state(w, batch=SMALL_BATCH).numpy()
+    perm = O.rank_rows(fmt, S_small)
+    pos = _sample_positions(n, w.seed + 2)
+    src = [(i % SMALL_BATCH, p % H) for i, p in enumerate(pos)]
+    pages = [O.quantize_page(fmt, S_small[b, h], perm[h]) for b, h in src]
+
+    qs = make_state(w)
+    qs.perm().copy_(torch.from_numpy(np.ascontiguousarray(perm, np.uint8)))
+    S_dev = W.initial_state(w, device="cuda")
+    B.stq_quantize_state(qs.state, S_dev)
+    del S_dev
+    torch.cuda.synchronize()
+    idx = torch.tensor(pos, dtype=torch.long, device="cuda")
+    qs.pages()[idx] = torch.from_numpy(np.stack([O.pack_page(fmt, pg) for pg in pages])).cuda()
+
+    xd = {k: torch.stack([W.step_inputs(w, 40 + l, device="cuda")[k] for l in range(L)]).contiguous()
+          for k in ("q", "k", "v", "alpha", "beta")}
+    xc = [W.step_inputs(w, 40 + l, batch=SMALL_BATCH) for l in range(L)]
+    for k in xd:
+        flat = xd[k].view(L, n, -1)
+        flat[:, idx] = torch.stack([torch.stack([xc[l][k][b, h].reshape(-1) for b, h in src]) for l in range(L)]).cuda()
+    seed = W.sr_seed(w)
+    o = torch.empty(L, w.batch, H, 128, device="cuda")
+    S_out = torch.empty(w.batch, H, 128, 128, device="cuda")
+    B.stq_prefill(qs.state, xd["q"], xd["k"], xd["v"], xd["alpha"], xd["beta"], o, S_out, seed=seed, step=3)
+    assert B.stq_device_status(qs.state) == B.STQ_OK
+    got_o = o.view(L, n, 128)[:, idx].cpu().numpy()
+    got_S = S_out.view(n, 128, 128)[idx].cpu().numpy()
+    torch.cuda.synchronize()
+    got_pages = qs.pages()[idx].cpu().numpy()
+    for i, (p, (b, h)) in enumerate(zip(pos, src)):
+        arr = {k: np.stack([xc[l][k][b, h].numpy().reshape(-1) for l in range(L)]) for k in xd}
+        o_ref, tp, margin = O.prefill_f32(fmt, pages[i], perm[h], arr["q"], arr["k"], arr["v"], arr["alpha"],
+                                          arr["beta"][:, 0], seed=seed, step=3, b=p // H, h=p % H, want_tp=True,
+                                          want_margin=True)
+        assert np.array_equal(got_o[:, i], o_ref), "o of page %d" % p
+        S_ref = np.zeros((128, 128), np.float32)
+        c = pages[i].c if fmt.col_scales else np.ones(128, np.float32)
+        S_ref[perm[h]] = tp * c[None, :]
+        assert np.array_equal(got_S[i], S_ref), "state of page %d" % p
+        if not np.array_equal(got_pages[i], O.pack_page(fmt, pages[i])):
+            pg = O.unpack_page(fmt, got_pages[i])
+            assert np.array_equal(pg.r.view(np.uint32), pages[i].r.view(np.uint32)), "r of page %d" % p
+            bad = pg.code != pages[i].code
+            assert np.all(margin[bad] < BAND), "codes of page %d outside the rounding band" % p
