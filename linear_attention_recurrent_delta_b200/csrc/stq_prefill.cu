@@ -50,6 +50,8 @@ struct PrefillSmem {
     float inv[kWarps][kRowsPerWarp];         // row maxima, then requant multipliers
     float red_u[2][kWarps][kD];              // per token parity and warp: chain sums of u
     float red_o[2][kWarps][kD];              // the same for o
+    float beta_t[kD];                        // beta of the page's tokens 128 m .. 128 m + 127
+    float alpha_t[kD];                       // the scalar gate of the same tokens (GDN)
     float ic[kD];                            // the page's 1 / c
     float cpg[kD];                           // the page's c
     uint64_t pfull[2];                       // page buffers
@@ -159,6 +161,17 @@ __global__ void __launch_bounds__(kThreads, 3) prefill_kernel(const DevFormat F,
         }
         Tile T;
         for (int l = 0; l < L; ++l) {
+            if ((l & (kD - 1)) == 0) {
+                // beta (and a scalar gate) of the next 128 tokens of the page,
+                // thread t: token l + t
+                __syncthreads();   // every warp is done with the previous ones
+                if (l + tid < L) {
+                    const size_t si = (size_t)(l + tid) * n + p;
+                    S.beta_t[tid] = __ldg(A.beta + si);
+                    if (!gate_vector) S.alpha_t[tid] = __ldg(A.alpha + si);
+                }
+                __syncthreads();
+            }
             const bool first = l == 0;   // token 0 dequantizes the page, later ones decay T
             const int st = g & (kTokenStages - 1);
             const int par = g & 1;
@@ -170,10 +183,9 @@ __global__ void __launch_bounds__(kThreads, 3) prefill_kernel(const DevFormat F,
             const float *k_s = q_s + kD;
             const float *v_s = q_s + 2 * kD;
             const float *al_s = q_s + 3 * kD;
-            const size_t sidx = (size_t)l * n + p;
-            const float beta = __ldg(A.beta + sidx);
+            const float beta = S.beta_t[l & (kD - 1)];
             {
-                const float al = gate_vector ? al_s[kap] : __ldg(A.alpha + sidx);
+                const float al = gate_vector ? al_s[kap] : S.alpha_t[l & (kD - 1)];
                 const float kk = k_s[kap];
                 S.a[warp][lane] = (first && (R.all_int || R.is_int)) ? __fmul_rn(al, r_me) : al;
                 S.kp[warp][lane] = kk;
