@@ -12,6 +12,10 @@ state alone 138 MB-2.5 GB) through the 126 MB L2, so no flush is needed
 between steps.  Under torchrun each rank runs its own batch (weak
 scaling, no collective on the data path); time is the max over ranks.
 
+The same line also reports the per-window path (stq_window_step, windows
+of 4, 8 and 16 steps) and the prefill (stq_prefill, prompts of 16 and 64
+tokens) on the default workload, each with its own roofline.
+
 --impl reference times the CPU oracle (single thread, as written) on a
 bounded sample of the same workload; only rank 0 runs it.
 """
