@@ -56,6 +56,7 @@ def lib():
         L.orc_step_f32.argtypes = [P, P, P, P, P, P, P, c_float, P, c_uint64, c_uint32,
                                    c_uint32, c_uint32, P, P]
         L.orc_step_f64.argtypes = [P, P, P, P, P, P, P, c_float, P, P]
+        L.orc_lifetime_weights.argtypes = [P, c_int, c_int, c_int, P, P]
         L.orc_prefill_f32.argtypes = [P, P, P, c_int, P, P, P, P, P, P, c_uint64, c_uint32, c_uint32, c_uint32,
                                       P, P]
         L.orc_window_step_f32.argtypes = [P, P, P, P, P, P, c_int, c_int, P, P, P, P, c_float, P, c_uint64,
@@ -149,6 +150,16 @@ def rank_rows(fmt, S, row_weight=None):
     rw = None if row_weight is None else np.ascontiguousarray(row_weight, np.float32)
     _ok(lib().orc_rank_rows(ctypes.byref(fmt), B, H, _p(S), _p(rw), _p(perm)), "rank_rows")
     return perm
+
+
+def lifetime_weights(fmt, alpha):
+    """Row weights [H, d_k] from gate samples alpha [n_samples, B, H] or
+    [n_samples, B, H, d_k] (gate_vector)."""
+    alpha = np.ascontiguousarray(alpha, np.float32)
+    n, B, H = alpha.shape[:3]
+    w = np.zeros((H, fmt.d_k), np.float32)
+    _ok(lib().orc_lifetime_weights(ctypes.byref(fmt), B, H, n, _p(alpha), _p(w)), "lifetime_weights")
+    return w
 
 
 def quantize_page(fmt, S_nat, perm):

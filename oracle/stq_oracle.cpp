@@ -680,6 +680,35 @@ extern "C" int orc_prefill_f32(const orc_format *f, orc_page *page, const int32_
     return 0;
 }
 
+/* ------------------------------------------------------------------------ */
+/* lifetime weights from gate samples                                       */
+/* ------------------------------------------------------------------------ */
+
+extern "C" int orc_lifetime_weights(const orc_format *f, int B, int H, int n_samples, const float *alpha,
+                                    float *row_weight)
+{
+    if (orc_format_check(f) != 0 || B < 1 || H < 1 || n_samples < 1 || !alpha || !row_weight) return -1;
+    const int d_k = f->d_k;
+    const int na = f->gate_vector ? d_k : 1;
+    for (int h = 0; h < H; ++h) {
+        for (int kap = 0; kap < d_k; ++kap) {
+            /* the mean gate over the samples and requests, summed sample by
+             * sample, requests ascending, in double */
+            double sum = 0.0;
+            for (int t = 0; t < n_samples; ++t)
+                for (int b = 0; b < B; ++b)
+                    sum += (double)alpha[(((size_t)t * B + b) * H + h) * na + (f->gate_vector ? kap : 0)];
+            const double mean = sum / ((double)n_samples * (double)B);
+            /* expected persistence under geometric decay: 1 / (1 - mean),
+             * capped at 2^24 (a gate of one keeps its content for ever) */
+            const double gap = 1.0 - mean;
+            const double w = (gap <= 0x1p-24) ? 0x1p24 : 1.0 / gap;
+            row_weight[(size_t)h * d_k + kap] = (float)w;
+        }
+    }
+    return 0;
+}
+
 extern "C" int orc_step_f64(const orc_format *f, const orc_page *page, const int32_t *perm,
                             const float *q, const float *k, const float *v,
                             const float *alpha, float beta, double *o_out, double *Sp_out)

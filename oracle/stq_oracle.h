@@ -79,6 +79,19 @@ long orc_page_bytes(const orc_format *f);          /* packed bytes per page (d =
 int orc_rank_rows(const orc_format *f, int B, int H, const float *S,
                   const float *row_weight, int32_t *perm_out);
 
+/* ---- lifetime weights (STEPQuant's temporal allocation) -----------------
+ * Per head h and key channel kappa, the expected persistence of what the
+ * channel stores under geometric decay with the mean gate,
+ * w = 1 / (1 - mean(alpha)) (capped at 2^24), as the row_weight of
+ * orc_rank_rows: channels that keep their content longer rank higher
+ * (STEPQuant landing page: errors in long-lived memory persist across many
+ * steps; Figure B1: long gate half-lives hold most of the quantization
+ * error).  alpha: [n_samples][B][H][d_k] (gate_vector) or [n_samples][B][H];
+ * the mean is a double sum over samples, then requests, ascending, divided
+ * by n_samples * B; row_weight: [H][d_k], rounded to float. */
+int orc_lifetime_weights(const orc_format *f, int B, int H, int n_samples, const float *alpha,
+                         float *row_weight);
+
 /* ---- quantize / dequantize one page ------------------------------------- */
 int orc_quantize_page(const orc_format *f, const float *S_nat, const int32_t *perm,
                       orc_page *out);

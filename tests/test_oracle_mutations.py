@@ -19,7 +19,7 @@ SRC = os.path.join(ROOT, "oracle", "stq_oracle.cpp")
 HDR = os.path.join(ROOT, "oracle", "stq_oracle.h")
 PIN_FILES = ["tests/test_oracle_scalars.py", "tests/test_oracle_format.py",
              "tests/test_oracle_quantize.py", "tests/test_oracle_step.py", "tests/test_oracle_window.py",
-             "tests/test_oracle_prefill.py"]
+             "tests/test_oracle_prefill.py", "tests/test_oracle_lifetime.py"]
 
 MUTANTS = {
     "error sign": ("e[j] = v[j] * ic[j] - u[j];", "e[j] = v[j] * ic[j] + u[j];"),
@@ -65,6 +65,11 @@ MUTANTS = {
                                          "for (int j = 0; j < d_v; ++j) T[(size_t)s * d_v + j] = T[(size_t)s * d_v + j];"),
     "prefill first beta for every token": ("const float bk = beta[l] * kl[perm[s]];", "const float bk = beta[0] * kl[perm[s]];"),
     "prefill readout with k": ("column_sum(f, perm, ql, T.data(), ot.data());", "column_sum(f, perm, kl, T.data(), ot.data());"),
+    "lifetime mean over samples only": ("const double mean = sum / ((double)n_samples * (double)B);",
+                                        "const double mean = sum / (double)n_samples;"),
+    "lifetime channel ignored": ("* H + h) * na + (f->gate_vector ? kap : 0)];", "* H + h) * na + 0];"),
+    "lifetime head ignored": ("* H + h) * na + (f->gate_vector ? kap : 0)];",
+                              "* H + 0) * na + (f->gate_vector ? kap : 0)];"),
     "window butterfly half": ("for (int off = lanes / 2; off >= 1; off /= 2) {",
                               "for (int off = lanes / 2; off >= 2; off /= 2) {"),
 }
