@@ -692,12 +692,19 @@ extern "C" int orc_lifetime_weights(const orc_format *f, int B, int H, int n_sam
     const int na = f->gate_vector ? d_k : 1;
     for (int h = 0; h < H; ++h) {
         for (int kap = 0; kap < d_k; ++kap) {
-            /* the mean gate over the samples and requests, summed sample by
-             * sample, requests ascending, in double */
-            double sum = 0.0;
-            for (int t = 0; t < n_samples; ++t)
-                for (int b = 0; b < B; ++b)
-                    sum += (double)alpha[(((size_t)t * B + b) * H + h) * na + (f->gate_vector ? kap : 0)];
+            /* the mean gate over the samples and requests, in double: the
+             * requests in eight slices [j B / 8, (j + 1) B / 8); per slice the
+             * samples, then its requests, ascending, from 0; the slice sums
+             * added as ((p0 + p1) + (p2 + p3)) + ((p4 + p5) + (p6 + p7)) */
+            double part[8];
+            for (int j = 0; j < 8; ++j) {
+                double acc = 0.0;
+                for (int t = 0; t < n_samples; ++t)
+                    for (int b = j * B / 8; b < (j + 1) * B / 8; ++b)
+                        acc += (double)alpha[(((size_t)t * B + b) * H + h) * na + (f->gate_vector ? kap : 0)];
+                part[j] = acc;
+            }
+            const double sum = ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
             const double mean = sum / ((double)n_samples * (double)B);
             /* expected persistence under geometric decay: 1 / (1 - mean),
              * capped at 2^24 (a gate of one keeps its content for ever) */

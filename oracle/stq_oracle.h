@@ -87,8 +87,10 @@ int orc_rank_rows(const orc_format *f, int B, int H, const float *S,
  * (STEPQuant landing page: errors in long-lived memory persist across many
  * steps; Figure B1: long gate half-lives hold most of the quantization
  * error).  alpha: [n_samples][B][H][d_k] (gate_vector) or [n_samples][B][H];
- * the mean is a double sum over samples, then requests, ascending, divided
- * by n_samples * B; row_weight: [H][d_k], rounded to float. */
+ * the mean is a double sum divided by n_samples * B: the requests in eight
+ * slices [j B / 8, (j + 1) B / 8), per slice the samples then its requests
+ * ascending, the slice sums added as a fixed pairwise tree;
+ * row_weight: [H][d_k], rounded to float. */
 int orc_lifetime_weights(const orc_format *f, int B, int H, int n_samples, const float *alpha,
                          float *row_weight);
 

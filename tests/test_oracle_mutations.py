@@ -70,6 +70,7 @@ MUTANTS = {
     "lifetime channel ignored": ("* H + h) * na + (f->gate_vector ? kap : 0)];", "* H + h) * na + 0];"),
     "lifetime head ignored": ("* H + h) * na + (f->gate_vector ? kap : 0)];",
                               "* H + 0) * na + (f->gate_vector ? kap : 0)];"),
+    "lifetime slice dropped": ("((part[4] + part[5]) + (part[6] + part[7]))", "((part[4] + part[5]) + part[6])"),
     "window butterfly half": ("for (int off = lanes / 2; off >= 1; off /= 2) {",
                               "for (int off = lanes / 2; off >= 2; off /= 2) {"),
 }
