@@ -374,6 +374,32 @@ def run_prefill(w, L, steps, warmup, rank, world):
     return {"ms": ms, "steps": steps}
 
 
+def run_lifetime(samples=32, batch=64, reps=20):
+    """stq_lifetime_weights over `samples` gate samples of a `batch`-request
+    stepquant4-kda state (vector gates): device time per call."""
+    from linear_attention_recurrent_delta_b200 import binding as B
+    w = [x for x in W.WORKLOADS if x.fmt == "stepquant4_kda"][0].resized(batch=batch)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    qs = B.QuantizedState(w.format, w.batch, w.heads, device=dev)
+    alpha = torch.stack([W.step_inputs(w, t, device=dev)["alpha"] for t in range(samples)]).contiguous()
+    out = torch.empty(w.heads, 128, device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(3):
+        B.stq_lifetime_weights(qs.state, alpha, out, stream)
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(reps):
+        B.stq_lifetime_weights(qs.state, alpha, out, stream)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    ms = ev0.elapsed_time(ev1) / reps
+    nbytes = alpha.numel() * 4
+    del qs, alpha
+    return {"ms": ms, "gbs": nbytes / (ms / 1000.0) / 1e9, "samples": samples, "requests": batch,
+            "heads": w.heads, "format": w.fmt, "bytes_read": nbytes}
+
+
 class OracleSample:
     """The CPU oracle (single thread, as written) stepping a sample of the
     workload's pages: the first ``n_pages`` pages of a batch whose fp32 state
@@ -600,6 +626,8 @@ def main():
                                                "frac": rate * fl / 1e12 / FP32_PEAK_TFLOPS,
                                                "flops_per_head_token": fl}}
 
+    lifetime = run_lifetime() if not args.only else None
+
     others = {}
     if not args.only:
         for i in (1, 2, 3, 4):
@@ -645,6 +673,9 @@ def main():
         "clocks": res["clocks"],
         "other_workloads": others,
         "paged_step": paged,
+        "lifetime_weights": ({"entry_point": "stq_lifetime_weights", "kernel": "stq::lifetime_kernel",
+                              "note": "cold path, once per calibration; one thread per (head, channel)",
+                              **lifetime} if lifetime else None),
         "prefill": ({"entry_point": "stq_prefill", "kernel": "stq::prefill_kernel",
                      "peak_kind": "derived: 148 SMs x 128 FP32 lanes x 2 x 1.965 GHz", "prompts": prefill}
                     if prefill else None),

@@ -153,6 +153,21 @@ stq_status stq_calibrate(stq_state *s, const float *d_S, const float *d_row_weig
  * Arguments and other errors as stq_calibrate. */
 stq_status stq_calibrate_noalloc(stq_state *s, const float *d_S, const float *d_row_weight, void *stream);
 
+/* Lifetime row weights for stq_calibrate (STEPQuant's temporal allocation,
+ * landing page Figure B1: long gate half-lives hold most of the quantization
+ * error).  Per head h and key channel kappa,
+ *     w[h][kappa] = 1 / (1 - mean alpha)     (capped at 2^24),
+ * the expected persistence of what the channel stores under geometric decay
+ * with the mean gate; the mean runs over the samples and the state's
+ * requests (a double sum, samples then requests ascending).  Pass w as
+ * stq_calibrate's d_row_weight to rank long-lived channels into the widest
+ * groups.  d_alpha: device, [n_samples][B][H] (GDN) or [n_samples][B][H][128]
+ * (gate_vector, 16-byte aligned), gates in [0, 1]; d_row_weight: [H][128]
+ * fp32, 16-byte aligned.  Neither may overlap the state or each other.
+ * Errors: INVALID_ARG (nulls, n_samples < 1, overlap), MISALIGNED, CUDA. */
+stq_status stq_lifetime_weights(const stq_state *s, const float *d_alpha, int n_samples, float *d_row_weight,
+                                void *stream);
+
 /* Quantize an fp32 state into every page using the state's precision map:
  * c_j = max_i |S_ij| (1 if 0; 1 without column scales); T = S * (1/c);
  * INT rows: r = max_j |T| / qmax, codes = round-to-nearest-even of

@@ -61,6 +61,7 @@ def lib():
         "stq_request_pages": (c_int, [P, c_int, POINTER(c_size_t), POINTER(c_size_t)]),
         "stq_window_buffer_bytes": (c_size_t, [P, c_int]),
         "stq_window_step": (c_int, [P, P, c_size_t, c_int, c_int, c_int, P, P, P, P, P, P, c_uint64, c_uint32, P]),
+        "stq_lifetime_weights": (c_int, [P, P, c_int, P, P]),
         "stq_prefill": (c_int, [P, c_int, P, P, P, P, P, P, P, c_uint64, c_uint32, P]),
         "stq_decode_io_bytes": (c_size_t, [P]),
         "stq_decode_step_host": (c_int, [P, P, P, P, P, P, P, P, c_size_t, c_uint64, c_uint32, P]),
@@ -205,6 +206,12 @@ def stq_window_step(state, buf, window, t, commit, q, k, v, alpha, beta, o, seed
     _check(lib().stq_window_step(state.handle, _ptr(buf), buf.numel() * buf.element_size(), int(window), int(t),
                                  int(bool(commit)), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(o),
                                  int(seed), int(step), _stream(stream)), "stq_window_step")
+
+
+def stq_lifetime_weights(state, alpha, row_weight, stream=None):
+    """Row weights [H, 128] from gate samples alpha [n_samples, B, H(, 128)]."""
+    _check(lib().stq_lifetime_weights(state.handle, _ptr(alpha), int(alpha.shape[0]), _ptr(row_weight),
+                                      _stream(stream)), "stq_lifetime_weights")
 
 
 def stq_prefill(state, q, k, v, alpha, beta, o, S_out=None, seed=0, step=0, stream=None):

@@ -2,6 +2,7 @@
 // Nothing here allocates device memory or synchronizes (except
 // stq_device_status, which is documented to).
 #include "stq_internal.h"
+#include "stq_lifetime.h"
 
 #include <cstring>
 #include <mutex>
@@ -176,6 +177,20 @@ stq_status stq_calibrate(stq_state *s, const float *d_S, const float *d_row_weig
         return STQ_ERR_INVALID_ARG;
     cudaError_t err = launch_calibrate(s, d_S, d_row_weight, static_cast<double *>(d_workspace),
                                        static_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? STQ_OK : STQ_ERR_CUDA;
+}
+
+stq_status stq_lifetime_weights(const stq_state *s, const float *d_alpha, int n_samples, float *d_row_weight,
+                                void *stream) {
+    if (!s || !d_alpha || !d_row_weight || n_samples < 1) return STQ_ERR_INVALID_ARG;
+    if (!aligned(d_alpha, s->fmt.gate_vector ? 16 : 4) || !aligned(d_row_weight, 16)) return STQ_ERR_MISALIGNED;
+    const size_t na = s->fmt.gate_vector ? kD : 1;
+    const size_t n_alpha = (size_t)n_samples * s->batch * s->heads * na * sizeof(float);
+    const size_t n_w = (size_t)s->heads * kD * sizeof(float);
+    if (overlaps(d_alpha, n_alpha, s->base, state_span(s)) || overlaps(d_row_weight, n_w, s->base, state_span(s)) ||
+        overlaps(d_row_weight, n_w, d_alpha, n_alpha))
+        return STQ_ERR_INVALID_ARG;
+    cudaError_t err = launch_lifetime(s, d_alpha, n_samples, d_row_weight, static_cast<cudaStream_t>(stream));
     return err == cudaSuccess ? STQ_OK : STQ_ERR_CUDA;
 }
 

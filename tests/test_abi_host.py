@@ -237,3 +237,18 @@ def test_prefill_checks_arguments(lib):
     assert call(o=FAKE + 512) == B.STQ_ERR_INVALID_ARG            # output overlaps the state
     assert call(S_out=o) == B.STQ_ERR_INVALID_ARG                 # the state output overlaps o
     lib.stq_state_free(h)
+
+
+def test_lifetime_weights_checks_arguments(lib):
+    fmt = B.format_from_spec(W.FORMATS["stepquant4_kda"])
+    st, h = _alloc(lib, fmt, 2, 3)
+    P = ctypes.c_void_p
+    a, w = 1 << 41, 1 << 42
+    assert lib.stq_lifetime_weights(None, P(a), 4, P(w), None) == B.STQ_ERR_INVALID_ARG
+    assert lib.stq_lifetime_weights(h, None, 4, P(w), None) == B.STQ_ERR_INVALID_ARG
+    assert lib.stq_lifetime_weights(h, P(a), 0, P(w), None) == B.STQ_ERR_INVALID_ARG
+    assert lib.stq_lifetime_weights(h, P(a + 4), 4, P(w), None) == B.STQ_ERR_MISALIGNED   # vector gates: 16 bytes
+    assert lib.stq_lifetime_weights(h, P(a), 4, P(w + 8), None) == B.STQ_ERR_MISALIGNED
+    assert lib.stq_lifetime_weights(h, P(a), 4, P(a + 256), None) == B.STQ_ERR_INVALID_ARG   # output overlaps the gates
+    assert lib.stq_lifetime_weights(h, P(FAKE), 4, P(w), None) == B.STQ_ERR_INVALID_ARG     # gates overlap the state
+    lib.stq_state_free(h)
