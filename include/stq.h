@@ -296,6 +296,26 @@ stq_status stq_decode_step_host(stq_state *s, const float *h_q, const float *h_k
                                 float *h_o, void *d_io, size_t io_bytes,
                                 uint64_t seed, uint32_t step, void *stream);
 
+/* n_steps consecutive steps with host-resident inputs and outputs, the
+ * copies overlapped with the steps: step i's inputs are read from h_x +
+ * i * (one step's elements) (the layouts of stq_decode_step_host, steps
+ * outermost), its o is written to h_o + i * B*H*128, and its stochastic-
+ * rounding step index is step + i.  Two staging slots alternate: while step
+ * i runs on `stream`, the inputs of step i + 1 are copied in and the o of
+ * step i - 1 is copied out on two streams the call creates (and releases),
+ * ordered by events, so every copy of every step still happens inside the
+ * call.  The steps are the stq_decode_step kernel, so the results equal
+ * n_steps calls of stq_decode_step_host.  d_io: >= 2 * stq_decode_io_bytes,
+ * 256-byte aligned, caller-owned; host buffers pinned.  All work is ordered
+ * before any later work on `stream`; the caller synchronizes it before
+ * reading h_o.  Errors as stq_decode_step_host (BUFFER_TOO_SMALL below two
+ * slots; INVALID_ARG for n_steps < 1); a CUDA error mid-way returns
+ * STQ_ERR_CUDA with the steps so far enqueued. */
+stq_status stq_decode_steps_host(stq_state *s, int n_steps, const float *h_q, const float *h_k,
+                                 const float *h_v, const float *h_alpha, const float *h_beta,
+                                 float *h_o, void *d_io, size_t io_bytes,
+                                 uint64_t seed, uint32_t step, void *stream);
+
 /* Dequantize every page to fp32 [B][H][128][128] in natural key order:
  * S_ij = (z_ij * r_i) * c_j (FP16 rows: h_ij * c_j).  d_S 16-byte aligned. */
 stq_status stq_dequantize_state(const stq_state *s, float *d_S, void *stream);

@@ -65,6 +65,7 @@ def lib():
         "stq_prefill": (c_int, [P, c_int, P, P, P, P, P, P, P, c_uint64, c_uint32, P]),
         "stq_decode_io_bytes": (c_size_t, [P]),
         "stq_decode_step_host": (c_int, [P, P, P, P, P, P, P, P, c_size_t, c_uint64, c_uint32, P]),
+        "stq_decode_steps_host": (c_int, [P, c_int, P, P, P, P, P, P, P, c_size_t, c_uint64, c_uint32, P]),
         "stq_dequantize_state": (c_int, [P, P, P]),
         "stq_device_status": (c_int, [P, P, c_int]),
         "stq_set_wait_limit": (c_int, [P, c_uint64, c_int]),
@@ -228,6 +229,13 @@ def stq_decode_step_host(state, hq, hk, hv, halpha, hbeta, ho, io, seed=0, step=
     _check(lib().stq_decode_step_host(state.handle, _ptr(hq), _ptr(hk), _ptr(hv), _ptr(halpha), _ptr(hbeta),
                                       _ptr(ho), _ptr(io), io.numel() * io.element_size(), int(seed),
                                       int(step), _stream(stream)), "stq_decode_step_host")
+
+
+def stq_decode_steps_host(state, hq, hk, hv, halpha, hbeta, ho, io, seed=0, step=0, stream=None):
+    """hq.shape[0] steps from pinned host tensors [n, B, H, ...], copies overlapped with the steps."""
+    _check(lib().stq_decode_steps_host(state.handle, int(hq.shape[0]), _ptr(hq), _ptr(hk), _ptr(hv), _ptr(halpha),
+                                       _ptr(hbeta), _ptr(ho), _ptr(io), io.numel() * io.element_size(), int(seed),
+                                       int(step), _stream(stream)), "stq_decode_steps_host")
 
 
 def stq_dequantize_state(state, S, stream=None):

@@ -371,6 +371,83 @@ stq_status stq_decode_step_host(stq_state *s, const float *h_q, const float *h_k
     return STQ_OK;
 }
 
+// Events and streams of one pipelined call, released on every return path.
+namespace {
+struct Pipe {
+    cudaStream_t h2d = nullptr, d2h = nullptr;
+    cudaEvent_t in_ready[2] = {nullptr, nullptr}, step_done[2] = {nullptr, nullptr},
+                out_done[2] = {nullptr, nullptr};
+    bool ok = true;
+    Pipe() {
+        ok = cudaStreamCreateWithFlags(&h2d, cudaStreamNonBlocking) == cudaSuccess &&
+             cudaStreamCreateWithFlags(&d2h, cudaStreamNonBlocking) == cudaSuccess;
+        for (int i = 0; i < 2 && ok; ++i)
+            ok = cudaEventCreateWithFlags(&in_ready[i], cudaEventDisableTiming) == cudaSuccess &&
+                 cudaEventCreateWithFlags(&step_done[i], cudaEventDisableTiming) == cudaSuccess &&
+                 cudaEventCreateWithFlags(&out_done[i], cudaEventDisableTiming) == cudaSuccess;
+    }
+    ~Pipe() {   // destroying them does not wait: the work in flight completes
+        for (int i = 0; i < 2; ++i) {
+            if (in_ready[i]) cudaEventDestroy(in_ready[i]);
+            if (step_done[i]) cudaEventDestroy(step_done[i]);
+            if (out_done[i]) cudaEventDestroy(out_done[i]);
+        }
+        if (h2d) cudaStreamDestroy(h2d);
+        if (d2h) cudaStreamDestroy(d2h);
+    }
+};
+}  // namespace
+
+stq_status stq_decode_steps_host(stq_state *s, int n_steps, const float *h_q, const float *h_k, const float *h_v,
+                                 const float *h_alpha, const float *h_beta, float *h_o, void *d_io, size_t io_bytes,
+                                 uint64_t seed, uint32_t step, void *stream) {
+    if (!s || !h_q || !h_k || !h_v || !h_alpha || !h_beta || !h_o || !d_io || n_steps < 1)
+        return STQ_ERR_INVALID_ARG;
+    if (!aligned(d_io, 256)) return STQ_ERR_MISALIGNED;
+    const IoLayout L = io_layout(s);
+    if (io_bytes < 2 * L.total) return STQ_ERR_BUFFER_TOO_SMALL;
+    if (overlaps(d_io, 2 * L.total, s->base, state_span(s))) return STQ_ERR_INVALID_ARG;
+    Pipe P;
+    if (!P.ok) return STQ_ERR_CUDA;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    const size_t per_vec = L.vec / sizeof(float), per_na = L.na / sizeof(float), per_sc = L.sc / sizeof(float);
+    for (int i = 0; i < n_steps; ++i) {
+        const int slot = i & 1;
+        uint8_t *io = static_cast<uint8_t *>(d_io) + slot * L.total;
+        // inputs of step i into the slot, once step i - 2 (the slot's last
+        // reader) is done
+        if (i >= 2 && cudaStreamWaitEvent(P.h2d, P.step_done[slot], 0) != cudaSuccess) return STQ_ERR_CUDA;
+        if (i == 0 && (cudaEventRecord(P.in_ready[1], cs) != cudaSuccess ||
+                       cudaStreamWaitEvent(P.h2d, P.in_ready[1], 0) != cudaSuccess))
+            return STQ_ERR_CUDA;   // the first copies follow the work already on `stream`
+        const struct { size_t off; const void *src; size_t n; } in[5] = {
+            {L.q, h_q + i * per_vec, L.vec}, {L.k, h_k + i * per_vec, L.vec}, {L.v, h_v + i * per_vec, L.vec},
+            {L.alpha, h_alpha + i * per_na, L.na}, {L.beta, h_beta + i * per_sc, L.sc}};
+        for (int j = 0; j < 5; ++j)
+            if (cudaMemcpyAsync(io + in[j].off, in[j].src, in[j].n, cudaMemcpyHostToDevice, P.h2d) != cudaSuccess)
+                return STQ_ERR_CUDA;
+        if (cudaEventRecord(P.in_ready[slot], P.h2d) != cudaSuccess) return STQ_ERR_CUDA;
+        // step i, once its inputs are in and the slot's o of step i - 2 is out
+        if (cudaStreamWaitEvent(cs, P.in_ready[slot], 0) != cudaSuccess) return STQ_ERR_CUDA;
+        if (i >= 2 && cudaStreamWaitEvent(cs, P.out_done[slot], 0) != cudaSuccess) return STQ_ERR_CUDA;
+        stq_status st = decode_step(s, nullptr, s->batch, reinterpret_cast<float *>(io + L.q),
+                                    reinterpret_cast<float *>(io + L.k), reinterpret_cast<float *>(io + L.v),
+                                    reinterpret_cast<float *>(io + L.alpha), reinterpret_cast<float *>(io + L.beta),
+                                    reinterpret_cast<float *>(io + L.o), seed, step + (uint32_t)i, stream, false);
+        if (st != STQ_OK) return st;
+        if (cudaEventRecord(P.step_done[slot], cs) != cudaSuccess) return STQ_ERR_CUDA;
+        // o of step i out
+        if (cudaStreamWaitEvent(P.d2h, P.step_done[slot], 0) != cudaSuccess) return STQ_ERR_CUDA;
+        if (cudaMemcpyAsync(h_o + i * per_vec, io + L.o, L.vec, cudaMemcpyDeviceToHost, P.d2h) != cudaSuccess)
+            return STQ_ERR_CUDA;
+        if (cudaEventRecord(P.out_done[slot], P.d2h) != cudaSuccess) return STQ_ERR_CUDA;
+    }
+    // everything of the call precedes later work on `stream`
+    for (int slot = 0; slot < 2 && slot < n_steps; ++slot)
+        if (cudaStreamWaitEvent(cs, P.out_done[slot], 0) != cudaSuccess) return STQ_ERR_CUDA;
+    return STQ_OK;
+}
+
 stq_status stq_dequantize_state(const stq_state *s, float *d_S, void *stream) {
     if (!s || !d_S) return STQ_ERR_INVALID_ARG;
     if (!aligned(d_S, 16)) return STQ_ERR_MISALIGNED;

@@ -252,3 +252,21 @@ def test_lifetime_weights_checks_arguments(lib):
     assert lib.stq_lifetime_weights(h, P(a), 4, P(a + 256), None) == B.STQ_ERR_INVALID_ARG   # output overlaps the gates
     assert lib.stq_lifetime_weights(h, P(FAKE), 4, P(w), None) == B.STQ_ERR_INVALID_ARG     # gates overlap the state
     lib.stq_state_free(h)
+
+
+def test_pipelined_host_steps_check_arguments(lib):
+    fmt = B.format_from_spec(W.FORMATS["int8row"])
+    st, h = _alloc(lib, fmt, 2, 3)
+    P = ctypes.c_void_p
+    hp = P(1 << 45)
+    io = 1 << 44
+    need = lib.stq_decode_io_bytes(h)
+
+    def call(n=3, io=io, nbytes=2 * need):
+        return lib.stq_decode_steps_host(h, n, hp, hp, hp, hp, hp, hp, P(io), nbytes, 0, 0, None)
+
+    assert call(n=0) == B.STQ_ERR_INVALID_ARG
+    assert call(nbytes=2 * need - 1) == B.STQ_ERR_BUFFER_TOO_SMALL   # two staging slots
+    assert call(io=io + 16) == B.STQ_ERR_MISALIGNED
+    assert call(io=FAKE) == B.STQ_ERR_INVALID_ARG                    # staging overlaps the state
+    lib.stq_state_free(h)
