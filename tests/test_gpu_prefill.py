@@ -154,3 +154,9 @@ def test_bounded_wait_times_out_and_writes_nothing():
     ref, o_ref, _, margins = _oracle(fmt, perm, pages, w.heads, x, 0, 1)
     assert np.array_equal(o.cpu().numpy().reshape(L, -1, 128), o_ref)
     _check_pages(fmt, download(qs), ref, margins)
+
+
+@pytest.mark.parametrize("name,L", [("stepquant6", 130), ("stepquant4_kda", 131)])
+def test_prompt_longer_than_the_scalar_chunk(name, L):
+    # beta and the scalar gate are staged 128 tokens at a time: cross a chunk boundary
+    _run(name, 5, 3, L)
