@@ -314,7 +314,8 @@ def test_steps_captured_in_a_cuda_graph_match_eager_steps():
     assert torch.equal(qb.pages(), qa.pages())
 
 
-def test_pipelined_host_steps_equal_device_steps():
+@pytest.mark.parametrize("n", [1, 2, 5])
+def test_pipelined_host_steps_equal_device_steps(n):
     """stq_decode_steps_host (copies overlapped with the steps on side
     streams) gives the o and pages of the same steps run on the device."""
     w = _small("stepquant4_kda", batch=8, heads=6, steps=5)
@@ -323,13 +324,13 @@ def test_pipelined_host_steps_equal_device_steps():
     qa, qb = make_state(w), make_state(w)
     upload(qa, perm, pages)
     upload(qb, perm, pages)
-    xs = [W.step_inputs(w, t) for t in range(5)]
+    xs = [W.step_inputs(w, t) for t in range(n)]
     o_dev = []
     for t, x in enumerate(xs):
         xd = {k: v.cuda() for k, v in x.items()}
         o_dev.append(qa.step(xd["q"], xd["k"], xd["v"], xd["alpha"], xd["beta"], seed=4, step=10 + t).cpu())
     host = {k: torch.stack([x[k] for x in xs]).contiguous().pin_memory() for k in xs[0]}
-    ho = torch.empty(5, 8, 6, 128).pin_memory()
+    ho = torch.empty(n, 8, 6, 128).pin_memory()
     io_bytes = 2 * B.stq_decode_io_bytes(qb.state)
     io_raw = torch.empty(io_bytes + 256, dtype=torch.uint8, device="cuda")
     off = (-io_raw.data_ptr()) % 256
@@ -337,6 +338,6 @@ def test_pipelined_host_steps_equal_device_steps():
                             io_raw[off:off + io_bytes], seed=4, step=10)
     torch.cuda.synchronize()
     assert B.stq_device_status(qb.state) == B.STQ_OK
-    for t in range(5):
+    for t in range(n):
         assert torch.equal(ho[t], o_dev[t]), t
     assert torch.equal(qa.pages(), qb.pages())
