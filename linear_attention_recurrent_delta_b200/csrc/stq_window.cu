@@ -34,7 +34,7 @@ namespace stq {
 
 constexpr int kWindowMax = STQ_WINDOW_MAX;
 constexpr int kWindowStages = 4;          // ring depth at most
-constexpr int kRebuildGroup = 4;          // blocks per pass of a commit's entry loop (measured: 1, 2, 4)
+constexpr int kRebuildGroup = 4;          // blocks per pass of a commit's entry loop (measured: 1, 2, 4, 8)
 
 struct WindowArgs {
     uint8_t *pages;
@@ -211,8 +211,8 @@ __device__ __forceinline__ void codes_slice(const uint8_t *blk, int w, int lane,
 // The first phase of a page, per warp: the operands of this lane's row, the
 // entries' dot products (warp w: entries w, w + 4, ...) and one pass over the
 // warp's slices (dequantize, u's and o's chains), whose sums go to the
-// stage's scratch.  A commit also keeps P' and the row's decayed keys (kd:
-// this warp's [tau][32] table).
+// stage's scratch.  A commit also keeps the row factor a' and the row's
+// decayed keys (kd: this warp's [tau][32] table).
 template <class FMT, bool COMMIT>
 __device__ __forceinline__ void window_first_phase(const DevFormat &F, const WindowArgs &A, WindowSmem &S,
                                                    const uint8_t *stg, const StageView &V, const RowCtx &R,
@@ -423,8 +423,9 @@ __global__ void __launch_bounds__(kThreads, 4) window_step_kernel(const DevForma
 // every warp needs this step's delta D[t] for its own rows.  After it each
 // warp dequantizes its slices again with the row factor, T = RN(z a') (the
 // page is intact in the stage until the warp requantizes them), adds the
-// entries in order, takes the row maxima and requantizes in place; the stage is stored
-// at the next page's barrier and refilled once the store has read it.
+// entries in order, takes the row maxima and requantizes in place; the
+// stage is stored at the next page's barrier and refilled once the store has
+// read it.
 template <class FMT>
 __global__ void __launch_bounds__(kThreads, 3) window_commit_kernel(const DevFormat F, const WindowArgs A) {
     extern __shared__ __align__(128) uint8_t smem[];
@@ -502,8 +503,9 @@ __global__ void __launch_bounds__(kThreads, 3) window_commit_kernel(const DevFor
             *reinterpret_cast<float4 *>(A.o + (size_t)p * kD + 4 * lane) = window_out(X, V.D, V.c, t, dt, lane);
 
         // T = RN(z a'), then the entries in order (per element one chain;
-        // block by block, so that a block's codes and keys are the only
-        // operands in registers besides T), and the row maxima
+        // a group of blocks at a time, so that the group's keys and one
+        // delta row are the only operands in registers besides T), and the
+        // row maxima
         const float2 dt01 = make_float2(dt.x, dt.y), dt23 = make_float2(dt.z, dt.w);
         Tile T;
         // blocks in groups of kRebuildGroup: each entry's delta row is read
