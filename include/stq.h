@@ -233,7 +233,14 @@ stq_status stq_request_pages(const stq_state *s, int slot, size_t *offset, size_
  *   u = S0^T (P' k) + sum_{tau<t} (K[tau] . k) D[tau]
  *   D[t] = beta (v / c - u);   K[t] = k
  *   o = c (S0^T (P' q) + sum_{tau<=t} (K[tau] . q) D[tau])
- * i.e. the gated delta rule run exactly from the page for t + 1 steps.  A
+ * i.e. the gated delta rule run exactly from the page for t + 1 steps.  In
+ * fp32 the decay is folded into the row scale, one factor a' = RN(P' r) per
+ * stored row (FP16 rows: P'), as stq_decode_step folds alpha into r: the
+ * page's column sums take row weights RN(k a') and RN(q a') on the exact
+ * codes in stq_decode_step's order; an entry's dot product is a 4-channel fma
+ * chain per lane plus an xor butterfly over 32 lanes; the entries' terms are
+ * added by fma in entry order; the commit rebuilds RN(z a') and adds
+ * fma(K[tau], D[tau], .) for tau = 0 .. t.  A
  * step that does not commit writes P', K[0 .. t] and D[t] to the buffer and
  * leaves the pages unchanged.  A committing step (commit != 0; required at
  * t = W - 1, allowed at any t to end a window early) writes no buffer row;
