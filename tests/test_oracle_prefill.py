@@ -146,3 +146,29 @@ def test_basis_keys_store_and_return_values():
     for l in range(len(idx)):
         np.testing.assert_allclose(o[l], v[l], rtol=4e-7, atol=1e-30)
     np.testing.assert_allclose(o[-1], v[3], rtol=4e-7, atol=1e-30)
+
+
+@pytest.mark.parametrize("name", ["stepquant6", "stepquant4_kda"])
+def test_prefill_and_a_window_of_the_same_steps_agree(name):
+    """A window of L steps and a prefill of the same L tokens run the same
+    exact rule in two fp32 orders: o of every token, and the state before the
+    one requantization (the window's rebuilt from its buffer), agree to
+    rounding."""
+    w, fmt, perm, page = _workload(name)
+    L = 8
+    q, k, v, alpha, beta = _prompt(w, 60, L)
+    o_p, tp, _ = O.prefill_f32(fmt, page.copy(), perm, q, k, v, alpha, beta, want_tp=True)
+    P = np.ones(128, np.float32)
+    K = np.zeros((L, 128), np.float32)
+    D = np.zeros((L, 128), np.float32)
+    pw = page.copy()
+    for t in range(L):
+        o_w, _ = O.window_step_f32(fmt, pw, perm, P, K, D, t, False, q[t], k[t], v[t], alpha[t], float(beta[t]))
+        assert _rel_l2(o_w, o_p[t]) <= 1e-5, t
+    # the window's state after step L - 1, rebuilt in fp64 from its buffer: P' S0 + sum K D^T
+    S0 = _dequant64(fmt, page, perm)
+    c = page.c.astype(np.float64) if fmt.col_scales else np.ones(128)
+    Sw = P.astype(np.float64)[:, None] * S0 + (K.astype(np.float64).T @ D.astype(np.float64)) * c[None, :]
+    Sp = np.zeros((128, 128))
+    Sp[perm] = tp.astype(np.float64) * c
+    assert _rel_l2(Sw, Sp) <= 1e-5
