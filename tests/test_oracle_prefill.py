@@ -172,3 +172,37 @@ def test_prefill_and_a_window_of_the_same_steps_agree(name):
     Sp = np.zeros((128, 128))
     Sp[perm] = tp.astype(np.float64) * c
     assert _rel_l2(Sw, Sp) <= 1e-5
+
+
+FORMATS_D4 = [
+    ([(1, "int", 8), (2, "int", 6), (1, "int", 4)], True),
+    ([(2, "fp16", 0), (2, "int", 8)], False),
+    ([(4, "int", 3)], True),
+]
+
+
+@pytest.mark.parametrize("groups,col", FORMATS_D4)
+@pytest.mark.parametrize("gate_vector", [False, True])
+def test_brute_force_d4(groups, col, gate_vector):
+    """4 x 4 states, five tokens: every token's o against the fp64 rule
+    within a few ulps of the state's scale."""
+    U = 2.0**-24
+    for seed in range(6):
+        rng = np.random.default_rng(300 + seed)
+        fmt = O.make_format(groups, d_k=4, d_v=4, col_scales=col, gate_vector=gate_vector)
+        S = (rng.normal(size=(4, 4)) * np.exp(rng.normal(size=(4, 1)))).astype(np.float32)
+        perm = rng.permutation(4).astype(np.int32)
+        page = O.quantize_page(fmt, S, perm)
+        L = 5
+        q = rng.normal(size=(L, 4)).astype(np.float32)
+        k = rng.normal(size=(L, 4)).astype(np.float32)
+        q /= np.linalg.norm(q, axis=1, keepdims=True)
+        k /= np.linalg.norm(k, axis=1, keepdims=True)
+        v = rng.normal(size=(L, 4)).astype(np.float32)
+        alpha = (1 / (1 + np.exp(rng.normal(-2, 1, size=(L, 4 if gate_vector else 1))))).astype(np.float32)
+        beta = (1 / (1 + np.exp(-rng.normal(size=L)))).astype(np.float32)
+        S0 = _dequant64(fmt, page, perm)
+        o64, S64 = _evolve64(S0, q, k, v, alpha, beta)
+        o, tp, _ = O.prefill_f32(fmt, page.copy(), perm, q, k, v, alpha, beta, want_tp=True)
+        scale = max(np.abs(S0).max(), np.abs(S64).max(), 1.0)
+        assert np.abs(o - o64).max() <= 256 * U * scale, seed
