@@ -23,7 +23,12 @@
  *     (dev.to post, "The state is a running sum, not a buffer"), here in the
  *     d_k x d_v convention with a decay gate alpha and a write strength beta:
  *       S' = A S + beta k (v - (A S)^T k)^T,  A = alpha I (GDN) or diag(alpha) (KDA),
- *       o  = S'^T q.
+ *       o  = S'^T q;
+ *   - around the step: the per-window variant that requantizes once per
+ *     window (LeapQuant abstract, paper-cards page), the prefill of a prompt
+ *     with one requantization at its end (repeated prefill: DASC card), and
+ *     the calibration's lifetime row weights (STEPQuant landing page,
+ *     Figure B1).
  *
  * Conventions: stored row s (group order), natural key channel perm[s].
  * Codes of INT rows are signed integers z in [-qmax, qmax], qmax = 2^(b-1)-1.
