@@ -55,16 +55,20 @@ def lib():
         L.orc_dequantize_page.argtypes = [P, P, P, P]
         L.orc_step_f32.argtypes = [P, P, P, P, P, P, P, c_float, P, c_uint64, c_uint32,
                                    c_uint32, c_uint32, P, P]
+        L.orc_step_f32_plain.argtypes = L.orc_step_f32.argtypes
         L.orc_step_f64.argtypes = [P, P, P, P, P, P, P, c_float, P, P]
         L.orc_lifetime_weights.argtypes = [P, c_int, c_int, c_int, P, P]
         L.orc_prefill_f32.argtypes = [P, P, P, c_int, P, P, P, P, P, P, c_uint64, c_uint32, c_uint32, c_uint32,
                                       P, P]
         L.orc_window_step_f32.argtypes = [P, P, P, P, P, P, c_int, c_int, P, P, P, P, c_float, P, c_uint64,
                                           c_uint32, c_uint32, c_uint32, P]
+        L.orc_window_step_f32_plain.argtypes = L.orc_window_step_f32.argtypes
+        L.orc_prefill_f32_plain.argtypes = L.orc_prefill_f32.argtypes
         L.orc_pack_page.argtypes = [P, P, P]
         L.orc_unpack_page.argtypes = [P, P, P]
         L.orc_decode_step_pages.argtypes = [P, c_int, c_int, P, P, P, P, P, P, P, P,
                                             c_uint64, c_uint32, c_long, c_long]
+        L.orc_decode_step_pages_plain.argtypes = L.orc_decode_step_pages.argtypes
         L.orc_f32_to_f16_rn.argtypes = [c_float]
         L.orc_f32_to_f16_rn.restype = c_uint16
         L.orc_f16_to_f32.argtypes = [c_uint16]
@@ -186,8 +190,10 @@ def _gate(fmt, alpha):
 
 
 def step_f32(fmt, page, perm, q, k, v, alpha, beta, seed=0, step=0, b=0, h=0,
-             want_tp=False, want_margin=False):
-    """Canonical fp32 step; updates ``page`` in place.  Returns (o, Tp, margin)."""
+             want_tp=False, want_margin=False, plain=False):
+    """fp32 step; updates ``page`` in place.  Returns (o, Tp, margin).  The
+    canonical (kernel) summation order, or with plain=True every column sum
+    one fma chain over the key channels in natural order."""
     perm = np.ascontiguousarray(perm, np.int32)
     q, k, v = (np.ascontiguousarray(x, np.float32) for x in (q, k, v))
     a = _gate(fmt, alpha)
@@ -195,14 +201,15 @@ def step_f32(fmt, page, perm, q, k, v, alpha, beta, seed=0, step=0, b=0, h=0,
     tp = np.zeros((fmt.d_k, fmt.d_v), np.float32) if want_tp else None
     mg = np.zeros((fmt.d_k, fmt.d_v), np.float64) if want_margin else None
     st = page._struct()
-    _ok(lib().orc_step_f32(ctypes.byref(fmt), ctypes.byref(st), _p(perm), _p(q), _p(k), _p(v),
-                           _p(a), float(beta), _p(o), int(seed), int(step), int(b), int(h),
-                           _p(tp), _p(mg)), "step_f32")
+    fn = lib().orc_step_f32_plain if plain else lib().orc_step_f32
+    _ok(fn(ctypes.byref(fmt), ctypes.byref(st), _p(perm), _p(q), _p(k), _p(v),
+           _p(a), float(beta), _p(o), int(seed), int(step), int(b), int(h),
+           _p(tp), _p(mg)), "step_f32")
     return o, tp, mg
 
 
 def window_step_f32(fmt, page, perm, P, K, D, t, commit, q, k, v, alpha, beta, seed=0, step=0, b=0, h=0,
-                    want_margin=False):
+                    want_margin=False, plain=False):
     """Per-window decode step t (0-based) on one page; P [d_k], K [W, d_k], D [W, d_v]
     (float32, updated in place; page updated in place when commit).  Returns (o, margin)."""
     perm = np.ascontiguousarray(perm, np.int32)
@@ -213,14 +220,15 @@ def window_step_f32(fmt, page, perm, P, K, D, t, commit, q, k, v, alpha, beta, s
     o = np.zeros(fmt.d_v, np.float32)
     mg = np.zeros((fmt.d_k, fmt.d_v), np.float64) if (want_margin and commit) else None
     st = page._struct()
-    _ok(lib().orc_window_step_f32(ctypes.byref(fmt), ctypes.byref(st), _p(perm), _p(P), _p(K), _p(D), int(t),
-                                  int(commit), _p(q), _p(k), _p(v), _p(a), float(beta), _p(o), int(seed),
-                                  int(step), int(b), int(h), _p(mg)), "window_step_f32")
+    fn = lib().orc_window_step_f32_plain if plain else lib().orc_window_step_f32
+    _ok(fn(ctypes.byref(fmt), ctypes.byref(st), _p(perm), _p(P), _p(K), _p(D), int(t),
+           int(commit), _p(q), _p(k), _p(v), _p(a), float(beta), _p(o), int(seed),
+           int(step), int(b), int(h), _p(mg)), "window_step_f32")
     return o, mg
 
 
 def prefill_f32(fmt, page, perm, q, k, v, alpha, beta, seed=0, step=0, b=0, h=0, want_tp=False,
-                want_margin=False):
+                want_margin=False, plain=False):
     """A prompt of L tokens through one page (page requantized in place at
     the end).  q, k, v: [L, 128]; alpha: [L] or [L, 128]; beta: [L].
     Returns (o [L, d_v], T before requantization or None, margin or None)."""
@@ -233,8 +241,9 @@ def prefill_f32(fmt, page, perm, q, k, v, alpha, beta, seed=0, step=0, b=0, h=0,
     tp = np.zeros((fmt.d_k, fmt.d_v), np.float32) if want_tp else None
     mg = np.zeros((fmt.d_k, fmt.d_v), np.float64) if want_margin else None
     st = page._struct()
-    _ok(lib().orc_prefill_f32(ctypes.byref(fmt), ctypes.byref(st), _p(perm), int(L), _p(q), _p(k), _p(v), _p(a),
-                              _p(bt), _p(o), int(seed), int(step), int(b), int(h), _p(tp), _p(mg)), "prefill_f32")
+    fn = lib().orc_prefill_f32_plain if plain else lib().orc_prefill_f32
+    _ok(fn(ctypes.byref(fmt), ctypes.byref(st), _p(perm), int(L), _p(q), _p(k), _p(v), _p(a),
+           _p(bt), _p(o), int(seed), int(step), int(b), int(h), _p(tp), _p(mg)), "prefill_f32")
     return o, tp, mg
 
 
@@ -268,8 +277,9 @@ def unpack_page(fmt, data):
 
 
 def decode_step_pages(fmt, B, H, pages, perm, q, k, v, alpha, beta, o, seed, step,
-                      page_begin=0, page_end=None):
-    """Canonical step over packed pages [page_begin, page_end) in place (one thread)."""
+                      page_begin=0, page_end=None, plain=False):
+    """fp32 step over packed pages [page_begin, page_end) in place (one
+    thread); canonical order, or the plain order with plain=True."""
     if page_end is None:
         page_end = B * H
     for name, arr, dt in (("pages", pages, np.uint8), ("perm", perm, np.int32), ("q", q, np.float32),
@@ -277,9 +287,10 @@ def decode_step_pages(fmt, B, H, pages, perm, q, k, v, alpha, beta, o, seed, ste
                           ("beta", beta, np.float32), ("o", o, np.float32)):
         if arr.dtype != dt or not arr.flags["C_CONTIGUOUS"]:
             raise TypeError("%s must be a C-contiguous %s array" % (name, np.dtype(dt).name))
-    _ok(lib().orc_decode_step_pages(ctypes.byref(fmt), B, H, _p(pages), _p(perm), _p(q), _p(k),
-                                    _p(v), _p(alpha), _p(beta), _p(o), int(seed), int(step),
-                                    int(page_begin), int(page_end)), "decode_step_pages")
+    fn = lib().orc_decode_step_pages_plain if plain else lib().orc_decode_step_pages
+    _ok(fn(ctypes.byref(fmt), B, H, _p(pages), _p(perm), _p(q), _p(k),
+           _p(v), _p(alpha), _p(beta), _p(o), int(seed), int(step),
+           int(page_begin), int(page_end)), "decode_step_pages")
 
 
 def f32_to_f16_rn(x):

@@ -7,12 +7,19 @@
  * evaluated exactly as written: one IEEE rounding per +, -, *, /, and fmaf
  * only where it is spelled out.
  *
- * Two evaluations of the step live here:
- *   orc_step_f64  the plain definition in double precision, natural key order;
- *   orc_step_f32  the canonical fp32 evaluation that the GPU kernel must
- *                 reproduce bit for bit.  The pages fix no fp32 evaluation
- *                 order; requiring bit-identical integer codes forces one, so
- *                 the order is part of the definition here:
+ * Three evaluations of the step live here:
+ *   orc_step_f64        the plain definition in double precision, natural key
+ *                       order;
+ *   orc_step_f32_plain  the plain fp32 evaluation: every column sum one fma
+ *                       chain over the key channels in natural order; the
+ *                       anchor the GPU is compared with under the rounding-
+ *                       band rule (codes may differ only where the fp32
+ *                       rounding of any evaluation order can move the
+ *                       pre-rounding value across a boundary);
+ *   orc_step_f32        the canonical fp32 evaluation, the decode kernel's own
+ *                       summation order, which the GPU must reproduce bit for
+ *                       bit (a second, stricter check).  The pages fix no fp32
+ *                       evaluation order; this one is the kernel's:
  *                   - the state is handled in column-normalised units
  *                     T = S / c (so the value-column scale c_j leaves the
  *                     inner loops);
@@ -28,7 +35,7 @@
  *                     (to an integer, ties to even);
  *                   - inv = qmax / m rounded toward zero, which keeps every
  *                     scaled value inside [-qmax, qmax].
- *                 orc_step_f64 pins this evaluation to the mathematics.
+ *                 orc_step_f64 pins both fp32 evaluations to the mathematics.
  *
  * parity pins: every function here is pinned by tests/test_oracle_*.py
  * (closed forms, brute force at d_k = d_v = 4, invariants, library
@@ -45,7 +52,6 @@
 static const int ORC_BLOCK_ROWS = 16;   /* rows of a block */
 static const int ORC_SLICE_ROWS = 4;    /* consecutive rows of a block in one slice */
 static const int ORC_HALF_ROWS = 64;    /* rows whose slice rows form one chain */
-static const int ORC_CALIB_CHUNK = 32;  /* requests per partial sum of a calibration score */
 
 /* ------------------------------------------------------------------------ */
 /* format helpers                                                           */
@@ -352,21 +358,15 @@ extern "C" int orc_rank_rows(const orc_format *f, int B, int H, const float *S,
     for (int h = 0; h < H; ++h) {
         /* score = row-mean-square summed over the batch, times the optional
          * retention weight; the constant 1 / (B d_v) is left out (it does
-         * not change the ranking).  The batch sum is taken in chunks of
-         * ORC_CALIB_CHUNK requests (each chunk from 0, requests ascending),
-         * and the chunk sums are added in chunk order: a fixed double
-         * evaluation order, so that equal inputs give one ranking. */
+         * not change the ranking).  In double: per request the row's sum of
+         * squares (columns in order), added over the requests in order. */
         for (int kap = 0; kap < d_k; ++kap) {
             double acc = 0.0;
-            for (int b0 = 0; b0 < B; b0 += ORC_CALIB_CHUNK) {
-                double part = 0.0;
-                for (int b = b0; b < std::min(B, b0 + ORC_CALIB_CHUNK); ++b) {
-                    const float *row = S + (((size_t)b * H + h) * d_k + kap) * d_v;
-                    double rs = 0.0;
-                    for (int j = 0; j < d_v; ++j) rs += (double)row[j] * (double)row[j];
-                    part += rs;
-                }
-                acc += part;
+            for (int b = 0; b < B; ++b) {
+                const float *row = S + (((size_t)b * H + h) * d_k + kap) * d_v;
+                double rs = 0.0;
+                for (int j = 0; j < d_v; ++j) rs += (double)row[j] * (double)row[j];
+                acc += rs;
             }
             if (row_weight) acc *= (double)row_weight[(size_t)h * d_k + kap];
             score[kap] = acc;
@@ -482,11 +482,36 @@ static void column_sum(const orc_format *f, const int32_t *perm, const float *w_
     }
 }
 
-extern "C" int orc_step_f32(const orc_format *f, orc_page *page, const int32_t *perm,
-                            const float *q, const float *k, const float *v,
-                            const float *alpha, float beta, float *o_out,
-                            uint64_t seed, uint32_t step, uint32_t b, uint32_t h,
-                            float *Tp_out, double *margin_out)
+/* The plain evaluation: out_j = sum over key channels kappa = 0 .. d_k - 1 in
+ * natural order of w[kappa] * X[s(kappa)][j] (s(kappa): the stored row that
+ * holds channel kappa), one fma chain from +0.  Nothing in it follows a
+ * thread mapping; it is the sum of the definition written left to right. */
+static void column_sum_plain(const orc_format *f, const int32_t *perm, const float *w_nat,
+                             const float *X, float *out)
+{
+    const int d_k = f->d_k, d_v = f->d_v;
+    std::vector<int> row_of(d_k);
+    for (int s = 0; s < d_k; ++s) row_of[perm[s]] = s;
+    for (int j = 0; j < d_v; ++j) {
+        float acc = 0.0f;
+        for (int kap = 0; kap < d_k; ++kap)
+            acc = std::fmaf(w_nat[kap], X[(size_t)row_of[kap] * d_v + j], acc);
+        out[j] = acc;
+    }
+}
+
+static void column_sum_in(int plain, const orc_format *f, const int32_t *perm, const float *w_nat,
+                          const float *X, float *out)
+{
+    if (plain) column_sum_plain(f, perm, w_nat, X, out);
+    else column_sum(f, perm, w_nat, X, out);
+}
+
+static int step_f32(int plain, const orc_format *f, orc_page *page, const int32_t *perm,
+                    const float *q, const float *k, const float *v,
+                    const float *alpha, float beta, float *o_out,
+                    uint64_t seed, uint32_t step, uint32_t b, uint32_t h,
+                    float *Tp_out, double *margin_out)
 {
     if (orc_format_check(f) != 0 || !page || !perm || !q || !k || !v || !alpha || !o_out)
         return -1;
@@ -504,7 +529,7 @@ extern "C" int orc_step_f32(const orc_format *f, orc_page *page, const int32_t *
             T[(size_t)s * d_v + j] = element_value(f, page, s, j) * a[s];
     }
     /* prediction (A S)^T k, then the error e = v - prediction (both / c) */
-    column_sum(f, perm, k, T.data(), u.data());
+    column_sum_in(plain, f, perm, k, T.data(), u.data());
     for (int j = 0; j < d_v; ++j) e[j] = v[j] * ic[j] - u[j];
     /* rank-1 delta update T' = T + (beta k) e^T */
     for (int s = 0; s < d_k; ++s) {
@@ -515,7 +540,7 @@ extern "C" int orc_step_f32(const orc_format *f, orc_page *page, const int32_t *
         }
     }
     /* readout o = S'^T q */
-    column_sum(f, perm, q, Tp.data(), ot.data());
+    column_sum_in(plain, f, perm, q, Tp.data(), ot.data());
     for (int j = 0; j < d_v; ++j) o_out[j] = f->col_scales ? page->c[j] * ot[j] : ot[j];
     if (Tp_out) std::memcpy(Tp_out, Tp.data(), sizeof(float) * Tp.size());
     /* requantize in place; c is unchanged */
@@ -523,6 +548,24 @@ extern "C" int orc_step_f32(const orc_format *f, orc_page *page, const int32_t *
         requant_row(f, s, Tp.data() + (size_t)s * d_v, page, seed, step, b, h,
                     f->stochastic, margin_out ? margin_out + (size_t)s * d_v : nullptr);
     return 0;
+}
+
+extern "C" int orc_step_f32(const orc_format *f, orc_page *page, const int32_t *perm,
+                            const float *q, const float *k, const float *v,
+                            const float *alpha, float beta, float *o_out,
+                            uint64_t seed, uint32_t step, uint32_t b, uint32_t h,
+                            float *Tp_out, double *margin_out)
+{
+    return step_f32(0, f, page, perm, q, k, v, alpha, beta, o_out, seed, step, b, h, Tp_out, margin_out);
+}
+
+extern "C" int orc_step_f32_plain(const orc_format *f, orc_page *page, const int32_t *perm,
+                                  const float *q, const float *k, const float *v,
+                                  const float *alpha, float beta, float *o_out,
+                                  uint64_t seed, uint32_t step, uint32_t b, uint32_t h,
+                                  float *Tp_out, double *margin_out)
+{
+    return step_f32(1, f, page, perm, q, k, v, alpha, beta, o_out, seed, step, b, h, Tp_out, margin_out);
 }
 
 /* ------------------------------------------------------------------------ */
@@ -552,12 +595,20 @@ static float lane_dot(const float *x, const float *y, int n)
     return p[0];
 }
 
-extern "C" int orc_window_step_f32(const orc_format *f, orc_page *page, const int32_t *perm,
-                                   float *P, float *K, float *D, int t, int commit,
-                                   const float *q, const float *k, const float *v,
-                                   const float *alpha, float beta, float *o_out,
-                                   uint64_t seed, uint32_t step, uint32_t b, uint32_t h,
-                                   double *margin_out)
+/* x . y over n channels as one fma chain in channel order, from +0 */
+static float plain_dot(const float *x, const float *y, int n)
+{
+    float acc = 0.0f;
+    for (int i = 0; i < n; ++i) acc = std::fmaf(x[i], y[i], acc);
+    return acc;
+}
+
+static int window_step_f32(int plain, const orc_format *f, orc_page *page, const int32_t *perm,
+                           float *P, float *K, float *D, int t, int commit,
+                           const float *q, const float *k, const float *v,
+                           const float *alpha, float beta, float *o_out,
+                           uint64_t seed, uint32_t step, uint32_t b, uint32_t h,
+                           double *margin_out)
 {
     if (orc_format_check(f) != 0 || !page || !perm || !P || !K || !D || t < 0 || !q || !k || !v ||
         !alpha || !o_out)
@@ -590,9 +641,9 @@ extern "C" int orc_window_step_f32(const orc_format *f, orc_page *page, const in
         wq[kap] = q[kap] * af[s];
     }
     /* prediction from the page and the earlier entries */
-    column_sum(f, perm, wk.data(), Z.data(), u.data());
+    column_sum_in(plain, f, perm, wk.data(), Z.data(), u.data());
     for (int tau = 0; tau < t; ++tau) {
-        const float a = lane_dot(K + (size_t)tau * d_k, k, d_k);
+        const float a = plain ? plain_dot(K + (size_t)tau * d_k, k, d_k) : lane_dot(K + (size_t)tau * d_k, k, d_k);
         for (int j = 0; j < d_v; ++j) u[j] = std::fmaf(a, D[(size_t)tau * d_v + j], u[j]);
     }
     /* this step's entry */
@@ -602,9 +653,9 @@ extern "C" int orc_window_step_f32(const orc_format *f, orc_page *page, const in
     }
     for (int kap = 0; kap < d_k; ++kap) K[(size_t)t * d_k + kap] = k[kap];
     /* readout from the page and every entry */
-    column_sum(f, perm, wq.data(), Z.data(), ot.data());
+    column_sum_in(plain, f, perm, wq.data(), Z.data(), ot.data());
     for (int tau = 0; tau <= t; ++tau) {
-        const float bq = lane_dot(K + (size_t)tau * d_k, q, d_k);
+        const float bq = plain ? plain_dot(K + (size_t)tau * d_k, q, d_k) : lane_dot(K + (size_t)tau * d_k, q, d_k);
         for (int j = 0; j < d_v; ++j) ot[j] = std::fmaf(bq, D[(size_t)tau * d_v + j], ot[j]);
     }
     for (int j = 0; j < d_v; ++j) o_out[j] = f->col_scales ? page->c[j] * ot[j] : ot[j];
@@ -628,15 +679,38 @@ extern "C" int orc_window_step_f32(const orc_format *f, orc_page *page, const in
     return 0;
 }
 
+extern "C" int orc_window_step_f32(const orc_format *f, orc_page *page, const int32_t *perm,
+                                   float *P, float *K, float *D, int t, int commit,
+                                   const float *q, const float *k, const float *v,
+                                   const float *alpha, float beta, float *o_out,
+                                   uint64_t seed, uint32_t step, uint32_t b, uint32_t h,
+                                   double *margin_out)
+{
+    return window_step_f32(0, f, page, perm, P, K, D, t, commit, q, k, v, alpha, beta, o_out, seed, step, b, h,
+                           margin_out);
+}
+
+extern "C" int orc_window_step_f32_plain(const orc_format *f, orc_page *page, const int32_t *perm,
+                                         float *P, float *K, float *D, int t, int commit,
+                                         const float *q, const float *k, const float *v,
+                                         const float *alpha, float beta, float *o_out,
+                                         uint64_t seed, uint32_t step, uint32_t b, uint32_t h,
+                                         double *margin_out)
+{
+    return window_step_f32(1, f, page, perm, P, K, D, t, commit, q, k, v, alpha, beta, o_out, seed, step, b, h,
+                           margin_out);
+}
+
+
 /* ------------------------------------------------------------------------ */
 /* prefill: a prompt of L tokens through one page, one requantization       */
 /* ------------------------------------------------------------------------ */
 
-extern "C" int orc_prefill_f32(const orc_format *f, orc_page *page, const int32_t *perm, int L,
-                               const float *q, const float *k, const float *v,
-                               const float *alpha, const float *beta, float *o_out,
-                               uint64_t seed, uint32_t step, uint32_t b, uint32_t h,
-                               float *Tp_out, double *margin_out)
+static int prefill_f32(int plain, const orc_format *f, orc_page *page, const int32_t *perm, int L,
+                       const float *q, const float *k, const float *v,
+                       const float *alpha, const float *beta, float *o_out,
+                       uint64_t seed, uint32_t step, uint32_t b, uint32_t h,
+                       float *Tp_out, double *margin_out)
 {
     if (orc_format_check(f) != 0 || !page || !perm || L < 1 || !q || !k || !v || !alpha || !beta || !o_out)
         return -1;
@@ -661,7 +735,7 @@ extern "C" int orc_prefill_f32(const orc_format *f, orc_page *page, const int32_
             }
         }
         /* the decode step's prediction, rank-1 update and readout */
-        column_sum(f, perm, kl, T.data(), u.data());
+        column_sum_in(plain, f, perm, kl, T.data(), u.data());
         for (int j = 0; j < d_v; ++j) e[j] = vl[j] * ic[j] - u[j];
         for (int s = 0; s < d_k; ++s) {
             const float bk = beta[l] * kl[perm[s]];
@@ -670,7 +744,7 @@ extern "C" int orc_prefill_f32(const orc_format *f, orc_page *page, const int32_
                 T[i] = std::fmaf(bk, e[j], T[i]);
             }
         }
-        column_sum(f, perm, ql, T.data(), ot.data());
+        column_sum_in(plain, f, perm, ql, T.data(), ot.data());
         for (int j = 0; j < d_v; ++j) o_out[(size_t)l * d_v + j] = f->col_scales ? page->c[j] * ot[j] : ot[j];
     }
     if (Tp_out) std::memcpy(Tp_out, T.data(), sizeof(float) * T.size());
@@ -679,6 +753,25 @@ extern "C" int orc_prefill_f32(const orc_format *f, orc_page *page, const int32_
                     margin_out ? margin_out + (size_t)s * d_v : nullptr);
     return 0;
 }
+
+extern "C" int orc_prefill_f32(const orc_format *f, orc_page *page, const int32_t *perm, int L,
+                               const float *q, const float *k, const float *v,
+                               const float *alpha, const float *beta, float *o_out,
+                               uint64_t seed, uint32_t step, uint32_t b, uint32_t h,
+                               float *Tp_out, double *margin_out)
+{
+    return prefill_f32(0, f, page, perm, L, q, k, v, alpha, beta, o_out, seed, step, b, h, Tp_out, margin_out);
+}
+
+extern "C" int orc_prefill_f32_plain(const orc_format *f, orc_page *page, const int32_t *perm, int L,
+                                     const float *q, const float *k, const float *v,
+                                     const float *alpha, const float *beta, float *o_out,
+                                     uint64_t seed, uint32_t step, uint32_t b, uint32_t h,
+                                     float *Tp_out, double *margin_out)
+{
+    return prefill_f32(1, f, page, perm, L, q, k, v, alpha, beta, o_out, seed, step, b, h, Tp_out, margin_out);
+}
+
 
 /* ------------------------------------------------------------------------ */
 /* lifetime weights from gate samples                                       */
@@ -692,19 +785,12 @@ extern "C" int orc_lifetime_weights(const orc_format *f, int B, int H, int n_sam
     const int na = f->gate_vector ? d_k : 1;
     for (int h = 0; h < H; ++h) {
         for (int kap = 0; kap < d_k; ++kap) {
-            /* the mean gate over the samples and requests, in double: the
-             * requests in eight slices [j B / 8, (j + 1) B / 8); per slice the
-             * samples, then its requests, ascending, from 0; the slice sums
-             * added as ((p0 + p1) + (p2 + p3)) + ((p4 + p5) + (p6 + p7)) */
-            double part[8];
-            for (int j = 0; j < 8; ++j) {
-                double acc = 0.0;
-                for (int t = 0; t < n_samples; ++t)
-                    for (int b = j * B / 8; b < (j + 1) * B / 8; ++b)
-                        acc += (double)alpha[(((size_t)t * B + b) * H + h) * na + (f->gate_vector ? kap : 0)];
-                part[j] = acc;
-            }
-            const double sum = ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
+            /* the mean gate over the samples and requests, in double: one
+             * sum from 0, samples in order, the requests of each in order */
+            double sum = 0.0;
+            for (int t = 0; t < n_samples; ++t)
+                for (int b = 0; b < B; ++b)
+                    sum += (double)alpha[(((size_t)t * B + b) * H + h) * na + (f->gate_vector ? kap : 0)];
             const double mean = sum / ((double)n_samples * (double)B);
             /* expected persistence under geometric decay: 1 / (1 - mean),
              * capped at 2^24 (a gate of one keeps its content for ever) */
@@ -900,11 +986,11 @@ extern "C" int orc_unpack_page(const orc_format *f, const uint8_t *bytes, orc_pa
     return 0;
 }
 
-extern "C" int orc_decode_step_pages(const orc_format *f, int B, int H, uint8_t *pages,
-                                     const int32_t *perm, const float *q, const float *k,
-                                     const float *v, const float *alpha, const float *beta,
-                                     float *o, uint64_t seed, uint32_t step,
-                                     long page_begin, long page_end)
+static int decode_step_pages(int plain, const orc_format *f, int B, int H, uint8_t *pages,
+                             const int32_t *perm, const float *q, const float *k,
+                             const float *v, const float *alpha, const float *beta,
+                             float *o, uint64_t seed, uint32_t step,
+                             long page_begin, long page_end)
 {
     if (!packable(f) || B < 1 || H < 1 || !pages || !perm) return -1;
     long pb = orc_page_bytes(f);
@@ -918,10 +1004,28 @@ extern "C" int orc_decode_step_pages(const orc_format *f, int B, int H, uint8_t 
         uint8_t *bytes = pages + (size_t)pi * pb;
         orc_unpack_page(f, bytes, &pg);
         const float *al = f->gate_vector ? alpha + (size_t)pi * 128 : alpha + pi;
-        orc_step_f32(f, &pg, perm + (size_t)h * 128, q + (size_t)pi * 128, k + (size_t)pi * 128,
-                     v + (size_t)pi * 128, al, beta[pi], o + (size_t)pi * 128,
-                     seed, step, b, h, nullptr, nullptr);
+        step_f32(plain, f, &pg, perm + (size_t)h * 128, q + (size_t)pi * 128, k + (size_t)pi * 128,
+                 v + (size_t)pi * 128, al, beta[pi], o + (size_t)pi * 128,
+                 seed, step, b, h, nullptr, nullptr);
         orc_pack_page(f, &pg, bytes);
     }
     return 0;
+}
+
+extern "C" int orc_decode_step_pages(const orc_format *f, int B, int H, uint8_t *pages,
+                                     const int32_t *perm, const float *q, const float *k,
+                                     const float *v, const float *alpha, const float *beta,
+                                     float *o, uint64_t seed, uint32_t step,
+                                     long page_begin, long page_end)
+{
+    return decode_step_pages(0, f, B, H, pages, perm, q, k, v, alpha, beta, o, seed, step, page_begin, page_end);
+}
+
+extern "C" int orc_decode_step_pages_plain(const orc_format *f, int B, int H, uint8_t *pages,
+                                           const int32_t *perm, const float *q, const float *k,
+                                           const float *v, const float *alpha, const float *beta,
+                                           float *o, uint64_t seed, uint32_t step,
+                                           long page_begin, long page_end)
+{
+    return decode_step_pages(1, f, B, H, pages, perm, q, k, v, alpha, beta, o, seed, step, page_begin, page_end);
 }

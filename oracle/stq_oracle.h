@@ -92,10 +92,8 @@ int orc_rank_rows(const orc_format *f, int B, int H, const float *S,
  * (STEPQuant landing page: errors in long-lived memory persist across many
  * steps; Figure B1: long gate half-lives hold most of the quantization
  * error).  alpha: [n_samples][B][H][d_k] (gate_vector) or [n_samples][B][H];
- * the mean is a double sum divided by n_samples * B: the requests in eight
- * slices [j B / 8, (j + 1) B / 8), per slice the samples then its requests
- * ascending, the slice sums added as a fixed pairwise tree;
- * row_weight: [H][d_k], rounded to float. */
+ * the mean is one double sum (samples in order, the requests of each in
+ * order) divided by n_samples * B; row_weight: [H][d_k], rounded to float. */
 int orc_lifetime_weights(const orc_format *f, int B, int H, int n_samples, const float *alpha,
                          float *row_weight);
 
@@ -106,6 +104,13 @@ int orc_dequantize_page(const orc_format *f, const orc_page *p, const int32_t *p
                         float *S_nat);
 
 /* ---- one decode step on one page: canonical fp32 evaluation -------------
+ * The pages fix no fp32 summation order.  The canonical order is the decode
+ * kernel's (a column sum deals the stored rows of every 16-row block into
+ * four slices of four consecutive rows; the rows of one slice in one half of
+ * the page form an fma chain in ascending stored row; per slice the two half
+ * chains are added, the four slice sums as (R0 + R1) + (R2 + R3)), kept so
+ * that the kernel can be checked bit for bit; orc_step_f32_plain below is the
+ * order-free anchor.
  * page is updated in place.  alpha points to 1 value (GDN) or d_k values in
  * natural key order (KDA).  q, k, v: d_k, d_k, d_v values.  o_out: d_v.
  * Tp_out (optional, d_k*d_v, stored order): the updated state in
@@ -119,6 +124,19 @@ int orc_step_f32(const orc_format *f, orc_page *page, const int32_t *perm,
                  const float *alpha, float beta, float *o_out,
                  uint64_t seed, uint32_t step, uint32_t b, uint32_t h,
                  float *Tp_out, double *margin_out);
+
+/* ---- the same step, plain fp32 evaluation ------------------------------
+ * As orc_step_f32 in every operation except the two column sums: each is one
+ * fma chain from +0 over the key channels in natural order (kappa = 0, 1,
+ * ...), the sum of the definition written left to right, with no blocking
+ * or tree.  Any correct fp32 evaluation of the step lies within the fp32
+ * rounding bound of this one; it anchors the GPU comparison, and the
+ * canonical order above is a second, stricter check. */
+int orc_step_f32_plain(const orc_format *f, orc_page *page, const int32_t *perm,
+                       const float *q, const float *k, const float *v,
+                       const float *alpha, float beta, float *o_out,
+                       uint64_t seed, uint32_t step, uint32_t b, uint32_t h,
+                       float *Tp_out, double *margin_out);
 
 /* ---- the same step from the plain definition in fp64 -------------------
  * Dequantizes the page in double, then S' = A S + beta k (v - (A S)^T k)^T,
@@ -157,6 +175,14 @@ int orc_window_step_f32(const orc_format *f, orc_page *page, const int32_t *perm
                         const float *alpha, float beta, float *o_out,
                         uint64_t seed, uint32_t step, uint32_t b, uint32_t h,
                         double *margin_out);
+/* The same with the plain column sums of orc_step_f32_plain and every buffer
+ * dot product one fma chain in channel order. */
+int orc_window_step_f32_plain(const orc_format *f, orc_page *page, const int32_t *perm,
+                              float *P, float *K, float *D, int t, int commit,
+                              const float *q, const float *k, const float *v,
+                              const float *alpha, float beta, float *o_out,
+                              uint64_t seed, uint32_t step, uint32_t b, uint32_t h,
+                              double *margin_out);
 
 /* ---- prefill: a prompt of L tokens through one page --------------------
  * The page's state runs through L decode steps in fp32 without being
@@ -176,6 +202,12 @@ int orc_prefill_f32(const orc_format *f, orc_page *page, const int32_t *perm, in
                     const float *alpha, const float *beta, float *o_out,
                     uint64_t seed, uint32_t step, uint32_t b, uint32_t h,
                     float *Tp_out, double *margin_out);
+/* The same with the plain column sums of orc_step_f32_plain. */
+int orc_prefill_f32_plain(const orc_format *f, orc_page *page, const int32_t *perm, int L,
+                          const float *q, const float *k, const float *v,
+                          const float *alpha, const float *beta, float *o_out,
+                          uint64_t seed, uint32_t step, uint32_t b, uint32_t h,
+                          float *Tp_out, double *margin_out);
 
 /* ---- packed byte layout (d_k = d_v = 128, row groups multiples of 16) ---- */
 int orc_pack_page(const orc_format *f, const orc_page *p, uint8_t *bytes);
@@ -189,6 +221,12 @@ int orc_decode_step_pages(const orc_format *f, int B, int H, uint8_t *pages,
                           const float *v, const float *alpha, const float *beta,
                           float *o, uint64_t seed, uint32_t step,
                           long page_begin, long page_end);
+/* The same with orc_step_f32_plain. */
+int orc_decode_step_pages_plain(const orc_format *f, int B, int H, uint8_t *pages,
+                                const int32_t *perm, const float *q, const float *k,
+                                const float *v, const float *alpha, const float *beta,
+                                float *o, uint64_t seed, uint32_t step,
+                                long page_begin, long page_end);
 
 /* ---- scalar building blocks, exported so tests can pin them ------------- */
 uint16_t orc_f32_to_f16_rn(float x);

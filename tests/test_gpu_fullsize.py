@@ -25,7 +25,7 @@ import oracle as O
 from linear_attention_recurrent_delta_b200 import binding as B
 from linear_attention_recurrent_delta_b200 import workloads as W
 
-from parity_util import BAND, make_state
+from parity_util import BAND, add_counts, assert_plain_ok, check_against_plain, make_state, maps_agree, plain_step
 
 pytestmark = pytest.mark.gpu
 
@@ -80,6 +80,7 @@ def test_full_size_step_on_sampled_pages(index):
 
     seed = W.sr_seed(w)
     o = torch.empty(w.batch, H, 128, device="cuda")
+    plain_total = {}
     for step in range(2):
         xd = W.step_inputs(w, step, device="cuda")
         xc = W.step_inputs(w, step, batch=SMALL_BATCH)
@@ -93,6 +94,13 @@ def test_full_size_step_on_sampled_pages(index):
         got_pages = qs.pages()[idx].cpu().numpy()
         band = 0
         for i, (p, (b, h)) in enumerate(zip(pos, src)):
+            # against the plain oracle, from the same packed input
+            ref = plain_step(fmt, pages[i], perm[h], xc["q"][b, h].numpy(), xc["k"][b, h].numpy(),
+                             xc["v"][b, h].numpy(), xc["alpha"][b, h].numpy(), float(xc["beta"][b, h]),
+                             seed, step, p // H, p % H)
+            res = check_against_plain(fmt, O.unpack_page(fmt, got_pages[i]), got_o[i], ref, perm[h])
+            assert_plain_ok(res, (w.name, step, p))
+            add_counts(plain_total, res)
             # the oracle steps its own page in place (each side continues from its own result)
             o_ref, _, margin = O.step_f32(fmt, pages[i], perm[h], xc["q"][b, h].numpy(), xc["k"][b, h].numpy(),
                                           xc["v"][b, h].numpy(), xc["alpha"][b, h].numpy(),
@@ -106,11 +114,16 @@ def test_full_size_step_on_sampled_pages(index):
                 assert np.all(margin[bad] < BAND), "codes of page %d outside the rounding band" % p
                 band += int(bad.sum())
         assert band == 0, "%d codes inside the rounding band differ (step %d)" % (band, step)
+    print("\n%s, %d sampled pages x 2 steps vs the plain oracle: code flips %d (in the 1e-5 band %d, by the "
+          "order bound %d), row scales differing %d, max o rel-L2 %.2e, max state rel-L2 %.2e"
+          % (w.name, len(pos), plain_total["flips"], plain_total["in_band"], plain_total["by_bound"],
+             plain_total["r_diff"], plain_total["o_rel"], plain_total["state_rel"]))
 
 
 def test_full_size_calibration_map():
-    """The precision map of the full int8row batch (256 requests = 8 chunks of
-    the calibration sum) from the CUDA path equals the oracle's, bit for bit."""
+    """The precision map of the full int8row batch (256 requests, summed by
+    the GPU in chunks of 32) from the CUDA path equals the oracle's (one
+    sequential double sum), except at a tie of scores at a group boundary."""
     w = W.WORKLOADS[1]
     S = W.initial_state(w)
     fmt = O.format_from_spec(w.format)
@@ -118,7 +131,8 @@ def test_full_size_calibration_map():
     qs = make_state(w)
     B.stq_calibrate(qs.state, S.cuda())
     torch.cuda.synchronize()
-    assert np.array_equal(qs.perm().cpu().numpy(), perm)
+    equal, tied = maps_agree(fmt, S.numpy(), qs.perm().cpu().numpy(), perm)
+    assert equal + tied == w.heads
 
 
 @pytest.mark.parametrize("index,window", [(1, 8), (2, 4), (3, 4), (4, 4)])

@@ -18,8 +18,8 @@ import oracle as O
 from linear_attention_recurrent_delta_b200 import binding as B
 from linear_attention_recurrent_delta_b200 import workloads as W
 
-from parity_util import (compare_pages, download, make_state, oracle_quantize, oracle_step, rel_l2,
-                         step_inputs_gpu, upload)
+from parity_util import (add_counts, assert_plain_ok, check_against_plain, compare_pages, download, make_state,
+                         maps_agree, oracle_quantize, oracle_step, plain_step, rel_l2, step_inputs_gpu, upload)
 
 pytestmark = pytest.mark.gpu
 
@@ -95,6 +95,40 @@ def test_step_matches_oracle_from_the_same_input(name):
         pages = expect
 
 
+@pytest.mark.parametrize("name", NAMES)
+def test_step_within_the_plain_oracle_band(name):
+    """The same steps against the oracle's plain evaluation (every column sum
+    one fma chain over the key channels in natural order): o and the
+    dequantized state within rel-L2 1e-5; codes and row scales identical
+    except inside the 1e-5 band or the fp32 bound of any summation order
+    around a rounding boundary; the flips are counted and printed."""
+    w = _small(name)
+    S = W.initial_state(w).numpy()
+    fmt, perm, pages = oracle_quantize(w, S)
+    qs = make_state(w)
+    seed = W.sr_seed(w)
+    total = {}
+    for step in range(w.steps):
+        x, xd = step_inputs_gpu(w, step)
+        upload(qs, perm, pages)
+        o_gpu = qs.step(xd["q"], xd["k"], xd["v"], xd["alpha"], xd["beta"], seed=seed, step=step)
+        got = download(qs)
+        o_gpu = o_gpu.cpu().numpy().reshape(w.pages, 128)
+        xs = {k: v.numpy().reshape(w.pages, -1) for k, v in x.items()}
+        for i in range(w.pages):
+            b, h = divmod(i, w.heads)
+            ref = plain_step(fmt, O.unpack_page(fmt, pages[i]), perm[h], xs["q"][i], xs["k"][i], xs["v"][i],
+                             xs["alpha"][i], float(xs["beta"][i][0]), seed, step, b, h)
+            res = check_against_plain(fmt, O.unpack_page(fmt, got[i]), o_gpu[i], ref, perm[h])
+            assert_plain_ok(res, (name, step, i))
+            add_counts(total, res)
+        pages = got
+    print("\n%s vs the plain oracle, %d page-steps: code flips %d (in the 1e-5 band %d, by the order bound %d), "
+          "row scales differing %d, max o rel-L2 %.2e, max state rel-L2 %.2e"
+          % (name, w.pages * w.steps, total["flips"], total["in_band"], total["by_bound"], total["r_diff"],
+             total["o_rel"], total["state_rel"]))
+
+
 def test_tiny_trajectory_free_running():
     """Workload 0 (1 x 4 pages, 64 steps): GPU and oracle each run free from
     their own quantization of the same fp32 state."""
@@ -117,9 +151,13 @@ def test_tiny_trajectory_free_running():
     print("trajectory: worst rel-L2 %.3g, bit-identical o on %d/%d steps" % (worst, exact, w.steps))
 
 
-@pytest.mark.parametrize("name", ["stepquant4_kda", "damp"])
+@pytest.mark.parametrize("name", ["int8row", "stepquant4_kda", "damp"])
 def test_long_trajectory_other_formats(name):
-    w = _small(name, batch=3, heads=4, steps=64)
+    """Free-running trajectories of the other formats at a small batch, over
+    their workload's step count and at least 64 steps (the uniform INT8
+    workload runs 128)."""
+    full = [x for x in W.WORKLOADS if x.fmt == name and x.index > 0][0]
+    w = _small(name, batch=3, heads=4, steps=max(64, full.steps))
     S = W.initial_state(w)
     fmt, perm, pages = oracle_quantize(w, S.numpy())
     qs = make_state(w)

@@ -24,8 +24,8 @@ PIN_FILES = ["tests/test_oracle_scalars.py", "tests/test_oracle_format.py",
 MUTANTS = {
     "error sign": ("e[j] = v[j] * ic[j] - u[j];", "e[j] = v[j] * ic[j] + u[j];"),
     "key index not permuted": ("float bk = beta * k[perm[s]];", "float bk = beta * k[s];"),
-    "readout with k": ("column_sum(f, perm, q, Tp.data(), ot.data());",
-                       "column_sum(f, perm, k, Tp.data(), ot.data());"),
+    "readout with k": ("column_sum_in(plain, f, perm, q, Tp.data(), ot.data());",
+                       "column_sum_in(plain, f, perm, k, Tp.data(), ot.data());"),
     "f32 decay dropped": ("a[s] = (orc_row_kind(f, s) == ORC_KIND_INT) ? al * page->r[s] : al;",
                           "a[s] = (orc_row_kind(f, s) == ORC_KIND_INT) ? page->r[s] : 1.0f;"),
     "f64 decay dropped": ("AS[(size_t)kap * d_v + j] = al * Sij;", "AS[(size_t)kap * d_v + j] = Sij;"),
@@ -49,8 +49,9 @@ MUTANTS = {
                                    "float a = std::fabs(S_nat[(size_t)j]);"),
     "window key decay dropped": ("K[(size_t)tau * d_k + kap] = K[(size_t)tau * d_k + kap] * al;",
                                  "K[(size_t)tau * d_k + kap] = K[(size_t)tau * d_k + kap];"),
-    "window prediction with q": ("const float a = lane_dot(K + (size_t)tau * d_k, k, d_k);",
-                                 "const float a = lane_dot(K + (size_t)tau * d_k, q, d_k);"),
+    "window prediction with q": (
+        "const float a = plain ? plain_dot(K + (size_t)tau * d_k, k, d_k) : lane_dot(K + (size_t)tau * d_k, k, d_k);",
+        "const float a = plain ? plain_dot(K + (size_t)tau * d_k, q, d_k) : lane_dot(K + (size_t)tau * d_k, q, d_k);"),
     "window delta without beta": ("D[(size_t)t * d_v + j] = beta * e;", "D[(size_t)t * d_v + j] = e;"),
     "window readout skips this step": ("for (int tau = 0; tau <= t; ++tau) {\n        const float bq",
                                        "for (int tau = 0; tau < t; ++tau) {\n        const float bq"),
@@ -64,13 +65,23 @@ MUTANTS = {
     "prefill later tokens not decayed": ("for (int j = 0; j < d_v; ++j) T[(size_t)s * d_v + j] = a_s * T[(size_t)s * d_v + j];",
                                          "for (int j = 0; j < d_v; ++j) T[(size_t)s * d_v + j] = T[(size_t)s * d_v + j];"),
     "prefill first beta for every token": ("const float bk = beta[l] * kl[perm[s]];", "const float bk = beta[0] * kl[perm[s]];"),
-    "prefill readout with k": ("column_sum(f, perm, ql, T.data(), ot.data());", "column_sum(f, perm, kl, T.data(), ot.data());"),
+    "prefill readout with k": ("column_sum_in(plain, f, perm, ql, T.data(), ot.data());",
+                               "column_sum_in(plain, f, perm, kl, T.data(), ot.data());"),
     "lifetime mean over samples only": ("const double mean = sum / ((double)n_samples * (double)B);",
                                         "const double mean = sum / (double)n_samples;"),
     "lifetime channel ignored": ("* H + h) * na + (f->gate_vector ? kap : 0)];", "* H + h) * na + 0];"),
     "lifetime head ignored": ("* H + h) * na + (f->gate_vector ? kap : 0)];",
                               "* H + 0) * na + (f->gate_vector ? kap : 0)];"),
-    "lifetime slice dropped": ("((part[4] + part[5]) + (part[6] + part[7]))", "((part[4] + part[5]) + part[6])"),
+    "lifetime first sample skipped": ("for (int t = 0; t < n_samples; ++t)\n                for (int b = 0; b < B; ++b)",
+                                      "for (int t = 1; t < n_samples; ++t)\n                for (int b = 0; b < B; ++b)"),
+    "plain chain skips channel 0": ("for (int kap = 0; kap < d_k; ++kap)\n            acc = std::fmaf(w_nat[kap], X[",
+                                    "for (int kap = 1; kap < d_k; ++kap)\n            acc = std::fmaf(w_nat[kap], X["),
+    "plain chain rows not permuted": ("for (int s = 0; s < d_k; ++s) row_of[perm[s]] = s;",
+                                      "for (int s = 0; s < d_k; ++s) row_of[s] = s;"),
+    "plain dot skips the last channel": ("for (int i = 0; i < n; ++i) acc = std::fmaf(x[i], y[i], acc);",
+                                         "for (int i = 0; i < n - 1; ++i) acc = std::fmaf(x[i], y[i], acc);"),
+    "calibration skips request 0": ("for (int b = 0; b < B; ++b) {\n                const float *row",
+                                    "for (int b = 1; b < B; ++b) {\n                const float *row"),
     "window butterfly half": ("for (int off = lanes / 2; off >= 1; off /= 2) {",
                               "for (int off = lanes / 2; off >= 2; off /= 2) {"),
 }

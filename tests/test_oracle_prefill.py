@@ -78,14 +78,15 @@ def test_one_token_is_the_decode_step(name):
     assert np.array_equal(pa.r, pb.r)
 
 
+@pytest.mark.parametrize("plain", [False, True])
 @pytest.mark.parametrize("name", list(W.FORMATS))
-def test_prompt_follows_the_f64_rule(name):
+def test_prompt_follows_the_f64_rule(name, plain):
     w, fmt, perm, page = _workload(name)
     q, k, v, alpha, beta = _prompt(w, 30, 32)
     S0 = _dequant64(fmt, page, perm)
     o64, S64 = _evolve64(S0, q, k, v, alpha, beta)
     pg = page.copy()
-    o, tp, _ = O.prefill_f32(fmt, pg, perm, q, k, v, alpha, beta, want_tp=True)
+    o, tp, _ = O.prefill_f32(fmt, pg, perm, q, k, v, alpha, beta, want_tp=True, plain=plain)
     for l in range(len(q)):
         assert _rel_l2(o[l], o64[l]) <= 1e-5, (l, _rel_l2(o[l], o64[l]))
     c = page.c.astype(np.float64) if fmt.col_scales else np.ones(fmt.d_v)

@@ -106,14 +106,17 @@ def _workload_case(name, rng):
             x["alpha"][0, 0].numpy(), float(x["beta"][0, 0]))
 
 
+@pytest.mark.parametrize("plain", [False, True])
 @pytest.mark.parametrize("name", list(W.FORMATS))
-def test_canonical_f32_matches_f64_definition(name):
+def test_canonical_f32_matches_f64_definition(name, plain):
+    """Both fp32 evaluations (the kernel's canonical order and the plain
+    natural-order chains) follow the fp64 definition to rel-L2 1e-5."""
     rng = np.random.default_rng(21)
     w, fmt, page, perm, q, k, v, alpha, beta = _workload_case(name, rng)
     for step in range(8):
         o64, sp64 = O.step_f64(fmt, page, perm, q, k, v, alpha, beta)
         o32, tp, _ = O.step_f32(fmt, page, perm, q, k, v, alpha, beta, seed=3, step=step,
-                                want_tp=True)
+                                want_tp=True, plain=plain)
         sp32 = np.zeros_like(sp64)
         sp32[perm] = tp.astype(np.float64) * (page.c.astype(np.float64) if fmt.col_scales else 1.0)
         assert _rel_l2(o32, o64) <= 1e-5
@@ -124,13 +127,14 @@ def test_canonical_f32_matches_f64_definition(name):
         alpha, beta = x["alpha"][0, 0].numpy(), float(x["beta"][0, 0])
 
 
+@pytest.mark.parametrize("plain", [False, True])
 @pytest.mark.parametrize("gate_vector", [False, True])
-def test_canonical_f32_matches_f64_d4(gate_vector):
+def test_canonical_f32_matches_f64_d4(gate_vector, plain):
     for seed in range(20):
         fmt = O.make_format(FORMATS_D4[0][0], d_k=4, d_v=4, col_scales=True, gate_vector=gate_vector)
         page, perm, q, k, v, alpha, beta = _random_case(fmt, np.random.default_rng(seed), gate_vector)
         o64, sp64 = O.step_f64(fmt, page, perm, q, k, v, alpha, beta)
-        o32, tp, _ = O.step_f32(fmt, page, perm, q, k, v, alpha, beta, want_tp=True)
+        o32, tp, _ = O.step_f32(fmt, page, perm, q, k, v, alpha, beta, want_tp=True, plain=plain)
         sp32 = np.zeros_like(sp64)
         sp32[perm] = tp.astype(np.float64) * page.c
         scale = np.abs(sp64).max()

@@ -82,7 +82,7 @@ def _inputs(w, first, n):
     return steps
 
 
-def _run_window(fmt, page, perm, steps, seed=0, step0=0, b=0, h=0):
+def _run_window(fmt, page, perm, steps, seed=0, step0=0, b=0, h=0, plain=False):
     """Run one window over steps (commit at the last); returns per-step (o, P, K, D) copies."""
     n = len(steps)
     P = np.ones(fmt.d_k, np.float32)
@@ -91,7 +91,7 @@ def _run_window(fmt, page, perm, steps, seed=0, step0=0, b=0, h=0):
     rec = []
     for t, (q, k, v, alpha, beta) in enumerate(steps):
         o, _ = O.window_step_f32(fmt, page, perm, P, K, D, t, t == n - 1, q, k, v, alpha, beta, seed=seed,
-                                 step=step0 + t, b=b, h=h)
+                                 step=step0 + t, b=b, h=h, plain=plain)
         rec.append((o, P.copy(), K.copy(), D.copy()))
     return rec
 
@@ -105,15 +105,16 @@ def _cumdecay(steps, first, last, d_k):
     return p
 
 
+@pytest.mark.parametrize("plain", [False, True])
 @pytest.mark.parametrize("name", list(W.FORMATS))
 @pytest.mark.parametrize("n", [1, 4, 8])
-def test_window_outputs_follow_the_f64_rule(name, n):
+def test_window_outputs_follow_the_f64_rule(name, n, plain):
     w, fmt, perm, page = _workload(name)
     steps = _inputs(w, 40, n)
     S0 = _dequant64(fmt, page, perm)
     c = _colscale(fmt, page)
     ref = _evolve64(S0, steps)
-    rec = _run_window(fmt, page.copy(), perm, steps)
+    rec = _run_window(fmt, page.copy(), perm, steps, plain=plain)
     for t in range(n):
         o, P, K, D = rec[t]
         o64, d64, _ = ref[t]
