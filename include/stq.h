@@ -144,9 +144,12 @@ stq_status stq_calibrate(stq_state *s, const float *d_S, const float *d_row_weig
  *     present on every GPU that loads the library until the process exits.
  *     States needing more (stq_calibrate_workspace_bytes(s) >
  *     STQ_CALIBRATE_NOALLOC_MAX_BYTES) get STQ_ERR_BUFFER_TOO_SMALL.
- *   - The first call on a device looks up the array's device address (a
- *     CUDA runtime query, with that device current); make that first call
- *     before capturing the stream into a graph.
+ *   - A call looks up the array's device address (a CUDA runtime query,
+ *     with the call's device current) unless its stream is being captured,
+ *     so a context rebuilt after a device reset is seen; a call made during
+ *     capture uses the address found by the device's last call outside it,
+ *     so make the first call on a device before capturing the stream into
+ *     a graph.
  *   - All calls share the array: calls that overlap on the GPU (other streams,
  *     other threads, other states) race on it and must be serialized by the
  *     caller.  Nothing in it needs clearing between calls.

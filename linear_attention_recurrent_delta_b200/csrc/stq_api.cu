@@ -164,16 +164,28 @@ static size_t state_span(const stq_state *s) {
     return state_bytes_for(s->dev, s->batch, s->heads);
 }
 
+}  // extern "C"
+
+stq_status stq::check_calibrate_input(const stq_state *s, const float *d_S, const float *d_row_weight) {
+    if (!s || !d_S) return STQ_ERR_INVALID_ARG;
+    if (!aligned(d_S, 16) || (d_row_weight && !aligned(d_row_weight, 4))) return STQ_ERR_MISALIGNED;
+    const size_t nS = (size_t)s->batch * s->heads * kD * kD * sizeof(float);
+    if (overlaps(d_S, nS, s->base, state_span(s))) return STQ_ERR_INVALID_ARG;
+    return STQ_OK;
+}
+
+extern "C" {
+
 stq_status stq_calibrate(stq_state *s, const float *d_S, const float *d_row_weight, void *d_workspace,
                          size_t workspace_bytes, void *stream) {
     if (!s || !d_S || !d_workspace) return STQ_ERR_INVALID_ARG;
-    if (!aligned(d_S, 16) || !aligned(d_workspace, 8) || (d_row_weight && !aligned(d_row_weight, 4)))
-        return STQ_ERR_MISALIGNED;
+    const stq_status in = stq::check_calibrate_input(s, d_S, d_row_weight);
+    if (in != STQ_OK) return in;
+    if (!aligned(d_workspace, 8)) return STQ_ERR_MISALIGNED;
     const size_t need = calibrate_workspace_bytes(s->batch, s->heads);
     if (workspace_bytes < need) return STQ_ERR_BUFFER_TOO_SMALL;
     const size_t nS = (size_t)s->batch * s->heads * kD * kD * sizeof(float);
-    if (overlaps(d_S, nS, s->base, state_span(s)) || overlaps(d_workspace, need, s->base, state_span(s)) ||
-        overlaps(d_workspace, need, d_S, nS))
+    if (overlaps(d_workspace, need, s->base, state_span(s)) || overlaps(d_workspace, need, d_S, nS))
         return STQ_ERR_INVALID_ARG;
     cudaError_t err = launch_calibrate(s, d_S, d_row_weight, static_cast<double *>(d_workspace),
                                        static_cast<cudaStream_t>(stream));

@@ -49,6 +49,10 @@ cudaError_t launch_prefill(const stq_state *s, int L, const float *q, const floa
                            uint32_t step, int stall_first_wait, bool early_launch, cudaStream_t stream);
 cudaError_t launch_calibrate(const stq_state *s, const float *S, const float *row_weight,
                              double *workspace, cudaStream_t stream);
+// The checks every calibration entry point makes of its fp32 state and row
+// weight: d_S non-null, 16-byte aligned and clear of the state's bytes;
+// d_row_weight (may be null) 4-byte aligned.  STQ_OK or the error to return.
+stq_status check_calibrate_input(const stq_state *s, const float *d_S, const float *d_row_weight);
 size_t calibrate_workspace_bytes(int batch, int heads);
 cudaError_t launch_quantize(const stq_state *s, const float *S, cudaStream_t stream);
 cudaError_t launch_dequantize(const stq_state *s, float *S, cudaStream_t stream);

@@ -101,21 +101,28 @@ static __device__ __align__(256) double g_calib_scratch[STQ_CALIBRATE_NOALLOC_MA
 
 // Device address of g_calib_scratch on the current device.  Host code must
 // not hand the symbol itself to a kernel (on the host it names a host-side
-// stand-in); the address is looked up once per device, with that device
-// current, and cached.
-static cudaError_t noalloc_scratch(double **out) {
+// stand-in).  The address is looked up with the device current, on every
+// call whose stream is not being captured (so a context rebuilt after a
+// device reset, which loads the module again, is seen), and kept per device
+// for calls made while a stream is captured, which use the address of the
+// device's last uncaptured call.
+static cudaError_t noalloc_scratch(cudaStream_t stream, double **out) {
     static std::mutex mu;
     static std::map<int, double *> addr;
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    err = cudaStreamIsCapturing(stream, &cs);
+    if (err != cudaSuccess) return err;
     std::lock_guard<std::mutex> lock(mu);
     auto it = addr.find(dev);
-    if (it == addr.end()) {
+    if (cs == cudaStreamCaptureStatusNone || it == addr.end()) {
         void *p = nullptr;
         err = cudaGetSymbolAddress(&p, g_calib_scratch);
         if (err != cudaSuccess) return err;
-        it = addr.emplace(dev, static_cast<double *>(p)).first;
+        addr[dev] = static_cast<double *>(p);
+        it = addr.find(dev);
     }
     *out = it->second;
     return cudaSuccess;
@@ -126,16 +133,12 @@ static cudaError_t noalloc_scratch(double **out) {
 extern "C" stq_status stq_calibrate_noalloc(stq_state *s, const float *d_S, const float *d_row_weight,
                                             void *stream) {
     using namespace stq;
-    if (!s || !d_S) return STQ_ERR_INVALID_ARG;
-    if (!((uintptr_t)d_S % 16 == 0) || (d_row_weight && (uintptr_t)d_row_weight % 4 != 0))
-        return STQ_ERR_MISALIGNED;
+    const stq_status in = check_calibrate_input(s, d_S, d_row_weight);
+    if (in != STQ_OK) return in;
     if (calibrate_workspace_bytes(s->batch, s->heads) > STQ_CALIBRATE_NOALLOC_MAX_BYTES)
         return STQ_ERR_BUFFER_TOO_SMALL;
-    const uintptr_t S0 = (uintptr_t)d_S, S1 = S0 + (size_t)s->batch * s->heads * kD * kD * sizeof(float);
-    const uintptr_t B0 = (uintptr_t)s->base, B1 = B0 + s->buf_bytes;
-    if (S0 < B1 && B0 < S1) return STQ_ERR_INVALID_ARG;
     double *ws = nullptr;
-    if (noalloc_scratch(&ws) != cudaSuccess) return STQ_ERR_CUDA;
+    if (noalloc_scratch(static_cast<cudaStream_t>(stream), &ws) != cudaSuccess) return STQ_ERR_CUDA;
     return launch_calibrate(s, d_S, d_row_weight, ws, static_cast<cudaStream_t>(stream)) == cudaSuccess
                ? STQ_OK : STQ_ERR_CUDA;
 }

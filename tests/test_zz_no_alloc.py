@@ -50,6 +50,24 @@ def test_noalloc_matches_the_workspace_entry_point_twice(index, batch, heads):
         np.testing.assert_array_equal(qs.perm().cpu().numpy(), expect, err_msg="call %d" % call)
 
 
+@pytest.mark.parametrize("batch,heads", [(1, 1024), (33, 512)])
+def test_noalloc_at_exactly_its_scratch_limit(batch, heads):
+    """States whose scratch need is exactly the array's size (1 MiB: one
+    chunk of requests x 1,024 heads, or two chunks, the second ragged, x 512
+    heads) are served, and give stq_calibrate's map on two calls in a row."""
+    w = W.WORKLOADS[2].resized(batch=batch, heads=heads)
+    ref, qs = _state(w), _state(w)
+    L = B.lib()
+    assert L.stq_calibrate_workspace_bytes(qs.state.handle) == (1 << 20)
+    S = W.initial_state(w, device="cuda")
+    B.stq_calibrate(ref.state, S)
+    for call in range(2):
+        qs.perm().zero_()
+        B.stq_calibrate_noalloc(qs.state, S)
+        torch.cuda.synchronize()
+        assert torch.equal(qs.perm(), ref.perm()), "call %d" % call
+
+
 def test_noalloc_with_row_weight_matches():
     w = W.WORKLOADS[3].resized(batch=20, heads=6)
     S = W.initial_state(w).cuda()
@@ -72,5 +90,13 @@ def test_noalloc_refuses_states_beyond_its_scratch():
     assert L.stq_state_alloc(ctypes.byref(fmt), w.batch, w.heads, fake, B.stq_state_bytes(fmt, w.batch, w.heads),
                              ctypes.byref(h)) == B.STQ_OK
     assert L.stq_calibrate_workspace_bytes(h) > (1 << 20)
+    assert L.stq_calibrate_noalloc(h, ctypes.c_void_p(1 << 42), None, None) == B.STQ_ERR_BUFFER_TOO_SMALL
+    L.stq_state_free(h)
+    # one head past the limit: 1 MiB + 1 KiB
+    w = W.WORKLOADS[2].resized(batch=1, heads=1025)
+    fmt = B.format_from_spec(w.format)
+    assert L.stq_state_alloc(ctypes.byref(fmt), w.batch, w.heads, fake, B.stq_state_bytes(fmt, w.batch, w.heads),
+                             ctypes.byref(h)) == B.STQ_OK
+    assert L.stq_calibrate_workspace_bytes(h) == (1 << 20) + 1024
     assert L.stq_calibrate_noalloc(h, ctypes.c_void_p(1 << 42), None, None) == B.STQ_ERR_BUFFER_TOO_SMALL
     L.stq_state_free(h)
