@@ -50,3 +50,22 @@ def test_plain_step_bytes_match_the_page_layout():
 def test_prefill_flops_and_peak():
     assert bench.prefill_flops_per_head_token() == 128 * 128 * 7
     assert abs(bench.FP32_PEAK_TFLOPS - 148 * 128 * 2 * 1.965e9 / 1e12) < 1e-9
+
+
+@pytest.mark.parametrize("k", [1, 2, 3, 5, 7, 20, 2000, 2003])
+def test_repetitions_cover_exactly_the_timed_steps(k):
+    sizes = bench.split_reps(k)
+    assert sum(sizes) == k
+    assert len(sizes) == min(5, k)
+    assert max(sizes) - min(sizes) <= 1
+
+
+def test_roofline_object_against_both_peaks():
+    spec = W.FORMATS["damp"]
+    pages, ms = 131072, 1.5
+    r = bench.hbm_roofline(spec, pages, ms, "damp-gdn")
+    gbs = bench.algorithmic_bytes_per_page(spec) * pages / (ms / 1000.0) / 1e9
+    assert abs(r["achieved"] - gbs) < 1e-9 * gbs
+    assert abs(r["frac"] - gbs / r["peak"]) < 1e-12
+    assert abs(r["frac_of_nominal_8tbs"] - gbs / 8000.0) < 1e-12
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s"
