@@ -53,6 +53,7 @@ def lib():
         L.orc_rank_rows.argtypes = [P, c_int, c_int, P, P, P]
         L.orc_quantize_page.argtypes = [P, P, P, P]
         L.orc_dequantize_page.argtypes = [P, P, P, P]
+        L.orc_quantize_page_fit.argtypes = [P, P, P, P, c_int, P, P]
         L.orc_step_f32.argtypes = [P, P, P, P, P, P, P, c_float, P, c_uint64, c_uint32,
                                    c_uint32, c_uint32, P, P]
         L.orc_step_f32_plain.argtypes = L.orc_step_f32.argtypes
@@ -173,6 +174,20 @@ def quantize_page(fmt, S_nat, perm):
     st = page._struct()
     _ok(lib().orc_quantize_page(ctypes.byref(fmt), _p(S_nat), _p(perm), ctypes.byref(st)), "quantize")
     return page
+
+
+def quantize_page_fit(fmt, S_nat, perm, impact=None, iters=4):
+    """Joint fit of the row and column scales (alternating weighted least
+    squares from the absmax scales).  Returns (page, objective per round)."""
+    S_nat = np.ascontiguousarray(S_nat, np.float32)
+    perm = np.ascontiguousarray(perm, np.int32)
+    w = None if impact is None else np.ascontiguousarray(impact, np.float32)
+    page = Page(fmt)
+    st = page._struct()
+    err = np.zeros(iters + 1, np.float64)
+    _ok(lib().orc_quantize_page_fit(ctypes.byref(fmt), _p(S_nat), _p(perm), _p(w), int(iters), ctypes.byref(st),
+                                    _p(err)), "quantize_page_fit")
+    return page, err
 
 
 def dequantize_page(fmt, page, perm):

@@ -441,6 +441,114 @@ extern "C" int orc_dequantize_page(const orc_format *f, const orc_page *p,
 }
 
 /* ------------------------------------------------------------------------ */
+/* joint fit of the row and column scales (STEPQuant's scale fitting)       */
+/* ------------------------------------------------------------------------ */
+
+/* Codes of INT row s for float scales r and c: the nearest code to
+ * S / (r c) (the product r c exact in double, one correctly rounded double
+ * division, ties to even), clamped to [-qmax, qmax]; 0 where r c is 0. */
+static void fit_codes_row(const orc_format *f, int s, const float *S_row, float r, const float *c, int32_t *z)
+{
+    const int qmax = orc_row_qmax(f, s);
+    for (int j = 0; j < f->d_v; ++j) {
+        const double d = (double)r * (double)c[j];
+        double n = (d > 0.0) ? std::nearbyint((double)S_row[j] / d) : 0.0;
+        if (n > qmax) n = qmax;
+        if (n < -qmax) n = -qmax;
+        z[j] = (int32_t)n;
+    }
+}
+
+/* sum over INT rows of w_kappa sum_j (S - z r c)^2, in double */
+static double fit_objective(const orc_format *f, const float *S_nat, const int32_t *perm, const float *w_nat,
+                            const std::vector<int32_t> &z, const std::vector<float> &r, const std::vector<float> &c)
+{
+    double e = 0.0;
+    for (int s = 0; s < f->d_k; ++s) {
+        if (orc_row_kind(f, s) != ORC_KIND_INT) continue;
+        const int kap = perm[s];
+        double row = 0.0;
+        for (int j = 0; j < f->d_v; ++j) {
+            const double d = (double)S_nat[(size_t)kap * f->d_v + j]
+                             - (double)z[(size_t)s * f->d_v + j] * (double)r[s] * (double)c[j];
+            row += d * d;
+        }
+        e += (w_nat ? (double)w_nat[kap] : 1.0) * row;
+    }
+    return e;
+}
+
+extern "C" int orc_quantize_page_fit(const orc_format *f, const float *S_nat, const int32_t *perm,
+                                     const float *impact_nat, int iters, orc_page *out, double *err_out)
+{
+    if (orc_format_check(f) != 0 || !S_nat || !perm || !out || iters < 0) return -1;
+    const int d_k = f->d_k, d_v = f->d_v;
+    /* start from the absmax scales */
+    int rc = orc_quantize_page(f, S_nat, perm, out);
+    if (rc != 0) return rc;
+    std::vector<float> r(out->r, out->r + d_k), c(out->c, out->c + d_v);
+    std::vector<int32_t> z((size_t)d_k * d_v, 0);
+    std::vector<int> row_of(d_k);
+    for (int s = 0; s < d_k; ++s) row_of[perm[s]] = s;
+    for (int it = 0; it < iters; ++it) {
+        /* the nearest codes for the current scales */
+        for (int s = 0; s < d_k; ++s)
+            if (orc_row_kind(f, s) == ORC_KIND_INT)
+                fit_codes_row(f, s, S_nat + (size_t)perm[s] * d_v, r[s], c.data(), z.data() + (size_t)s * d_v);
+        if (err_out) err_out[it] = fit_objective(f, S_nat, perm, impact_nat, z, r, c);
+        /* row scales: least squares of each row with its codes and c fixed,
+         * r_s = sum_j S z c / sum_j (z c)^2 (the row's impact weight cancels) */
+        for (int s = 0; s < d_k; ++s) {
+            if (orc_row_kind(f, s) != ORC_KIND_INT) continue;
+            const float *Sr = S_nat + (size_t)perm[s] * d_v;
+            double num = 0.0, den = 0.0;
+            for (int j = 0; j < d_v; ++j) {
+                const double zc = (double)z[(size_t)s * d_v + j] * (double)c[j];
+                num += (double)Sr[j] * zc;
+                den += zc * zc;
+            }
+            if (den > 0.0) r[s] = (float)(num / den);
+        }
+        /* column scales: impact-weighted least squares of each column with
+         * the codes and r fixed, c_j = sum_kappa w S z r / sum_kappa w (z r)^2,
+         * over the INT rows in natural key order */
+        if (f->col_scales) {
+            for (int j = 0; j < d_v; ++j) {
+                double num = 0.0, den = 0.0;
+                for (int kap = 0; kap < d_k; ++kap) {
+                    const int s = row_of[kap];
+                    if (orc_row_kind(f, s) != ORC_KIND_INT) continue;
+                    const double w = impact_nat ? (double)impact_nat[kap] : 1.0;
+                    const double zr = (double)z[(size_t)s * d_v + j] * (double)r[s];
+                    num += w * ((double)S_nat[(size_t)kap * d_v + j] * zr);
+                    den += w * (zr * zr);
+                }
+                if (den > 0.0) c[j] = (float)(num / den);
+            }
+        }
+    }
+    /* final codes for the fitted scales; float rows as the quantizer stores them */
+    for (int s = 0; s < d_k; ++s) {
+        const float *Sr = S_nat + (size_t)perm[s] * d_v;
+        if (orc_row_kind(f, s) == ORC_KIND_INT) {
+            if (iters > 0) fit_codes_row(f, s, Sr, r[s], c.data(), out->code + (size_t)s * d_v);
+            else for (int j = 0; j < d_v; ++j) z[(size_t)s * d_v + j] = out->code[(size_t)s * d_v + j];
+            out->r[s] = r[s];
+        } else if (iters > 0) {
+            std::vector<float> T(d_v);
+            for (int j = 0; j < d_v; ++j) T[j] = Sr[j] * (f->col_scales ? 1.0f / c[j] : 1.0f);
+            requant_row(f, s, T.data(), out, 0, 0, 0, 0, 0, nullptr);
+        }
+    }
+    for (int j = 0; j < d_v; ++j) out->c[j] = c[j];
+    if (err_out) {
+        std::vector<int32_t> zf(out->code, out->code + (size_t)d_k * d_v);
+        err_out[iters] = fit_objective(f, S_nat, perm, impact_nat, zf, r, c);
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
 /* decode step: canonical fp32 evaluation                                   */
 /* ------------------------------------------------------------------------ */
 

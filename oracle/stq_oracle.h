@@ -103,6 +103,28 @@ int orc_quantize_page(const orc_format *f, const float *S_nat, const int32_t *pe
 int orc_dequantize_page(const orc_format *f, const orc_page *p, const int32_t *perm,
                         float *S_nat);
 
+/* ---- joint fit of row and column scales (STEPQuant) ---------------------
+ * STEPQuant fits key-row and value-column scales jointly from the state's
+ * distribution and each key row's impact on the output error (paper-cards
+ * page, STEPQuant abstract; freedom251 post, "STEPQuant: precision can be
+ * allocated selectively").  The pages give no objective; the one used: the
+ * impact-weighted squared reconstruction error over the INT rows,
+ *     E = sum_kappa w_kappa sum_j (S_kappa,j - z r c)^2,
+ * w_kappa the row's readout impact (E[q_kappa^2] over calibration queries:
+ * o = S^T q, so a row's error reaches o scaled by q_kappa), minimized by
+ * alternating exact steps from the absmax scales, each of which cannot
+ * raise E:  z <- the nearest codes for (r, c) (clamped);  r_s <- the least
+ * squares row scale for z, c;  c_j <- the w-weighted least squares column
+ * scale for z, r (col_scales formats).  After `iters` rounds the codes are
+ * taken once more for the final scales.  Arithmetic in double with one
+ * rounding of each scale to float per update; sums in order (j ascending for
+ * rows, kappa ascending for columns); codes as S / (r c) by one double
+ * division.  impact_nat: [d_k] natural order, or NULL for uniform weights.
+ * err_out (optional, iters + 1 values): E before each round's scale updates
+ * and for the final page.  iters = 0 is orc_quantize_page. */
+int orc_quantize_page_fit(const orc_format *f, const float *S_nat, const int32_t *perm,
+                          const float *impact_nat, int iters, orc_page *out, double *err_out);
+
 /* ---- one decode step on one page: canonical fp32 evaluation -------------
  * The pages fix no fp32 summation order.  The canonical order is the decode
  * kernel's (a column sum deals the stored rows of every 16-row block into

@@ -19,7 +19,7 @@ SRC = os.path.join(ROOT, "oracle", "stq_oracle.cpp")
 HDR = os.path.join(ROOT, "oracle", "stq_oracle.h")
 PIN_FILES = ["tests/test_oracle_scalars.py", "tests/test_oracle_format.py",
              "tests/test_oracle_quantize.py", "tests/test_oracle_step.py", "tests/test_oracle_window.py",
-             "tests/test_oracle_prefill.py", "tests/test_oracle_lifetime.py"]
+             "tests/test_oracle_prefill.py", "tests/test_oracle_lifetime.py", "tests/test_oracle_fit.py"]
 
 MUTANTS = {
     "error sign": ("e[j] = v[j] * ic[j] - u[j];", "e[j] = v[j] * ic[j] + u[j];"),
@@ -82,6 +82,12 @@ MUTANTS = {
                                          "for (int i = 0; i < n - 1; ++i) acc = std::fmaf(x[i], y[i], acc);"),
     "calibration skips request 0": ("for (int b = 0; b < B; ++b) {\n                const float *row",
                                     "for (int b = 1; b < B; ++b) {\n                const float *row"),
+    "fit row scale ignores c": ("const double zc = (double)z[(size_t)s * d_v + j] * (double)c[j];",
+                                "const double zc = (double)z[(size_t)s * d_v + j];"),
+    "fit impact weights ignored": ("const double w = impact_nat ? (double)impact_nat[kap] : 1.0;",
+                                   "const double w = 1.0;"),
+    "fit codes truncate": ("double n = (d > 0.0) ? std::nearbyint((double)S_row[j] / d) : 0.0;",
+                           "double n = (d > 0.0) ? std::trunc((double)S_row[j] / d) : 0.0;"),
     "window butterfly half": ("for (int off = lanes / 2; off >= 1; off /= 2) {",
                               "for (int off = lanes / 2; off >= 2; off /= 2) {"),
 }
