@@ -76,8 +76,10 @@ MUTANTS = {
                                       "for (int t = 1; t < n_samples; ++t)\n                for (int b = 0; b < B; ++b)"),
     "plain chain skips channel 0": ("for (int kap = 0; kap < d_k; ++kap)\n            acc = std::fmaf(w_nat[kap], X[",
                                     "for (int kap = 1; kap < d_k; ++kap)\n            acc = std::fmaf(w_nat[kap], X["),
-    "plain chain rows not permuted": ("for (int s = 0; s < d_k; ++s) row_of[perm[s]] = s;",
-                                      "for (int s = 0; s < d_k; ++s) row_of[s] = s;"),
+    "plain chain rows not permuted": ("for (int s = 0; s < d_k; ++s) row_of[perm[s]] = s;\n    for (int j = 0;",
+                                      "for (int s = 0; s < d_k; ++s) row_of[s] = s;\n    for (int j = 0;"),
+    "fit column rows not permuted": ("for (int s = 0; s < d_k; ++s) row_of[perm[s]] = s;\n    for (int it = 0;",
+                                     "for (int s = 0; s < d_k; ++s) row_of[s] = s;\n    for (int it = 0;"),
     "plain dot skips the last channel": ("for (int i = 0; i < n; ++i) acc = std::fmaf(x[i], y[i], acc);",
                                          "for (int i = 0; i < n - 1; ++i) acc = std::fmaf(x[i], y[i], acc);"),
     "calibration skips request 0": ("for (int b = 0; b < B; ++b) {\n                const float *row",
