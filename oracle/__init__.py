@@ -65,6 +65,7 @@ def lib():
                                           c_uint32, c_uint32, c_uint32, P]
         L.orc_window_step_f32_plain.argtypes = L.orc_window_step_f32.argtypes
         L.orc_prefill_f32_plain.argtypes = L.orc_prefill_f32.argtypes
+        L.orc_prefill_chunked_f64.argtypes = [P, P, P, c_int, c_int, P, P, P, P, P, P, P]
         L.orc_pack_page.argtypes = [P, P, P]
         L.orc_unpack_page.argtypes = [P, P, P]
         L.orc_decode_step_pages.argtypes = [P, c_int, c_int, P, P, P, P, P, P, P, P,
@@ -260,6 +261,22 @@ def prefill_f32(fmt, page, perm, q, k, v, alpha, beta, seed=0, step=0, b=0, h=0,
     _ok(fn(ctypes.byref(fmt), ctypes.byref(st), _p(perm), int(L), _p(q), _p(k), _p(v), _p(a),
            _p(bt), _p(o), int(seed), int(step), int(b), int(h), _p(tp), _p(mg)), "prefill_f32")
     return o, tp, mg
+
+
+def prefill_chunked_f64(fmt, page, perm, q, k, v, alpha, beta, chunk):
+    """The chunk algebra of a prompt in fp64 from the page (unchanged).
+    Returns (o [L, d_v], final state [d_k, d_v] natural order), double."""
+    perm = np.ascontiguousarray(perm, np.int32)
+    q, k, v = (np.ascontiguousarray(x, np.float32) for x in (q, k, v))
+    L = q.shape[0]
+    a = np.ascontiguousarray(np.asarray(alpha, np.float32).reshape(L, -1)[:, :fmt.d_k if fmt.gate_vector else 1])
+    bt = np.ascontiguousarray(np.asarray(beta, np.float32).reshape(L))
+    o = np.zeros((L, fmt.d_v), np.float64)
+    sp = np.zeros((fmt.d_k, fmt.d_v), np.float64)
+    st = page._struct()
+    _ok(lib().orc_prefill_chunked_f64(ctypes.byref(fmt), ctypes.byref(st), _p(perm), int(L), int(chunk), _p(q), _p(k),
+                                      _p(v), _p(a), _p(bt), _p(o), _p(sp)), "prefill_chunked_f64")
+    return o, sp
 
 
 def step_f64(fmt, page, perm, q, k, v, alpha, beta):

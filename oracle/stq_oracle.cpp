@@ -882,6 +882,90 @@ extern "C" int orc_prefill_f32_plain(const orc_format *f, orc_page *page, const 
 
 
 /* ------------------------------------------------------------------------ */
+/* prefill, chunkwise form (the chunk algebra in fp64)                      */
+/* ------------------------------------------------------------------------ */
+
+extern "C" int orc_prefill_chunked_f64(const orc_format *f, const orc_page *page, const int32_t *perm, int L, int C,
+                                       const float *q, const float *k, const float *v,
+                                       const float *alpha, const float *beta, double *o_out, double *Sp_out)
+{
+    if (orc_format_check(f) != 0 || !page || !perm || L < 1 || C < 1 || !q || !k || !v || !alpha || !beta || !o_out)
+        return -1;
+    const int d_k = f->d_k, d_v = f->d_v;
+    const int na = f->gate_vector ? d_k : 1;
+    /* the page's state in natural key order, in double */
+    std::vector<double> S((size_t)d_k * d_v);
+    for (int s = 0; s < d_k; ++s) {
+        const double rs = (orc_row_kind(f, s) == ORC_KIND_INT) ? (double)page->r[s] : 1.0;
+        for (int j = 0; j < d_v; ++j)
+            S[(size_t)perm[s] * d_v + j] = (double)element_value(f, page, s, j) * rs
+                                           * (f->col_scales ? (double)page->c[j] : 1.0);
+    }
+    for (int t0 = 0; t0 < L; t0 += C) {
+        const int n = std::min(C, L - t0);
+        /* cumulative decay of the chunk's tokens per key channel: gam[i][c] =
+         * prod of the gates of tokens t0 .. t0 + i */
+        std::vector<double> gam((size_t)n * d_k);
+        for (int i = 0; i < n; ++i)
+            for (int c = 0; c < d_k; ++c) {
+                const double a = (double)alpha[(size_t)(t0 + i) * na + (f->gate_vector ? c : 0)];
+                gam[(size_t)i * d_k + c] = (i == 0 ? 1.0 : gam[(size_t)(i - 1) * d_k + c]) * a;
+            }
+        /* A[i][j] (j < i) = beta_i sum_c k_ic k_jc gam_ic / gam_jc;
+         * E = (I + A)^-1 R, R_i = beta_i (v_i - (gam_i k_i)^T S0), by forward
+         * substitution: E_i = R_i - sum_{j<i} A_ij E_j */
+        std::vector<double> E((size_t)n * d_v);
+        for (int i = 0; i < n; ++i) {
+            const float *ki = k + (size_t)(t0 + i) * d_k;
+            const double bi = (double)beta[t0 + i];
+            for (int j = 0; j < d_v; ++j) {
+                double pred = 0.0;
+                for (int c = 0; c < d_k; ++c) pred += gam[(size_t)i * d_k + c] * (double)ki[c] * S[(size_t)c * d_v + j];
+                E[(size_t)i * d_v + j] = bi * ((double)v[(size_t)(t0 + i) * d_v + j] - pred);
+            }
+            for (int jt = 0; jt < i; ++jt) {
+                const float *kj = k + (size_t)(t0 + jt) * d_k;
+                double a = 0.0;
+                for (int c = 0; c < d_k; ++c)
+                    a += (double)ki[c] * (double)kj[c] * (gam[(size_t)i * d_k + c] / gam[(size_t)jt * d_k + c]);
+                a *= bi;
+                for (int j = 0; j < d_v; ++j) E[(size_t)i * d_v + j] -= a * E[(size_t)jt * d_v + j];
+            }
+        }
+        /* o_i = (gam_i q_i)^T S0 + sum_{j<=i} (sum_c q_ic k_jc gam_ic / gam_jc) E_j */
+        for (int i = 0; i < n; ++i) {
+            const float *qi = q + (size_t)(t0 + i) * d_k;
+            double *oi = o_out + (size_t)(t0 + i) * d_v;
+            for (int j = 0; j < d_v; ++j) {
+                double acc = 0.0;
+                for (int c = 0; c < d_k; ++c) acc += gam[(size_t)i * d_k + c] * (double)qi[c] * S[(size_t)c * d_v + j];
+                oi[j] = acc;
+            }
+            for (int jt = 0; jt <= i; ++jt) {
+                const float *kj = k + (size_t)(t0 + jt) * d_k;
+                double pw = 0.0;
+                for (int c = 0; c < d_k; ++c)
+                    pw += (double)qi[c] * (double)kj[c] * (gam[(size_t)i * d_k + c] / gam[(size_t)jt * d_k + c]);
+                for (int j = 0; j < d_v; ++j) oi[j] += pw * E[(size_t)jt * d_v + j];
+            }
+        }
+        /* S <- diag(gam_n) S0 + sum_j (gam_n / gam_j k_j) E_j^T */
+        for (int c = 0; c < d_k; ++c) {
+            const double gn = gam[(size_t)(n - 1) * d_k + c];
+            for (int j = 0; j < d_v; ++j) {
+                double acc = gn * S[(size_t)c * d_v + j];
+                for (int jt = 0; jt < n; ++jt)
+                    acc += (gn / gam[(size_t)jt * d_k + c]) * (double)k[(size_t)(t0 + jt) * d_k + c]
+                           * E[(size_t)jt * d_v + j];
+                S[(size_t)c * d_v + j] = acc;
+            }
+        }
+    }
+    if (Sp_out) std::memcpy(Sp_out, S.data(), sizeof(double) * S.size());
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
 /* lifetime weights from gate samples                                       */
 /* ------------------------------------------------------------------------ */
 

@@ -19,7 +19,8 @@ SRC = os.path.join(ROOT, "oracle", "stq_oracle.cpp")
 HDR = os.path.join(ROOT, "oracle", "stq_oracle.h")
 PIN_FILES = ["tests/test_oracle_scalars.py", "tests/test_oracle_format.py",
              "tests/test_oracle_quantize.py", "tests/test_oracle_step.py", "tests/test_oracle_window.py",
-             "tests/test_oracle_prefill.py", "tests/test_oracle_lifetime.py", "tests/test_oracle_fit.py"]
+             "tests/test_oracle_prefill.py", "tests/test_oracle_lifetime.py", "tests/test_oracle_fit.py",
+             "tests/test_oracle_chunked.py"]
 
 MUTANTS = {
     "error sign": ("e[j] = v[j] * ic[j] - u[j];", "e[j] = v[j] * ic[j] + u[j];"),
@@ -90,6 +91,14 @@ MUTANTS = {
                                    "const double w = 1.0;"),
     "fit codes truncate": ("double n = (d > 0.0) ? std::nearbyint((double)S_row[j] / d) : 0.0;",
                            "double n = (d > 0.0) ? std::trunc((double)S_row[j] / d) : 0.0;"),
+    "chunk A without beta": ("                a *= bi;\n", "                a *= 1.0;\n"),
+    "chunk decay ratio inverted": (
+        "a += (double)ki[c] * (double)kj[c] * (gam[(size_t)i * d_k + c] / gam[(size_t)jt * d_k + c]);",
+        "a += (double)ki[c] * (double)kj[c] * (gam[(size_t)jt * d_k + c] / gam[(size_t)i * d_k + c]);"),
+    "chunk readout skips the diagonal": ("for (int jt = 0; jt <= i; ++jt) {\n                const float *kj = k + (size_t)(t0 + jt) * d_k;\n                double pw",
+                                         "for (int jt = 0; jt < i; ++jt) {\n                const float *kj = k + (size_t)(t0 + jt) * d_k;\n                double pw"),
+    "chunk state keeps the old state undecayed": ("double acc = gn * S[(size_t)c * d_v + j];",
+                                                  "double acc = S[(size_t)c * d_v + j];"),
     "window butterfly half": ("for (int off = lanes / 2; off >= 1; off /= 2) {",
                               "for (int off = lanes / 2; off >= 2; off /= 2) {"),
 }
