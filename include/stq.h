@@ -178,6 +178,36 @@ stq_status stq_lifetime_weights(const stq_state *s, const float *d_alpha, int n_
  * Clears the status word.  d_S as in stq_calibrate. */
 stq_status stq_quantize_state(stq_state *s, const float *d_S, void *stream);
 
+/* Largest number of fitting rounds stq_quantize_state_fit accepts. */
+#define STQ_FIT_MAX_ITERS 16
+
+/* Quantize with jointly fitted row and column scales (STEPQuant's scale
+ * fitting: key-row and value-column scales fitted to the state's
+ * distribution and to each key row's impact on the output error; paper-cards
+ * page, STEPQuant abstract; freedom251 post, "STEPQuant: precision can be
+ * allocated selectively").  The pages give no objective; the one minimized
+ * is the impact-weighted squared reconstruction error over the INT rows,
+ *     E = sum_kappa w_kappa sum_j (S_kappa,j - z r c)^2,
+ * from the absmax scales of stq_quantize_state by `iters` rounds of three
+ * exact steps, none of which can raise E: the nearest codes for (r, c)
+ * (z = RNE(S / (r c)) in double, clamped to +-qmax), the least-squares row
+ * scale of each row for its codes, and the w-weighted least-squares column
+ * scale of each column for the codes and the new r (column-scale formats);
+ * then the codes once more for the final scales.  Double arithmetic, sums in
+ * a fixed order, each scale rounded to float once per update.  FP16 rows are
+ * stored as binary16(S / c) with the final c.  iters = 0 is
+ * stq_quantize_state.  The decode step re-derives r from the row maximum at
+ * its first requantization; c stays as fitted.
+ *   d_S: as stq_quantize_state.  d_row_impact: device, [H][128] fp32 in
+ *   natural key order (a row's readout impact, e.g. the mean of q_kappa^2
+ *   over calibration queries: o = S^T q, so row kappa's error reaches o
+ *   scaled by q_kappa), >= 0, 4-byte aligned, or NULL for equal weights;
+ *   it must not overlap the state or d_S.
+ * Errors: INVALID_ARG (null s or d_S, iters outside [0, STQ_FIT_MAX_ITERS],
+ * overlap), MISALIGNED, CUDA.  Clears the status word. */
+stq_status stq_quantize_state_fit(stq_state *s, const float *d_S, const float *d_row_impact, int iters,
+                                  void *stream);
+
 /* One decode step on every page, in place (see the header comment).
  * d_q, d_k, d_v, d_o: [B][H][128], 16-byte aligned.  d_alpha: [B][H]
  * (4-byte aligned) or [B][H][128] (16-byte aligned, gate_vector).  d_beta:

@@ -56,6 +56,7 @@ def lib():
         "stq_calibrate": (c_int, [P, P, P, P, c_size_t, P]),
         "stq_calibrate_noalloc": (c_int, [P, P, P, P]),
         "stq_quantize_state": (c_int, [P, P, P]),
+        "stq_quantize_state_fit": (c_int, [P, P, P, c_int, P]),
         "stq_decode_step": (c_int, [P, P, P, P, P, P, P, c_uint64, c_uint32, P]),
         "stq_decode_step_slots": (c_int, [P, P, c_int, P, P, P, P, P, P, c_uint64, c_uint32, P]),
         "stq_request_pages": (c_int, [P, c_int, POINTER(c_size_t), POINTER(c_size_t)]),
@@ -176,6 +177,12 @@ def stq_calibrate_noalloc(state, S, row_weight=None, stream=None):
 
 def stq_quantize_state(state, S, stream=None):
     _check(lib().stq_quantize_state(state.handle, _ptr(S), _stream(stream)), "stq_quantize_state")
+
+
+def stq_quantize_state_fit(state, S, row_impact=None, iters=4, stream=None):
+    """Quantize with jointly fitted row and column scales (row_impact: [H, 128] or None)."""
+    _check(lib().stq_quantize_state_fit(state.handle, _ptr(S), _ptr(row_impact), int(iters), _stream(stream)),
+           "stq_quantize_state_fit")
 
 
 def stq_decode_step(state, q, k, v, alpha, beta, o, seed=0, step=0, stream=None):

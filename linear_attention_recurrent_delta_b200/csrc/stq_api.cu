@@ -217,6 +217,21 @@ stq_status stq_quantize_state(stq_state *s, const float *d_S, void *stream) {
     return err == cudaSuccess ? STQ_OK : STQ_ERR_CUDA;
 }
 
+stq_status stq_quantize_state_fit(stq_state *s, const float *d_S, const float *d_row_impact, int iters,
+                                  void *stream) {
+    if (!s || !d_S || iters < 0 || iters > STQ_FIT_MAX_ITERS) return STQ_ERR_INVALID_ARG;
+    if (!aligned(d_S, 16) || (d_row_impact && !aligned(d_row_impact, 4))) return STQ_ERR_MISALIGNED;
+    const size_t nS = (size_t)s->batch * s->heads * kD * kD * sizeof(float);
+    const size_t nW = (size_t)s->heads * kD * sizeof(float);
+    if (overlaps(d_S, nS, s->base, state_span(s))) return STQ_ERR_INVALID_ARG;
+    if (d_row_impact && (overlaps(d_row_impact, nW, s->base, state_span(s)) || overlaps(d_row_impact, nW, d_S, nS)))
+        return STQ_ERR_INVALID_ARG;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(s->base + s->status_offset, 0, sizeof(uint32_t), cs) != cudaSuccess) return STQ_ERR_CUDA;
+    cudaError_t err = launch_fit(s, d_S, d_row_impact, iters, cs);
+    return err == cudaSuccess ? STQ_OK : STQ_ERR_CUDA;
+}
+
 // n_rows: request rows of the inputs and of o (the state's batch, or the
 // length of a slot table)
 static stq_status check_step_args(const stq_state *s, int n_rows, const float *q, const float *k,

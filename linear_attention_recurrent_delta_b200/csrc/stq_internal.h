@@ -55,6 +55,8 @@ cudaError_t launch_calibrate(const stq_state *s, const float *S, const float *ro
 stq_status check_calibrate_input(const stq_state *s, const float *d_S, const float *d_row_weight);
 size_t calibrate_workspace_bytes(int batch, int heads);
 cudaError_t launch_quantize(const stq_state *s, const float *S, cudaStream_t stream);
+// Quantize with jointly fitted scales (iters rounds; 0: launch_quantize).
+cudaError_t launch_fit(const stq_state *s, const float *S, const float *impact, int iters, cudaStream_t stream);
 cudaError_t launch_dequantize(const stq_state *s, float *S, cudaStream_t stream);
 
 }  // namespace stq
