@@ -212,8 +212,9 @@ stq_status stq_quantize_state_fit(stq_state *s, const float *d_S, const float *d
  * d_q, d_k, d_v, d_o: [B][H][128], 16-byte aligned.  d_alpha: [B][H]
  * (4-byte aligned) or [B][H][128] (16-byte aligned, gate_vector).  d_beta:
  * [B][H].  None may overlap the state buffer, and d_o may overlap no input.
- * seed and step feed the stochastic-rounding generator only (Philox-4x32-10,
- * key = seed, counter = (tile, step, request, head)).  q is used as given.
+ * seed and step feed the stochastic-rounding generator only (the pcg4d hash
+ * of Jarzynski and Olano, JCGT 2020, of (tile, step, request ^ low seed word,
+ * head ^ high seed word)).  q is used as given.
  * The kernel is launched as a programmatic dependent launch: it may become
  * resident while the previous kernel on `stream` finishes, and reads nothing
  * from global memory until that kernel has completed and its writes are
@@ -321,6 +322,28 @@ stq_status stq_window_step(stq_state *s, void *d_buf, size_t buf_bytes, int wind
 stq_status stq_prefill(stq_state *s, int L, const float *d_q, const float *d_k, const float *d_v,
                        const float *d_alpha, const float *d_beta, float *d_o, float *d_S_out, uint64_t seed,
                        uint32_t step, void *stream);
+
+/* The same prefill in chunkwise form on the tensor cores (GDN states: a
+ * scalar gate per token and page).  The prompt runs in chunks of 128 tokens;
+ * per chunk, with gam_i the product of the chunk's gates up to token i, the
+ * chunk's deltas E are the triangular solve (I + A) E = R,
+ *     A_ij = beta_i (gam_i / gam_j) (k_i . k_j)  (j < i),
+ *     R_i  = beta_i (v_i - gam_i S0^T k_i),
+ * o_i = gam_i S0^T q_i + sum_{j<=i} (gam_i / gam_j) (q_i . k_j) E_j, and the
+ * state becomes gam_n S0 + sum_j (gam_n / gam_j) k_j E_j^T, the token
+ * recurrence of stq_prefill resolved a chunk at a time (repeated prefill,
+ * DASC card page).  The products run as tf32 tensor-core MMAs with split
+ * operands (fp32 = tf32 part + remainder, three products), the solve on the
+ * CUDA cores; results agree with stq_prefill to fp32 rounding, not bit for
+ * bit (the summation order differs), and the one requantization after the
+ * last token is stq_prefill's.  Arguments, layouts and errors as
+ * stq_prefill, plus UNSUPPORTED for gate_vector formats (KDA: use
+ * stq_prefill).  One CTA per page (the whole shared memory and tensor
+ * memory of an SM); a bounded wait that ran out is reported by
+ * stq_device_status. */
+stq_status stq_prefill_chunked(stq_state *s, int L, const float *d_q, const float *d_k, const float *d_v,
+                               const float *d_alpha, const float *d_beta, float *d_o, float *d_S_out,
+                               uint64_t seed, uint32_t step, void *stream);
 
 /* Device staging bytes stq_decode_step_host needs (q, k, v, alpha, beta, o). */
 size_t stq_decode_io_bytes(const stq_state *s);

@@ -8,7 +8,7 @@
 //   S3 column sums u = sum_s k_s T_s        e = v (1/c) - u
 //   S4 T' = T + (beta k_s) e                 S5 o = c * sum_s q_s T'_s
 //   S6 row absmax -> r' = m/qmax, inv = qmax/m rounded toward zero
-//   S7 requant (RNE of the exact product, or Philox stochastic rounding on
+//   S7 requant (RNE of the exact product, or pcg4d stochastic rounding on
 //      INT rows; binary16 on FP16 rows)    S8 repack.
 // The requantized codes and r' are written back into the page's ring stage,
 // and one bulk copy stores the stage to HBM at the next page's barrier, so
@@ -137,7 +137,7 @@ __device__ __forceinline__ void write_o(const float (*red_o)[kD], const DecodeAr
 }
 
 // Resident CTAs per SM the register budget is sized for: 3 (168 registers);
-// the stochastic-rounding variant carries the Philox state and gets 2.
+// the stochastic-rounding variant carries the hash state and gets 2.
 template <bool SR>
 constexpr int decode_ctas_per_sm() { return SR ? 2 : 3; }
 

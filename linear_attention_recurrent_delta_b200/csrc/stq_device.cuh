@@ -1,6 +1,6 @@
 // stq_device.cuh -- device building blocks of the quantized Delta-rule
 // decode step for sm_100a: page format, plane unpack/pack, dequant/requant,
-// Philox-4x32-10, bulk-copy staging with bounded mbarrier waits.
+// the pcg4d stochastic-rounding hash, bulk-copy staging with bounded mbarrier waits.
 //
 // In every page kernel lane l of a warp owns value columns 4l .. 4l+3.  The
 // packed layout is built so that a lane reads and writes its columns as
@@ -242,19 +242,30 @@ __device__ __forceinline__ uint32_t low_bytes(float y0, float y1, float y2, floa
     return __byte_perm(lo, hi, 0x5410u);
 }
 
-// --------------------------------------------------------------- Philox --
-// Philox-4x32-10 (Salmon, Moraes, Dror, Shaw, SC'11): ten rounds of a
-// multiply-xor bijection on a 128-bit counter; the 64-bit key is bumped by
-// the Weyl constants between rounds.
-__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
-#pragma unroll
-    for (int round = 0; round < 10; ++round) {
-        if (round > 0) { k0 += 0x9E3779B9u; k1 += 0xBB67AE85u; }
-        uint32_t hi0 = __umulhi(0xD2511F53u, c.x), lo0 = 0xD2511F53u * c.x;
-        uint32_t hi1 = __umulhi(0xCD9E8D57u, c.z), lo1 = 0xCD9E8D57u * c.z;
-        c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
-    }
-    return c;
+// ------------------------------------------------- stochastic-rounding hash --
+// pcg4d (Jarzynski and Olano, "Hash Functions for GPU Rendering", JCGT 9(3),
+// 2020): a linear congruential step on each word, each word plus the product
+// of two others, a 16-bit xorshift of every word, the products once more.
+// Input: the counter (c.x, c.y) and (c.z, c.w) xor the 64-bit seed (k0, k1).
+__device__ __forceinline__ uint4 sr_hash4(uint4 c, uint32_t k0, uint32_t k1) {
+    uint32_t x = c.x, y = c.y, z = c.z ^ k0, w = c.w ^ k1;
+    x = x * 1664525u + 1013904223u;
+    y = y * 1664525u + 1013904223u;
+    z = z * 1664525u + 1013904223u;
+    w = w * 1664525u + 1013904223u;
+    x += y * w;
+    y += z * x;
+    z += x * y;
+    w += y * z;
+    x ^= x >> 16;
+    y ^= y >> 16;
+    z ^= z >> 16;
+    w ^= w >> 16;
+    x += y * w;
+    y += z * x;
+    z += x * y;
+    w += y * z;
+    return make_uint4(x, y, z, w);
 }
 
 // Stochastic-rounding offsets of the two columns held by one 32-bit word:

@@ -11,7 +11,7 @@
 //   token l   T = RN(alpha T)          (the fp32 state decayed in place)
 //   each      u = T^T k (canonical column sums), e = v (1/c) - u,
 //             T = fma(beta k, e, T), o = c T^T q
-// then the decode step's row scales and requantization (RTN or Philox SR
+// then the decode step's row scales and requantization (RTN or pcg4d SR
 // with `step`), in place in the page's buffer, and one bulk store.
 // Pages are double-buffered in shared memory; each token's q, k, v (and KDA
 // gate) rows stream through a ring of token stages, all by cp.async.bulk (no

@@ -1,7 +1,7 @@
 // stq_slices.cuh -- per-slice device pieces of the packed-state kernels (sm_100a):
 // the compile-time formats, plane unpack / pack of one slice (rows 4w .. 4w+3 of a
 // 16-row block, lane l holding columns 4l .. 4l+3), dequantization, requantization
-// (round to nearest or Philox stochastic rounding), the readout chains and the
+// (round to nearest or pcg4d stochastic rounding), the readout chains and the
 // divisions of the row-scale step.  Included by the decode and window kernels.
 #pragma once
 
@@ -292,7 +292,7 @@ __device__ __forceinline__ void requant_slice(uint8_t *blk, int w, int lane, con
             float2 y0, y1, y2, y3;
             if constexpr (SR) {
                 const uint32_t s = 16u * B + 4u * (uint32_t)w + (uint32_t)i;   // stored row, even
-                const uint4 h = philox4x32_10(make_uint4((s >> 1) * 32u + (uint32_t)lane, sr.step, sr.b, sr.h),
+                const uint4 h = sr_hash4(make_uint4((s >> 1) * 32u + (uint32_t)lane, sr.step, sr.b, sr.h),
                                               sr.k0, sr.k1);
                 y0 = __fadd2_rn(__ffma2_rn(T[B][i][0], i0, sr_delta_pair(h.x)), M2);
                 y1 = __fadd2_rn(__ffma2_rn(T[B][i][1], i0, sr_delta_pair(h.y)), M2);

@@ -80,7 +80,7 @@ def lib():
         L.orc_f32_to_f16_rn_n.argtypes = [P, P, c_long]
         L.orc_f16_to_f32_n.argtypes = [P, P, c_long]
         L.orc_div_rz_n.argtypes = [P, P, P, c_long]
-        L.orc_philox4x32_10.argtypes = [P, P, P]
+        L.orc_pcg4d.argtypes = [P, P]
         L.orc_sr_delta.argtypes = [c_uint64, c_uint32, c_uint32, c_uint32, c_int, c_int, c_int]
         L.orc_sr_delta.restype = c_float
     return _lib
@@ -347,11 +347,11 @@ def div_rz(a, b):
     return out
 
 
-def philox4x32_10(ctr, key):
-    c = np.ascontiguousarray(ctr, np.uint32)
-    kk = np.ascontiguousarray(key, np.uint32)
+def pcg4d(v):
+    """pcg4d of a 4-word input (uint32 array of 4)."""
+    v = np.ascontiguousarray(v, np.uint32)
     out = np.zeros(4, np.uint32)
-    lib().orc_philox4x32_10(_p(c), _p(kk), _p(out))
+    lib().orc_pcg4d(_p(v), _p(out))
     return out
 
 

@@ -218,42 +218,47 @@ extern "C" void orc_div_rz_n(const float *a, const float *b, float *out, long n)
     for (long i = 0; i < n; ++i) out[i] = orc_div_rz(a[i], b[i]);
 }
 
-/* Philox-4x32-10, the counter-based generator of Salmon, Moraes, Dror and
- * Shaw, "Parallel random numbers: as easy as 1, 2, 3" (SC'11): ten rounds of
- * a multiply-xor bijection on a 128-bit counter, the 64-bit key bumped by the
- * Weyl constants between rounds. */
-extern "C" void orc_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4])
+/* pcg4d, the four-word hash of Jarzynski and Olano, "Hash Functions for GPU
+ * Rendering" (Journal of Computer Graphics Techniques 9(3), 2020): a linear
+ * congruential step on each word (multiplier 1664525, increment 1013904223),
+ * then each word plus the product of two others, a 16-bit xorshift of every
+ * word, and the products once more.  Every step is invertible, so the map is
+ * a bijection of the 128-bit input. */
+extern "C" void orc_pcg4d(const uint32_t in[4], uint32_t out[4])
 {
-    uint32_t x0 = ctr[0], x1 = ctr[1], x2 = ctr[2], x3 = ctr[3];
-    uint32_t k0 = key[0], k1 = key[1];
-    for (int round = 0; round < 10; ++round) {
-        if (round > 0) { k0 += 0x9E3779B9u; k1 += 0xBB67AE85u; }
-        uint64_t p0 = (uint64_t)0xD2511F53u * (uint64_t)x0;
-        uint64_t p1 = (uint64_t)0xCD9E8D57u * (uint64_t)x2;
-        uint32_t hi0 = (uint32_t)(p0 >> 32), lo0 = (uint32_t)p0;
-        uint32_t hi1 = (uint32_t)(p1 >> 32), lo1 = (uint32_t)p1;
-        uint32_t y0 = hi1 ^ x1 ^ k0;
-        uint32_t y1 = lo1;
-        uint32_t y2 = hi0 ^ x3 ^ k1;
-        uint32_t y3 = lo0;
-        x0 = y0; x1 = y1; x2 = y2; x3 = y3;
-    }
-    out[0] = x0; out[1] = x1; out[2] = x2; out[3] = x3;
+    uint32_t x = in[0], y = in[1], z = in[2], w = in[3];
+    x = x * 1664525u + 1013904223u;
+    y = y * 1664525u + 1013904223u;
+    z = z * 1664525u + 1013904223u;
+    w = w * 1664525u + 1013904223u;
+    x += y * w;
+    y += z * x;
+    z += x * y;
+    w += y * z;
+    x ^= x >> 16;
+    y ^= y >> 16;
+    z ^= z >> 16;
+    w ^= w >> 16;
+    x += y * w;
+    y += z * x;
+    z += x * y;
+    w += y * z;
+    out[0] = x; out[1] = y; out[2] = z; out[3] = w;
 }
 
 /* Stochastic-rounding offset for element (s, j) of page (b, h) at a step.
- * One Philox call serves a 2-row x 4-column tile: counter
- * (tile index, step, request, head), key = the 64-bit seed.  Word
- * 2*(s & 1) + ((j >> 1) & 1) of the output holds columns j & ~1 (high 16 bits)
- * and j | 1 (low 16 bits).  delta = (h16 - 32767.5) / 65536, exactly. */
+ * One hash serves a 2-row x 4-column tile: input (tile index, step,
+ * request ^ low seed word, head ^ high seed word).  Word 2*(s & 1) +
+ * ((j >> 1) & 1) of the output holds columns j & ~1 (high 16 bits) and j | 1
+ * (low 16 bits).  delta = (h16 - 32767.5) / 65536, exactly. */
 extern "C" float orc_sr_delta(uint64_t seed, uint32_t step, uint32_t b, uint32_t h,
                               int s, int j, int d_v)
 {
     uint32_t quads = (uint32_t)((d_v + 3) / 4);
-    uint32_t ctr[4] = { (uint32_t)(s >> 1) * quads + (uint32_t)(j >> 2), step, b, h };
-    uint32_t key[2] = { (uint32_t)seed, (uint32_t)(seed >> 32) };
+    uint32_t in[4] = { (uint32_t)(s >> 1) * quads + (uint32_t)(j >> 2), step,
+                       b ^ (uint32_t)seed, h ^ (uint32_t)(seed >> 32) };
     uint32_t out[4];
-    orc_philox4x32_10(ctr, key, out);
+    orc_pcg4d(in, out);
     uint32_t word = out[((s & 1) << 1) | ((j >> 1) & 1)];
     uint32_t h16 = (j & 1) ? (word & 0xFFFFu) : (word >> 16);
     return (float)(2 * (int)h16 - 65535) * 0x1p-17f;

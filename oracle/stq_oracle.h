@@ -277,7 +277,8 @@ float orc_div_rz(float a, float b);
 void orc_f32_to_f16_rn_n(const float *x, uint16_t *out, long n);
 void orc_f16_to_f32_n(const uint16_t *x, float *out, long n);
 void orc_div_rz_n(const float *a, const float *b, float *out, long n);
-void orc_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4]);
+/* pcg4d (Jarzynski and Olano, JCGT 2020), the stochastic-rounding hash */
+void orc_pcg4d(const uint32_t in[4], uint32_t out[4]);
 /* stochastic-rounding offset delta in (-1/2, 1/2) for element (s, j) */
 float orc_sr_delta(uint64_t seed, uint32_t step, uint32_t b, uint32_t h,
                    int s, int j, int d_v);

@@ -38,7 +38,8 @@ MUTANTS = {
     "rounding truncates": ("zr = std::nearbyint(x);", "zr = std::trunc(x);"),
     "bias wrong": ("int bias = (kind == ORC_KIND_INT) ? (1 << (bits - 1)) : 0;",
                    "int bias = (kind == ORC_KIND_INT) ? (1 << bits) - 1 : 0;"),
-    "philox key bump": ("k1 += 0xBB67AE85u;", "k1 += 0x9E3779B9u;"),
+    "pcg4d xorshift dropped": ("    w ^= w >> 16;\n    x += y * w;", "    x += y * w;"),
+    "pcg4d seed not mixed": ("b ^ (uint32_t)seed, h ^ (uint32_t)(seed >> 32) };", "b, h };"),
     "fp16 ties away": ("double n = std::nearbyint(t);\n    if (n >= 2048.0)",
                        "double n = std::floor(t + 0.5);\n    if (n >= 2048.0)"),
     "ranking ascending": ("return score[a] > score[b2];", "return score[a] < score[b2];"),

@@ -1,6 +1,6 @@
 """Pins of the oracle's scalar building blocks against things other than itself:
 library routines (numpy's IEEE binary16 conversion), exact rational arithmetic
-(fractions.Fraction), and Philox-4x32-10 against cuRAND's implementation.
+(fractions.Fraction), and the pcg4d hash by its inverse and its statistics.
 """
 from fractions import Fraction
 
@@ -80,72 +80,71 @@ def test_div_rz_exact_quotients_are_kept():
     np.testing.assert_array_equal(O.div_rz(a, m), (a.astype(np.float64) / m).astype(np.float32))
 
 
-# --------------------------------------------------------------- Philox ----
-# Philox-4x32-10 (Salmon, Moraes, Dror, Shaw, SC'11) pinned to an independent
-# implementation: cuRAND's host generator CURAND_RNG_PSEUDO_PHILOX4_32_10
-# (NVIDIA's CUDA library, run on the CPU).  With seed s it emits block m
-# (4 words) = Philox(counter = (x, y, z, 0), key = (s mod 2^32, s >> 32))
-# where m = (y * 2^32 + x) * 65536 + z: 65,536 interleaved subsequences.  A
-# generator offset of 4m starts the stream at block m, which reaches the
-# first three counter words; the fourth is pinned on the GPU
-# (tests/test_gpu_philox.py, cuRAND's device API).
-_CURAND = None
+# ---------------------------------------------------------------- pcg4d ----
+# pcg4d (Jarzynski and Olano, "Hash Functions for GPU Rendering", JCGT 2020):
+# the pins check what the stochastic rounding needs of it, each of which a
+# plausible slip (a dropped mixing step, a wrong shift, a swapped word)
+# breaks: every step is invertible, so the map is a bijection (the inverse,
+# written out here, recovers random inputs); the 16-bit halves the rounding
+# uses are uniform over consecutive counters (chi-square); neighbouring
+# counters give unrelated words (correlation of halves, and about half of the
+# output bits flip when one input bit flips).
+def _pcg4d_inverse(o):
+    x, y, z, w = (int(v) for v in o)
+    M = 0xFFFFFFFF
+    w = (w - y * z) & M
+    z = (z - x * y) & M
+    y = (y - z * x) & M
+    x = (x - y * w) & M
+
+    def unshift(v):
+        return v ^ (v >> 16)            # a 16-bit xorshift of a 32-bit word is its own inverse
+    x, y, z, w = unshift(x), unshift(y), unshift(z), unshift(w)
+    w = (w - y * z) & M
+    z = (z - x * y) & M
+    y = (y - z * x) & M
+    x = (x - y * w) & M
+    ainv = pow(1664525, -1, 2**32)
+    return [((v - 1013904223) * ainv) & M for v in (x, y, z, w)]
 
 
-def _curand():
-    global _CURAND
-    if _CURAND is None:
-        import ctypes
-        import glob
-        import os
-        import torch
-        paths = glob.glob(os.path.join(os.path.dirname(torch.__file__), "..", "nvidia", "curand", "lib",
-                                       "libcurand.so*")) + glob.glob("/usr/local/cuda/lib64/libcurand.so*")
-        for path in paths:
-            try:
-                _CURAND = ctypes.CDLL(path)
-                break
-            except OSError:
-                continue
-        if _CURAND is None:
-            pytest.skip("libcurand not found")
-    return _CURAND
+def test_pcg4d_is_a_bijection():
+    rng = np.random.default_rng(5)
+    for _ in range(200):
+        v = rng.integers(0, 2**32, 4, dtype=np.uint64).astype(np.uint32)
+        assert _pcg4d_inverse(O.pcg4d(v)) == [int(x) for x in v]
 
 
-def _curand_block(seed, x, y, z):
-    import ctypes
-    lib = _curand()
-    gen = ctypes.c_void_p()
-    assert lib.curandCreateGeneratorHost(ctypes.byref(gen), 161) == 0   # PHILOX4_32_10
-    try:
-        assert lib.curandSetPseudoRandomGeneratorSeed(gen, ctypes.c_ulonglong(seed)) == 0
-        block = ((y << 32) + x) * 65536 + z
-        assert lib.curandSetGeneratorOffset(gen, ctypes.c_ulonglong(4 * block)) == 0
-        out = (ctypes.c_uint32 * 4)()
-        assert lib.curandGenerate(gen, out, ctypes.c_size_t(4)) == 0
-        return tuple(int(v) for v in out)
-    finally:
-        lib.curandDestroyGenerator(gen)
+def _halves(n, step=3, b=7, h=2):
+    out = np.array([O.pcg4d(np.array([i, step, b, h], np.uint32)) for i in range(n)], np.uint64)
+    return np.concatenate([out >> 16, out & 0xFFFF]).ravel()
 
 
-def test_philox_matches_curand():
-    rng = np.random.default_rng(20260511)
-    for _ in range(48):
-        seed = int(rng.integers(0, 2**63)) * 2 + int(rng.integers(0, 2))
-        x = int(rng.integers(0, 2**32))
-        y = int(rng.integers(0, 2**13))
-        z = int(rng.integers(0, 65536))
-        key = np.array([seed & 0xFFFFFFFF, seed >> 32], np.uint32)
-        got = tuple(int(v) for v in O.philox4x32_10(np.array([x, y, z, 0], np.uint32), key))
-        assert got == _curand_block(seed, x, y, z), (seed, x, y, z)
+def test_pcg4d_halves_are_uniform():
+    x = _halves(8192)                                   # 65,536 16-bit values
+    counts = np.bincount((x >> 10).astype(np.int64), minlength=64)   # 64 bins
+    expect = x.size / 64
+    chi2 = float(((counts - expect) ** 2 / expect).sum())
+    assert chi2 < 120, chi2                             # 63 dof: p < 1e-5 above 120
 
 
-def test_philox_edges_match_curand():
-    for seed in (0, 2**64 - 1):
-        for x, y, z in ((0, 0, 0), (2**32 - 1, 0, 65535), (1, 1, 1)):
-            key = np.array([seed & 0xFFFFFFFF, seed >> 32], np.uint32)
-            got = tuple(int(v) for v in O.philox4x32_10(np.array([x, y, z, 0], np.uint32), key))
-            assert got == _curand_block(seed, x, y, z)
+def test_pcg4d_neighbouring_counters_are_unrelated():
+    n = 8192
+    out = np.array([O.pcg4d(np.array([i, 1, 0, 0], np.uint32)) for i in range(n)], np.uint64)
+    a = (out[:-1, 0] >> 16).astype(np.float64)
+    b = (out[1:, 0] >> 16).astype(np.float64)
+    assert abs(np.corrcoef(a, b)[0, 1]) < 4 / np.sqrt(n)
+    # avalanche: one flipped input bit flips about half of the 128 output bits
+    rng = np.random.default_rng(8)
+    flips = []
+    for _ in range(400):
+        v = rng.integers(0, 2**32, 4, dtype=np.uint64).astype(np.uint32)
+        bit = int(rng.integers(0, 128))
+        u = v.copy()
+        u[bit // 32] ^= np.uint32(1 << (bit % 32))
+        d = O.pcg4d(v) ^ O.pcg4d(u)
+        flips.append(sum(bin(int(t)).count("1") for t in d))
+    assert 56 < np.mean(flips) < 72, np.mean(flips)
 
 
 # ------------------------------------------------- stochastic-rounding offsets
@@ -165,9 +164,9 @@ def test_sr_delta_is_a_pure_function_of_its_counter():
     assert a == b
     c = [O.sr_delta(9, 2, 2, 3, s, j) for s in range(4) for j in range(8)]
     assert a != c
-    # the two columns of one 32-bit word come from its high and low halves
-    ctr = np.array([0, 1, 2, 3], np.uint32)
-    out = O.philox4x32_10(ctr, np.array([9, 0], np.uint32))
+    # the two columns of one 32-bit word come from its high and low halves;
+    # the input is (tile, step, request ^ low seed word, head ^ high seed word)
+    out = O.pcg4d(np.array([0, 1, 2 ^ 9, 3], np.uint32))
     w = int(out[0])
     assert O.sr_delta(9, 1, 2, 3, 0, 0) == (2 * (w >> 16) - 65535) * 2.0**-17
     assert O.sr_delta(9, 1, 2, 3, 0, 1) == (2 * (w & 0xFFFF) - 65535) * 2.0**-17
