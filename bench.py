@@ -428,6 +428,18 @@ def run_window(w, window, steps, warmup, rank, world):
     return {"ms": ms, "steps": steps, "per_t_ms": per_t}
 
 
+def tf32_peak():
+    """Dense tf32 tensor-core peak: the measured bf16 GEMM rate (burst) x the
+    nominal tf32 / bf16 ratio (1.1 / 2.25 PFLOP/s dense)."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            bf16 = float(json.load(fh)["bf16_tflops"])
+        return bf16 * 1.1 / 2.25, "measured bf16 x nominal tf32/bf16 ratio"
+    except (OSError, KeyError, ValueError):
+        return 1590.0 * 1.1 / 2.25, "fallback bf16 x nominal tf32/bf16 ratio"
+
+
 # FP32 peak of the CUDA cores for the prefill's plain arithmetic: 148 SMs x
 # 128 FP32 lanes x 2 flops per fma x 1.965 GHz (clocks.max.sm).
 FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
@@ -440,9 +452,18 @@ def prefill_flops_per_head_token():
     return 128 * 128 * (1 + 2 + 2 + 2)
 
 
-def run_prefill(w, L, steps, warmup, rank, world):
-    """stq_prefill of an L-token prompt over the whole batch, K times (each
-    from the state the previous left).  Returns the device time (max over ranks)."""
+def chunked_flops_per_head_token():
+    """Tensor-core work per page and token of the chunkwise prefill, counted
+    as the fp32 products it computes (each run as three tf32 MMAs on split
+    operands): per 128-token chunk, K K^T, S^T K^T, (gam Q) K^T, S^T (gam Q)^T,
+    E^T P~^T and E^T K~, six 128 x 128 x 128 products, divided by 128 tokens."""
+    return 6 * 2 * 128 * 128 * 128 // 128
+
+
+def run_prefill(w, L, steps, warmup, rank, world, chunked=False):
+    """stq_prefill (or, chunked, stq_prefill_chunked) of an L-token prompt over
+    the whole batch, K times (each from the state the previous left).  Returns
+    the device time (max over ranks)."""
     from linear_attention_recurrent_delta_b200 import binding as B
     dev = torch.device("cuda", torch.cuda.current_device())
     wr = R.rank_workload(w, rank)
@@ -450,21 +471,26 @@ def run_prefill(w, L, steps, warmup, rank, world):
     S = W.initial_state(wr, device=dev)
     qs.calibrate_and_quantize(S)
     del S
-    xs = [W.step_inputs(wr, l, device=dev) for l in range(L)]
-    x = {k: torch.stack([xi[k] for xi in xs]).contiguous() for k in xs[0]}
-    del xs
+    x = None
+    for l in range(L):   # [L][B][H][...] filled token by token (no second copy)
+        xl = W.step_inputs(wr, l, device=dev)
+        if x is None:
+            x = {k: torch.empty((L,) + tuple(v.shape), dtype=v.dtype, device=dev) for k, v in xl.items()}
+        for k in xl:
+            x[k][l].copy_(xl[k])
     o = torch.empty(L, wr.batch, wr.heads, 128, device=dev)
     seed = W.sr_seed(wr)
     stream = torch.cuda.current_stream()
+    fn = B.stq_prefill_chunked if chunked else B.stq_prefill
     for i in range(max(warmup, 3)):
-        B.stq_prefill(qs.state, x["q"], x["k"], x["v"], x["alpha"], x["beta"], o, None, seed, i, stream)
+        fn(qs.state, x["q"], x["k"], x["v"], x["alpha"], x["beta"], o, None, seed, i, stream)
     torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev0.record(stream)
     for i in range(steps):
-        B.stq_prefill(qs.state, x["q"], x["k"], x["v"], x["alpha"], x["beta"], o, None, seed, 100 + i, stream)
+        fn(qs.state, x["q"], x["k"], x["v"], x["alpha"], x["beta"], o, None, seed, 100 + i, stream)
     ev1.record(stream)
     torch.cuda.synchronize()
     status = B.stq_device_status(qs.state)
@@ -625,6 +651,8 @@ def main():
                     help="with --profile: per-window steps (stq_window_step) of this window length")
     ap.add_argument("--prefill", type=int, default=0,
                     help="with --profile: stq_prefill of a prompt of this many tokens")
+    ap.add_argument("--chunked", action="store_true",
+                    help="with --profile --prefill: the chunkwise tensor-core form (stq_prefill_chunked)")
     ap.add_argument("--profile", action="store_true",
                     help="decode steps only: no clock sampling, e2e, CPU baseline or other workloads")
     args = ap.parse_args()
@@ -674,10 +702,10 @@ def main():
         build_mod.build()
     barrier(world)
     if args.profile and args.prefill:
-        r = run_prefill(w, args.prefill, args.steps, args.warmup, rank, world)
+        r = run_prefill(w, args.prefill, args.steps, args.warmup, rank, world, chunked=args.chunked)
         if rank == 0:
             print(json.dumps({"workload": w.name, "batch": w.batch, "prompt": args.prefill,
-                              "ms_per_prefill": r["ms"] / r["steps"]}))
+                              "chunked": args.chunked, "ms_per_prefill": r["ms"] / r["steps"]}))
         R.finish(world)
         return
     if args.profile and args.window:
@@ -731,6 +759,27 @@ def main():
                                                "peak": FP32_PEAK_TFLOPS, "unit": "TFLOP/s",
                                                "frac": rate * fl / 1e12 / FP32_PEAK_TFLOPS,
                                                "flops_per_head_token": fl}}
+        # the chunkwise tensor-core form against the recurrent one: the
+        # headline batch with a 512-token prompt, and one request x 32 heads
+        # with a 1,024-token prompt (32 pages: few CTAs for the recurrent form)
+        if not spec["gate_vector"]:
+            tf = chunked_flops_per_head_token()
+            tc_peak = tf32_peak()
+            for tag, wl, L, n in (("batch256_L512", w.resized(batch=min(w.batch, 256)), 512, 3),
+                                  ("one_request_L1024", w.resized(batch=1), 1024, 5)):
+                rr = run_prefill(wl, L, n, 2, rank, world)
+                rc = run_prefill(wl, L, n, 2, rank, world, chunked=True)
+                rate_r = R.aggregate_rate(wl.pages * L, world, rr["steps"], rr["ms"])
+                rate_c = R.aggregate_rate(wl.pages * L, world, rc["steps"], rc["ms"])
+                prefill["chunked_" + tag] = {
+                    "value": rate_c, "unit": "head-tokens/s", "prompt": L, "pages": wl.pages,
+                    "entry_point": "stq_prefill_chunked", "kernel": "stq::prefill_tc_kernel",
+                    "ms_per_prefill": rc["ms"] / rc["steps"],
+                    "recurrent_value": rate_r, "speedup_vs_recurrent": rate_c / rate_r,
+                    "roofline": {"bound": "tensor", "achieved": rate_c * tf / 1e12, "peak": tc_peak[0],
+                                 "unit": "TFLOP/s", "frac": rate_c * tf / 1e12 / tc_peak[0],
+                                 "peak_kind": tc_peak[1], "flops_per_head_token": tf,
+                                 "note": "fp32 products counted once; each runs as three tf32 MMAs"}}
 
     lifetime = run_lifetime() if not args.only else None
 

@@ -64,6 +64,7 @@ def lib():
         "stq_window_step": (c_int, [P, P, c_size_t, c_int, c_int, c_int, P, P, P, P, P, P, c_uint64, c_uint32, P]),
         "stq_lifetime_weights": (c_int, [P, P, c_int, P, P]),
         "stq_prefill": (c_int, [P, c_int, P, P, P, P, P, P, P, c_uint64, c_uint32, P]),
+        "stq_prefill_chunked": (c_int, [P, c_int, P, P, P, P, P, P, P, c_uint64, c_uint32, P]),
         "stq_decode_io_bytes": (c_size_t, [P]),
         "stq_decode_step_host": (c_int, [P, P, P, P, P, P, P, P, c_size_t, c_uint64, c_uint32, P]),
         "stq_decode_steps_host": (c_int, [P, c_int, P, P, P, P, P, P, P, c_size_t, c_uint64, c_uint32, P]),
@@ -226,6 +227,13 @@ def stq_prefill(state, q, k, v, alpha, beta, o, S_out=None, seed=0, step=0, stre
     """A prompt of L = q.shape[0] tokens through every page (q, k, v, o: [L, B, H, 128])."""
     _check(lib().stq_prefill(state.handle, int(q.shape[0]), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),
                              _ptr(o), _ptr(S_out), int(seed), int(step), _stream(stream)), "stq_prefill")
+
+
+def stq_prefill_chunked(state, q, k, v, alpha, beta, o, S_out=None, seed=0, step=0, stream=None):
+    """The same prompt in chunkwise form on the tensor cores (scalar-gate formats)."""
+    _check(lib().stq_prefill_chunked(state.handle, int(q.shape[0]), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
+                                     _ptr(beta), _ptr(o), _ptr(S_out), int(seed), int(step), _stream(stream)),
+           "stq_prefill_chunked")
 
 
 def stq_decode_io_bytes(state):

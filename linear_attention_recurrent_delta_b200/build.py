@@ -13,8 +13,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB = os.path.join(HERE, "libstq.so")
-SOURCES = ["stq_api.cu", "stq_decode.cu", "stq_quant.cu", "stq_window.cu", "stq_prefill.cu", "stq_lifetime.cu", "stq_fit.cu"]
-HEADERS = ["stq_device.cuh", "stq_internal.h", "stq_slices.cuh", "stq_rows.cuh", "stq_lifetime.h"]
+SOURCES = ["stq_api.cu", "stq_decode.cu", "stq_quant.cu", "stq_window.cu", "stq_prefill.cu", "stq_lifetime.cu", "stq_fit.cu", "stq_prefill_tc.cu"]
+HEADERS = ["stq_device.cuh", "stq_internal.h", "stq_slices.cuh", "stq_rows.cuh", "stq_lifetime.h", "stq_tc.cuh"]
 
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "--fmad=false",
               "-std=c++17", "-Xcompiler", "-fPIC,-O2", "-shared"]

@@ -47,6 +47,10 @@ cudaError_t launch_window(const stq_state *s, uint8_t *buf, int window, int t, b
 cudaError_t launch_prefill(const stq_state *s, int L, const float *q, const float *k, const float *v,
                            const float *alpha, const float *beta, float *o, float *S_out, uint64_t seed,
                            uint32_t step, int stall_first_wait, bool early_launch, cudaStream_t stream);
+// Prefill in chunkwise form on the tensor cores (scalar-gate formats).
+cudaError_t launch_prefill_tc(const stq_state *s, int L, const float *q, const float *k, const float *v,
+                              const float *alpha, const float *beta, float *o, float *S_out, uint64_t seed,
+                              uint32_t step, int stall_first_wait, cudaStream_t stream);
 cudaError_t launch_calibrate(const stq_state *s, const float *S, const float *row_weight,
                              double *workspace, cudaStream_t stream);
 // The checks every calibration entry point makes of its fp32 state and row

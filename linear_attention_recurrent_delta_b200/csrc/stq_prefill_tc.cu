@@ -1,0 +1,473 @@
+// stq_prefill_tc.cu -- the chunkwise prefill on the fifth-generation tensor
+// cores (sm_100a, tcgen05): a prompt of L tokens through every page of a
+// GDN (scalar-gate) state, 128 tokens per chunk, one requantization after
+// the last token.
+//
+// Per chunk of n <= 128 tokens from the state S0 (T = S / c units, key rows
+// in natural order), with gam_i = prod of the gates of tokens 0..i of the
+// chunk (the UT-transform form of the delta rule, "repeated prefill": DASC):
+//   G  = K K^T,  A_ij = beta_i (gam_i / gam_j) G_ij  (j < i)
+//   E  = (I + A)^-1 R,  R_i = beta_i (v_i / c - gam_i (S0^T k_i))
+//   o_i = c (gam_i S0^T q_i + sum_{j<=i} (gam_i / gam_j) (q_i . k_j) E_j)
+//   S  <- gam_n S0 + sum_j (gam_n / gam_j) k_j E_j^T
+// The products run on the tensor cores in tf32 with each fp32 operand split
+// into a tf32 part and its remainder (three MMAs per product: hi hi, hi lo,
+// lo hi), which keeps fp32-level accuracy; the triangular solve runs on the
+// CUDA cores (thread v owns value column v of E).
+//
+// One CTA of 128 threads per page (persistent over pages; its 168 KB of
+// shared memory and all 512 tensor-memory columns keep it alone on its SM).
+// Thread t owns row t of whatever a phase computes: token t, value column
+// t, or key channel t, which is also tensor-memory lane t.
+//   shared memory: six 16 KB operand tiles (128 rows x 32 fp32, 128-byte
+//   swizzled, K-major), reused as the solve's matrix A and as the page
+//   buffer; the state X = S^T (X[v][kappa], fp32, rows padded to 129
+//   floats); per-token scalars.
+//   tensor memory: G | Y^T = S0^T K^T | P' = (gam Q) K^T | O^T, then the
+//   state's increment in G's columns.
+#include "stq_rows.cuh"
+#include "stq_tc.cuh"
+
+namespace stq {
+
+constexpr int kChunk = 128;                    // tokens per chunk
+constexpr int kXStride = kD + 1;               // floats per state row
+constexpr int kAStride = kChunk + 4;           // floats per row of the solve's matrix (16-byte rows)
+constexpr uint32_t kTiles = 6;
+constexpr uint32_t kTileRegion = kTiles * tc::kTileBytes;
+
+struct TcArgs {
+    uint8_t *pages;
+    const uint8_t *perm;
+    uint32_t *status;
+    const float *q, *k, *v, *alpha, *beta;
+    float *o, *S_out;
+    int L, n_pages, heads;
+    uint32_t store_bytes;
+    uint32_t seed_lo, seed_hi, step;
+    uint64_t wait_limit_ns;
+    int stall_first_wait;
+};
+
+struct TcSmall {
+    float gam[kChunk];       // cumulative gate of the chunk's tokens
+    float igam[kChunk];      // 1 / gam
+    float bet[kChunk];       // beta (0 for padding)
+    float kts[kChunk];       // gam_n / gam_j: a key's decay to the chunk's end
+    float c[kD], ic[kD];     // column scale and its inverse
+    float inv[kWarps][kRowsPerWarp];
+    int kap[kD];             // stored row -> key channel
+    uint64_t mma_bar, page_bar, never;
+    uint32_t tmem;
+};
+
+constexpr size_t kTcSmem = kTileRegion + (size_t)kD * kXStride * 4 + sizeof(TcSmall) + 1024;
+
+__device__ __forceinline__ void put_split(uint8_t *hi_tile, uint8_t *lo_tile, uint32_t row, uint32_t k, float x) {
+    float h, l;
+    tc::split_tf32(x, h, l);
+    const uint32_t off = tc::sw128_offset(row, k);
+    *reinterpret_cast<float *>(hi_tile + off) = h;
+    *reinterpret_cast<float *>(lo_tile + off) = l;
+}
+
+// D (+)= A B^T over one 32-wide K slab, split operands: hi hi, hi lo, lo hi
+__device__ __forceinline__ void mma_split(uint32_t d, uint32_t a_hi, uint32_t a_lo, uint32_t b_hi, uint32_t b_lo,
+                                          bool accumulate) {
+    const uint32_t idesc = tc::idesc_tf32(128, 128);
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+        const uint32_t off = 32u * kk;
+        tc::mma_tf32(d, tc::desc_k_sw128(a_hi + off), tc::desc_k_sw128(b_hi + off), idesc, accumulate || kk > 0);
+        tc::mma_tf32(d, tc::desc_k_sw128(a_hi + off), tc::desc_k_sw128(b_lo + off), idesc, true);
+        tc::mma_tf32(d, tc::desc_k_sw128(a_lo + off), tc::desc_k_sw128(b_hi + off), idesc, true);
+    }
+}
+
+// 128 columns of this thread's tensor-memory lane, 32 at a time
+template <class Fn>
+__device__ __forceinline__ void tmem_row(uint32_t taddr_lane, Fn &&fn) {
+#pragma unroll
+    for (int c = 0; c < kChunk; c += 32) {
+        float x[32];
+        tc::ld32(taddr_lane + (uint32_t)c, x);
+        fn(c, x);
+    }
+}
+
+template <class FMT>
+__global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const DevFormat F, const TcArgs A) {
+    extern __shared__ uint8_t tc_smem_raw[];
+    const uint32_t raw = smem_u32(tc_smem_raw);
+    uint8_t *base = tc_smem_raw + (((raw + 1023u) & ~1023u) - raw);
+    uint8_t *tiles = base;                                            // six operand tiles / A / page buffer
+    float *XS = reinterpret_cast<float *>(base + kTileRegion);       // X[v][kappa]
+    TcSmall &M = *reinterpret_cast<TcSmall *>(base + kTileRegion + (size_t)kD * kXStride * 4);
+    float *Amat = reinterpret_cast<float *>(tiles);
+    const uint32_t t_base = smem_u32(tiles);
+    auto tile = [&](int i) { return tiles + i * tc::kTileBytes; };
+    auto tile_addr = [&](int i) { return t_base + (uint32_t)i * tc::kTileBytes; };
+
+    constexpr bool SR = FMT::kSr;
+    bool col_scales, gate_vector;
+    format_flags<FMT>(F, col_scales, gate_vector);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const RowCtx R = row_ctx<FMT>(F, warp, lane);
+
+    if (tid == 0) {
+        mbar_init(&M.mma_bar, 1);
+        mbar_init(&M.page_bar, 1);
+        mbar_init(&M.never, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tc::tmem_alloc(&M.tmem, 512);
+        tc::tmem_relinquish();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = M.tmem;
+    const uint32_t lane_addr = tmem + ((uint32_t)(32 * warp) << 16);   // this thread's lane, column 0
+    const uint32_t RG = 0, RY = 128, RP = 256, RO = 384;               // column regions
+
+    const int n = A.n_pages, H = A.heads;
+    uint32_t mma_phase = 0, page_phase = 0;
+    bool failed = false;
+    int pending_mma = -1, pending_page = -1;      // a phase this thread gave up on (exit path waits again)
+
+    auto wait_mma = [&]() {
+        const uint32_t ph = mma_phase;
+        mma_phase ^= 1u;
+        const bool ok = mbar_wait_bounded(&M.mma_bar, ph, A.wait_limit_ns);
+        if (!ok) pending_mma = (int)ph;
+        tc::fence_after_sync();
+        return ok;
+    };
+
+    for (int p = blockIdx.x; p < n; p += gridDim.x) {
+        const int ph = p % H, pb = p / H;
+        // ---- the page: bulk copy into the tile region, dequantize into X
+        if (tid == 0) {
+            mbar_expect_tx(&M.page_bar, (uint32_t)F.page_bytes);
+            bulk_g2s(tiles, A.pages + (size_t)p * F.page_bytes, (uint32_t)F.page_bytes, &M.page_bar);
+        }
+        M.kap[tid] = A.perm[(size_t)ph * kD + tid] & (kD - 1);
+        bool ok;
+        const uint32_t pp = page_phase;
+        page_phase ^= 1u;
+        if (A.stall_first_wait && p == (int)blockIdx.x) ok = mbar_wait_bounded(&M.never, 0, A.wait_limit_ns);
+        else ok = mbar_wait_bounded(&M.page_bar, pp, A.wait_limit_ns);
+        if (!ok) pending_page = (int)pp;
+        {
+            const float c = col_scales ? reinterpret_cast<const float *>(tiles + F.c_off)[tid] : 1.f;
+            M.c[tid] = c;
+            M.ic[tid] = col_scales ? __frcp_rn(c) : 1.f;
+        }
+        if (__syncthreads_or(!ok)) { failed = true; break; }
+        {
+            // warp w dequantizes slice w (rows 16 b + 4 w + i) of every block:
+            // T = z r (FP16 rows: h), written to X[v][kappa]
+            const float *r_s = reinterpret_cast<const float *>(tiles + F.r_off);
+            static_for<0, kBlocks>([&](auto bc) {
+                constexpr int b = decltype(bc)::value;
+                float av[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int s = 16 * b + 4 * warp + i;
+                    const int blk_r = (R.all_int || F.blk_kind(b) == kKindInt) ? F.blk_rbase(b) + 4 * warp + i : -1;
+                    av[i] = blk_r >= 0 ? r_s[blk_r] : 1.f;
+                    (void)s;
+                }
+                Tile T;
+                const uint8_t *blk = tiles + fmt_offset<FMT, b>(F);
+                with_width<FMT, b>(F, [&](auto wc) {
+                    constexpr int W = decltype(wc)::value;
+                    dequant_slice<W, b>(blk, warp, lane, make_float4(av[0], av[1], av[2], av[3]), T);
+                });
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int kap = M.kap[16 * b + 4 * warp + i];
+                    XS[(4 * lane + 0) * kXStride + kap] = T[b][i][0].x;
+                    XS[(4 * lane + 1) * kXStride + kap] = T[b][i][0].y;
+                    XS[(4 * lane + 2) * kXStride + kap] = T[b][i][1].x;
+                    XS[(4 * lane + 3) * kXStride + kap] = T[b][i][1].y;
+                }
+            });
+        }
+        __syncthreads();
+
+        for (int t0 = 0; t0 < A.L && !failed; t0 += kChunk) {
+            const int cn = min(kChunk, A.L - t0);
+            // ---- per-token scalars of the chunk
+            {
+                const bool real = tid < cn;
+                const size_t row = (size_t)(t0 + tid) * n + p;
+                M.bet[tid] = real ? A.beta[row] : 0.f;
+                M.gam[tid] = real ? A.alpha[row] : 1.f;    // the gate; made cumulative below
+            }
+            __syncthreads();
+            if (tid == 0) {
+                float g = 1.f;
+                for (int i = 0; i < kChunk; ++i) {
+                    g = __fmul_rn(g, M.gam[i]);
+                    M.gam[i] = g;
+                }
+            }
+            __syncthreads();
+            {
+                const float gi = M.gam[tid];
+                M.igam[tid] = __frcp_rn(gi);
+                M.kts[tid] = __fdiv_rn(M.gam[kChunk - 1], gi);
+            }
+            __syncthreads();
+
+            // ---- phase A: G = K K^T, Y^T = X K^T, P' = (gam Q) K^T, O^T = X (gam Q)^T
+            for (int ks = 0; ks < kD / 32; ++ks) {
+                {
+                    const bool real = tid < cn;
+                    const size_t row = ((size_t)(t0 + tid) * n + p) * kD + 32 * ks;
+                    const float gi = M.gam[tid];
+#pragma unroll
+                    for (int j4 = 0; j4 < 8; ++j4) {
+                        float4 kx = make_float4(0.f, 0.f, 0.f, 0.f), qx = kx;
+                        if (real) {
+                            kx = __ldg(reinterpret_cast<const float4 *>(A.k + row) + j4);
+                            qx = __ldg(reinterpret_cast<const float4 *>(A.q + row) + j4);
+                        }
+                        const float kv[4] = {kx.x, kx.y, kx.z, kx.w}, qv[4] = {qx.x, qx.y, qx.z, qx.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            put_split(tile(0), tile(1), tid, 4 * j4 + e, kv[e]);
+                            put_split(tile(2), tile(3), tid, 4 * j4 + e, __fmul_rn(gi, qv[e]));
+                        }
+                    }
+                    const float *xr = XS + tid * kXStride + 32 * ks;
+#pragma unroll 8
+                    for (int j = 0; j < 32; ++j) put_split(tile(4), tile(5), tid, j, xr[j]);
+                }
+                fence_proxy_async_smem();
+                tc::fence_before_sync();
+                __syncthreads();
+                tc::fence_after_sync();
+                if (tid == 0) {
+                    const bool acc = ks > 0;
+                    mma_split(tmem + RG, tile_addr(0), tile_addr(1), tile_addr(0), tile_addr(1), acc);
+                    mma_split(tmem + RY, tile_addr(4), tile_addr(5), tile_addr(0), tile_addr(1), acc);
+                    mma_split(tmem + RP, tile_addr(2), tile_addr(3), tile_addr(0), tile_addr(1), acc);
+                    mma_split(tmem + RO, tile_addr(4), tile_addr(5), tile_addr(2), tile_addr(3), acc);
+                    tc::commit(&M.mma_bar);
+                }
+                if (__syncthreads_or(!wait_mma())) { failed = true; break; }
+            }
+            if (failed) break;
+
+            // ---- phase B: A from G (thread i: token i), R from Y^T (thread v), the solve
+            {
+                const float bi = M.bet[tid], gi = M.gam[tid];
+                float *arow = Amat + tid * kAStride;
+                tmem_row(lane_addr + RG, [&](int c0, const float (&x)[32]) {
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj) {
+                        const int j = c0 + jj;
+                        const float a = __fmul_rn(bi, __fmul_rn(__fmul_rn(gi, M.igam[j]), x[jj]));
+                        arow[j] = j < tid ? a : 0.f;
+                    }
+                });
+            }
+            float e[kChunk];
+            {
+                const float icv = M.ic[tid];
+                tmem_row(lane_addr + RY, [&](int c0, const float (&x)[32]) {
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj) {
+                        const int i = c0 + jj;
+                        const float vv = (i < cn) ? __ldg(A.v + ((size_t)(t0 + i) * n + p) * kD + tid) : 0.f;
+                        // R_i = beta_i (v_i / c - gam_i y_i)
+                        e[i] = __fmul_rn(M.bet[i], __fsub_rn(__fmul_rn(vv, icv), __fmul_rn(M.gam[i], x[jj])));
+                    }
+                });
+            }
+            __syncthreads();
+            // forward substitution: E_i = R_i - sum_{j<i} A_ij E_j (thread v: column v)
+#pragma unroll
+            for (int i = 1; i < kChunk; ++i) {
+                const float *arow = Amat + i * kAStride;
+                float acc = e[i];
+#pragma unroll
+                for (int j4 = 0; j4 < (i + 3) / 4; ++j4) {
+                    const float4 a4 = *reinterpret_cast<const float4 *>(arow + 4 * j4);
+                    const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj)
+                        if (4 * j4 + jj < i) acc = __fmaf_rn(-av[jj], e[4 * j4 + jj], acc);
+                }
+                e[i] = acc;
+            }
+            __syncthreads();   // the matrix A's space becomes operand tiles again
+
+            // ---- phase C: O^T += E^T P~^T, dX = E^T K~ (K = tokens)
+            for (int js = 0; js < kChunk / 32; ++js) {
+                {
+                    // E^T row v (thread v)
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj) put_split(tile(0), tile(1), tid, jj, e[32 * js + jj]);
+                    // P~ row i (thread i): P'_ij / gam_j for j <= i, else 0
+                    float x[32];
+                    tc::ld32(lane_addr + RP + 32 * js, x);
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj) {
+                        const int j = 32 * js + jj;
+                        put_split(tile(2), tile(3), tid, jj, j <= tid ? __fmul_rn(x[jj], M.igam[j]) : 0.f);
+                    }
+                    // K~^T row kappa (thread kappa): k_j[kappa] gam_n / gam_j
+#pragma unroll 8
+                    for (int jj = 0; jj < 32; ++jj) {
+                        const int j = 32 * js + jj;
+                        const float kk = (j < cn) ? __ldg(A.k + ((size_t)(t0 + j) * n + p) * kD + tid) : 0.f;
+                        put_split(tile(4), tile(5), tid, jj, __fmul_rn(kk, M.kts[j]));
+                    }
+                }
+                fence_proxy_async_smem();
+                tc::fence_before_sync();
+                __syncthreads();
+                tc::fence_after_sync();
+                if (tid == 0) {
+                    mma_split(tmem + RO, tile_addr(0), tile_addr(1), tile_addr(2), tile_addr(3), true);
+                    mma_split(tmem + RG, tile_addr(0), tile_addr(1), tile_addr(4), tile_addr(5), js > 0);
+                    tc::commit(&M.mma_bar);
+                }
+                if (__syncthreads_or(!wait_mma())) { failed = true; break; }
+            }
+            if (failed) break;
+
+            // ---- phase D: o of the chunk's tokens; X <- gam_n X + dX
+            {
+                const float cv = M.c[tid];
+                tmem_row(lane_addr + RO, [&](int c0, const float (&x)[32]) {
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj) {
+                        const int i = c0 + jj;
+                        if (i < cn) A.o[((size_t)(t0 + i) * n + p) * kD + tid] = __fmul_rn(cv, x[jj]);
+                    }
+                });
+                const float gn = M.gam[kChunk - 1];
+                float *xr = XS + tid * kXStride;
+                tmem_row(lane_addr + RG, [&](int c0, const float (&x)[32]) {
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj) xr[c0 + jj] = __fmaf_rn(gn, xr[c0 + jj], x[jj]);
+                });
+            }
+            tc::fence_before_sync();
+            __syncthreads();
+            tc::fence_after_sync();
+        }
+        if (failed) break;
+
+        // ---- the page's end: the state (optional), one requantization, the store
+        if (A.S_out) {
+            const float cv = M.c[tid];
+            const float *xr = XS + tid * kXStride;
+            for (int kap = 0; kap < kD; ++kap)
+                A.S_out[((size_t)p * kD + kap) * kD + tid] = __fmul_rn(xr[kap], cv);
+        }
+        // the page buffer starts from zero (the 1-bit plane's words are
+        // updated by xor of each slice's bits)
+        for (int i = tid; i < (int)(F.page_bytes / 16); i += kThreads)
+            reinterpret_cast<uint4 *>(tiles)[i] = make_uint4(0u, 0u, 0u, 0u);
+        Tile T;
+        static_for<0, kBlocks>([&](auto bc) {
+            constexpr int b = decltype(bc)::value;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int kap = M.kap[16 * b + 4 * warp + i];
+                T[b][i][0] = make_float2(XS[(4 * lane + 0) * kXStride + kap], XS[(4 * lane + 1) * kXStride + kap]);
+                T[b][i][1] = make_float2(XS[(4 * lane + 2) * kXStride + kap], XS[(4 * lane + 3) * kXStride + kap]);
+                M.inv[warp][4 * b + i] = warp_absmax(absmax4(T[b][i][0], T[b][i][1]));
+            }
+        });
+        __syncthreads();
+        {
+            float *r_s = reinterpret_cast<float *>(tiles + F.r_off);
+            const float m = M.inv[warp][lane];
+            float inv = 0.f;
+            if (R.all_int || R.is_int) {
+                const float r = div_by_qmax(m, R.qmax, R.rcp_qmax);
+                inv = m > 0.f ? div_rz_qmax<false>(R.qmax, m) : 0.f;
+                r_s[R.rix] = r;
+            }
+            M.inv[warp][lane] = inv;
+        }
+        __syncwarp();
+        SrCtx sr;
+        sr.k0 = A.seed_lo; sr.k1 = A.seed_hi; sr.step = A.step;
+        sr.b = (uint32_t)pb;
+        sr.h = (uint32_t)ph;
+        static_for<0, kBlocks>([&](auto bc) {
+            constexpr int b = decltype(bc)::value;
+            const float4 i4 = *reinterpret_cast<const float4 *>(&M.inv[warp][4 * b]);
+            uint8_t *blk = tiles + fmt_offset<FMT, b>(F);
+            with_width<FMT, b>(F, [&](auto wc) {
+                constexpr int W = decltype(wc)::value;
+                requant_slice<W, b, SR>(blk, warp, lane, i4, T, sr);
+            });
+        });
+        fence_proxy_async_smem();
+        __syncthreads();
+        if (tid == 0) {
+            bulk_s2g(A.pages + (size_t)p * F.page_bytes, tiles, A.store_bytes);
+            bulk_commit();
+            bulk_wait<0>();
+        }
+        __syncthreads();
+    }
+    if (failed && tid == 0) {
+        atomicOr(A.status, kStatusTimeout);
+        // the MMAs or the page copy still outstanding get a second bounded
+        // wait before the tensor memory is released and the CTA exits
+        if (pending_mma >= 0) mbar_wait_bounded(&M.mma_bar, (uint32_t)pending_mma, A.wait_limit_ns);
+        if (pending_page >= 0) mbar_wait_bounded(&M.page_bar, (uint32_t)pending_page, A.wait_limit_ns);
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (warp == 0) tc::tmem_dealloc(tmem, 512);
+}
+
+template <class FMT>
+static cudaError_t launch_prefill_tc_with(const DevFormat &F, const TcArgs &A, cudaStream_t stream) {
+    const void *fn = (const void *)prefill_tc_kernel<FMT>;
+    cudaError_t err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTcSmem);
+    if (err != cudaSuccess) return err;
+    const int grid = persistent_grid(fn, kThreads, kTcSmem, A.n_pages);
+    if (grid <= 0) return cudaErrorInvalidConfiguration;
+    prefill_tc_kernel<FMT><<<grid, kThreads, kTcSmem, stream>>>(F, A);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_prefill_tc(const stq_state *s, int L, const float *q, const float *k, const float *v,
+                              const float *alpha, const float *beta, float *o, float *S_out, uint64_t seed,
+                              uint32_t step, int stall_first_wait, cudaStream_t stream) {
+    const DevFormat &F = s->dev;
+    TcArgs A;
+    A.pages = s->base + s->pages_offset;
+    A.perm = s->base + s->perm_offset;
+    A.status = reinterpret_cast<uint32_t *>(s->base + s->status_offset);
+    A.q = q; A.k = k; A.v = v; A.alpha = alpha; A.beta = beta; A.o = o; A.S_out = S_out;
+    A.L = L;
+    A.n_pages = s->batch * s->heads;
+    A.heads = s->heads;
+    A.store_bytes = (uint32_t)(F.col_scales ? F.c_off : F.page_bytes);
+    A.seed_lo = (uint32_t)seed;
+    A.seed_hi = (uint32_t)(seed >> 32);
+    A.step = step;
+    A.wait_limit_ns = s->wait_limit_ns;
+    A.stall_first_wait = stall_first_wait;
+    if (format_is<FmtStepQuant6>(F)) return launch_prefill_tc_with<FmtStepQuant6>(F, A, stream);
+    if (format_is<FmtInt8Row>(F)) return launch_prefill_tc_with<FmtInt8Row>(F, A, stream);
+    if (format_is<FmtDamp>(F)) return launch_prefill_tc_with<FmtDamp>(F, A, stream);
+    if (F.stochastic) return launch_prefill_tc_with<RuntimeFmt<true>>(F, A, stream);
+    return launch_prefill_tc_with<RuntimeFmt<false>>(F, A, stream);
+}
+
+}  // namespace stq

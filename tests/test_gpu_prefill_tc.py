@@ -1,0 +1,179 @@
+"""GPU parity of the chunkwise tensor-core prefill (stq_prefill_chunked).
+
+The kernel resolves the prompt 128 tokens at a time with tf32 tensor-core
+products on split operands and a triangular solve, so it agrees with the
+token recurrence to fp32 rounding, not bit for bit.  The bar, per page:
+  * o of every token and the final fp32 state (the optional state output)
+    within rel-L2 1e-5 of the oracle's chunk algebra in fp64
+    (orc_prefill_chunked_f64, itself pinned against the recurrence), and
+    within 1e-5 of the recurrent GPU prefill run on the same inputs;
+  * the requantized page is the requantization of the kernel's own final
+    state: each row scale is that state's row maximum / qmax (to 2 ulps), each
+    INT code the nearest integer to x = T qmax / m (with the stochastic
+    offset of the oracle's generator for stochastic formats) except within
+    1e-5 of a rounding midpoint, each FP16 row element the binary16 rounding
+    of T except at a near-tie.
+Prompts of 1, 37, 128, 130 and 300 tokens (one chunk, a ragged chunk, two
+and three chunks); the GDN formats; more pages than SMs for the persistent
+grid; the bounded-wait hook.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from linear_attention_recurrent_delta_b200 import binding as B
+from linear_attention_recurrent_delta_b200 import workloads as W
+
+from parity_util import download, make_state, oracle_quantize, rel_l2, upload
+
+pytestmark = pytest.mark.gpu
+
+GDN = ["int8row", "stepquant6", "damp"]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from linear_attention_recurrent_delta_b200 import build
+    build.build()
+    B.lib()
+    assert torch.cuda.is_available()
+
+
+def _setup(name, batch, heads):
+    w = [x for x in W.WORKLOADS if x.fmt == name and x.index > 0][0].resized(batch=batch, heads=heads, steps=2)
+    S = W.initial_state(w).numpy()
+    fmt, perm, pages = oracle_quantize(w, S)
+    qs = make_state(w)
+    upload(qs, perm, pages)
+    return w, fmt, perm, pages, qs
+
+
+def _prompt(w, L, first=0):
+    xs = [W.step_inputs(w, first + l) for l in range(L)]
+    return {k: torch.stack([x[k] for x in xs]).contiguous() for k in xs[0]}
+
+
+def _check_requant(fmt, page, T, seed, step, b, h):
+    """page: the kernel's packed page (unpacked); T: its final state in stored
+    order, column-normalised (double).  Returns the number of codes within
+    the near-tie band (allowed either way)."""
+    ties = 0
+    for s in range(128):
+        kind = O.row_kind(fmt, s)
+        t = T[s]
+        if kind == 1:
+            h16 = O.f16_to_f32(page.code[s].astype(np.uint16)).astype(np.float64)
+            ax = np.abs(t)
+            sp = np.where(ax < 2.0 ** -14, 2.0 ** -24, 2.0 ** (np.floor(np.log2(np.maximum(ax, 2.0 ** -14))) - 10))
+            err = np.abs(h16 - t) / sp
+            assert np.all(err <= 0.5 + 1e-5), (s, err.max())
+            ties += int(np.sum(err > 0.5 - 1e-5))
+            continue
+        qmax = O.row_qmax(fmt, s)
+        m = np.abs(t).max()
+        r = float(page.r[s])
+        assert abs(r - m / qmax) <= 2 * np.spacing(np.float32(m / qmax)), (s, r, m / qmax)
+        if m == 0:
+            assert np.all(page.code[s] == 0)
+            continue
+        x = t * qmax / m
+        if fmt.stochastic:
+            x = x + np.array([O.sr_delta(seed, step, b, h, s, j) for j in range(128)], np.float64)
+        z = page.code[s].astype(np.float64)
+        d = np.abs(z - x)
+        assert np.all(d <= 0.5 + 1e-5), (s, d.max())
+        ties += int(np.sum(d > 0.5 - 1e-5))
+    return ties
+
+
+@pytest.mark.parametrize("L", [1, 37, 128, 130, 300])
+@pytest.mark.parametrize("name", GDN)
+def test_chunked_prefill_matches_the_chunk_algebra(name, L):
+    w, fmt, perm, pages, qs = _setup(name, 3, 5)
+    x = _prompt(w, L)
+    xd = {k: v.cuda() for k, v in x.items()}
+    o = torch.full((L, w.batch, w.heads, 128), float("nan"), device="cuda")
+    S_out = torch.empty(w.batch, w.heads, 128, 128, device="cuda")
+    seed = W.sr_seed(w)
+    B.stq_prefill_chunked(qs.state, xd["q"], xd["k"], xd["v"], xd["alpha"], xd["beta"], o, S_out, seed, 7)
+    assert B.stq_device_status(qs.state) == B.STQ_OK
+    got = download(qs)
+    o_g, S_g = o.cpu().numpy(), S_out.cpu().numpy()
+    # the recurrent GPU prefill on the same inputs
+    qr = make_state(w)
+    upload(qr, perm, pages)
+    o_r = torch.empty_like(o)
+    S_r = torch.empty_like(S_out)
+    B.stq_prefill(qr.state, xd["q"], xd["k"], xd["v"], xd["alpha"], xd["beta"], o_r, S_r, seed, 7)
+    o_r, S_r = o_r.cpu().numpy(), S_r.cpu().numpy()
+    ties, worst_o, worst_s = 0, 0.0, 0.0
+    for i in range(w.pages):
+        b, h = divmod(i, w.heads)
+        page0 = O.unpack_page(fmt, pages[i])
+        o64, S64 = O.prefill_chunked_f64(fmt, page0, perm[h], x["q"][:, b, h].numpy(), x["k"][:, b, h].numpy(),
+                                         x["v"][:, b, h].numpy(), x["alpha"][:, b, h].numpy(),
+                                         x["beta"][:, b, h].numpy(), 128)
+        worst_o = max(worst_o, rel_l2(o_g[:, b, h], o64))
+        worst_s = max(worst_s, rel_l2(S_g[b, h], S64))
+        assert rel_l2(o_g[:, b, h], o64) <= 1e-5, ("o", i, rel_l2(o_g[:, b, h], o64))
+        assert rel_l2(S_g[b, h], S64) <= 1e-5, ("state", i, rel_l2(S_g[b, h], S64))
+        assert rel_l2(o_g[:, b, h], o_r[:, b, h]) <= 1e-5
+        assert rel_l2(S_g[b, h], S_r[b, h]) <= 1e-5
+        pg = O.unpack_page(fmt, got[i])
+        c = page0.c.astype(np.float64) if fmt.col_scales else np.ones(128)
+        T = S_g[b, h].astype(np.float64)[perm[h]] / c           # stored order, column-normalised
+        assert np.array_equal(pg.c.view(np.uint32), page0.c.view(np.uint32))
+        ties += _check_requant(fmt, pg, T, seed, 7, b, h)
+    print("\n%s, L = %d: max o rel-L2 %.2e, max state rel-L2 %.2e, near-tie codes %d"
+          % (name, L, worst_o, worst_s, ties))
+
+
+def test_many_pages_per_cta():
+    """More pages than SMs: every CTA takes several pages in turn."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    w, fmt, perm, pages, qs = _setup("int8row", (sms * 2) // 4 + 3, 4)
+    L = 20
+    x = _prompt(w, L)
+    xd = {k: v.cuda() for k, v in x.items()}
+    o = torch.empty(L, w.batch, w.heads, 128, device="cuda")
+    B.stq_prefill_chunked(qs.state, xd["q"], xd["k"], xd["v"], xd["alpha"], xd["beta"], o, None, 0, 3)
+    assert B.stq_device_status(qs.state) == B.STQ_OK
+    o_g = o.cpu().numpy()
+    for i in (0, w.pages // 2, w.pages - 1):
+        b, h = divmod(i, w.heads)
+        o64, _ = O.prefill_chunked_f64(fmt, O.unpack_page(fmt, pages[i]), perm[h], x["q"][:, b, h].numpy(),
+                                       x["k"][:, b, h].numpy(), x["v"][:, b, h].numpy(),
+                                       x["alpha"][:, b, h].numpy(), x["beta"][:, b, h].numpy(), 128)
+        assert rel_l2(o_g[:, b, h], o64) <= 1e-5
+
+
+def test_vector_gate_formats_are_refused():
+    w, fmt, perm, pages, qs = _setup("stepquant4_kda", 2, 2)
+    x = {k: v.cuda() for k, v in _prompt(w, 3).items()}
+    o = torch.empty(3, 2, 2, 128, device="cuda")
+    st = B.lib().stq_prefill_chunked(qs.state.handle, 3, B._ptr(x["q"]), B._ptr(x["k"]), B._ptr(x["v"]),
+                                     B._ptr(x["alpha"]), B._ptr(x["beta"]), B._ptr(o), None, 0, 0, None)
+    assert st == B.STQ_ERR_UNSUPPORTED
+
+
+def test_bounded_wait_times_out_and_writes_nothing():
+    w, fmt, perm, pages, qs = _setup("stepquant6", 4, 3)
+    L = 40
+    x = _prompt(w, L)
+    xd = {k: v.cuda() for k, v in x.items()}
+    o = torch.full((L, 4, 3, 128), 7.0, device="cuda")
+    B.stq_set_wait_limit(qs.state, 20_000_000, stall_first_wait=True)
+    B.stq_prefill_chunked(qs.state, xd["q"], xd["k"], xd["v"], xd["alpha"], xd["beta"], o, None, 0, 1)
+    assert B.stq_device_status(qs.state, clear=True) == B.STQ_ERR_DEVICE_TIMEOUT
+    assert np.array_equal(download(qs), pages)
+    assert bool((o == 7.0).all())
+    B.stq_set_wait_limit(qs.state, 0, stall_first_wait=False)
+    B.stq_prefill_chunked(qs.state, xd["q"], xd["k"], xd["v"], xd["alpha"], xd["beta"], o, None, 0, 1)
+    assert B.stq_device_status(qs.state) == B.STQ_OK
+    o_g = o.cpu().numpy()
+    b, h = 1, 2
+    o64, _ = O.prefill_chunked_f64(fmt, O.unpack_page(fmt, pages[b * 3 + h]), perm[h], x["q"][:, b, h].numpy(),
+                                   x["k"][:, b, h].numpy(), x["v"][:, b, h].numpy(), x["alpha"][:, b, h].numpy(),
+                                   x["beta"][:, b, h].numpy(), 128)
+    assert rel_l2(o_g[:, b, h], o64) <= 1e-5
