@@ -262,58 +262,147 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const DevFormat
             }
             if (failed) break;
 
-            // ---- phase B: A from G (thread i: token i), R from Y^T (thread v), the solve
-            {
-                const float bi = M.bet[tid], gi = M.gam[tid];
-                float *arow = Amat + tid * kAStride;
-                tmem_row(lane_addr + RG, [&](int c0, const float (&x)[32]) {
-#pragma unroll
-                    for (int jj = 0; jj < 32; ++jj) {
-                        const int j = c0 + jj;
-                        const float a = __fmul_rn(bi, __fmul_rn(__fmul_rn(gi, M.igam[j]), x[jj]));
-                        arow[j] = j < tid ? a : 0.f;
-                    }
-                });
-            }
-            float e[kChunk];
+            // ---- phase B: R from Y^T in place (thread v), then the solve
+            // (I + A) E = R in two halves of 64 tokens: each half by forward
+            // substitution with thread v holding column v of the half in
+            // registers; between them the off-diagonal block, R2 -= A21 E1,
+            // as a tensor-core product.  E^T ends up in Y^T's columns.
             {
                 const float icv = M.ic[tid];
-                tmem_row(lane_addr + RY, [&](int c0, const float (&x)[32]) {
+                const uint32_t ry = lane_addr + RY;
+#pragma unroll
+                for (int c0 = 0; c0 < kChunk; c0 += 32) {
+                    float x[32];
+                    tc::ld32(ry + c0, x);
 #pragma unroll
                     for (int jj = 0; jj < 32; ++jj) {
                         const int i = c0 + jj;
                         const float vv = (i < cn) ? __ldg(A.v + ((size_t)(t0 + i) * n + p) * kD + tid) : 0.f;
                         // R_i = beta_i (v_i / c - gam_i y_i)
-                        e[i] = __fmul_rn(M.bet[i], __fsub_rn(__fmul_rn(vv, icv), __fmul_rn(M.gam[i], x[jj])));
+                        x[jj] = __fmul_rn(M.bet[i], __fsub_rn(__fmul_rn(vv, icv), __fmul_rn(M.gam[i], x[jj])));
                     }
-                });
-            }
-            __syncthreads();
-            // forward substitution: E_i = R_i - sum_{j<i} A_ij E_j (thread v: column v)
-#pragma unroll
-            for (int i = 1; i < kChunk; ++i) {
-                const float *arow = Amat + i * kAStride;
-                float acc = e[i];
-#pragma unroll
-                for (int j4 = 0; j4 < (i + 3) / 4; ++j4) {
-                    const float4 a4 = *reinterpret_cast<const float4 *>(arow + 4 * j4);
-                    const float av[4] = {a4.x, a4.y, a4.z, a4.w};
-#pragma unroll
-                    for (int jj = 0; jj < 4; ++jj)
-                        if (4 * j4 + jj < i) acc = __fmaf_rn(-av[jj], e[4 * j4 + jj], acc);
+                    tc::st32(ry + c0, x);
                 }
-                e[i] = acc;
             }
-            __syncthreads();   // the matrix A's space becomes operand tiles again
+            for (int sb = 0; sb < 2; ++sb) {
+                // the diagonal block of this half: A_ij, i, j in [64 sb, 64 sb + 64)
+                if (tid >= 64 * sb && tid < 64 * sb + 64) {
+                    const float bi = M.bet[tid], gi = M.gam[tid];
+                    float *arow = Amat + (tid - 64 * sb) * kAStride;
+#pragma unroll
+                    for (int c0 = 0; c0 < 64; c0 += 32) {
+                        float x[32];
+                        tc::ld32(lane_addr + RG + 64 * sb + c0, x);
+#pragma unroll
+                        for (int jj = 0; jj < 32; ++jj) {
+                            const int j = 64 * sb + c0 + jj;
+                            const float a = __fmul_rn(bi, __fmul_rn(__fmul_rn(gi, M.igam[j]), x[jj]));
+                            arow[c0 + jj] = j < tid ? a : 0.f;
+                        }
+                    }
+                }
+                __syncthreads();
+                float e[64];
+                {
+                    float x[32];
+                    tc::ld32(lane_addr + RY + 64 * sb, x);
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj) e[jj] = x[jj];
+                    tc::ld32(lane_addr + RY + 64 * sb + 32, x);
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj) e[32 + jj] = x[jj];
+                }
+                // forward substitution: E_i = R_i - sum_{j<i} A_ij E_j
+#pragma unroll
+                for (int i = 1; i < 64; ++i) {
+                    const float *arow = Amat + i * kAStride;
+                    float acc = e[i];
+#pragma unroll
+                    for (int j4 = 0; j4 < (i + 3) / 4; ++j4) {
+                        const float4 a4 = *reinterpret_cast<const float4 *>(arow + 4 * j4);
+                        const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+                        for (int jj = 0; jj < 4; ++jj)
+                            if (4 * j4 + jj < i) acc = __fmaf_rn(-av[jj], e[4 * j4 + jj], acc);
+                    }
+                    e[i] = acc;
+                }
+                {
+                    float x[32];
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj) x[jj] = e[jj];
+                    tc::st32(lane_addr + RY + 64 * sb, x);
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj) x[jj] = e[32 + jj];
+                    tc::st32(lane_addr + RY + 64 * sb + 32, x);
+                }
+                if (sb == 1) break;
+                __syncthreads();   // the diagonal block's space becomes operand tiles
+                // R2 -= A21 E1 on the tensor cores: D = R2^T (columns 64..127 of
+                // Y^T) += (-E1^T) A21^T, M = 128 (v), N = 64 (i), K = 64 (j).
+                // Tiles: E1^T hi / lo (rows v, two K slabs) at 0 .. 64 KB; A21
+                // hi / lo (rows i - 64, 64-row tiles of 8 KB) at 64 .. 96 KB.
+#pragma unroll
+                for (int kb = 0; kb < 2; ++kb) {
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj)
+                        put_split(tile(2 * kb), tile(2 * kb + 1), tid, jj, e[32 * kb + jj]);
+                }
+                if (tid >= 64) {
+                    const float bi = M.bet[tid], gi = M.gam[tid];
+                    uint8_t *a21 = tiles + 4 * tc::kTileBytes;
+#pragma unroll
+                    for (int kb = 0; kb < 2; ++kb) {
+                        float x[32];
+                        tc::ld32(lane_addr + RG + 32 * kb, x);
+#pragma unroll
+                        for (int jj = 0; jj < 32; ++jj) {
+                            const int j = 32 * kb + jj;
+                            const float a = __fmul_rn(bi, __fmul_rn(__fmul_rn(gi, M.igam[j]), x[jj]));
+                            put_split(a21 + (2 * kb) * (tc::kTileBytes / 2), a21 + (2 * kb + 1) * (tc::kTileBytes / 2),
+                                      tid - 64, jj, a);
+                        }
+                    }
+                }
+                fence_proxy_async_smem();
+                tc::fence_before_sync();
+                __syncthreads();
+                tc::fence_after_sync();
+                if (tid == 0) {
+                    const uint32_t idesc = tc::idesc_tf32(128, 64, true);
+                    const uint32_t a21 = tile_addr(4);
+#pragma unroll
+                    for (int kb = 0; kb < 2; ++kb) {
+                        const uint32_t e_hi = tile_addr(2 * kb), e_lo = tile_addr(2 * kb + 1);
+                        const uint32_t b_hi = a21 + (2 * kb) * (tc::kTileBytes / 2);
+                        const uint32_t b_lo = a21 + (2 * kb + 1) * (tc::kTileBytes / 2);
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk) {
+                            const uint32_t off = 32u * kk;
+                            tc::mma_tf32(tmem + RY + 64, tc::desc_k_sw128(e_hi + off), tc::desc_k_sw128(b_hi + off),
+                                         idesc, true);
+                            tc::mma_tf32(tmem + RY + 64, tc::desc_k_sw128(e_hi + off), tc::desc_k_sw128(b_lo + off),
+                                         idesc, true);
+                            tc::mma_tf32(tmem + RY + 64, tc::desc_k_sw128(e_lo + off), tc::desc_k_sw128(b_hi + off),
+                                         idesc, true);
+                        }
+                    }
+                    tc::commit(&M.mma_bar);
+                }
+                if (__syncthreads_or(!wait_mma())) { failed = true; break; }
+            }
+            if (failed) break;
+            __syncthreads();   // the solve's space becomes operand tiles again
 
             // ---- phase C: O^T += E^T P~^T, dX = E^T K~ (K = tokens)
             for (int js = 0; js < kChunk / 32; ++js) {
                 {
-                    // E^T row v (thread v)
-#pragma unroll
-                    for (int jj = 0; jj < 32; ++jj) put_split(tile(0), tile(1), tid, jj, e[32 * js + jj]);
-                    // P~ row i (thread i): P'_ij / gam_j for j <= i, else 0
+                    // E^T row v (thread v), from Y^T's columns
                     float x[32];
+                    tc::ld32(lane_addr + RY + 32 * js, x);
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj) put_split(tile(0), tile(1), tid, jj, x[jj]);
+                    // P~ row i (thread i): P'_ij / gam_j for j <= i, else 0
                     tc::ld32(lane_addr + RP + 32 * js, x);
 #pragma unroll
                     for (int jj = 0; jj < 32; ++jj) {
