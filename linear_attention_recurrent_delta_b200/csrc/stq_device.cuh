@@ -268,16 +268,14 @@ __device__ __forceinline__ uint4 sr_hash4(uint4 c, uint32_t k0, uint32_t k1) {
     return make_uint4(x, y, z, w);
 }
 
-// Stochastic-rounding offsets of the two columns held by one 32-bit word:
-// delta = (h16 - 32767.5) / 65536 for the high and the low 16-bit half,
-// built exactly: a byte permute makes the float 2^23 + h16, one f32x2 fma
-// scales it by 2^-16 and removes 128 (exact: h16 / 65536), one f32x2 add
-// subtracts 32767.5 / 65536 (exact: a multiple of 2^-17 below 1/2).
-__device__ __forceinline__ float2 sr_delta_pair(uint32_t word) {
-    const float hi = __int_as_float(__byte_perm(word, 0x4B000000u, 0x7632u));   // 2^23 + high half
-    const float lo = __int_as_float(__byte_perm(word, 0x4B000000u, 0x7610u));   // 2^23 + low half
-    const float2 d = __ffma2_rn(make_float2(hi, lo), make_float2(0x1p-16f, 0x1p-16f), make_float2(-128.f, -128.f));
-    return __fadd2_rn(d, make_float2(-32767.5f / 65536.f, -32767.5f / 65536.f));
+// Stochastic-rounding offsets of the two columns held by one 32-bit word, as
+// the floats 128 + u, u = h16 / 65536 in [0, 1) for the high and the low
+// 16-bit half: a byte permute puts h16 under the exponent of 128.0f (the
+// float 128 (1 + h16 2^-23) = 128 + h16 2^-16, exact).
+__device__ __forceinline__ float2 sr_offset_pair(uint32_t word) {
+    const float hi = __int_as_float(__byte_perm(word, 0x43000000u, 0x7632u));   // 128 + high half / 2^16
+    const float lo = __int_as_float(__byte_perm(word, 0x43000000u, 0x7610u));   // 128 + low half / 2^16
+    return make_float2(hi, lo);
 }
 
 // ------------------------------------------------------- bulk-copy staging --

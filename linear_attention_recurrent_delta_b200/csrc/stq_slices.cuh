@@ -284,6 +284,11 @@ __device__ __forceinline__ void requant_slice(uint8_t *blk, int w, int lane, con
     } else {
         const float M = 12582912.0f + (float)(1 << (W - 1));   // 1.5 * 2^23 + bias
         const float2 M2 = make_float2(M, M);
+        // stochastic rounding: floor(x + u) of the exact x = T inv.  The fma
+        // rounds x + 128 + u down (in [1, 256): |x| <= qmax < 128), which keeps
+        // its floor, and the add of M - 128 rounds down to the integer grid
+        // of [2^23, 2^24): floor(x + u) + M in one rounding each.
+        const float2 Mf2 = make_float2(M - 128.0f, M - 128.0f);
         const float iv[4] = {inv4.x, inv4.y, inv4.z, inv4.w};
         uint32_t ub[4];
 #pragma unroll
@@ -294,10 +299,10 @@ __device__ __forceinline__ void requant_slice(uint8_t *blk, int w, int lane, con
                 const uint32_t s = 16u * B + 4u * (uint32_t)w + (uint32_t)i;   // stored row, even
                 const uint4 h = sr_hash4(make_uint4((s >> 1) * 32u + (uint32_t)lane, sr.step, sr.b, sr.h),
                                               sr.k0, sr.k1);
-                y0 = __fadd2_rn(__ffma2_rn(T[B][i][0], i0, sr_delta_pair(h.x)), M2);
-                y1 = __fadd2_rn(__ffma2_rn(T[B][i][1], i0, sr_delta_pair(h.y)), M2);
-                y2 = __fadd2_rn(__ffma2_rn(T[B][i + 1][0], i1, sr_delta_pair(h.z)), M2);
-                y3 = __fadd2_rn(__ffma2_rn(T[B][i + 1][1], i1, sr_delta_pair(h.w)), M2);
+                y0 = __fadd2_rd(__ffma2_rd(T[B][i][0], i0, sr_offset_pair(h.x)), Mf2);
+                y1 = __fadd2_rd(__ffma2_rd(T[B][i][1], i0, sr_offset_pair(h.y)), Mf2);
+                y2 = __fadd2_rd(__ffma2_rd(T[B][i + 1][0], i1, sr_offset_pair(h.z)), Mf2);
+                y3 = __fadd2_rd(__ffma2_rd(T[B][i + 1][1], i1, sr_offset_pair(h.w)), Mf2);
             } else {
                 y0 = __ffma2_rn(T[B][i][0], i0, M2);
                 y1 = __ffma2_rn(T[B][i][1], i0, M2);

@@ -81,8 +81,8 @@ def lib():
         L.orc_f16_to_f32_n.argtypes = [P, P, c_long]
         L.orc_div_rz_n.argtypes = [P, P, P, c_long]
         L.orc_pcg4d.argtypes = [P, P]
-        L.orc_sr_delta.argtypes = [c_uint64, c_uint32, c_uint32, c_uint32, c_int, c_int, c_int]
-        L.orc_sr_delta.restype = c_float
+        L.orc_sr_offset.argtypes = [c_uint64, c_uint32, c_uint32, c_uint32, c_int, c_int, c_int]
+        L.orc_sr_offset.restype = c_float
     return _lib
 
 
@@ -355,5 +355,5 @@ def pcg4d(v):
     return out
 
 
-def sr_delta(seed, step, b, h, s, j, d_v=128):
-    return lib().orc_sr_delta(int(seed), int(step), int(b), int(h), int(s), int(j), int(d_v))
+def sr_offset(seed, step, b, h, s, j, d_v=128):
+    return lib().orc_sr_offset(int(seed), int(step), int(b), int(h), int(s), int(j), int(d_v))

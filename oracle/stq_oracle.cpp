@@ -250,9 +250,10 @@ extern "C" void orc_pcg4d(const uint32_t in[4], uint32_t out[4])
  * One hash serves a 2-row x 4-column tile: input (tile index, step,
  * request ^ low seed word, head ^ high seed word).  Word 2*(s & 1) +
  * ((j >> 1) & 1) of the output holds columns j & ~1 (high 16 bits) and j | 1
- * (low 16 bits).  delta = (h16 - 32767.5) / 65536, exactly. */
-extern "C" float orc_sr_delta(uint64_t seed, uint32_t step, uint32_t b, uint32_t h,
-                              int s, int j, int d_v)
+ * (low 16 bits).  u = h16 / 65536 in [0, 1), exactly; the rounded code is
+ * floor(x + u), x the exact scaled value. */
+extern "C" float orc_sr_offset(uint64_t seed, uint32_t step, uint32_t b, uint32_t h,
+                               int s, int j, int d_v)
 {
     uint32_t quads = (uint32_t)((d_v + 3) / 4);
     uint32_t in[4] = { (uint32_t)(s >> 1) * quads + (uint32_t)(j >> 2), step,
@@ -261,7 +262,7 @@ extern "C" float orc_sr_delta(uint64_t seed, uint32_t step, uint32_t b, uint32_t
     orc_pcg4d(in, out);
     uint32_t word = out[((s & 1) << 1) | ((j >> 1) & 1)];
     uint32_t h16 = (j & 1) ? (word & 0xFFFFu) : (word >> 16);
-    return (float)(2 * (int)h16 - 65535) * 0x1p-17f;
+    return (float)h16 * 0x1p-16f;
 }
 
 /* ------------------------------------------------------------------------ */
@@ -271,6 +272,11 @@ extern "C" float orc_sr_delta(uint64_t seed, uint32_t step, uint32_t b, uint32_t
 static double dist_to_half(double x)
 {
     return std::fabs(x - (std::floor(x) + 0.5));
+}
+
+static double dist_to_int(double x)
+{
+    return std::fabs(x - std::nearbyint(x));
 }
 
 static double f16_margin(float x)
@@ -327,10 +333,12 @@ static void requant_row(const orc_format *f, int s, const float *Tp, orc_page *p
             zr = std::nearbyint(x);
             if (margin) margin[j] = dist_to_half(x);
         } else {
-            float delta = orc_sr_delta(seed, step, b, h, s, j, d_v);
-            float w = std::fmaf(Tp[j], inv, delta);
-            zr = std::nearbyint((double)w);
-            if (margin) margin[j] = dist_to_half(x + (double)delta);
+            /* floor(x + u) of the exact sum: x >= fl + 1 - u compares two
+             * exact doubles (fl an integer, u on the 2^-16 grid) */
+            double u = (double)orc_sr_offset(seed, step, b, h, s, j, d_v);
+            double fl = std::floor(x);
+            zr = (x >= fl + 1.0 - u) ? fl + 1.0 : fl;
+            if (margin) margin[j] = dist_to_int(x + u);
         }
         if (!(zr == zr)) zr = 0.0;                 /* non-finite input */
         if (zr > qmax) zr = qmax;

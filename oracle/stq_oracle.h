@@ -279,9 +279,10 @@ void orc_f16_to_f32_n(const uint16_t *x, float *out, long n);
 void orc_div_rz_n(const float *a, const float *b, float *out, long n);
 /* pcg4d (Jarzynski and Olano, JCGT 2020), the stochastic-rounding hash */
 void orc_pcg4d(const uint32_t in[4], uint32_t out[4]);
-/* stochastic-rounding offset delta in (-1/2, 1/2) for element (s, j) */
-float orc_sr_delta(uint64_t seed, uint32_t step, uint32_t b, uint32_t h,
-                   int s, int j, int d_v);
+/* stochastic-rounding offset u in [0, 1) (a multiple of 2^-16) for element
+ * (s, j); the code is floor(x + u) */
+float orc_sr_offset(uint64_t seed, uint32_t step, uint32_t b, uint32_t h,
+                    int s, int j, int d_v);
 
 #ifdef __cplusplus
 }

@@ -79,7 +79,8 @@ def _check_requant(fmt, page, T, seed, step, b, h):
             continue
         x = t * qmax / m
         if fmt.stochastic:
-            x = x + np.array([O.sr_delta(seed, step, b, h, s, j) for j in range(128)], np.float64)
+            # floor(x + u) lies within 1/2 of x + u - 1/2
+            x = x + np.array([O.sr_offset(seed, step, b, h, s, j) for j in range(128)], np.float64) - 0.5
         z = page.code[s].astype(np.float64)
         d = np.abs(z - x)
         assert np.all(d <= 0.5 + 1e-5), (s, d.max())

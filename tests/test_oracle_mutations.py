@@ -45,6 +45,8 @@ MUTANTS = {
     "ranking ascending": ("return score[a] > score[b2];", "return score[a] < score[b2];"),
     "dequantize drops c": ("S_nat[(size_t)perm[s] * d_v + j] = (x * rs) * c;",
                            "S_nat[(size_t)perm[s] * d_v + j] = x * rs;"),
+    "sr rounds up with 1 - frac": ("zr = (x >= fl + 1.0 - u) ? fl + 1.0 : fl;", "zr = (x >= fl + u) ? fl + 1.0 : fl;"),
+    "sr offset on a 2^-17 grid": ("return (float)h16 * 0x1p-16f;", "return (float)h16 * 0x1p-17f;"),
     "sr halves swapped": ("uint32_t h16 = (j & 1) ? (word & 0xFFFFu) : (word >> 16);",
                           "uint32_t h16 = (j & 1) ? (word >> 16) : (word & 0xFFFFu);"),
     "column absmax over one row": ("float a = std::fabs(S_nat[(size_t)kap * d_v + j]);",

@@ -149,24 +149,28 @@ def test_pcg4d_neighbouring_counters_are_unrelated():
 
 # ------------------------------------------------- stochastic-rounding offsets
 
-def test_sr_delta_grid_and_range():
-    vals = np.array([O.sr_delta(123, 5, 7, 3, s, j) for s in range(8) for j in range(128)])
-    scaled = vals * 2.0**17
-    assert np.all(np.abs(vals) < 0.5)
-    assert np.all(scaled == np.round(scaled))              # multiples of 2^-17
-    assert np.all(np.mod(np.round(scaled), 2) == 1)        # odd multiples: never 0, symmetric
-    assert abs(vals.mean()) < 4 * 0.29 / np.sqrt(vals.size)
+def test_sr_offset_grid_and_range():
+    vals = np.array([O.sr_offset(123, 5, 7, 3, s, j) for s in range(8) for j in range(128)])
+    scaled = vals * 2.0**16
+    assert np.all((vals >= 0.0) & (vals < 1.0))
+    assert np.all(scaled == np.round(scaled))              # multiples of 2^-16
+    # uniform on the grid: mean (1 - 2^-16) / 2, variance ~ 1/12
+    assert abs(vals.mean() - (0.5 - 2.0**-17)) < 4 * 0.29 / np.sqrt(vals.size)
+    assert abs(vals.var() - 1.0 / 12) < 0.01
+    counts = np.histogram(vals, bins=8, range=(0.0, 1.0))[0]
+    exp = vals.size / 8
+    assert np.sum((counts - exp) ** 2 / exp) < 24.3        # chi-square, 7 dof, p ~ 0.001
 
 
-def test_sr_delta_is_a_pure_function_of_its_counter():
-    a = [O.sr_delta(9, 1, 2, 3, s, j) for s in range(4) for j in range(8)]
-    b = [O.sr_delta(9, 1, 2, 3, s, j) for s in range(4) for j in range(8)]
+def test_sr_offset_is_a_pure_function_of_its_counter():
+    a = [O.sr_offset(9, 1, 2, 3, s, j) for s in range(4) for j in range(8)]
+    b = [O.sr_offset(9, 1, 2, 3, s, j) for s in range(4) for j in range(8)]
     assert a == b
-    c = [O.sr_delta(9, 2, 2, 3, s, j) for s in range(4) for j in range(8)]
+    c = [O.sr_offset(9, 2, 2, 3, s, j) for s in range(4) for j in range(8)]
     assert a != c
     # the two columns of one 32-bit word come from its high and low halves;
     # the input is (tile, step, request ^ low seed word, head ^ high seed word)
     out = O.pcg4d(np.array([0, 1, 2 ^ 9, 3], np.uint32))
     w = int(out[0])
-    assert O.sr_delta(9, 1, 2, 3, 0, 0) == (2 * (w >> 16) - 65535) * 2.0**-17
-    assert O.sr_delta(9, 1, 2, 3, 0, 1) == (2 * (w & 0xFFFF) - 65535) * 2.0**-17
+    assert O.sr_offset(9, 1, 2, 3, 0, 0) == (w >> 16) * 2.0**-16
+    assert O.sr_offset(9, 1, 2, 3, 0, 1) == (w & 0xFFFF) * 2.0**-16
