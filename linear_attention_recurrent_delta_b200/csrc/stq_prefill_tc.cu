@@ -15,10 +15,12 @@
 // lo hi), which keeps fp32-level accuracy; the triangular solve runs on the
 // CUDA cores (thread v owns value column v of E).
 //
-// One CTA of 128 threads per page (persistent over pages; its 168 KB of
+// One CTA of 256 threads per page (persistent over pages; its 168 KB of
 // shared memory and all 512 tensor-memory columns keep it alone on its SM).
-// Thread t owns row t of whatever a phase computes: token t, value column
-// t, or key channel t, which is also tensor-memory lane t.
+// Thread t of each 128-thread half owns row t of whatever a phase computes:
+// token t, value column t, or key channel t, which is also tensor-memory
+// lane t (warps w and w + 4 see the same 32 lanes); the two halves split the
+// row's columns between them.  The triangular solve runs on the first half.
 //   shared memory: six 16 KB operand tiles (128 rows x 32 fp32, 128-byte
 //   swizzled, K-major), reused as the solve's matrix A and as the page
 //   buffer; the state X = S^T (X[v][kappa], fp32, rows padded to 129
@@ -31,6 +33,7 @@
 namespace stq {
 
 constexpr int kChunk = 128;                    // tokens per chunk
+constexpr int kTcThreads = 256;                // two halves of 128 threads
 constexpr int kXStride = kD + 1;               // floats per state row
 constexpr int kAStride = kChunk + 4;           // floats per row of the solve's matrix (16-byte rows)
 constexpr uint32_t kTiles = 6;
@@ -96,7 +99,7 @@ __device__ __forceinline__ void tmem_row(uint32_t taddr_lane, Fn &&fn) {
 }
 
 template <class FMT>
-__global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const DevFormat F, const TcArgs A) {
+__global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const DevFormat F, const TcArgs A) {
     extern __shared__ uint8_t tc_smem_raw[];
     const uint32_t raw = smem_u32(tc_smem_raw);
     uint8_t *base = tc_smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -112,7 +115,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const DevFormat
     bool col_scales, gate_vector;
     format_flags<FMT>(F, col_scales, gate_vector);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const RowCtx R = row_ctx<FMT>(F, warp, lane);
+    const int t = tid & (kD - 1), hf = tid >> 7;   // row t, half hf of its columns
+    const int wq = warp & 3;                        // lanes 32 wq .. + 31; slice wq of the page
+    const RowCtx R = row_ctx<FMT>(F, wq, lane);
 
     if (tid == 0) {
         mbar_init(&M.mma_bar, 1);
@@ -128,7 +133,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const DevFormat
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = M.tmem;
-    const uint32_t lane_addr = tmem + ((uint32_t)(32 * warp) << 16);   // this thread's lane, column 0
+    const uint32_t lane_addr = tmem + ((uint32_t)(32 * wq) << 16);     // this thread's lane, column 0
     const uint32_t RG = 0, RY = 128, RP = 256, RO = 384;               // column regions
 
     const int n = A.n_pages, H = A.heads;
@@ -152,42 +157,42 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const DevFormat
             mbar_expect_tx(&M.page_bar, (uint32_t)F.page_bytes);
             bulk_g2s(tiles, A.pages + (size_t)p * F.page_bytes, (uint32_t)F.page_bytes, &M.page_bar);
         }
-        M.kap[tid] = A.perm[(size_t)ph * kD + tid] & (kD - 1);
+        if (tid < kD) M.kap[tid] = A.perm[(size_t)ph * kD + tid] & (kD - 1);
         bool ok;
         const uint32_t pp = page_phase;
         page_phase ^= 1u;
         if (A.stall_first_wait && p == (int)blockIdx.x) ok = mbar_wait_bounded(&M.never, 0, A.wait_limit_ns);
         else ok = mbar_wait_bounded(&M.page_bar, pp, A.wait_limit_ns);
         if (!ok) pending_page = (int)pp;
-        {
+        if (tid < kD) {
             const float c = col_scales ? reinterpret_cast<const float *>(tiles + F.c_off)[tid] : 1.f;
             M.c[tid] = c;
             M.ic[tid] = col_scales ? __frcp_rn(c) : 1.f;
         }
         if (__syncthreads_or(!ok)) { failed = true; break; }
         {
-            // warp w dequantizes slice w (rows 16 b + 4 w + i) of every block:
-            // T = z r (FP16 rows: h), written to X[v][kappa]
+            // warp w dequantizes slice w % 4 (rows 16 b + 4 (w % 4) + i) of
+            // blocks 4 (w / 4) .. + 3: T = z r (FP16 rows: h), written to
+            // X[v][kappa]
             const float *r_s = reinterpret_cast<const float *>(tiles + F.r_off);
             static_for<0, kBlocks>([&](auto bc) {
                 constexpr int b = decltype(bc)::value;
+                if ((b >> 2) != hf) return;
                 float av[4];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    const int s = 16 * b + 4 * warp + i;
-                    const int blk_r = (R.all_int || F.blk_kind(b) == kKindInt) ? F.blk_rbase(b) + 4 * warp + i : -1;
+                    const int blk_r = (R.all_int || F.blk_kind(b) == kKindInt) ? F.blk_rbase(b) + 4 * wq + i : -1;
                     av[i] = blk_r >= 0 ? r_s[blk_r] : 1.f;
-                    (void)s;
                 }
                 Tile T;
                 const uint8_t *blk = tiles + fmt_offset<FMT, b>(F);
                 with_width<FMT, b>(F, [&](auto wc) {
                     constexpr int W = decltype(wc)::value;
-                    dequant_slice<W, b>(blk, warp, lane, make_float4(av[0], av[1], av[2], av[3]), T);
+                    dequant_slice<W, b>(blk, wq, lane, make_float4(av[0], av[1], av[2], av[3]), T);
                 });
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    const int kap = M.kap[16 * b + 4 * warp + i];
+                    const int kap = M.kap[16 * b + 4 * wq + i];
                     XS[(4 * lane + 0) * kXStride + kap] = T[b][i][0].x;
                     XS[(4 * lane + 1) * kXStride + kap] = T[b][i][0].y;
                     XS[(4 * lane + 2) * kXStride + kap] = T[b][i][1].x;
@@ -200,7 +205,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const DevFormat
         for (int t0 = 0; t0 < A.L && !failed; t0 += kChunk) {
             const int cn = min(kChunk, A.L - t0);
             // ---- per-token scalars of the chunk
-            {
+            if (tid < kChunk) {
                 const bool real = tid < cn;
                 const size_t row = (size_t)(t0 + tid) * n + p;
                 M.bet[tid] = real ? A.beta[row] : 0.f;
@@ -215,7 +220,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const DevFormat
                 }
             }
             __syncthreads();
-            {
+            if (tid < kChunk) {
                 const float gi = M.gam[tid];
                 M.igam[tid] = __frcp_rn(gi);
                 M.kts[tid] = __fdiv_rn(M.gam[kChunk - 1], gi);
@@ -225,26 +230,33 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const DevFormat
             // ---- phase A: G = K K^T, Y^T = X K^T, P' = (gam Q) K^T, O^T = X (gam Q)^T
             for (int ks = 0; ks < kD / 32; ++ks) {
                 {
-                    const bool real = tid < cn;
-                    const size_t row = ((size_t)(t0 + tid) * n + p) * kD + 32 * ks;
-                    const float gi = M.gam[tid];
+                    // row t of the K, gam Q and X slabs, columns 16 hf .. + 15
+                    const bool real = t < cn;
+                    const size_t row = ((size_t)(t0 + t) * n + p) * kD + 32 * ks + 16 * hf;
+                    const float gi = M.gam[t];
+                    float4 kx[4], qx[4];
 #pragma unroll
-                    for (int j4 = 0; j4 < 8; ++j4) {
-                        float4 kx = make_float4(0.f, 0.f, 0.f, 0.f), qx = kx;
+                    for (int j4 = 0; j4 < 4; ++j4) {
+                        kx[j4] = qx[j4] = make_float4(0.f, 0.f, 0.f, 0.f);
                         if (real) {
-                            kx = __ldg(reinterpret_cast<const float4 *>(A.k + row) + j4);
-                            qx = __ldg(reinterpret_cast<const float4 *>(A.q + row) + j4);
-                        }
-                        const float kv[4] = {kx.x, kx.y, kx.z, kx.w}, qv[4] = {qx.x, qx.y, qx.z, qx.w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            put_split(tile(0), tile(1), tid, 4 * j4 + e, kv[e]);
-                            put_split(tile(2), tile(3), tid, 4 * j4 + e, __fmul_rn(gi, qv[e]));
+                            kx[j4] = __ldg(reinterpret_cast<const float4 *>(A.k + row) + j4);
+                            qx[j4] = __ldg(reinterpret_cast<const float4 *>(A.q + row) + j4);
                         }
                     }
-                    const float *xr = XS + tid * kXStride + 32 * ks;
+#pragma unroll
+                    for (int j4 = 0; j4 < 4; ++j4) {
+                        const float kv[4] = {kx[j4].x, kx[j4].y, kx[j4].z, kx[j4].w};
+                        const float qv[4] = {qx[j4].x, qx[j4].y, qx[j4].z, qx[j4].w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int j = 16 * hf + 4 * j4 + e;
+                            put_split(tile(0), tile(1), t, j, kv[e]);
+                            put_split(tile(2), tile(3), t, j, __fmul_rn(gi, qv[e]));
+                        }
+                    }
+                    const float *xr = XS + t * kXStride + 32 * ks;
 #pragma unroll 8
-                    for (int j = 0; j < 32; ++j) put_split(tile(4), tile(5), tid, j, xr[j]);
+                    for (int j = 16 * hf; j < 16 * hf + 16; ++j) put_split(tile(4), tile(5), t, j, xr[j]);
                 }
                 fence_proxy_async_smem();
                 tc::fence_before_sync();
@@ -268,16 +280,17 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const DevFormat
             // registers; between them the off-diagonal block, R2 -= A21 E1,
             // as a tensor-core product.  E^T ends up in Y^T's columns.
             {
-                const float icv = M.ic[tid];
+                // column t of R, tokens 64 hf .. + 63
+                const float icv = M.ic[t];
                 const uint32_t ry = lane_addr + RY;
 #pragma unroll
-                for (int c0 = 0; c0 < kChunk; c0 += 32) {
+                for (int c0 = 64 * hf; c0 < 64 * hf + 64; c0 += 32) {
                     float x[32];
                     tc::ld32(ry + c0, x);
 #pragma unroll
                     for (int jj = 0; jj < 32; ++jj) {
                         const int i = c0 + jj;
-                        const float vv = (i < cn) ? __ldg(A.v + ((size_t)(t0 + i) * n + p) * kD + tid) : 0.f;
+                        const float vv = (i < cn) ? __ldg(A.v + ((size_t)(t0 + i) * n + p) * kD + t) : 0.f;
                         // R_i = beta_i (v_i / c - gam_i y_i)
                         x[jj] = __fmul_rn(M.bet[i], __fsub_rn(__fmul_rn(vv, icv), __fmul_rn(M.gam[i], x[jj])));
                     }
@@ -286,70 +299,73 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const DevFormat
             }
             for (int sb = 0; sb < 2; ++sb) {
                 // the diagonal block of this half: A_ij, i, j in [64 sb, 64 sb + 64)
-                if (tid >= 64 * sb && tid < 64 * sb + 64) {
-                    const float bi = M.bet[tid], gi = M.gam[tid];
-                    float *arow = Amat + (tid - 64 * sb) * kAStride;
+                // (row t, columns 32 hf .. + 31 of the block)
+                if (t >= 64 * sb && t < 64 * sb + 64) {
+                    const float bi = M.bet[t], gi = M.gam[t];
+                    float *arow = Amat + (t - 64 * sb) * kAStride;
+                    const int c0 = 32 * hf;
+                    float x[32];
+                    tc::ld32(lane_addr + RG + 64 * sb + c0, x);
 #pragma unroll
-                    for (int c0 = 0; c0 < 64; c0 += 32) {
-                        float x[32];
-                        tc::ld32(lane_addr + RG + 64 * sb + c0, x);
-#pragma unroll
-                        for (int jj = 0; jj < 32; ++jj) {
-                            const int j = 64 * sb + c0 + jj;
-                            const float a = __fmul_rn(bi, __fmul_rn(__fmul_rn(gi, M.igam[j]), x[jj]));
-                            arow[c0 + jj] = j < tid ? a : 0.f;
-                        }
+                    for (int jj = 0; jj < 32; ++jj) {
+                        const int j = 64 * sb + c0 + jj;
+                        const float a = __fmul_rn(bi, __fmul_rn(__fmul_rn(gi, M.igam[j]), x[jj]));
+                        arow[c0 + jj] = j < t ? a : 0.f;
                     }
                 }
                 __syncthreads();
-                float e[64];
-                {
-                    float x[32];
-                    tc::ld32(lane_addr + RY + 64 * sb, x);
+                float e[64];   // the first half's threads: column t of this half of E
+                if (hf == 0) {
+                    {
+                        float x[32];
+                        tc::ld32(lane_addr + RY + 64 * sb, x);
 #pragma unroll
-                    for (int jj = 0; jj < 32; ++jj) e[jj] = x[jj];
-                    tc::ld32(lane_addr + RY + 64 * sb + 32, x);
+                        for (int jj = 0; jj < 32; ++jj) e[jj] = x[jj];
+                        tc::ld32(lane_addr + RY + 64 * sb + 32, x);
 #pragma unroll
-                    for (int jj = 0; jj < 32; ++jj) e[32 + jj] = x[jj];
-                }
-                // forward substitution: E_i = R_i - sum_{j<i} A_ij E_j
-#pragma unroll
-                for (int i = 1; i < 64; ++i) {
-                    const float *arow = Amat + i * kAStride;
-                    float acc = e[i];
-#pragma unroll
-                    for (int j4 = 0; j4 < (i + 3) / 4; ++j4) {
-                        const float4 a4 = *reinterpret_cast<const float4 *>(arow + 4 * j4);
-                        const float av[4] = {a4.x, a4.y, a4.z, a4.w};
-#pragma unroll
-                        for (int jj = 0; jj < 4; ++jj)
-                            if (4 * j4 + jj < i) acc = __fmaf_rn(-av[jj], e[4 * j4 + jj], acc);
+                        for (int jj = 0; jj < 32; ++jj) e[32 + jj] = x[jj];
                     }
-                    e[i] = acc;
-                }
-                {
-                    float x[32];
+                    // forward substitution: E_i = R_i - sum_{j<i} A_ij E_j
 #pragma unroll
-                    for (int jj = 0; jj < 32; ++jj) x[jj] = e[jj];
-                    tc::st32(lane_addr + RY + 64 * sb, x);
+                    for (int i = 1; i < 64; ++i) {
+                        const float *arow = Amat + i * kAStride;
+                        float acc = e[i];
 #pragma unroll
-                    for (int jj = 0; jj < 32; ++jj) x[jj] = e[32 + jj];
-                    tc::st32(lane_addr + RY + 64 * sb + 32, x);
+                        for (int j4 = 0; j4 < (i + 3) / 4; ++j4) {
+                            const float4 a4 = *reinterpret_cast<const float4 *>(arow + 4 * j4);
+                            const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+                            for (int jj = 0; jj < 4; ++jj)
+                                if (4 * j4 + jj < i) acc = __fmaf_rn(-av[jj], e[4 * j4 + jj], acc);
+                        }
+                        e[i] = acc;
+                    }
+                    {
+                        float x[32];
+#pragma unroll
+                        for (int jj = 0; jj < 32; ++jj) x[jj] = e[jj];
+                        tc::st32(lane_addr + RY + 64 * sb, x);
+#pragma unroll
+                        for (int jj = 0; jj < 32; ++jj) x[jj] = e[32 + jj];
+                        tc::st32(lane_addr + RY + 64 * sb + 32, x);
+                    }
                 }
                 if (sb == 1) break;
                 __syncthreads();   // the diagonal block's space becomes operand tiles
                 // R2 -= A21 E1 on the tensor cores: D = R2^T (columns 64..127 of
                 // Y^T) += (-E1^T) A21^T, M = 128 (v), N = 64 (i), K = 64 (j).
-                // Tiles: E1^T hi / lo (rows v, two K slabs) at 0 .. 64 KB; A21
-                // hi / lo (rows i - 64, 64-row tiles of 8 KB) at 64 .. 96 KB.
+                // Tiles: E1^T hi / lo (rows v, two K slabs) at 0 .. 64 KB, written
+                // by the first half from its columns of E; A21 hi / lo (rows
+                // i - 64, 64-row tiles of 8 KB) at 64 .. 96 KB, by the second.
+                if (hf == 0) {
 #pragma unroll
-                for (int kb = 0; kb < 2; ++kb) {
+                    for (int kb = 0; kb < 2; ++kb) {
 #pragma unroll
-                    for (int jj = 0; jj < 32; ++jj)
-                        put_split(tile(2 * kb), tile(2 * kb + 1), tid, jj, e[32 * kb + jj]);
-                }
-                if (tid >= 64) {
-                    const float bi = M.bet[tid], gi = M.gam[tid];
+                        for (int jj = 0; jj < 32; ++jj)
+                            put_split(tile(2 * kb), tile(2 * kb + 1), t, jj, e[32 * kb + jj]);
+                    }
+                } else if (t >= 64) {
+                    const float bi = M.bet[t], gi = M.gam[t];
                     uint8_t *a21 = tiles + 4 * tc::kTileBytes;
 #pragma unroll
                     for (int kb = 0; kb < 2; ++kb) {
@@ -360,7 +376,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const DevFormat
                             const int j = 32 * kb + jj;
                             const float a = __fmul_rn(bi, __fmul_rn(__fmul_rn(gi, M.igam[j]), x[jj]));
                             put_split(a21 + (2 * kb) * (tc::kTileBytes / 2), a21 + (2 * kb + 1) * (tc::kTileBytes / 2),
-                                      tid - 64, jj, a);
+                                      t - 64, jj, a);
                         }
                     }
                 }
@@ -392,30 +408,39 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const DevFormat
                 if (__syncthreads_or(!wait_mma())) { failed = true; break; }
             }
             if (failed) break;
-            __syncthreads();   // the solve's space becomes operand tiles again
+            // the solve's space becomes operand tiles again; E^T (stored by the
+            // first half) is read by both halves
+            tc::fence_before_sync();
+            __syncthreads();
+            tc::fence_after_sync();
 
             // ---- phase C: O^T += E^T P~^T, dX = E^T K~ (K = tokens)
             for (int js = 0; js < kChunk / 32; ++js) {
                 {
+                    // columns 16 hf .. + 15 of the slab
+                    const int c0 = 16 * hf;
                     // E^T row v (thread v), from Y^T's columns
-                    float x[32];
-                    tc::ld32(lane_addr + RY + 32 * js, x);
+                    float x[16];
+                    tc::ld16(lane_addr + RY + 32 * js + c0, x);
 #pragma unroll
-                    for (int jj = 0; jj < 32; ++jj) put_split(tile(0), tile(1), tid, jj, x[jj]);
+                    for (int jj = 0; jj < 16; ++jj) put_split(tile(0), tile(1), t, c0 + jj, x[jj]);
                     // P~ row i (thread i): P'_ij / gam_j for j <= i, else 0
-                    tc::ld32(lane_addr + RP + 32 * js, x);
+                    tc::ld16(lane_addr + RP + 32 * js + c0, x);
 #pragma unroll
-                    for (int jj = 0; jj < 32; ++jj) {
-                        const int j = 32 * js + jj;
-                        put_split(tile(2), tile(3), tid, jj, j <= tid ? __fmul_rn(x[jj], M.igam[j]) : 0.f);
+                    for (int jj = 0; jj < 16; ++jj) {
+                        const int j = 32 * js + c0 + jj;
+                        put_split(tile(2), tile(3), t, c0 + jj, j <= t ? __fmul_rn(x[jj], M.igam[j]) : 0.f);
                     }
                     // K~^T row kappa (thread kappa): k_j[kappa] gam_n / gam_j
-#pragma unroll 8
-                    for (int jj = 0; jj < 32; ++jj) {
-                        const int j = 32 * js + jj;
-                        const float kk = (j < cn) ? __ldg(A.k + ((size_t)(t0 + j) * n + p) * kD + tid) : 0.f;
-                        put_split(tile(4), tile(5), tid, jj, __fmul_rn(kk, M.kts[j]));
+                    float kk[16];
+#pragma unroll
+                    for (int jj = 0; jj < 16; ++jj) {
+                        const int j = 32 * js + c0 + jj;
+                        kk[jj] = (j < cn) ? __ldg(A.k + ((size_t)(t0 + j) * n + p) * kD + t) : 0.f;
                     }
+#pragma unroll
+                    for (int jj = 0; jj < 16; ++jj)
+                        put_split(tile(4), tile(5), t, c0 + jj, __fmul_rn(kk[jj], M.kts[32 * js + c0 + jj]));
                 }
                 fence_proxy_async_smem();
                 tc::fence_before_sync();
@@ -432,20 +457,27 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const DevFormat
 
             // ---- phase D: o of the chunk's tokens; X <- gam_n X + dX
             {
-                const float cv = M.c[tid];
-                tmem_row(lane_addr + RO, [&](int c0, const float (&x)[32]) {
+                // column t: tokens (o) and key channels (X) 64 hf .. + 63
+                const float cv = M.c[t];
+#pragma unroll
+                for (int c0 = 64 * hf; c0 < 64 * hf + 64; c0 += 32) {
+                    float x[32];
+                    tc::ld32(lane_addr + RO + c0, x);
 #pragma unroll
                     for (int jj = 0; jj < 32; ++jj) {
                         const int i = c0 + jj;
-                        if (i < cn) A.o[((size_t)(t0 + i) * n + p) * kD + tid] = __fmul_rn(cv, x[jj]);
+                        if (i < cn) A.o[((size_t)(t0 + i) * n + p) * kD + t] = __fmul_rn(cv, x[jj]);
                     }
-                });
+                }
                 const float gn = M.gam[kChunk - 1];
-                float *xr = XS + tid * kXStride;
-                tmem_row(lane_addr + RG, [&](int c0, const float (&x)[32]) {
+                float *xr = XS + t * kXStride;
+#pragma unroll
+                for (int c0 = 64 * hf; c0 < 64 * hf + 64; c0 += 32) {
+                    float x[32];
+                    tc::ld32(lane_addr + RG + c0, x);
 #pragma unroll
                     for (int jj = 0; jj < 32; ++jj) xr[c0 + jj] = __fmaf_rn(gn, xr[c0 + jj], x[jj]);
-                });
+                }
             }
             tc::fence_before_sync();
             __syncthreads();
@@ -455,52 +487,63 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const DevFormat
 
         // ---- the page's end: the state (optional), one requantization, the store
         if (A.S_out) {
-            const float cv = M.c[tid];
-            const float *xr = XS + tid * kXStride;
-            for (int kap = 0; kap < kD; ++kap)
-                A.S_out[((size_t)p * kD + kap) * kD + tid] = __fmul_rn(xr[kap], cv);
+            const float cv = M.c[t];
+            const float *xr = XS + t * kXStride;
+            for (int kap = 64 * hf; kap < 64 * hf + 64; ++kap)
+                A.S_out[((size_t)p * kD + kap) * kD + t] = __fmul_rn(xr[kap], cv);
         }
         // the page buffer starts from zero (the 1-bit plane's words are
         // updated by xor of each slice's bits)
-        for (int i = tid; i < (int)(F.page_bytes / 16); i += kThreads)
+        for (int i = tid; i < (int)(F.page_bytes / 16); i += kTcThreads)
             reinterpret_cast<uint4 *>(tiles)[i] = make_uint4(0u, 0u, 0u, 0u);
-        Tile T;
-        static_for<0, kBlocks>([&](auto bc) {
-            constexpr int b = decltype(bc)::value;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int kap = M.kap[16 * b + 4 * warp + i];
-                T[b][i][0] = make_float2(XS[(4 * lane + 0) * kXStride + kap], XS[(4 * lane + 1) * kXStride + kap]);
-                T[b][i][1] = make_float2(XS[(4 * lane + 2) * kXStride + kap], XS[(4 * lane + 3) * kXStride + kap]);
-                M.inv[warp][4 * b + i] = warp_absmax(absmax4(T[b][i][0], T[b][i][1]));
-            }
-        });
-        __syncthreads();
-        {
-            float *r_s = reinterpret_cast<float *>(tiles + F.r_off);
-            const float m = M.inv[warp][lane];
-            float inv = 0.f;
-            if (R.all_int || R.is_int) {
-                const float r = div_by_qmax(m, R.qmax, R.rcp_qmax);
-                inv = m > 0.f ? div_rz_qmax<false>(R.qmax, m) : 0.f;
-                r_s[R.rix] = r;
-            }
-            M.inv[warp][lane] = inv;
-        }
-        __syncwarp();
+        __syncthreads();   // the buffer is zero before any slice packs into it
+        // warp w: slice w % 4 of blocks 4 (w / 4) .. + 3, as at the page's
+        // start; its lanes 0 .. 15 finish those blocks' 16 rows (row maxima
+        // in M.inv[w % 4][4 b + i])
         SrCtx sr;
         sr.k0 = A.seed_lo; sr.k1 = A.seed_hi; sr.step = A.step;
         sr.b = (uint32_t)pb;
         sr.h = (uint32_t)ph;
-        static_for<0, kBlocks>([&](auto bc) {
-            constexpr int b = decltype(bc)::value;
-            const float4 i4 = *reinterpret_cast<const float4 *>(&M.inv[warp][4 * b]);
-            uint8_t *blk = tiles + fmt_offset<FMT, b>(F);
-            with_width<FMT, b>(F, [&](auto wc) {
-                constexpr int W = decltype(wc)::value;
-                requant_slice<W, b, SR>(blk, warp, lane, i4, T, sr);
+        auto finish_half = [&](auto hc) {
+            constexpr int H = decltype(hc)::value;
+            Tile T;
+            static_for<4 * H, 4 * H + 4>([&](auto bc) {
+                constexpr int b = decltype(bc)::value;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int kap = M.kap[16 * b + 4 * wq + i];
+                    T[b][i][0] = make_float2(XS[(4 * lane + 0) * kXStride + kap], XS[(4 * lane + 1) * kXStride + kap]);
+                    T[b][i][1] = make_float2(XS[(4 * lane + 2) * kXStride + kap], XS[(4 * lane + 3) * kXStride + kap]);
+                    M.inv[wq][4 * b + i] = warp_absmax(absmax4(T[b][i][0], T[b][i][1]));
+                }
             });
-        });
+            __syncwarp();
+            if (lane < 16) {
+                const int vl = 16 * H + lane;   // row vl of the slice: block vl / 4, row vl % 4
+                const RowCtx Rv = row_ctx<FMT>(F, wq, vl);
+                float *r_s = reinterpret_cast<float *>(tiles + F.r_off);
+                const float m = M.inv[wq][vl];
+                float inv = 0.f;
+                if (Rv.all_int || Rv.is_int) {
+                    const float r = div_by_qmax(m, Rv.qmax, Rv.rcp_qmax);
+                    inv = m > 0.f ? div_rz_qmax<false>(Rv.qmax, m) : 0.f;
+                    r_s[Rv.rix] = r;
+                }
+                M.inv[wq][vl] = inv;
+            }
+            __syncwarp();
+            static_for<4 * H, 4 * H + 4>([&](auto bc) {
+                constexpr int b = decltype(bc)::value;
+                const float4 i4 = *reinterpret_cast<const float4 *>(&M.inv[wq][4 * b]);
+                uint8_t *blk = tiles + fmt_offset<FMT, b>(F);
+                with_width<FMT, b>(F, [&](auto wc) {
+                    constexpr int W = decltype(wc)::value;
+                    requant_slice<W, b, SR>(blk, wq, lane, i4, T, sr);
+                });
+            });
+        };
+        if (hf == 0) finish_half(IC<0>{});
+        else finish_half(IC<1>{});
         fence_proxy_async_smem();
         __syncthreads();
         if (tid == 0) {
@@ -528,9 +571,9 @@ static cudaError_t launch_prefill_tc_with(const DevFormat &F, const TcArgs &A, c
     const void *fn = (const void *)prefill_tc_kernel<FMT>;
     cudaError_t err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTcSmem);
     if (err != cudaSuccess) return err;
-    const int grid = persistent_grid(fn, kThreads, kTcSmem, A.n_pages);
+    const int grid = persistent_grid(fn, kTcThreads, kTcSmem, A.n_pages);
     if (grid <= 0) return cudaErrorInvalidConfiguration;
-    prefill_tc_kernel<FMT><<<grid, kThreads, kTcSmem, stream>>>(F, A);
+    prefill_tc_kernel<FMT><<<grid, kTcThreads, kTcSmem, stream>>>(F, A);
     return cudaGetLastError();
 }
 
