@@ -228,21 +228,26 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const DevForm
             __syncthreads();
 
             // ---- phase A: G = K K^T, Y^T = X K^T, P' = (gam Q) K^T, O^T = X (gam Q)^T
+            // row t of the K and Q slabs, columns 16 hf .. + 15: the next slab's
+            // are loaded while the tensor cores work on this one
+            float4 kx[4], qx[4];
+            auto load_kq = [&](int ks) {
+                const bool real = t < cn;
+                const size_t row = ((size_t)(t0 + t) * n + p) * kD + 32 * ks + 16 * hf;
+#pragma unroll
+                for (int j4 = 0; j4 < 4; ++j4) {
+                    kx[j4] = qx[j4] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (real) {
+                        kx[j4] = __ldg(reinterpret_cast<const float4 *>(A.k + row) + j4);
+                        qx[j4] = __ldg(reinterpret_cast<const float4 *>(A.q + row) + j4);
+                    }
+                }
+            };
+            load_kq(0);
             for (int ks = 0; ks < kD / 32; ++ks) {
                 {
                     // row t of the K, gam Q and X slabs, columns 16 hf .. + 15
-                    const bool real = t < cn;
-                    const size_t row = ((size_t)(t0 + t) * n + p) * kD + 32 * ks + 16 * hf;
                     const float gi = M.gam[t];
-                    float4 kx[4], qx[4];
-#pragma unroll
-                    for (int j4 = 0; j4 < 4; ++j4) {
-                        kx[j4] = qx[j4] = make_float4(0.f, 0.f, 0.f, 0.f);
-                        if (real) {
-                            kx[j4] = __ldg(reinterpret_cast<const float4 *>(A.k + row) + j4);
-                            qx[j4] = __ldg(reinterpret_cast<const float4 *>(A.q + row) + j4);
-                        }
-                    }
 #pragma unroll
                     for (int j4 = 0; j4 < 4; ++j4) {
                         const float kv[4] = {kx[j4].x, kx[j4].y, kx[j4].z, kx[j4].w};
@@ -270,6 +275,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const DevForm
                     mma_split(tmem + RO, tile_addr(4), tile_addr(5), tile_addr(2), tile_addr(3), acc);
                     tc::commit(&M.mma_bar);
                 }
+                if (ks + 1 < kD / 32) load_kq(ks + 1);
                 if (__syncthreads_or(!wait_mma())) { failed = true; break; }
             }
             if (failed) break;
@@ -415,6 +421,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const DevForm
             tc::fence_after_sync();
 
             // ---- phase C: O^T += E^T P~^T, dX = E^T K~ (K = tokens)
+            // key channel t of tokens 32 js + 16 hf .. + 15, the next slab's
+            // loaded while the tensor cores work on this one
+            float kk[16];
+            auto load_kt = [&](int js) {
+#pragma unroll
+                for (int jj = 0; jj < 16; ++jj) {
+                    const int j = 32 * js + 16 * hf + jj;
+                    kk[jj] = (j < cn) ? __ldg(A.k + ((size_t)(t0 + j) * n + p) * kD + t) : 0.f;
+                }
+            };
+            load_kt(0);
             for (int js = 0; js < kChunk / 32; ++js) {
                 {
                     // columns 16 hf .. + 15 of the slab
@@ -432,12 +449,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const DevForm
                         put_split(tile(2), tile(3), t, c0 + jj, j <= t ? __fmul_rn(x[jj], M.igam[j]) : 0.f);
                     }
                     // K~^T row kappa (thread kappa): k_j[kappa] gam_n / gam_j
-                    float kk[16];
-#pragma unroll
-                    for (int jj = 0; jj < 16; ++jj) {
-                        const int j = 32 * js + c0 + jj;
-                        kk[jj] = (j < cn) ? __ldg(A.k + ((size_t)(t0 + j) * n + p) * kD + t) : 0.f;
-                    }
 #pragma unroll
                     for (int jj = 0; jj < 16; ++jj)
                         put_split(tile(4), tile(5), t, c0 + jj, __fmul_rn(kk[jj], M.kts[32 * js + c0 + jj]));
@@ -451,6 +462,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const DevForm
                     mma_split(tmem + RG, tile_addr(0), tile_addr(1), tile_addr(4), tile_addr(5), js > 0);
                     tc::commit(&M.mma_bar);
                 }
+                if (js + 1 < kChunk / 32) load_kt(js + 1);
                 if (__syncthreads_or(!wait_mma())) { failed = true; break; }
             }
             if (failed) break;
