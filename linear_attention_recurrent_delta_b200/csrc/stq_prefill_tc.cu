@@ -66,12 +66,22 @@ struct TcSmall {
 
 constexpr size_t kTcSmem = kTileRegion + (size_t)kD * kXStride * 4 + sizeof(TcSmall) + 1024;
 
-__device__ __forceinline__ void put_split(uint8_t *hi_tile, uint8_t *lo_tile, uint32_t row, uint32_t k, float x) {
-    float h, l;
-    tc::split_tf32(x, h, l);
+// four consecutive columns k .. k + 3 (k a multiple of 4) of a row: one
+// 16-byte unit of the swizzled row, so a warp's 32 rows take 4 conflict-free
+// shared-memory wavefronts (a float at a time, 8 banks serve the 32 rows)
+__device__ __forceinline__ void put_split4(uint8_t *hi_tile, uint8_t *lo_tile, uint32_t row, uint32_t k, float4 x) {
+    float4 h, l;
+    tc::split_tf32(x.x, h.x, l.x);
+    tc::split_tf32(x.y, h.y, l.y);
+    tc::split_tf32(x.z, h.z, l.z);
+    tc::split_tf32(x.w, h.w, l.w);
     const uint32_t off = tc::sw128_offset(row, k);
-    *reinterpret_cast<float *>(hi_tile + off) = h;
-    *reinterpret_cast<float *>(lo_tile + off) = l;
+    *reinterpret_cast<float4 *>(hi_tile + off) = h;
+    *reinterpret_cast<float4 *>(lo_tile + off) = l;
+}
+
+__device__ __forceinline__ float4 mul4(float a, float4 x) {
+    return make_float4(__fmul_rn(a, x.x), __fmul_rn(a, x.y), __fmul_rn(a, x.z), __fmul_rn(a, x.w));
 }
 
 // D (+)= A B^T over one 32-wide K slab, split operands: hi hi, hi lo, lo hi
@@ -248,20 +258,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const DevForm
                 {
                     // row t of the K, gam Q and X slabs, columns 16 hf .. + 15
                     const float gi = M.gam[t];
+                    const float *xr = XS + t * kXStride + 32 * ks;
 #pragma unroll
                     for (int j4 = 0; j4 < 4; ++j4) {
-                        const float kv[4] = {kx[j4].x, kx[j4].y, kx[j4].z, kx[j4].w};
-                        const float qv[4] = {qx[j4].x, qx[j4].y, qx[j4].z, qx[j4].w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int j = 16 * hf + 4 * j4 + e;
-                            put_split(tile(0), tile(1), t, j, kv[e]);
-                            put_split(tile(2), tile(3), t, j, __fmul_rn(gi, qv[e]));
-                        }
+                        const int j = 16 * hf + 4 * j4;
+                        put_split4(tile(0), tile(1), t, j, kx[j4]);
+                        put_split4(tile(2), tile(3), t, j, mul4(gi, qx[j4]));
+                        put_split4(tile(4), tile(5), t, j, make_float4(xr[j], xr[j + 1], xr[j + 2], xr[j + 3]));
                     }
-                    const float *xr = XS + t * kXStride + 32 * ks;
-#pragma unroll 8
-                    for (int j = 16 * hf; j < 16 * hf + 16; ++j) put_split(tile(4), tile(5), t, j, xr[j]);
                 }
                 fence_proxy_async_smem();
                 tc::fence_before_sync();
@@ -313,10 +317,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const DevForm
                     float x[32];
                     tc::ld32(lane_addr + RG + 64 * sb + c0, x);
 #pragma unroll
-                    for (int jj = 0; jj < 32; ++jj) {
-                        const int j = 64 * sb + c0 + jj;
-                        const float a = __fmul_rn(bi, __fmul_rn(__fmul_rn(gi, M.igam[j]), x[jj]));
-                        arow[c0 + jj] = j < t ? a : 0.f;
+                    for (int u = 0; u < 8; ++u) {
+                        float a[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int j = 64 * sb + c0 + 4 * u + e;
+                            const float v = __fmul_rn(bi, __fmul_rn(__fmul_rn(gi, M.igam[j]), x[4 * u + e]));
+                            a[e] = j < t ? v : 0.f;
+                        }
+                        *reinterpret_cast<float4 *>(arow + c0 + 4 * u) = make_float4(a[0], a[1], a[2], a[3]);
                     }
                 }
                 __syncthreads();
@@ -367,8 +376,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const DevForm
 #pragma unroll
                     for (int kb = 0; kb < 2; ++kb) {
 #pragma unroll
-                        for (int jj = 0; jj < 32; ++jj)
-                            put_split(tile(2 * kb), tile(2 * kb + 1), t, jj, e[32 * kb + jj]);
+                        for (int u = 0; u < 8; ++u) {
+                            const int j = 32 * kb + 4 * u;
+                            put_split4(tile(2 * kb), tile(2 * kb + 1), t, 4 * u,
+                                       make_float4(e[j], e[j + 1], e[j + 2], e[j + 3]));
+                        }
                     }
                 } else if (t >= 64) {
                     const float bi = M.bet[t], gi = M.gam[t];
@@ -378,11 +390,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const DevForm
                         float x[32];
                         tc::ld32(lane_addr + RG + 32 * kb, x);
 #pragma unroll
-                        for (int jj = 0; jj < 32; ++jj) {
-                            const int j = 32 * kb + jj;
-                            const float a = __fmul_rn(bi, __fmul_rn(__fmul_rn(gi, M.igam[j]), x[jj]));
-                            put_split(a21 + (2 * kb) * (tc::kTileBytes / 2), a21 + (2 * kb + 1) * (tc::kTileBytes / 2),
-                                      t - 64, jj, a);
+                        for (int u = 0; u < 8; ++u) {
+                            float a[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int j = 32 * kb + 4 * u + e;
+                                a[e] = __fmul_rn(bi, __fmul_rn(__fmul_rn(gi, M.igam[j]), x[4 * u + e]));
+                            }
+                            put_split4(a21 + (2 * kb) * (tc::kTileBytes / 2), a21 + (2 * kb + 1) * (tc::kTileBytes / 2),
+                                       t - 64, 4 * u, make_float4(a[0], a[1], a[2], a[3]));
                         }
                     }
                 }
@@ -440,18 +456,29 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const DevForm
                     float x[16];
                     tc::ld16(lane_addr + RY + 32 * js + c0, x);
 #pragma unroll
-                    for (int jj = 0; jj < 16; ++jj) put_split(tile(0), tile(1), t, c0 + jj, x[jj]);
+                    for (int u = 0; u < 4; ++u)
+                        put_split4(tile(0), tile(1), t, c0 + 4 * u,
+                                   make_float4(x[4 * u], x[4 * u + 1], x[4 * u + 2], x[4 * u + 3]));
                     // P~ row i (thread i): P'_ij / gam_j for j <= i, else 0
                     tc::ld16(lane_addr + RP + 32 * js + c0, x);
 #pragma unroll
-                    for (int jj = 0; jj < 16; ++jj) {
-                        const int j = 32 * js + c0 + jj;
-                        put_split(tile(2), tile(3), t, c0 + jj, j <= t ? __fmul_rn(x[jj], M.igam[j]) : 0.f);
+                    for (int u = 0; u < 4; ++u) {
+                        float pv[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int j = 32 * js + c0 + 4 * u + e;
+                            pv[e] = j <= t ? __fmul_rn(x[4 * u + e], M.igam[j]) : 0.f;
+                        }
+                        put_split4(tile(2), tile(3), t, c0 + 4 * u, make_float4(pv[0], pv[1], pv[2], pv[3]));
                     }
                     // K~^T row kappa (thread kappa): k_j[kappa] gam_n / gam_j
 #pragma unroll
-                    for (int jj = 0; jj < 16; ++jj)
-                        put_split(tile(4), tile(5), t, c0 + jj, __fmul_rn(kk[jj], M.kts[32 * js + c0 + jj]));
+                    for (int u = 0; u < 4; ++u) {
+                        const float *kt = M.kts + 32 * js + c0 + 4 * u;
+                        put_split4(tile(4), tile(5), t, c0 + 4 * u,
+                                   make_float4(__fmul_rn(kk[4 * u], kt[0]), __fmul_rn(kk[4 * u + 1], kt[1]),
+                                               __fmul_rn(kk[4 * u + 2], kt[2]), __fmul_rn(kk[4 * u + 3], kt[3])));
+                    }
                 }
                 fence_proxy_async_smem();
                 tc::fence_before_sync();
