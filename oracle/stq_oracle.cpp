@@ -918,13 +918,24 @@ extern "C" int orc_prefill_chunked_f64(const orc_format *f, const orc_page *page
         const int n = std::min(C, L - t0);
         /* cumulative decay of the chunk's tokens per key channel: gam[i][c] =
          * prod of the gates of tokens t0 .. t0 + i */
+        auto gate = [&](int i, int c) {
+            return (double)alpha[(size_t)(t0 + i) * na + (f->gate_vector ? c : 0)];
+        };
         std::vector<double> gam((size_t)n * d_k);
         for (int i = 0; i < n; ++i)
+            for (int c = 0; c < d_k; ++c)
+                gam[(size_t)i * d_k + c] = (i == 0 ? 1.0 : gam[(size_t)(i - 1) * d_k + c]) * gate(i, c);
+        /* the decay from token j to token i (j <= i), gam_i / gam_j, taken as
+         * the product of the gates of tokens j + 1 .. i (1 for j = i): defined
+         * where a gate is zero or the cumulative decay vanishes */
+        std::vector<double> rho((size_t)n * n * d_k);
+        auto R = [&](int i, int j, int c) -> double & { return rho[((size_t)i * n + j) * d_k + c]; };
+        for (int i = 0; i < n; ++i)
             for (int c = 0; c < d_k; ++c) {
-                const double a = (double)alpha[(size_t)(t0 + i) * na + (f->gate_vector ? c : 0)];
-                gam[(size_t)i * d_k + c] = (i == 0 ? 1.0 : gam[(size_t)(i - 1) * d_k + c]) * a;
+                R(i, i, c) = 1.0;
+                for (int j = i - 1; j >= 0; --j) R(i, j, c) = R(i, j + 1, c) * gate(j + 1, c);
             }
-        /* A[i][j] (j < i) = beta_i sum_c k_ic k_jc gam_ic / gam_jc;
+        /* A[i][j] (j < i) = beta_i sum_c k_ic k_jc rho_ijc;
          * E = (I + A)^-1 R, R_i = beta_i (v_i - (gam_i k_i)^T S0), by forward
          * substitution: E_i = R_i - sum_{j<i} A_ij E_j */
         std::vector<double> E((size_t)n * d_v);
@@ -940,12 +951,12 @@ extern "C" int orc_prefill_chunked_f64(const orc_format *f, const orc_page *page
                 const float *kj = k + (size_t)(t0 + jt) * d_k;
                 double a = 0.0;
                 for (int c = 0; c < d_k; ++c)
-                    a += (double)ki[c] * (double)kj[c] * (gam[(size_t)i * d_k + c] / gam[(size_t)jt * d_k + c]);
+                    a += (double)ki[c] * (double)kj[c] * R(i, jt, c);
                 a *= bi;
                 for (int j = 0; j < d_v; ++j) E[(size_t)i * d_v + j] -= a * E[(size_t)jt * d_v + j];
             }
         }
-        /* o_i = (gam_i q_i)^T S0 + sum_{j<=i} (sum_c q_ic k_jc gam_ic / gam_jc) E_j */
+        /* o_i = (gam_i q_i)^T S0 + sum_{j<=i} (sum_c q_ic k_jc rho_ijc) E_j */
         for (int i = 0; i < n; ++i) {
             const float *qi = q + (size_t)(t0 + i) * d_k;
             double *oi = o_out + (size_t)(t0 + i) * d_v;
@@ -958,17 +969,17 @@ extern "C" int orc_prefill_chunked_f64(const orc_format *f, const orc_page *page
                 const float *kj = k + (size_t)(t0 + jt) * d_k;
                 double pw = 0.0;
                 for (int c = 0; c < d_k; ++c)
-                    pw += (double)qi[c] * (double)kj[c] * (gam[(size_t)i * d_k + c] / gam[(size_t)jt * d_k + c]);
+                    pw += (double)qi[c] * (double)kj[c] * R(i, jt, c);
                 for (int j = 0; j < d_v; ++j) oi[j] += pw * E[(size_t)jt * d_v + j];
             }
         }
-        /* S <- diag(gam_n) S0 + sum_j (gam_n / gam_j k_j) E_j^T */
+        /* S <- diag(gam_n) S0 + sum_j (rho_nj k_j) E_j^T */
         for (int c = 0; c < d_k; ++c) {
             const double gn = gam[(size_t)(n - 1) * d_k + c];
             for (int j = 0; j < d_v; ++j) {
                 double acc = gn * S[(size_t)c * d_v + j];
                 for (int jt = 0; jt < n; ++jt)
-                    acc += (gn / gam[(size_t)jt * d_k + c]) * (double)k[(size_t)(t0 + jt) * d_k + c]
+                    acc += R(n - 1, jt, c) * (double)k[(size_t)(t0 + jt) * d_k + c]
                            * E[(size_t)jt * d_v + j];
                 S[(size_t)c * d_v + j] = acc;
             }

@@ -235,12 +235,14 @@ int orc_prefill_f32_plain(const orc_format *f, orc_page *page, const int32_t *pe
  * The same L tokens as orc_prefill_f32, from the page's dequantized state,
  * in chunks of C tokens (the form a tensor-core prefill computes; repeated
  * prefill: DASC card page).  Within a chunk of n tokens from state S0, with
- * gam_i = prod of the gates of the chunk's tokens up to i (per key channel):
- *   A_ij = beta_i sum_c k_ic k_jc gam_ic / gam_jc          (j < i)
+ * gam_i = prod of the gates of the chunk's tokens up to i (per key channel)
+ * and rho_ij = gam_i / gam_j, evaluated as the product of the gates of tokens
+ * j + 1 .. i (so defined where a gate is zero or gam vanishes):
+ *   A_ij = beta_i sum_c k_ic k_jc rho_ijc                  (j < i)
  *   E    = (I + A)^-1 R,  R_i = beta_i (v_i - (gam_i k_i)^T S0)
  *          (forward substitution: E_i = R_i - sum_{j<i} A_ij E_j)
- *   o_i  = (gam_i q_i)^T S0 + sum_{j<=i} (sum_c q_ic k_jc gam_ic / gam_jc) E_j
- *   S    = diag(gam_n) S0 + sum_j (gam_n / gam_j k_j) E_j^T;
+ *   o_i  = (gam_i q_i)^T S0 + sum_{j<=i} (sum_c q_ic k_jc rho_ijc) E_j
+ *   S    = diag(gam_n) S0 + sum_j (rho_nj k_j) E_j^T;
  * E_i is the step's delta beta_i (v_i - S_{i-1}^T k_i) after the decay, so
  * the chunk reproduces the token recurrence exactly in exact arithmetic.
  * q, k: [L][d_k]; v: [L][d_v]; alpha: [L][d_k] or [L]; beta: [L];

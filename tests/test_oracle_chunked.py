@@ -76,3 +76,24 @@ def test_chunked_f64_and_the_f32_prefill_agree(name):
     S32 = np.zeros_like(Sc)
     S32[perm] = tp.astype(np.float64) * c
     assert _rel_l2(S32, Sc) <= 1e-5
+
+
+@pytest.mark.parametrize("name", ["stepquant6", "stepquant4_kda"])
+def test_zero_and_vanishing_gates(name):
+    """Gates of zero, and runs of small gates whose cumulative product leaves
+    the double range within a chunk (0.002^128 ~ 1e-345), still give the
+    recurrence: the decay between two tokens is a product of gates, never a
+    quotient of cumulative decays."""
+    w, fmt, perm, page = _workload(name)
+    L, C = 200, 128
+    q, k, v, alpha, beta = _prompt(w, 17, L)
+    alpha = alpha.copy()
+    alpha[5] = 0.0                      # one token forgets everything
+    alpha[20:150] = 0.002               # the cumulative decay underflows double
+    if alpha.shape[1] > 1:
+        alpha[60, ::3] = 0.0            # KDA: some channels only
+    o64, S64 = _evolve64(_dequant64(fmt, page, perm), q, k, v, alpha, beta)
+    oc, Sc = O.prefill_chunked_f64(fmt, page, perm, q, k, v, alpha, beta, C)
+    assert np.all(np.isfinite(oc)) and np.all(np.isfinite(Sc))
+    assert _rel_l2(oc, o64) <= 1e-12, _rel_l2(oc, o64)
+    assert _rel_l2(Sc, S64) <= 1e-12, _rel_l2(Sc, S64)

@@ -95,9 +95,10 @@ MUTANTS = {
     "fit codes truncate": ("double n = (d > 0.0) ? std::nearbyint((double)S_row[j] / d) : 0.0;",
                            "double n = (d > 0.0) ? std::trunc((double)S_row[j] / d) : 0.0;"),
     "chunk A without beta": ("                a *= bi;\n", "                a *= 1.0;\n"),
-    "chunk decay ratio inverted": (
-        "a += (double)ki[c] * (double)kj[c] * (gam[(size_t)i * d_k + c] / gam[(size_t)jt * d_k + c]);",
-        "a += (double)ki[c] * (double)kj[c] * (gam[(size_t)jt * d_k + c] / gam[(size_t)i * d_k + c]);"),
+    "chunk decay from the wrong token": ("R(i, j, c) = R(i, j + 1, c) * gate(j + 1, c);",
+                                         "R(i, j, c) = R(i, j + 1, c) * gate(j, c);"),
+    "chunk A without the decay": ("a += (double)ki[c] * (double)kj[c] * R(i, jt, c);",
+                                  "a += (double)ki[c] * (double)kj[c];"),
     "chunk readout skips the diagonal": ("for (int jt = 0; jt <= i; ++jt) {\n                const float *kj = k + (size_t)(t0 + jt) * d_k;\n                double pw",
                                          "for (int jt = 0; jt < i; ++jt) {\n                const float *kj = k + (size_t)(t0 + jt) * d_k;\n                double pw"),
     "chunk state keeps the old state undecayed": ("double acc = gn * S[(size_t)c * d_v + j];",
