@@ -6,10 +6,12 @@
 // Per chunk of n <= 128 tokens from the state S0 (T = S / c units, key rows
 // in natural order), with gam_i = prod of the gates of tokens 0..i of the
 // chunk (the UT-transform form of the delta rule, "repeated prefill": DASC):
-//   G  = K K^T,  A_ij = beta_i (gam_i / gam_j) G_ij  (j < i)
+//   G  = K K^T,  A_ij = beta_i rho_ij G_ij  (j < i)
 //   E  = (I + A)^-1 R,  R_i = beta_i (v_i / c - gam_i (S0^T k_i))
-//   o_i = c (gam_i S0^T q_i + sum_{j<=i} (gam_i / gam_j) (q_i . k_j) E_j)
-//   S  <- gam_n S0 + sum_j (gam_n / gam_j) k_j E_j^T
+//   o_i = c (gam_i S0^T q_i + sum_{j<=i} rho_ij (q_i . k_j) E_j)
+//   S  <- gam_n S0 + sum_j rho_nj k_j E_j^T
+// where rho_ij = gam_i / gam_j is formed as the product of the gates of
+// tokens j + 1 .. i (defined for zero gates and vanishing decays).
 // The products run on the tensor cores in tf32 with each fp32 operand split
 // into a tf32 part and its remainder (three MMAs per product: hi hi, hi lo,
 // lo hi), which keeps fp32-level accuracy; the triangular solve runs on the
@@ -25,7 +27,8 @@
 //   swizzled, K-major), reused as the solve's matrix A and as the page
 //   buffer; the state X = S^T (X[v][kappa], fp32, rows padded to 129
 //   floats); per-token scalars.
-//   tensor memory: G | Y^T = S0^T K^T | P' = (gam Q) K^T | O^T, then the
+//   tensor memory: G | Y^T = S0^T K^T | P = Q K^T | O^T (X Q^T, its column
+//   i then scaled by gam_i), then the
 //   state's increment in G's columns.
 #include "stq_rows.cuh"
 #include "stq_tc.cuh"
@@ -54,21 +57,30 @@ struct TcArgs {
 
 struct TcSmall {
     float gam[kChunk];       // cumulative gate of the chunk's tokens
-    float igam[kChunk];      // 1 / gam
+    float al[kChunk];        // the gate of each token (1 for padding)
     float bet[kChunk];       // beta (0 for padding)
-    float kts[kChunk];       // gam_n / gam_j: a key's decay to the chunk's end
+    float kts[kChunk];       // a key's decay to the chunk's end: the gates of tokens j + 1 .. n - 1
+    float igam[kChunk];      // 1 / gam (chunks whose decays stay in range)
     float c[kD], ic[kD];     // column scale and its inverse
-    float inv[kWarps][kRowsPerWarp];
+    alignas(16) float inv[kWarps][kRowsPerWarp];   // read as float4
     int kap[kD];             // stored row -> key channel
     uint64_t mma_bar, page_bar, never;
     uint32_t tmem;
+    int quot;                // this chunk's decays may be taken as gam_i / gam_j
 };
 
+static_assert(offsetof(TcSmall, inv) % 16 == 0, "inv is read as float4");
+static_assert(offsetof(TcSmall, mma_bar) % 8 == 0, "mbarriers are 8-byte aligned");
+static_assert((kTileRegion + (size_t)kD * kXStride * 4) % alignof(TcSmall) == 0, "TcSmall follows X aligned");
 constexpr size_t kTcSmem = kTileRegion + (size_t)kD * kXStride * 4 + sizeof(TcSmall) + 1024;
 
 // four consecutive columns k .. k + 3 (k a multiple of 4) of a row: one
 // 16-byte unit of the swizzled row, so a warp's 32 rows take 4 conflict-free
 // shared-memory wavefronts (a float at a time, 8 banks serve the 32 rows)
+__device__ __forceinline__ float4 mul4(float a, float4 x) {
+    return make_float4(__fmul_rn(a, x.x), __fmul_rn(a, x.y), __fmul_rn(a, x.z), __fmul_rn(a, x.w));
+}
+
 __device__ __forceinline__ void put_split4(uint8_t *hi_tile, uint8_t *lo_tile, uint32_t row, uint32_t k, float4 x) {
     float4 h, l;
     tc::split_tf32(x.x, h.x, l.x);
@@ -78,10 +90,6 @@ __device__ __forceinline__ void put_split4(uint8_t *hi_tile, uint8_t *lo_tile, u
     const uint32_t off = tc::sw128_offset(row, k);
     *reinterpret_cast<float4 *>(hi_tile + off) = h;
     *reinterpret_cast<float4 *>(lo_tile + off) = l;
-}
-
-__device__ __forceinline__ float4 mul4(float a, float4 x) {
-    return make_float4(__fmul_rn(a, x.x), __fmul_rn(a, x.y), __fmul_rn(a, x.z), __fmul_rn(a, x.w));
 }
 
 // D (+)= A B^T over one 32-wide K slab, split operands: hi hi, hi lo, lo hi
@@ -219,308 +227,396 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const DevForm
                 const bool real = tid < cn;
                 const size_t row = (size_t)(t0 + tid) * n + p;
                 M.bet[tid] = real ? A.beta[row] : 0.f;
-                M.gam[tid] = real ? A.alpha[row] : 1.f;    // the gate; made cumulative below
+                M.al[tid] = real ? A.alpha[row] : 1.f;
             }
             __syncthreads();
+            // The decay from token j to token i is gam_i / gam_j.  While every
+            // cumulative decay of the chunk lies in [2^-100, 2^100] it is taken
+            // as gam_i (1 / gam_j), with gam_i folded into q; otherwise (a zero
+            // gate, or a decay that leaves the float range inside the chunk) as
+            // the product of the gates of tokens j + 1 .. i, which is always
+            // defined.  The flag is the same for the whole CTA.
             if (tid == 0) {
                 float g = 1.f;
+                bool in_range = true;   // a NaN fails the test as well
                 for (int i = 0; i < kChunk; ++i) {
-                    g = __fmul_rn(g, M.gam[i]);
+                    g = __fmul_rn(g, M.al[i]);
                     M.gam[i] = g;
+                    in_range = in_range && g >= 0x1p-100f && g <= 0x1p100f;
                 }
+                M.quot = in_range ? 1 : 0;
             }
             __syncthreads();
-            if (tid < kChunk) {
-                const float gi = M.gam[tid];
-                M.igam[tid] = __frcp_rn(gi);
-                M.kts[tid] = __fdiv_rn(M.gam[kChunk - 1], gi);
-            }
-            __syncthreads();
-
-            // ---- phase A: G = K K^T, Y^T = X K^T, P' = (gam Q) K^T, O^T = X (gam Q)^T
-            // row t of the K and Q slabs, columns 16 hf .. + 15: the next slab's
-            // are loaded while the tensor cores work on this one
-            float4 kx[4], qx[4];
-            auto load_kq = [&](int ks) {
-                const bool real = t < cn;
-                const size_t row = ((size_t)(t0 + t) * n + p) * kD + 32 * ks + 16 * hf;
-#pragma unroll
-                for (int j4 = 0; j4 < 4; ++j4) {
-                    kx[j4] = qx[j4] = make_float4(0.f, 0.f, 0.f, 0.f);
-                    if (real) {
-                        kx[j4] = __ldg(reinterpret_cast<const float4 *>(A.k + row) + j4);
-                        qx[j4] = __ldg(reinterpret_cast<const float4 *>(A.q + row) + j4);
+            // the rest of the chunk, compiled once for each way of taking the
+            // decays, so that each runs as one contiguous stretch of code
+            auto chunk_body = [&](auto qc) {
+                constexpr bool quot = decltype(qc)::value != 0;
+                if (quot) {
+                    if (tid < kChunk) {
+                        const float gi = M.gam[tid];
+                        M.igam[tid] = __frcp_rn(gi);
+                        M.kts[tid] = __fdiv_rn(M.gam[kChunk - 1], gi);
+                    }
+                } else if (tid == 32) {
+                    float g = 1.f;
+                    M.kts[kChunk - 1] = g;
+                    for (int j = kChunk - 2; j >= 0; --j) {
+                        g = __fmul_rn(g, M.al[j + 1]);
+                        M.kts[j] = g;
                     }
                 }
-            };
-            load_kq(0);
-            for (int ks = 0; ks < kD / 32; ++ks) {
-                {
-                    // row t of the K, gam Q and X slabs, columns 16 hf .. + 15
-                    const float gi = M.gam[t];
-                    const float *xr = XS + t * kXStride + 32 * ks;
+                __syncthreads();
+
+                // ---- phase A: G = K K^T, Y^T = X K^T, P = (gam Q) K^T and
+                // O^T = X (gam Q)^T (gam = 1 here for a chunk of products)
+                // row t of the K and Q slabs, columns 16 hf .. + 15: the next slab's
+                // are loaded while the tensor cores work on this one
+                float4 kx[4], qx[4];
+                auto load_kq = [&](int ks) {
+                    const bool real = t < cn;
+                    const size_t row = ((size_t)(t0 + t) * n + p) * kD + 32 * ks + 16 * hf;
 #pragma unroll
                     for (int j4 = 0; j4 < 4; ++j4) {
-                        const int j = 16 * hf + 4 * j4;
-                        put_split4(tile(0), tile(1), t, j, kx[j4]);
-                        put_split4(tile(2), tile(3), t, j, mul4(gi, qx[j4]));
-                        put_split4(tile(4), tile(5), t, j, make_float4(xr[j], xr[j + 1], xr[j + 2], xr[j + 3]));
-                    }
-                }
-                fence_proxy_async_smem();
-                tc::fence_before_sync();
-                __syncthreads();
-                tc::fence_after_sync();
-                if (tid == 0) {
-                    const bool acc = ks > 0;
-                    mma_split(tmem + RG, tile_addr(0), tile_addr(1), tile_addr(0), tile_addr(1), acc);
-                    mma_split(tmem + RY, tile_addr(4), tile_addr(5), tile_addr(0), tile_addr(1), acc);
-                    mma_split(tmem + RP, tile_addr(2), tile_addr(3), tile_addr(0), tile_addr(1), acc);
-                    mma_split(tmem + RO, tile_addr(4), tile_addr(5), tile_addr(2), tile_addr(3), acc);
-                    tc::commit(&M.mma_bar);
-                }
-                if (ks + 1 < kD / 32) load_kq(ks + 1);
-                if (__syncthreads_or(!wait_mma())) { failed = true; break; }
-            }
-            if (failed) break;
-
-            // ---- phase B: R from Y^T in place (thread v), then the solve
-            // (I + A) E = R in two halves of 64 tokens: each half by forward
-            // substitution with thread v holding column v of the half in
-            // registers; between them the off-diagonal block, R2 -= A21 E1,
-            // as a tensor-core product.  E^T ends up in Y^T's columns.
-            {
-                // column t of R, tokens 64 hf .. + 63
-                const float icv = M.ic[t];
-                const uint32_t ry = lane_addr + RY;
-#pragma unroll
-                for (int c0 = 64 * hf; c0 < 64 * hf + 64; c0 += 32) {
-                    float x[32];
-                    tc::ld32(ry + c0, x);
-#pragma unroll
-                    for (int jj = 0; jj < 32; ++jj) {
-                        const int i = c0 + jj;
-                        const float vv = (i < cn) ? __ldg(A.v + ((size_t)(t0 + i) * n + p) * kD + t) : 0.f;
-                        // R_i = beta_i (v_i / c - gam_i y_i)
-                        x[jj] = __fmul_rn(M.bet[i], __fsub_rn(__fmul_rn(vv, icv), __fmul_rn(M.gam[i], x[jj])));
-                    }
-                    tc::st32(ry + c0, x);
-                }
-            }
-            for (int sb = 0; sb < 2; ++sb) {
-                // the diagonal block of this half: A_ij, i, j in [64 sb, 64 sb + 64)
-                // (row t, columns 32 hf .. + 31 of the block)
-                if (t >= 64 * sb && t < 64 * sb + 64) {
-                    const float bi = M.bet[t], gi = M.gam[t];
-                    float *arow = Amat + (t - 64 * sb) * kAStride;
-                    const int c0 = 32 * hf;
-                    float x[32];
-                    tc::ld32(lane_addr + RG + 64 * sb + c0, x);
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        float a[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int j = 64 * sb + c0 + 4 * u + e;
-                            const float v = __fmul_rn(bi, __fmul_rn(__fmul_rn(gi, M.igam[j]), x[4 * u + e]));
-                            a[e] = j < t ? v : 0.f;
+                        kx[j4] = qx[j4] = make_float4(0.f, 0.f, 0.f, 0.f);
+                        if (real) {
+                            kx[j4] = __ldg(reinterpret_cast<const float4 *>(A.k + row) + j4);
+                            qx[j4] = __ldg(reinterpret_cast<const float4 *>(A.q + row) + j4);
                         }
-                        *reinterpret_cast<float4 *>(arow + c0 + 4 * u) = make_float4(a[0], a[1], a[2], a[3]);
                     }
-                }
-                __syncthreads();
-                float e[64];   // the first half's threads: column t of this half of E
-                if (hf == 0) {
+                };
+                load_kq(0);
+                for (int ks = 0; ks < kD / 32; ++ks) {
                     {
-                        float x[32];
-                        tc::ld32(lane_addr + RY + 64 * sb, x);
+                        // row t of the K, gam Q and X slabs, columns 16 hf .. + 15
+                        const float gi = quot ? M.gam[t] : 1.f;
+                        const float *xr = XS + t * kXStride + 32 * ks;
 #pragma unroll
-                        for (int jj = 0; jj < 32; ++jj) e[jj] = x[jj];
-                        tc::ld32(lane_addr + RY + 64 * sb + 32, x);
-#pragma unroll
-                        for (int jj = 0; jj < 32; ++jj) e[32 + jj] = x[jj];
-                    }
-                    // forward substitution: E_i = R_i - sum_{j<i} A_ij E_j
-#pragma unroll
-                    for (int i = 1; i < 64; ++i) {
-                        const float *arow = Amat + i * kAStride;
-                        float acc = e[i];
-#pragma unroll
-                        for (int j4 = 0; j4 < (i + 3) / 4; ++j4) {
-                            const float4 a4 = *reinterpret_cast<const float4 *>(arow + 4 * j4);
-                            const float av[4] = {a4.x, a4.y, a4.z, a4.w};
-#pragma unroll
-                            for (int jj = 0; jj < 4; ++jj)
-                                if (4 * j4 + jj < i) acc = __fmaf_rn(-av[jj], e[4 * j4 + jj], acc);
+                        for (int j4 = 0; j4 < 4; ++j4) {
+                            const int j = 16 * hf + 4 * j4;
+                            put_split4(tile(0), tile(1), t, j, kx[j4]);
+                            put_split4(tile(2), tile(3), t, j, quot ? mul4(gi, qx[j4]) : qx[j4]);
+                            put_split4(tile(4), tile(5), t, j, make_float4(xr[j], xr[j + 1], xr[j + 2], xr[j + 3]));
                         }
-                        e[i] = acc;
                     }
-                    {
-                        float x[32];
-#pragma unroll
-                        for (int jj = 0; jj < 32; ++jj) x[jj] = e[jj];
-                        tc::st32(lane_addr + RY + 64 * sb, x);
-#pragma unroll
-                        for (int jj = 0; jj < 32; ++jj) x[jj] = e[32 + jj];
-                        tc::st32(lane_addr + RY + 64 * sb + 32, x);
+                    fence_proxy_async_smem();
+                    tc::fence_before_sync();
+                    __syncthreads();
+                    tc::fence_after_sync();
+                    if (tid == 0) {
+                        const bool acc = ks > 0;
+                        mma_split(tmem + RG, tile_addr(0), tile_addr(1), tile_addr(0), tile_addr(1), acc);
+                        mma_split(tmem + RY, tile_addr(4), tile_addr(5), tile_addr(0), tile_addr(1), acc);
+                        mma_split(tmem + RP, tile_addr(2), tile_addr(3), tile_addr(0), tile_addr(1), acc);
+                        mma_split(tmem + RO, tile_addr(4), tile_addr(5), tile_addr(2), tile_addr(3), acc);
+                        tc::commit(&M.mma_bar);
                     }
+                    if (ks + 1 < kD / 32) load_kq(ks + 1);
+                    if (__syncthreads_or(!wait_mma())) { failed = true; break; }
                 }
-                if (sb == 1) break;
-                __syncthreads();   // the diagonal block's space becomes operand tiles
-                // R2 -= A21 E1 on the tensor cores: D = R2^T (columns 64..127 of
-                // Y^T) += (-E1^T) A21^T, M = 128 (v), N = 64 (i), K = 64 (j).
-                // Tiles: E1^T hi / lo (rows v, two K slabs) at 0 .. 64 KB, written
-                // by the first half from its columns of E; A21 hi / lo (rows
-                // i - 64, 64-row tiles of 8 KB) at 64 .. 96 KB, by the second.
-                if (hf == 0) {
-#pragma unroll
-                    for (int kb = 0; kb < 2; ++kb) {
-#pragma unroll
-                        for (int u = 0; u < 8; ++u) {
-                            const int j = 32 * kb + 4 * u;
-                            put_split4(tile(2 * kb), tile(2 * kb + 1), t, 4 * u,
-                                       make_float4(e[j], e[j + 1], e[j + 2], e[j + 3]));
-                        }
-                    }
-                } else if (t >= 64) {
-                    const float bi = M.bet[t], gi = M.gam[t];
-                    uint8_t *a21 = tiles + 4 * tc::kTileBytes;
-#pragma unroll
-                    for (int kb = 0; kb < 2; ++kb) {
-                        float x[32];
-                        tc::ld32(lane_addr + RG + 32 * kb, x);
-#pragma unroll
-                        for (int u = 0; u < 8; ++u) {
-                            float a[4];
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const int j = 32 * kb + 4 * u + e;
-                                a[e] = __fmul_rn(bi, __fmul_rn(__fmul_rn(gi, M.igam[j]), x[4 * u + e]));
-                            }
-                            put_split4(a21 + (2 * kb) * (tc::kTileBytes / 2), a21 + (2 * kb + 1) * (tc::kTileBytes / 2),
-                                       t - 64, 4 * u, make_float4(a[0], a[1], a[2], a[3]));
-                        }
-                    }
-                }
-                fence_proxy_async_smem();
-                tc::fence_before_sync();
-                __syncthreads();
-                tc::fence_after_sync();
-                if (tid == 0) {
-                    const uint32_t idesc = tc::idesc_tf32(128, 64, true);
-                    const uint32_t a21 = tile_addr(4);
-#pragma unroll
-                    for (int kb = 0; kb < 2; ++kb) {
-                        const uint32_t e_hi = tile_addr(2 * kb), e_lo = tile_addr(2 * kb + 1);
-                        const uint32_t b_hi = a21 + (2 * kb) * (tc::kTileBytes / 2);
-                        const uint32_t b_lo = a21 + (2 * kb + 1) * (tc::kTileBytes / 2);
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk) {
-                            const uint32_t off = 32u * kk;
-                            tc::mma_tf32(tmem + RY + 64, tc::desc_k_sw128(e_hi + off), tc::desc_k_sw128(b_hi + off),
-                                         idesc, true);
-                            tc::mma_tf32(tmem + RY + 64, tc::desc_k_sw128(e_hi + off), tc::desc_k_sw128(b_lo + off),
-                                         idesc, true);
-                            tc::mma_tf32(tmem + RY + 64, tc::desc_k_sw128(e_lo + off), tc::desc_k_sw128(b_hi + off),
-                                         idesc, true);
-                        }
-                    }
-                    tc::commit(&M.mma_bar);
-                }
-                if (__syncthreads_or(!wait_mma())) { failed = true; break; }
-            }
-            if (failed) break;
-            // the solve's space becomes operand tiles again; E^T (stored by the
-            // first half) is read by both halves
-            tc::fence_before_sync();
-            __syncthreads();
-            tc::fence_after_sync();
+                if (failed) return;
 
-            // ---- phase C: O^T += E^T P~^T, dX = E^T K~ (K = tokens)
-            // key channel t of tokens 32 js + 16 hf .. + 15, the next slab's
-            // loaded while the tensor cores work on this one
-            float kk[16];
-            auto load_kt = [&](int js) {
-#pragma unroll
-                for (int jj = 0; jj < 16; ++jj) {
-                    const int j = 32 * js + 16 * hf + jj;
-                    kk[jj] = (j < cn) ? __ldg(A.k + ((size_t)(t0 + j) * n + p) * kD + t) : 0.f;
-                }
-            };
-            load_kt(0);
-            for (int js = 0; js < kChunk / 32; ++js) {
+                // ---- phase B: R from Y^T in place (thread v), then the solve
+                // (I + A) E = R in two halves of 64 tokens: each half by forward
+                // substitution with thread v holding column v of the half in
+                // registers; between them the off-diagonal block, R2 -= A21 E1,
+                // as a tensor-core product.  E^T ends up in Y^T's columns.
                 {
-                    // columns 16 hf .. + 15 of the slab
-                    const int c0 = 16 * hf;
-                    // E^T row v (thread v), from Y^T's columns
-                    float x[16];
-                    tc::ld16(lane_addr + RY + 32 * js + c0, x);
+                    // column t of R, tokens 64 hf .. + 63; in a chunk of products
+                    // the same columns of O^T get their token's decay (o_i's first
+                    // part is gam_i S0^T q_i)
+                    const float icv = M.ic[t];
+                    const uint32_t ry = lane_addr + RY, ro = lane_addr + RO;
 #pragma unroll
-                    for (int u = 0; u < 4; ++u)
-                        put_split4(tile(0), tile(1), t, c0 + 4 * u,
-                                   make_float4(x[4 * u], x[4 * u + 1], x[4 * u + 2], x[4 * u + 3]));
-                    // P~ row i (thread i): P'_ij / gam_j for j <= i, else 0
-                    tc::ld16(lane_addr + RP + 32 * js + c0, x);
+                    for (int c0 = 64 * hf; c0 < 64 * hf + 64; c0 += 32) {
+                        float x[32];
+                        tc::ld32(ry + c0, x);
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        float pv[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int j = 32 * js + c0 + 4 * u + e;
-                            pv[e] = j <= t ? __fmul_rn(x[4 * u + e], M.igam[j]) : 0.f;
+                        for (int jj = 0; jj < 32; ++jj) {
+                            const int i = c0 + jj;
+                            const float vv = (i < cn) ? __ldg(A.v + ((size_t)(t0 + i) * n + p) * kD + t) : 0.f;
+                            // R_i = beta_i (v_i / c - gam_i y_i)
+                            x[jj] = __fmul_rn(M.bet[i], __fsub_rn(__fmul_rn(vv, icv), __fmul_rn(M.gam[i], x[jj])));
                         }
-                        put_split4(tile(2), tile(3), t, c0 + 4 * u, make_float4(pv[0], pv[1], pv[2], pv[3]));
-                    }
-                    // K~^T row kappa (thread kappa): k_j[kappa] gam_n / gam_j
+                        tc::st32(ry + c0, x);
+                        if (!quot) {
+                            tc::ld32(ro + c0, x);
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const float *kt = M.kts + 32 * js + c0 + 4 * u;
-                        put_split4(tile(4), tile(5), t, c0 + 4 * u,
-                                   make_float4(__fmul_rn(kk[4 * u], kt[0]), __fmul_rn(kk[4 * u + 1], kt[1]),
-                                               __fmul_rn(kk[4 * u + 2], kt[2]), __fmul_rn(kk[4 * u + 3], kt[3])));
+                            for (int jj = 0; jj < 32; ++jj) x[jj] = __fmul_rn(M.gam[c0 + jj], x[jj]);
+                            tc::st32(ro + c0, x);
+                        }
                     }
                 }
-                fence_proxy_async_smem();
+                for (int sb = 0; sb < 2; ++sb) {
+                    // the diagonal block of this half: A_ij, i, j in [64 sb, 64 sb + 64)
+                    // (row t, columns 32 hf .. + 31 of the block).  rho = the decay
+                    // from token j to t, walked down from j = t: rho_{t,j-1} =
+                    // rho_{t,j} al_j
+                    if (t >= 64 * sb && t < 64 * sb + 64) {
+                        const float bi = M.bet[t];
+                        float *arow = Amat + (t - 64 * sb) * kAStride;
+                        const int c0 = 32 * hf;
+                        const int jlo = 64 * sb + c0;
+                        float x[32];
+                        tc::ld32(lane_addr + RG + jlo, x);
+                        float a[32];
+                        if (quot) {
+                            const float gi = M.gam[t];
+#pragma unroll
+                            for (int jj = 0; jj < 32; ++jj) {
+                                const int j = jlo + jj;
+                                a[jj] = j < t ? __fmul_rn(bi, __fmul_rn(__fmul_rn(gi, M.igam[j]), x[jj])) : 0.f;
+                            }
+                        } else {
+                            float rho = 1.f;   // rho_{t, jlo+31} when t is above the columns: the gates jlo+32 .. t
+#pragma unroll
+                            for (int d = 0; d < 32; ++d)
+                                if (jlo + 32 + d <= t) rho = __fmul_rn(rho, M.al[jlo + 32 + d]);
+#pragma unroll
+                            for (int jj = 31; jj >= 0; --jj) {
+                                const int j = jlo + jj;
+                                a[jj] = j < t ? __fmul_rn(bi, __fmul_rn(rho, x[jj])) : 0.f;
+                                if (j <= t) rho = __fmul_rn(rho, M.al[j]);
+                            }
+                        }
+#pragma unroll
+                        for (int u = 0; u < 8; ++u)
+                            *reinterpret_cast<float4 *>(arow + c0 + 4 * u) =
+                                make_float4(a[4 * u], a[4 * u + 1], a[4 * u + 2], a[4 * u + 3]);
+                    }
+                    __syncthreads();
+                    float e[64];   // the first half's threads: column t of this half of E
+                    if (hf == 0) {
+                        {
+                            float x[32];
+                            tc::ld32(lane_addr + RY + 64 * sb, x);
+#pragma unroll
+                            for (int jj = 0; jj < 32; ++jj) e[jj] = x[jj];
+                            tc::ld32(lane_addr + RY + 64 * sb + 32, x);
+#pragma unroll
+                            for (int jj = 0; jj < 32; ++jj) e[32 + jj] = x[jj];
+                        }
+                        // forward substitution: E_i = R_i - sum_{j<i} A_ij E_j
+#pragma unroll
+                        for (int i = 1; i < 64; ++i) {
+                            const float *arow = Amat + i * kAStride;
+                            float acc = e[i];
+#pragma unroll
+                            for (int j4 = 0; j4 < (i + 3) / 4; ++j4) {
+                                const float4 a4 = *reinterpret_cast<const float4 *>(arow + 4 * j4);
+                                const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+                                for (int jj = 0; jj < 4; ++jj)
+                                    if (4 * j4 + jj < i) acc = __fmaf_rn(-av[jj], e[4 * j4 + jj], acc);
+                            }
+                            e[i] = acc;
+                        }
+                        {
+                            float x[32];
+#pragma unroll
+                            for (int jj = 0; jj < 32; ++jj) x[jj] = e[jj];
+                            tc::st32(lane_addr + RY + 64 * sb, x);
+#pragma unroll
+                            for (int jj = 0; jj < 32; ++jj) x[jj] = e[32 + jj];
+                            tc::st32(lane_addr + RY + 64 * sb + 32, x);
+                        }
+                    }
+                    if (sb == 1) break;
+                    __syncthreads();   // the diagonal block's space becomes operand tiles
+                    // R2 -= A21 E1 on the tensor cores: D = R2^T (columns 64..127 of
+                    // Y^T) += (-E1^T) A21^T, M = 128 (v), N = 64 (i), K = 64 (j).
+                    // Tiles: E1^T hi / lo (rows v, two K slabs) at 0 .. 64 KB, written
+                    // by the first half from its columns of E; A21 hi / lo (rows
+                    // i - 64, 64-row tiles of 8 KB) at 64 .. 96 KB, by the second.
+                    if (hf == 0) {
+#pragma unroll
+                        for (int kb = 0; kb < 2; ++kb) {
+#pragma unroll
+                            for (int u = 0; u < 8; ++u) {
+                                const int j = 32 * kb + 4 * u;
+                                put_split4(tile(2 * kb), tile(2 * kb + 1), t, 4 * u,
+                                           make_float4(e[j], e[j + 1], e[j + 2], e[j + 3]));
+                            }
+                        }
+                    } else if (t >= 64) {
+                        // rho walked down from j = t to the block's columns 63 .. 0
+                        const float bi = M.bet[t];
+                        uint8_t *a21 = tiles + 4 * tc::kTileBytes;
+                        const float gi = M.gam[t];
+                        float rho = 1.f;   // rho_{t, 63}: the gates 64 .. t
+                        if (!quot) {
+#pragma unroll
+                            for (int d = 0; d < 64; ++d)
+                                if (64 + d <= t) rho = __fmul_rn(rho, M.al[64 + d]);
+                        }
+#pragma unroll
+                        for (int kb = 1; kb >= 0; --kb) {
+                            float x[32];
+                            tc::ld32(lane_addr + RG + 32 * kb, x);
+                            float a[32];
+                            if (quot) {
+#pragma unroll
+                                for (int jj = 0; jj < 32; ++jj)
+                                    a[jj] = __fmul_rn(bi, __fmul_rn(__fmul_rn(gi, M.igam[32 * kb + jj]), x[jj]));
+                            } else {
+#pragma unroll
+                                for (int jj = 31; jj >= 0; --jj) {
+                                    const int j = 32 * kb + jj;
+                                    a[jj] = __fmul_rn(bi, __fmul_rn(rho, x[jj]));
+                                    rho = __fmul_rn(rho, M.al[j]);
+                                }
+                            }
+#pragma unroll
+                            for (int u = 0; u < 8; ++u)
+                                put_split4(a21 + (2 * kb) * (tc::kTileBytes / 2), a21 + (2 * kb + 1) * (tc::kTileBytes / 2),
+                                           t - 64, 4 * u, make_float4(a[4 * u], a[4 * u + 1], a[4 * u + 2], a[4 * u + 3]));
+                        }
+                    }
+                    fence_proxy_async_smem();
+                    tc::fence_before_sync();
+                    __syncthreads();
+                    tc::fence_after_sync();
+                    if (tid == 0) {
+                        const uint32_t idesc = tc::idesc_tf32(128, 64, true);
+                        const uint32_t a21 = tile_addr(4);
+#pragma unroll
+                        for (int kb = 0; kb < 2; ++kb) {
+                            const uint32_t e_hi = tile_addr(2 * kb), e_lo = tile_addr(2 * kb + 1);
+                            const uint32_t b_hi = a21 + (2 * kb) * (tc::kTileBytes / 2);
+                            const uint32_t b_lo = a21 + (2 * kb + 1) * (tc::kTileBytes / 2);
+#pragma unroll
+                            for (int kk = 0; kk < 4; ++kk) {
+                                const uint32_t off = 32u * kk;
+                                tc::mma_tf32(tmem + RY + 64, tc::desc_k_sw128(e_hi + off), tc::desc_k_sw128(b_hi + off),
+                                             idesc, true);
+                                tc::mma_tf32(tmem + RY + 64, tc::desc_k_sw128(e_hi + off), tc::desc_k_sw128(b_lo + off),
+                                             idesc, true);
+                                tc::mma_tf32(tmem + RY + 64, tc::desc_k_sw128(e_lo + off), tc::desc_k_sw128(b_hi + off),
+                                             idesc, true);
+                            }
+                        }
+                        tc::commit(&M.mma_bar);
+                    }
+                    if (__syncthreads_or(!wait_mma())) { failed = true; break; }
+                }
+                if (failed) return;
+                // the solve's space becomes operand tiles again; E^T (stored by the
+                // first half) is read by both halves
                 tc::fence_before_sync();
                 __syncthreads();
                 tc::fence_after_sync();
-                if (tid == 0) {
-                    mma_split(tmem + RO, tile_addr(0), tile_addr(1), tile_addr(2), tile_addr(3), true);
-                    mma_split(tmem + RG, tile_addr(0), tile_addr(1), tile_addr(4), tile_addr(5), js > 0);
-                    tc::commit(&M.mma_bar);
-                }
-                if (js + 1 < kChunk / 32) load_kt(js + 1);
-                if (__syncthreads_or(!wait_mma())) { failed = true; break; }
-            }
-            if (failed) break;
 
-            // ---- phase D: o of the chunk's tokens; X <- gam_n X + dX
-            {
-                // column t: tokens (o) and key channels (X) 64 hf .. + 63
-                const float cv = M.c[t];
+                // ---- phase C: O^T += E^T P~^T, dX = E^T K~ (K = tokens); in a
+                // chunk of products the token slabs go from the last to the first,
+                // so that each thread walks the decay rho_{t,j} down from j = t.
+                // k of key channel t, tokens 32 js + 16 hf .. + 15: the next
+                // slab's loaded while the tensor cores work on this one
+                float kk[16];
+                auto load_kt = [&](int js) {
 #pragma unroll
-                for (int c0 = 64 * hf; c0 < 64 * hf + 64; c0 += 32) {
-                    float x[32];
-                    tc::ld32(lane_addr + RO + c0, x);
+                    for (int jj = 0; jj < 16; ++jj) {
+                        const int j = 32 * js + 16 * hf + jj;
+                        kk[jj] = (j < cn) ? __ldg(A.k + ((size_t)(t0 + j) * n + p) * kD + t) : 0.f;
+                    }
+                };
+                // slab order: ascending for quotients, descending for products
+                constexpr int kSlabs = kChunk / 32;
+                auto slab = [&](int n_done) { return quot ? n_done : kSlabs - 1 - n_done; };
+                load_kt(slab(0));
+                float rho = 1.f;   // rho_{t, j} for the next j below the columns done
+                for (int sdone = 0; sdone < kSlabs; ++sdone) {
+                    const int js = slab(sdone);
+                    {
+                        // columns 16 hf .. + 15 of the slab
+                        const int c0 = 16 * hf;
+                        // E^T row v (thread v), from Y^T's columns
+                        float x[16];
+                        tc::ld16(lane_addr + RY + 32 * js + c0, x);
 #pragma unroll
-                    for (int jj = 0; jj < 32; ++jj) {
-                        const int i = c0 + jj;
-                        if (i < cn) A.o[((size_t)(t0 + i) * n + p) * kD + t] = __fmul_rn(cv, x[jj]);
+                        for (int u = 0; u < 4; ++u)
+                            put_split4(tile(0), tile(1), t, c0 + 4 * u,
+                                       make_float4(x[4 * u], x[4 * u + 1], x[4 * u + 2], x[4 * u + 3]));
+                        // P~ row i (thread i), j <= i (else 0): P_ij / gam_j, or in a
+                        // chunk of products rho_ij P_ij, rho running through the
+                        // other half's columns of the slab too
+                        tc::ld16(lane_addr + RP + 32 * js + c0, x);
+                        float pv[16];
+                        if (quot) {
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) {
+                                const int j = 32 * js + c0 + e;
+                                pv[e] = j <= t ? __fmul_rn(x[e], M.igam[j]) : 0.f;
+                            }
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) pv[e] = 0.f;
+#pragma unroll
+                            for (int part = 1; part >= 0; --part) {
+#pragma unroll
+                                for (int e = 15; e >= 0; --e) {
+                                    const int j = 32 * js + 16 * part + e;
+                                    if (part == hf && j <= t) pv[e] = __fmul_rn(rho, x[e]);
+                                    if (j <= t) rho = __fmul_rn(rho, M.al[j]);
+                                }
+                            }
+                        }
+#pragma unroll
+                        for (int u = 0; u < 4; ++u)
+                            put_split4(tile(2), tile(3), t, c0 + 4 * u,
+                                       make_float4(pv[4 * u], pv[4 * u + 1], pv[4 * u + 2], pv[4 * u + 3]));
+                        // K~^T row kappa (thread kappa): k_j[kappa] times the decay of
+                        // token j to the chunk's end
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const float *kt = M.kts + 32 * js + c0 + 4 * u;
+                            put_split4(tile(4), tile(5), t, c0 + 4 * u,
+                                       make_float4(__fmul_rn(kk[4 * u], kt[0]), __fmul_rn(kk[4 * u + 1], kt[1]),
+                                                   __fmul_rn(kk[4 * u + 2], kt[2]), __fmul_rn(kk[4 * u + 3], kt[3])));
+                        }
+                    }
+                    fence_proxy_async_smem();
+                    tc::fence_before_sync();
+                    __syncthreads();
+                    tc::fence_after_sync();
+                    if (tid == 0) {
+                        mma_split(tmem + RO, tile_addr(0), tile_addr(1), tile_addr(2), tile_addr(3), true);
+                        mma_split(tmem + RG, tile_addr(0), tile_addr(1), tile_addr(4), tile_addr(5), sdone > 0);
+                        tc::commit(&M.mma_bar);
+                    }
+                    if (sdone + 1 < kSlabs) load_kt(slab(sdone + 1));
+                    if (__syncthreads_or(!wait_mma())) { failed = true; break; }
+                }
+                if (failed) return;
+
+                // ---- phase D: o of the chunk's tokens; X <- gam_n X + dX
+                {
+                    // column t: tokens (o) and key channels (X) 64 hf .. + 63
+                    const float cv = M.c[t];
+#pragma unroll
+                    for (int c0 = 64 * hf; c0 < 64 * hf + 64; c0 += 32) {
+                        float x[32];
+                        tc::ld32(lane_addr + RO + c0, x);
+#pragma unroll
+                        for (int jj = 0; jj < 32; ++jj) {
+                            const int i = c0 + jj;
+                            if (i < cn) A.o[((size_t)(t0 + i) * n + p) * kD + t] = __fmul_rn(cv, x[jj]);
+                        }
+                    }
+                    const float gn = M.gam[kChunk - 1];
+                    float *xr = XS + t * kXStride;
+#pragma unroll
+                    for (int c0 = 64 * hf; c0 < 64 * hf + 64; c0 += 32) {
+                        float x[32];
+                        tc::ld32(lane_addr + RG + c0, x);
+#pragma unroll
+                        for (int jj = 0; jj < 32; ++jj) xr[c0 + jj] = __fmaf_rn(gn, xr[c0 + jj], x[jj]);
                     }
                 }
-                const float gn = M.gam[kChunk - 1];
-                float *xr = XS + t * kXStride;
-#pragma unroll
-                for (int c0 = 64 * hf; c0 < 64 * hf + 64; c0 += 32) {
-                    float x[32];
-                    tc::ld32(lane_addr + RG + c0, x);
-#pragma unroll
-                    for (int jj = 0; jj < 32; ++jj) xr[c0 + jj] = __fmaf_rn(gn, xr[c0 + jj], x[jj]);
-                }
-            }
-            tc::fence_before_sync();
-            __syncthreads();
-            tc::fence_after_sync();
+                tc::fence_before_sync();
+                __syncthreads();
+                tc::fence_after_sync();
+            };
+            if (M.quot != 0) chunk_body(IC<1>{});
+            else chunk_body(IC<0>{});
         }
         if (failed) break;
 

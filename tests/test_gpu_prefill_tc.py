@@ -92,7 +92,27 @@ def _check_requant(fmt, page, T, seed, step, b, h):
 @pytest.mark.parametrize("name", GDN)
 def test_chunked_prefill_matches_the_chunk_algebra(name, L):
     w, fmt, perm, pages, qs = _setup(name, 3, 5)
+    _check_chunked(name, w, fmt, perm, pages, qs, _prompt(w, L), L)
+
+
+@pytest.mark.parametrize("name", ["stepquant6", "damp"])
+def test_zero_and_vanishing_gates(name):
+    """A gate of zero, and a run of 0.4 gates whose cumulative product leaves
+    the float range inside a chunk (0.4^128 ~ 1e-51): the decay between two
+    tokens is a product of gates in the kernel too, so o and the state stay
+    finite and within the bar of the chunk algebra and of the recurrence."""
+    w, fmt, perm, pages, qs = _setup(name, 3, 5)
+    L = 300
     x = _prompt(w, L)
+    a = x["alpha"].clone()
+    a[3, 0] = 0.0                       # request 0: one token forgets everything
+    a[10:200, 1] = 0.4                  # request 1: the cumulative decay underflows
+    a[130:260:7, 2] = 0.0               # request 2: zero gates in the second chunk
+    x["alpha"] = a.contiguous()
+    _check_chunked(name, w, fmt, perm, pages, qs, x, L)
+
+
+def _check_chunked(name, w, fmt, perm, pages, qs, x, L):
     xd = {k: v.cuda() for k, v in x.items()}
     o = torch.full((L, w.batch, w.heads, 128), float("nan"), device="cuda")
     S_out = torch.empty(w.batch, w.heads, 128, 128, device="cuda")
