@@ -332,7 +332,10 @@ stq_status stq_prefill(stq_state *s, int L, const float *d_q, const float *d_k, 
  * o_i = gam_i S0^T q_i + sum_{j<=i} (gam_i / gam_j) (q_i . k_j) E_j, and the
  * state becomes gam_n S0 + sum_j (gam_n / gam_j) k_j E_j^T, the token
  * recurrence of stq_prefill resolved a chunk at a time (repeated prefill,
- * DASC card page).  The products run as tf32 tensor-core MMAs with split
+ * DASC card page).  Any gates are accepted, zero included: a chunk whose
+ * cumulative gates leave [2^-100, 2^100] takes each gam_i / gam_j as the
+ * product of the gates of tokens j + 1 .. i (slower by about a sixth).
+ * The products run as tf32 tensor-core MMAs with split
  * operands (fp32 = tf32 part + remainder, three products), the solve on the
  * CUDA cores; results agree with stq_prefill to fp32 rounding, not bit for
  * bit (the summation order differs), and the one requantization after the
