@@ -89,7 +89,8 @@ typedef struct stq_state stq_state;   /* opaque host descriptor */
 size_t stq_page_bytes(const stq_format *f);
 
 /* Bytes of device memory a state of B requests x H heads needs: a 256-byte
- * header (status word), the precision map [H][128] (uint8, stored row ->
+ * header (word 0 the status word, word 1 used by stq_prefill_chunked
+ * between its two launches, the rest reserved), the precision map [H][128] (uint8, stored row ->
  * key channel) padded to 256 bytes, then B*H pages, page (b, h) at index
  * b*H + h.  0 on invalid arguments. */
 size_t stq_state_bytes(const stq_format *f, int batch, int heads);
@@ -332,9 +333,11 @@ stq_status stq_prefill(stq_state *s, int L, const float *d_q, const float *d_k, 
  * o_i = gam_i S0^T q_i + sum_{j<=i} (gam_i / gam_j) (q_i . k_j) E_j, and the
  * state becomes gam_n S0 + sum_j (gam_n / gam_j) k_j E_j^T, the token
  * recurrence of stq_prefill resolved a chunk at a time (repeated prefill,
- * DASC card page).  Any gates are accepted, zero included: a chunk whose
- * cumulative gates leave [2^-100, 2^100] takes each gam_i / gam_j as the
- * product of the gates of tokens j + 1 .. i (slower by about a sixth).
+ * DASC card page).  Any gates are accepted, zero included: a page with a
+ * chunk whose cumulative gates leave [2^-100, 2^100] takes each
+ * gam_i / gam_j as the product of the gates of tokens j + 1 .. i (in a
+ * second launch; slower by about a sixth for that page).  The two launches
+ * share the second 32-bit word of the state's header.
  * The products run as tf32 tensor-core MMAs with split
  * operands (fp32 = tf32 part + remainder, three products), the solve on the
  * CUDA cores; results agree with stq_prefill to fp32 rounding, not bit for

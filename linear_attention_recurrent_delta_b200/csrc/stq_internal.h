@@ -17,6 +17,7 @@ struct stq_state {
     stq::DevFormat dev;
     uint64_t wait_limit_ns;
     int stall_first_wait;
+    mutable uint32_t chunked_calls = 0;   // stq_prefill_chunked calls (the mark its two launches share)
 };
 
 namespace stq {

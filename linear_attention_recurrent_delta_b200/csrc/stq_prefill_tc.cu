@@ -37,6 +37,7 @@ namespace stq {
 
 constexpr int kChunk = 128;                    // tokens per chunk
 constexpr int kTcThreads = 256;                // two halves of 128 threads
+static_assert(kTcThreads == 2 * kChunk, "a page's gates are staged two chunks at a time");
 constexpr int kXStride = kD + 1;               // floats per state row
 constexpr int kAStride = kChunk + 4;           // floats per row of the solve's matrix (16-byte rows)
 constexpr uint32_t kTiles = 6;
@@ -46,6 +47,8 @@ struct TcArgs {
     uint8_t *pages;
     const uint8_t *perm;
     uint32_t *status;
+    uint32_t *pending;       // == call when the quotient launch left pages to the product launch
+    uint32_t call;           // this call's mark (never 0)
     const float *q, *k, *v, *alpha, *beta;
     float *o, *S_out;
     int L, n_pages, heads;
@@ -66,7 +69,7 @@ struct TcSmall {
     int kap[kD];             // stored row -> key channel
     uint64_t mma_bar, page_bar, never;
     uint32_t tmem;
-    int quot;                // this chunk's decays may be taken as gam_i / gam_j
+    int in_range;            // this chunk's cumulative decays lie in [2^-100, 2^100]
 };
 
 static_assert(offsetof(TcSmall, inv) % 16 == 0, "inv is read as float4");
@@ -116,7 +119,20 @@ __device__ __forceinline__ void tmem_row(uint32_t taddr_lane, Fn &&fn) {
     }
 }
 
-template <class FMT>
+// the test a chunk's cumulative decays (gam_0, gam_1, ... as thread 0 forms
+// them, padding gates 1) pass for the quotient form
+__device__ __forceinline__ bool decay_in_range(float g) { return g >= 0x1p-100f && g <= 0x1p100f; }
+
+// QUOT: every page, the decay from token j to token i taken as gam_i (1 /
+// gam_j) with gam_i folded into q; a page with a chunk whose cumulative
+// decays leave [2^-100, 2^100] is left as it was (before that chunk's first
+// product; its page bytes are not written) and *A.pending is set to A.call.
+// !QUOT (launched next, as a programmatic dependent launch: its CTAs may wait
+// on the SMs the first leaves idle): once the first has completed, nothing
+// unless *A.pending == A.call; then the pages the first launch left, each
+// decay the product of the gates of tokens j + 1 .. i (defined for zero gates
+// and decays below the float range).
+template <class FMT, bool QUOT>
 __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const DevFormat F, const TcArgs A) {
     extern __shared__ uint8_t tc_smem_raw[];
     const uint32_t raw = smem_u32(tc_smem_raw);
@@ -129,6 +145,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const DevForm
     auto tile = [&](int i) { return tiles + i * tc::kTileBytes; };
     auto tile_addr = [&](int i) { return t_base + (uint32_t)i * tc::kTileBytes; };
 
+    if constexpr (QUOT) {
+        asm volatile("griddepcontrol.launch_dependents;");
+    } else {
+        asm volatile("griddepcontrol.wait;" ::: "memory");   // the quotient launch has completed
+        if (*reinterpret_cast<volatile const uint32_t *>(A.pending) != A.call) return;   // nothing was left
+    }
     constexpr bool SR = FMT::kSr;
     bool col_scales, gate_vector;
     format_flags<FMT>(F, col_scales, gate_vector);
@@ -169,6 +191,28 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const DevForm
     };
 
     for (int p = blockIdx.x; p < n; p += gridDim.x) {
+        if (!QUOT) {
+            // was this page left by the quotient launch?  Its rule, replayed:
+            // a chunk's gates staged in shared memory, then one thread per
+            // chunk forms the cumulative decays in the same order
+            float *gst = reinterpret_cast<float *>(tiles);
+            bool left = false;
+            for (int base = 0; base < A.L; base += kTcThreads) {
+                const int i = base + tid;
+                gst[tid] = i < A.L ? __ldg(A.alpha + (size_t)i * n + p) : 1.f;
+                __syncthreads();
+                if (tid < 2 && base + kChunk * tid < A.L) {
+                    float g = 1.f;
+                    for (int k = 0; k < kChunk; ++k) {
+                        g = __fmul_rn(g, gst[kChunk * tid + k]);
+                        left = left || !decay_in_range(g);
+                    }
+                }
+                __syncthreads();
+            }
+            fence_proxy_async_smem();   // the staging writes before the page's bulk copy
+            if (!__syncthreads_or(left)) continue;
+        }
         const int ph = p % H, pb = p / H;
         // ---- the page: bulk copy into the tile region, dequantize into X
         if (tid == 0) {
@@ -220,6 +264,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const DevForm
         }
         __syncthreads();
 
+        bool leave = false;   // the quotient launch leaves this page to the product launch
         for (int t0 = 0; t0 < A.L && !failed; t0 += kChunk) {
             const int cn = min(kChunk, A.L - t0);
             // ---- per-token scalars of the chunk
@@ -230,27 +275,23 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const DevForm
                 M.al[tid] = real ? A.alpha[row] : 1.f;
             }
             __syncthreads();
-            // The decay from token j to token i is gam_i / gam_j.  While every
-            // cumulative decay of the chunk lies in [2^-100, 2^100] it is taken
-            // as gam_i (1 / gam_j), with gam_i folded into q; otherwise (a zero
-            // gate, or a decay that leaves the float range inside the chunk) as
-            // the product of the gates of tokens j + 1 .. i, which is always
-            // defined.  The flag is the same for the whole CTA.
             if (tid == 0) {
                 float g = 1.f;
-                bool in_range = true;   // a NaN fails the test as well
+                bool in_range = true;
                 for (int i = 0; i < kChunk; ++i) {
                     g = __fmul_rn(g, M.al[i]);
                     M.gam[i] = g;
-                    in_range = in_range && g >= 0x1p-100f && g <= 0x1p100f;
+                    in_range = in_range && decay_in_range(g);
                 }
-                M.quot = in_range ? 1 : 0;
+                M.in_range = in_range ? 1 : 0;
             }
             __syncthreads();
-            // the rest of the chunk, compiled once for each way of taking the
-            // decays, so that each runs as one contiguous stretch of code
-            auto chunk_body = [&](auto qc) {
-                constexpr bool quot = decltype(qc)::value != 0;
+            if (QUOT && M.in_range == 0) {   // for the product launch
+                leave = true;
+                break;
+            }
+            auto chunk_body = [&]() {
+                constexpr bool quot = QUOT;
                 if (quot) {
                     if (tid < kChunk) {
                         const float gi = M.gam[tid];
@@ -615,10 +656,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const DevForm
                 __syncthreads();
                 tc::fence_after_sync();
             };
-            if (M.quot != 0) chunk_body(IC<1>{});
-            else chunk_body(IC<0>{});
+            chunk_body();
         }
         if (failed) break;
+        if (QUOT && leave) {
+            // nothing of the page is stored (o of its earlier chunks is
+            // written again by the product launch)
+            if (tid == 0) *reinterpret_cast<volatile uint32_t *>(A.pending) = A.call;
+            fence_proxy_async_smem();   // the tiles' generic writes before the next bulk copy
+            __syncthreads();
+            continue;
+        }
 
         // ---- the page's end: the state (optional), one requantization, the store
         if (A.S_out) {
@@ -701,15 +749,33 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const DevForm
     if (warp == 0) tc::tmem_dealloc(tmem, 512);
 }
 
-template <class FMT>
-static cudaError_t launch_prefill_tc_with(const DevFormat &F, const TcArgs &A, cudaStream_t stream) {
-    const void *fn = (const void *)prefill_tc_kernel<FMT>;
+template <class FMT, bool QUOT>
+static cudaError_t launch_prefill_tc_form(const DevFormat &F, const TcArgs &A, cudaStream_t stream) {
+    const void *fn = (const void *)prefill_tc_kernel<FMT, QUOT>;
     cudaError_t err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTcSmem);
     if (err != cudaSuccess) return err;
     const int grid = persistent_grid(fn, kTcThreads, kTcSmem, A.n_pages);
     if (grid <= 0) return cudaErrorInvalidConfiguration;
-    prefill_tc_kernel<FMT><<<grid, kTcThreads, kTcSmem, stream>>>(F, A);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kTcThreads);
+    cfg.dynamicSmemBytes = kTcSmem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = QUOT ? 0 : 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, prefill_tc_kernel<FMT, QUOT>, F, A);
+}
+
+// the quotient form on every page it can take, then the pages it left (the
+// second launch returns at once when there are none)
+template <class FMT>
+static cudaError_t launch_prefill_tc_with(const DevFormat &F, const TcArgs &A, cudaStream_t stream) {
+    cudaError_t err = launch_prefill_tc_form<FMT, true>(F, A, stream);
+    if (err != cudaSuccess) return err;
+    return launch_prefill_tc_form<FMT, false>(F, A, stream);
 }
 
 cudaError_t launch_prefill_tc(const stq_state *s, int L, const float *q, const float *k, const float *v,
@@ -720,6 +786,9 @@ cudaError_t launch_prefill_tc(const stq_state *s, int L, const float *q, const f
     A.pages = s->base + s->pages_offset;
     A.perm = s->base + s->perm_offset;
     A.status = reinterpret_cast<uint32_t *>(s->base + s->status_offset);
+    A.pending = A.status + 1;   // the header's second word
+    A.call = ++s->chunked_calls;
+    if (A.call == 0) A.call = ++s->chunked_calls;   // a zeroed header never matches
     A.q = q; A.k = k; A.v = v; A.alpha = alpha; A.beta = beta; A.o = o; A.S_out = S_out;
     A.L = L;
     A.n_pages = s->batch * s->heads;
