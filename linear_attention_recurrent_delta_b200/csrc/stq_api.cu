@@ -355,16 +355,15 @@ stq_status stq_prefill_chunked(stq_state *s, int L, const float *d_q, const floa
                                const float *d_alpha, const float *d_beta, float *d_o, float *d_S_out,
                                uint64_t seed, uint32_t step, void *stream) {
     if (!s || !d_q || !d_k || !d_v || !d_alpha || !d_beta || !d_o) return STQ_ERR_INVALID_ARG;
-    if (s->fmt.gate_vector) return STQ_ERR_UNSUPPORTED;
     const long long n = (long long)s->batch * s->heads;
     if (L < 1 || (long long)(L + 128) * n > 0x7FFFFFF0LL) return STQ_ERR_INVALID_ARG;
     if (!aligned(d_q, 16) || !aligned(d_k, 16) || !aligned(d_v, 16) || !aligned(d_o, 16) || !aligned(d_beta, 4) ||
-        !aligned(d_alpha, 4) || (d_S_out && !aligned(d_S_out, 16)))
+        !aligned(d_alpha, s->fmt.gate_vector ? 16 : 4) || (d_S_out && !aligned(d_S_out, 16)))
         return STQ_ERR_MISALIGNED;
     const size_t vec = (size_t)L * n * kD * sizeof(float), sc = (size_t)L * n * sizeof(float);
     const size_t span = state_span(s);
     const void *in[5] = {d_q, d_k, d_v, d_alpha, d_beta};
-    const size_t len[5] = {vec, vec, vec, sc, sc};
+    const size_t len[5] = {vec, vec, vec, s->fmt.gate_vector ? vec : sc, sc};
     const size_t nS = (size_t)n * kD * kD * sizeof(float);
     for (int i = 0; i < 5; ++i) {
         if (overlaps(in[i], len[i], s->base, span) || overlaps(in[i], len[i], d_o, vec)) return STQ_ERR_INVALID_ARG;

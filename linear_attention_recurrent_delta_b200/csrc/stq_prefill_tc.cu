@@ -40,8 +40,11 @@ constexpr int kTcThreads = 256;                // two halves of 128 threads
 static_assert(kTcThreads == 2 * kChunk, "a page's gates are staged two chunks at a time");
 constexpr int kXStride = kD + 1;               // floats per state row
 constexpr int kAStride = kChunk + 4;           // floats per row of the solve's matrix (16-byte rows)
-constexpr uint32_t kTiles = 6;
-constexpr uint32_t kTileRegion = kTiles * tc::kTileBytes;
+// operand tiles: six for scalar gates (K, gam Q, X as hi / lo pairs), eight
+// for gate vectors (K Gam, Q Gam, X, K / Gam)
+template <bool GV>
+__host__ __device__ constexpr uint32_t tile_region() { return (GV ? 8u : 6u) * tc::kTileBytes; }
+constexpr int kGsStride = 33;                  // floats per token row of the staged decays
 
 struct TcArgs {
     uint8_t *pages;
@@ -70,16 +73,34 @@ struct TcSmall {
     uint64_t mma_bar, page_bar, never;
     uint32_t tmem;
     int in_range;            // this chunk's cumulative decays lie in [2^-100, 2^100]
+    float gn[kD];            // gate vectors: each key channel's decay to the chunk's end
+    float segp[8][32];       // gate vectors: products of 16-token segments of one slab's channels
+    float red[2][2][kD];     // gate vectors, token by token: the halves' partial sums (u, o)
+    alignas(16) float tok[2][4][kD];   // gate vectors, token by token: k, q, gate, v / c (two buffers; float4 reads)
 };
 
 static_assert(offsetof(TcSmall, inv) % 16 == 0, "inv is read as float4");
 static_assert(offsetof(TcSmall, mma_bar) % 8 == 0, "mbarriers are 8-byte aligned");
-static_assert((kTileRegion + (size_t)kD * kXStride * 4) % alignof(TcSmall) == 0, "TcSmall follows X aligned");
-constexpr size_t kTcSmem = kTileRegion + (size_t)kD * kXStride * 4 + sizeof(TcSmall) + 1024;
+static_assert((tile_region<false>() + (size_t)kD * kXStride * 4) % alignof(TcSmall) == 0, "TcSmall follows X aligned");
+static_assert((tile_region<true>() + (size_t)kD * kXStride * 4) % alignof(TcSmall) == 0, "TcSmall follows X aligned");
+static_assert(sizeof(TcSmall) % 16 == 0, "the staged decays follow TcSmall 16-byte aligned");
+static_assert(offsetof(TcSmall, tok) % 16 == 0, "tok is read as float4");
+// shared memory: tiles, X, TcSmall, (gate vectors) one slab's decays of the
+// chunk's tokens, 1 KB for the alignment of the tiles
+template <bool GV>
+constexpr size_t tc_smem() {
+    return tile_region<GV>() + (size_t)kD * kXStride * 4 + sizeof(TcSmall) +
+           (GV ? (size_t)kChunk * kGsStride * 4 : 0) + 1024;
+}
+static_assert(tc_smem<true>() <= 227 * 1024, "shared memory of one CTA");
 
 // four consecutive columns k .. k + 3 (k a multiple of 4) of a row: one
 // 16-byte unit of the swizzled row, so a warp's 32 rows take 4 conflict-free
 // shared-memory wavefronts (a float at a time, 8 banks serve the 32 rows)
+__device__ __forceinline__ float4 mul4e(float4 a, float4 x) {
+    return make_float4(__fmul_rn(a.x, x.x), __fmul_rn(a.y, x.y), __fmul_rn(a.z, x.z), __fmul_rn(a.w, x.w));
+}
+
 __device__ __forceinline__ float4 mul4(float a, float4 x) {
     return make_float4(__fmul_rn(a, x.x), __fmul_rn(a, x.y), __fmul_rn(a, x.z), __fmul_rn(a, x.w));
 }
@@ -132,14 +153,18 @@ __device__ __forceinline__ bool decay_in_range(float g) { return g >= 0x1p-100f 
 // unless *A.pending == A.call; then the pages the first launch left, each
 // decay the product of the gates of tokens j + 1 .. i (defined for zero gates
 // and decays below the float range).
-template <class FMT, bool QUOT>
+// GV (gate vectors, KDA): QUOT only; a chunk whose per-channel cumulative
+// decays leave the range runs token by token on the CUDA cores instead.
+template <class FMT, bool QUOT, bool GV>
 __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const DevFormat F, const TcArgs A) {
+    static_assert(QUOT || !GV, "gate vectors take the quotient form or the token recurrence");
     extern __shared__ uint8_t tc_smem_raw[];
     const uint32_t raw = smem_u32(tc_smem_raw);
     uint8_t *base = tc_smem_raw + (((raw + 1023u) & ~1023u) - raw);
-    uint8_t *tiles = base;                                            // six operand tiles / A / page buffer
-    float *XS = reinterpret_cast<float *>(base + kTileRegion);       // X[v][kappa]
-    TcSmall &M = *reinterpret_cast<TcSmall *>(base + kTileRegion + (size_t)kD * kXStride * 4);
+    uint8_t *tiles = base;                                            // operand tiles / A / page buffer
+    float *XS = reinterpret_cast<float *>(base + tile_region<GV>());  // X[v][kappa]
+    TcSmall &M = *reinterpret_cast<TcSmall *>(base + tile_region<GV>() + (size_t)kD * kXStride * 4);
+    float *Gs = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(&M) + sizeof(TcSmall));   // GV: [token][33]
     float *Amat = reinterpret_cast<float *>(tiles);
     const uint32_t t_base = smem_u32(tiles);
     auto tile = [&](int i) { return tiles + i * tc::kTileBytes; };
@@ -265,6 +290,75 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const DevForm
         __syncthreads();
 
         bool leave = false;   // the quotient launch leaves this page to the product launch
+        // Gate vectors, a chunk whose per-channel decays leave the range: the
+        // delta rule token by token on the CUDA cores, in the state's own
+        // units (X = S^T / c).  Thread (v, hf) holds X[v][64 hf .. + 63] in
+        // registers; each token: decay, prediction u = X k, e = beta (v / c -
+        // u), update X += e k^T, readout o = c X q, the halves' partial sums
+        // through shared memory.  The next token's vectors are staged while
+        // this one runs.
+        auto gv_tokens = [&](int t0, int cn) {
+            auto stage = [&](int i, int b) {
+                if (tid < kD) {
+                    const size_t row = ((size_t)(t0 + i) * n + p) * kD + tid;
+                    M.tok[b][0][tid] = __ldg(A.k + row);
+                    M.tok[b][1][tid] = __ldg(A.q + row);
+                    M.tok[b][2][tid] = __ldg(A.alpha + row);
+                    M.tok[b][3][tid] = __fmul_rn(__ldg(A.v + row), M.ic[tid]);
+                }
+            };
+            float x[64];
+            const float *xr = XS + t * kXStride + 64 * hf;
+#pragma unroll
+            for (int c = 0; c < 64; ++c) x[c] = xr[c];
+            stage(0, 0);
+            __syncthreads();
+            for (int i = 0; i < cn; ++i) {
+                const int b = i & 1;
+                if (i + 1 < cn) stage(i + 1, b ^ 1);   // read after the next token's first barrier
+                const float *kb = &M.tok[b][0][64 * hf], *qb = &M.tok[b][1][64 * hf], *ab = &M.tok[b][2][64 * hf];
+                float u = 0.f;
+#pragma unroll
+                for (int c = 0; c < 64; c += 4) {
+                    const float4 a4 = *reinterpret_cast<const float4 *>(ab + c);
+                    const float4 k4 = *reinterpret_cast<const float4 *>(kb + c);
+                    x[c] = __fmul_rn(x[c], a4.x);
+                    x[c + 1] = __fmul_rn(x[c + 1], a4.y);
+                    x[c + 2] = __fmul_rn(x[c + 2], a4.z);
+                    x[c + 3] = __fmul_rn(x[c + 3], a4.w);
+                    u = __fmaf_rn(k4.x, x[c], u);
+                    u = __fmaf_rn(k4.y, x[c + 1], u);
+                    u = __fmaf_rn(k4.z, x[c + 2], u);
+                    u = __fmaf_rn(k4.w, x[c + 3], u);
+                }
+                M.red[0][hf][t] = u;
+                __syncthreads();
+                const float e = __fmul_rn(M.bet[i], __fsub_rn(M.tok[b][3][t], __fadd_rn(M.red[0][0][t], M.red[0][1][t])));
+                float o = 0.f;
+#pragma unroll
+                for (int c = 0; c < 64; c += 4) {
+                    const float4 k4 = *reinterpret_cast<const float4 *>(kb + c);
+                    const float4 q4 = *reinterpret_cast<const float4 *>(qb + c);
+                    x[c] = __fmaf_rn(k4.x, e, x[c]);
+                    x[c + 1] = __fmaf_rn(k4.y, e, x[c + 1]);
+                    x[c + 2] = __fmaf_rn(k4.z, e, x[c + 2]);
+                    x[c + 3] = __fmaf_rn(k4.w, e, x[c + 3]);
+                    o = __fmaf_rn(q4.x, x[c], o);
+                    o = __fmaf_rn(q4.y, x[c + 1], o);
+                    o = __fmaf_rn(q4.z, x[c + 2], o);
+                    o = __fmaf_rn(q4.w, x[c + 3], o);
+                }
+                M.red[1][hf][t] = o;
+                __syncthreads();
+                if (hf == 0)
+                    A.o[((size_t)(t0 + i) * n + p) * kD + t] =
+                        __fmul_rn(M.c[t], __fadd_rn(M.red[1][0][t], M.red[1][1][t]));
+            }
+            float *xw = XS + t * kXStride + 64 * hf;
+#pragma unroll
+            for (int c = 0; c < 64; ++c) xw[c] = x[c];
+            __syncthreads();   // X is whole again before the next chunk
+        };
         for (int t0 = 0; t0 < A.L && !failed; t0 += kChunk) {
             const int cn = min(kChunk, A.L - t0);
             // ---- per-token scalars of the chunk
@@ -272,27 +366,57 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const DevForm
                 const bool real = tid < cn;
                 const size_t row = (size_t)(t0 + tid) * n + p;
                 M.bet[tid] = real ? A.beta[row] : 0.f;
-                M.al[tid] = real ? A.alpha[row] : 1.f;
+                if constexpr (!GV) M.al[tid] = real ? A.alpha[row] : 1.f;
             }
-            __syncthreads();
-            if (tid == 0) {
+            if constexpr (GV) {
+                // thread (kappa = t, hf) multiplies the gates of tokens 64 hf ..
+                // + 63 of key channel kappa; the decay to the chunk's end is the
+                // product of the halves.  The matrix form needs every cumulative
+                // decay in [2^-100, 2^100]: with every gate in [0, 1] and each
+                // channel's whole product at least 2^-90 (a margin for the other
+                // orders in which the kernel forms them) it is.
                 float g = 1.f;
                 bool in_range = true;
-                for (int i = 0; i < kChunk; ++i) {
-                    g = __fmul_rn(g, M.al[i]);
-                    M.gam[i] = g;
-                    in_range = in_range && decay_in_range(g);
+#pragma unroll 16
+                for (int i = 64 * hf; i < 64 * hf + 64; ++i) {
+                    const float a = i < cn ? __ldg(A.alpha + ((size_t)(t0 + i) * n + p) * kD + t) : 1.f;
+                    in_range = in_range && a >= 0.f && a <= 1.f;   // a NaN fails too
+                    g = __fmul_rn(g, a);
                 }
-                M.in_range = in_range ? 1 : 0;
-            }
-            __syncthreads();
-            if (QUOT && M.in_range == 0) {   // for the product launch
-                leave = true;
-                break;
+                M.red[0][hf][t] = g;
+                __syncthreads();
+                if (hf == 0) {
+                    const float gn = __fmul_rn(M.red[0][0][t], M.red[0][1][t]);
+                    M.gn[t] = gn;
+                    in_range = in_range && gn >= 0x1p-90f;
+                }
+                if (!__syncthreads_and(in_range)) {
+                    gv_tokens(t0, cn);   // this chunk token by token
+                    continue;
+                }
+            } else {
+                __syncthreads();
+                if (tid == 0) {
+                    float g = 1.f;
+                    bool in_range = true;
+                    for (int i = 0; i < kChunk; ++i) {
+                        g = __fmul_rn(g, M.al[i]);
+                        M.gam[i] = g;
+                        in_range = in_range && decay_in_range(g);
+                    }
+                    M.in_range = in_range ? 1 : 0;
+                }
+                __syncthreads();
+                if (QUOT && M.in_range == 0) {   // for the product launch
+                    leave = true;
+                    break;
+                }
             }
             auto chunk_body = [&]() {
                 constexpr bool quot = QUOT;
-                if (quot) {
+                if constexpr (GV) {
+                    // (the decays come per slab below)
+                } else if (quot) {
                     if (tid < kChunk) {
                         const float gi = M.gam[tid];
                         M.igam[tid] = __frcp_rn(gi);
@@ -325,9 +449,47 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const DevForm
                         }
                     }
                 };
+                // gate vectors: the decays Gam[token][channel] of one slab's 32
+                // channels staged in Gs; warp s takes tokens 16 s .. + 15 of
+                // channel 32 ks + lane (segment products, then their prefixes)
+                auto stage_gam = [&](int ks) {
+                    float av[16];
+                    float pr = 1.f;
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const int tk = 16 * warp + i;
+                        av[i] = tk < cn ? __ldg(A.alpha + ((size_t)(t0 + tk) * n + p) * kD + 32 * ks + lane) : 1.f;
+                        pr = __fmul_rn(pr, av[i]);
+                    }
+                    M.segp[warp][lane] = pr;
+                    __syncthreads();
+                    float g = 1.f;
+                    for (int s2 = 0; s2 < warp; ++s2) g = __fmul_rn(g, M.segp[s2][lane]);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        g = __fmul_rn(g, av[i]);
+                        Gs[(16 * warp + i) * kGsStride + lane] = g;
+                    }
+                    __syncthreads();
+                };
                 load_kq(0);
+                if constexpr (GV) stage_gam(0);
                 for (int ks = 0; ks < kD / 32; ++ks) {
-                    {
+                    if constexpr (GV) {
+                        // row t of the K Gam, Q Gam, X and K / Gam slabs, columns 16 hf .. + 15
+                        const float *xr = XS + t * kXStride + 32 * ks;
+                        const float *gr = Gs + t * kGsStride;
+#pragma unroll
+                        for (int j4 = 0; j4 < 4; ++j4) {
+                            const int j = 16 * hf + 4 * j4;
+                            const float4 g4 = make_float4(gr[j], gr[j + 1], gr[j + 2], gr[j + 3]);
+                            const float4 ig4 = make_float4(__frcp_rn(g4.x), __frcp_rn(g4.y), __frcp_rn(g4.z), __frcp_rn(g4.w));
+                            put_split4(tile(0), tile(1), t, j, mul4e(kx[j4], g4));
+                            put_split4(tile(2), tile(3), t, j, mul4e(qx[j4], g4));
+                            put_split4(tile(4), tile(5), t, j, make_float4(xr[j], xr[j + 1], xr[j + 2], xr[j + 3]));
+                            put_split4(tile(6), tile(7), t, j, mul4e(kx[j4], ig4));
+                        }
+                    } else {
                         // row t of the K, gam Q and X slabs, columns 16 hf .. + 15
                         const float gi = quot ? M.gam[t] : 1.f;
                         const float *xr = XS + t * kXStride + 32 * ks;
@@ -345,13 +507,24 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const DevForm
                     tc::fence_after_sync();
                     if (tid == 0) {
                         const bool acc = ks > 0;
-                        mma_split(tmem + RG, tile_addr(0), tile_addr(1), tile_addr(0), tile_addr(1), acc);
-                        mma_split(tmem + RY, tile_addr(4), tile_addr(5), tile_addr(0), tile_addr(1), acc);
-                        mma_split(tmem + RP, tile_addr(2), tile_addr(3), tile_addr(0), tile_addr(1), acc);
-                        mma_split(tmem + RO, tile_addr(4), tile_addr(5), tile_addr(2), tile_addr(3), acc);
+                        if constexpr (GV) {
+                            // G = (K Gam)(K / Gam)^T, Y^T = X (K Gam)^T, P = (Q Gam)(K / Gam)^T, O^T = X (Q Gam)^T
+                            mma_split(tmem + RG, tile_addr(0), tile_addr(1), tile_addr(6), tile_addr(7), acc);
+                            mma_split(tmem + RY, tile_addr(4), tile_addr(5), tile_addr(0), tile_addr(1), acc);
+                            mma_split(tmem + RP, tile_addr(2), tile_addr(3), tile_addr(6), tile_addr(7), acc);
+                            mma_split(tmem + RO, tile_addr(4), tile_addr(5), tile_addr(2), tile_addr(3), acc);
+                        } else {
+                            mma_split(tmem + RG, tile_addr(0), tile_addr(1), tile_addr(0), tile_addr(1), acc);
+                            mma_split(tmem + RY, tile_addr(4), tile_addr(5), tile_addr(0), tile_addr(1), acc);
+                            mma_split(tmem + RP, tile_addr(2), tile_addr(3), tile_addr(0), tile_addr(1), acc);
+                            mma_split(tmem + RO, tile_addr(4), tile_addr(5), tile_addr(2), tile_addr(3), acc);
+                        }
                         tc::commit(&M.mma_bar);
                     }
                     if (ks + 1 < kD / 32) load_kq(ks + 1);
+                    if constexpr (GV) {
+                        if (ks + 1 < kD / 32) stage_gam(ks + 1);   // Gs is free: this slab's tiles are written
+                    }
                     if (__syncthreads_or(!wait_mma())) { failed = true; break; }
                 }
                 if (failed) return;
@@ -375,8 +548,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const DevForm
                         for (int jj = 0; jj < 32; ++jj) {
                             const int i = c0 + jj;
                             const float vv = (i < cn) ? __ldg(A.v + ((size_t)(t0 + i) * n + p) * kD + t) : 0.f;
-                            // R_i = beta_i (v_i / c - gam_i y_i)
-                            x[jj] = __fmul_rn(M.bet[i], __fsub_rn(__fmul_rn(vv, icv), __fmul_rn(M.gam[i], x[jj])));
+                            // R_i = beta_i (v_i / c - gam_i y_i) (gate vectors: the decay is in y)
+                            const float gy = GV ? x[jj] : __fmul_rn(M.gam[i], x[jj]);
+                            x[jj] = __fmul_rn(M.bet[i], __fsub_rn(__fmul_rn(vv, icv), gy));
                         }
                         tc::st32(ry + c0, x);
                         if (!quot) {
@@ -400,7 +574,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const DevForm
                         float x[32];
                         tc::ld32(lane_addr + RG + jlo, x);
                         float a[32];
-                        if (quot) {
+                        if constexpr (GV) {
+#pragma unroll
+                            for (int jj = 0; jj < 32; ++jj) a[jj] = jlo + jj < t ? __fmul_rn(bi, x[jj]) : 0.f;
+                        } else if (quot) {
                             const float gi = M.gam[t];
 #pragma unroll
                             for (int jj = 0; jj < 32; ++jj) {
@@ -482,7 +659,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const DevForm
                         // rho walked down from j = t to the block's columns 63 .. 0
                         const float bi = M.bet[t];
                         uint8_t *a21 = tiles + 4 * tc::kTileBytes;
-                        const float gi = M.gam[t];
+                        const float gi = GV ? 1.f : M.gam[t];
                         float rho = 1.f;   // rho_{t, 63}: the gates 64 .. t
                         if (!quot) {
 #pragma unroll
@@ -494,7 +671,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const DevForm
                             float x[32];
                             tc::ld32(lane_addr + RG + 32 * kb, x);
                             float a[32];
-                            if (quot) {
+                            if constexpr (GV) {
+#pragma unroll
+                                for (int jj = 0; jj < 32; ++jj) a[jj] = __fmul_rn(bi, x[jj]);
+                            } else if (quot) {
 #pragma unroll
                                 for (int jj = 0; jj < 32; ++jj)
                                     a[jj] = __fmul_rn(bi, __fmul_rn(__fmul_rn(gi, M.igam[32 * kb + jj]), x[jj]));
@@ -564,6 +744,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const DevForm
                 auto slab = [&](int n_done) { return quot ? n_done : kSlabs - 1 - n_done; };
                 load_kt(slab(0));
                 float rho = 1.f;   // rho_{t, j} for the next j below the columns done
+                float gk = 1.f;    // gate vectors: Gam of channel t through the tokens done
                 for (int sdone = 0; sdone < kSlabs; ++sdone) {
                     const int js = slab(sdone);
                     {
@@ -581,7 +762,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const DevForm
                         // other half's columns of the slab too
                         tc::ld16(lane_addr + RP + 32 * js + c0, x);
                         float pv[16];
-                        if (quot) {
+                        if constexpr (GV) {
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) pv[e] = 32 * js + c0 + e <= t ? x[e] : 0.f;
+                        } else if (quot) {
 #pragma unroll
                             for (int e = 0; e < 16; ++e) {
                                 const int j = 32 * js + c0 + e;
@@ -605,13 +789,36 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const DevForm
                             put_split4(tile(2), tile(3), t, c0 + 4 * u,
                                        make_float4(pv[4 * u], pv[4 * u + 1], pv[4 * u + 2], pv[4 * u + 3]));
                         // K~^T row kappa (thread kappa): k_j[kappa] times the decay of
-                        // token j to the chunk's end
+                        // token j to the chunk's end (gate vectors: Gam_n / Gam_j of
+                        // channel kappa, Gam walked through the slab's tokens)
+                        if constexpr (GV) {
+                            float rt[16];
 #pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const float *kt = M.kts + 32 * js + c0 + 4 * u;
-                            put_split4(tile(4), tile(5), t, c0 + 4 * u,
-                                       make_float4(__fmul_rn(kk[4 * u], kt[0]), __fmul_rn(kk[4 * u + 1], kt[1]),
-                                                   __fmul_rn(kk[4 * u + 2], kt[2]), __fmul_rn(kk[4 * u + 3], kt[3])));
+                            for (int e = 0; e < 16; ++e) rt[e] = 0.f;
+#pragma unroll
+                            for (int part = 0; part < 2; ++part) {
+#pragma unroll
+                                for (int e = 0; e < 16; ++e) {
+                                    const int j = 32 * js + 16 * part + e;
+                                    const float a = j < cn ? __ldg(A.alpha + ((size_t)(t0 + j) * n + p) * kD + t) : 1.f;
+                                    gk = __fmul_rn(gk, a);
+                                    if (part == hf) rt[e] = __fdiv_rn(M.gn[t], gk);
+                                }
+                            }
+#pragma unroll
+                            for (int u = 0; u < 4; ++u)
+                                put_split4(tile(4), tile(5), t, c0 + 4 * u,
+                                           make_float4(__fmul_rn(kk[4 * u], rt[4 * u]), __fmul_rn(kk[4 * u + 1], rt[4 * u + 1]),
+                                                       __fmul_rn(kk[4 * u + 2], rt[4 * u + 2]),
+                                                       __fmul_rn(kk[4 * u + 3], rt[4 * u + 3])));
+                        } else {
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) {
+                                const float *kt = M.kts + 32 * js + c0 + 4 * u;
+                                put_split4(tile(4), tile(5), t, c0 + 4 * u,
+                                           make_float4(__fmul_rn(kk[4 * u], kt[0]), __fmul_rn(kk[4 * u + 1], kt[1]),
+                                                       __fmul_rn(kk[4 * u + 2], kt[2]), __fmul_rn(kk[4 * u + 3], kt[3])));
+                            }
                         }
                     }
                     fence_proxy_async_smem();
@@ -649,7 +856,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const DevForm
                         float x[32];
                         tc::ld32(lane_addr + RG + c0, x);
 #pragma unroll
-                        for (int jj = 0; jj < 32; ++jj) xr[c0 + jj] = __fmaf_rn(gn, xr[c0 + jj], x[jj]);
+                        for (int jj = 0; jj < 32; ++jj)
+                        xr[c0 + jj] = __fmaf_rn(GV ? M.gn[c0 + jj] : gn, xr[c0 + jj], x[jj]);
                     }
                 }
                 tc::fence_before_sync();
@@ -749,33 +957,47 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const DevForm
     if (warp == 0) tc::tmem_dealloc(tmem, 512);
 }
 
-template <class FMT, bool QUOT>
+template <class FMT, bool QUOT, bool GV>
 static cudaError_t launch_prefill_tc_form(const DevFormat &F, const TcArgs &A, cudaStream_t stream) {
-    const void *fn = (const void *)prefill_tc_kernel<FMT, QUOT>;
-    cudaError_t err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTcSmem);
+    const void *fn = (const void *)prefill_tc_kernel<FMT, QUOT, GV>;
+    constexpr size_t smem = tc_smem<GV>();
+    cudaError_t err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
-    const int grid = persistent_grid(fn, kTcThreads, kTcSmem, A.n_pages);
+    const int grid = persistent_grid(fn, kTcThreads, smem, A.n_pages);
     if (grid <= 0) return cudaErrorInvalidConfiguration;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(kTcThreads);
-    cfg.dynamicSmemBytes = kTcSmem;
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = QUOT ? 0 : 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, prefill_tc_kernel<FMT, QUOT>, F, A);
+    return cudaLaunchKernelEx(&cfg, prefill_tc_kernel<FMT, QUOT, GV>, F, A);
 }
 
 // the quotient form on every page it can take, then the pages it left (the
 // second launch returns at once when there are none)
 template <class FMT>
-static cudaError_t launch_prefill_tc_with(const DevFormat &F, const TcArgs &A, cudaStream_t stream) {
-    cudaError_t err = launch_prefill_tc_form<FMT, true>(F, A, stream);
+static cudaError_t launch_prefill_tc_scalar(const DevFormat &F, const TcArgs &A, cudaStream_t stream) {
+    cudaError_t err = launch_prefill_tc_form<FMT, true, false>(F, A, stream);
     if (err != cudaSuccess) return err;
-    return launch_prefill_tc_form<FMT, false>(F, A, stream);
+    return launch_prefill_tc_form<FMT, false, false>(F, A, stream);
+}
+
+// gate vectors: one launch (the token recurrence takes the chunks out of range)
+template <class FMT>
+static cudaError_t launch_prefill_tc_with(const DevFormat &F, const TcArgs &A, cudaStream_t stream) {
+    if constexpr (FMT::kRuntime) {
+        if (F.gate_vector) return launch_prefill_tc_form<FMT, true, true>(F, A, stream);
+        return launch_prefill_tc_scalar<FMT>(F, A, stream);
+    } else if constexpr (FMT::kGvec) {
+        return launch_prefill_tc_form<FMT, true, true>(F, A, stream);
+    } else {
+        return launch_prefill_tc_scalar<FMT>(F, A, stream);
+    }
 }
 
 cudaError_t launch_prefill_tc(const stq_state *s, int L, const float *q, const float *k, const float *v,
@@ -802,6 +1024,7 @@ cudaError_t launch_prefill_tc(const stq_state *s, int L, const float *q, const f
     if (format_is<FmtStepQuant6>(F)) return launch_prefill_tc_with<FmtStepQuant6>(F, A, stream);
     if (format_is<FmtInt8Row>(F)) return launch_prefill_tc_with<FmtInt8Row>(F, A, stream);
     if (format_is<FmtDamp>(F)) return launch_prefill_tc_with<FmtDamp>(F, A, stream);
+    if (format_is<FmtStepQuant4Kda>(F)) return launch_prefill_tc_with<FmtStepQuant4Kda>(F, A, stream);
     if (F.stochastic) return launch_prefill_tc_with<RuntimeFmt<true>>(F, A, stream);
     return launch_prefill_tc_with<RuntimeFmt<false>>(F, A, stream);
 }

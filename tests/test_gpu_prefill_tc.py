@@ -14,8 +14,9 @@ token recurrence to fp32 rounding, not bit for bit.  The bar, per page:
     1e-5 of a rounding midpoint, each FP16 row element the binary16 rounding
     of T except at a near-tie.
 Prompts of 1, 37, 128, 130 and 300 tokens (one chunk, a ragged chunk, two
-and three chunks); the GDN formats; more pages than SMs for the persistent
-grid; the bounded-wait hook.
+and three chunks); the GDN formats and KDA's gate vectors; zero and
+vanishing gates; more pages than SMs for the persistent grid; the
+bounded-wait hook.
 """
 import numpy as np
 import pytest
@@ -169,13 +170,27 @@ def test_many_pages_per_cta():
         assert rel_l2(o_g[:, b, h], o64) <= 1e-5
 
 
-def test_vector_gate_formats_are_refused():
-    w, fmt, perm, pages, qs = _setup("stepquant4_kda", 2, 2)
-    x = {k: v.cuda() for k, v in _prompt(w, 3).items()}
-    o = torch.empty(3, 2, 2, 128, device="cuda")
-    st = B.lib().stq_prefill_chunked(qs.state.handle, 3, B._ptr(x["q"]), B._ptr(x["k"]), B._ptr(x["v"]),
-                                     B._ptr(x["alpha"]), B._ptr(x["beta"]), B._ptr(o), None, 0, 0, None)
-    assert st == B.STQ_ERR_UNSUPPORTED
+@pytest.mark.parametrize("L", [1, 37, 128, 130, 300])
+def test_vector_gates_match_the_chunk_algebra(L):
+    """KDA gates (a vector over key channels): the decays Gam of every channel
+    folded into the operands (K Gam, Q Gam, K / Gam), the same bars."""
+    w, fmt, perm, pages, qs = _setup("stepquant4_kda", 3, 5)
+    _check_chunked("stepquant4_kda", w, fmt, perm, pages, qs, _prompt(w, L), L)
+
+
+def test_vector_gates_zero_and_vanishing():
+    """Chunks whose per-channel decays leave the range run token by token on
+    the CUDA cores: a zero gate on some channels, and a run of 0.2 gates on
+    others (0.2^128 ~ 1e-90), next to chunks of the matrix form."""
+    w, fmt, perm, pages, qs = _setup("stepquant4_kda", 3, 5)
+    L = 300
+    x = _prompt(w, L)
+    a = x["alpha"].clone()
+    a[3, 0, :, ::5] = 0.0               # request 0: some channels forget at token 3
+    a[10:200, 1, :, 7] = 0.2            # request 1: one channel's decay underflows
+    a[130:260:7, 2] = 0.0               # request 2: every channel forgets, second chunk
+    x["alpha"] = a.contiguous()
+    _check_chunked("stepquant4_kda", w, fmt, perm, pages, qs, x, L)
 
 
 def test_bounded_wait_times_out_and_writes_nothing():
