@@ -741,10 +741,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const DevForm
                 };
                 // slab order: ascending for quotients, descending for products
                 constexpr int kSlabs = kChunk / 32;
-                auto slab = [&](int n_done) { return quot ? n_done : kSlabs - 1 - n_done; };
+                // (gate vectors: descending too, a key's decay to the chunk's end
+                // being the product of the gates after it)
+                auto slab = [&](int n_done) { return (quot && !GV) ? n_done : kSlabs - 1 - n_done; };
                 load_kt(slab(0));
                 float rho = 1.f;   // rho_{t, j} for the next j below the columns done
-                float gk = 1.f;    // gate vectors: Gam of channel t through the tokens done
+                float gk = 1.f;    // gate vectors: channel t's gates after the next token down
                 for (int sdone = 0; sdone < kSlabs; ++sdone) {
                     const int js = slab(sdone);
                     {
@@ -792,17 +794,32 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const DevForm
                         // token j to the chunk's end (gate vectors: Gam_n / Gam_j of
                         // channel kappa, Gam walked through the slab's tokens)
                         if constexpr (GV) {
+                            // the slab's gates of every channel, [32 tokens][128] in
+                            // tile 6 (free in this phase): thread (t, hf) loads
+                            // channel t of tokens 16 hf .. + 15 in one batch
+                            float *ga = reinterpret_cast<float *>(tile(6));
+                            {
+                                float av[16];
+#pragma unroll
+                                for (int e = 0; e < 16; ++e) {
+                                    const int j = 32 * js + 16 * hf + e;
+                                    av[e] = j < cn ? __ldg(A.alpha + ((size_t)(t0 + j) * n + p) * kD + t) : 1.f;
+                                }
+#pragma unroll
+                                for (int e = 0; e < 16; ++e) ga[(16 * hf + e) * kD + t] = av[e];
+                            }
+                            __syncthreads();
+                            // Gam_n / Gam_j = the gates of tokens j + 1 .. n - 1, walked
+                            // down (padding gates are 1)
                             float rt[16];
 #pragma unroll
                             for (int e = 0; e < 16; ++e) rt[e] = 0.f;
 #pragma unroll
-                            for (int part = 0; part < 2; ++part) {
+                            for (int part = 1; part >= 0; --part) {
 #pragma unroll
-                                for (int e = 0; e < 16; ++e) {
-                                    const int j = 32 * js + 16 * part + e;
-                                    const float a = j < cn ? __ldg(A.alpha + ((size_t)(t0 + j) * n + p) * kD + t) : 1.f;
-                                    gk = __fmul_rn(gk, a);
-                                    if (part == hf) rt[e] = __fdiv_rn(M.gn[t], gk);
+                                for (int e = 15; e >= 0; --e) {
+                                    if (part == hf) rt[e] = gk;
+                                    gk = __fmul_rn(gk, ga[(16 * part + e) * kD + t]);
                                 }
                             }
 #pragma unroll
