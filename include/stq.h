@@ -324,8 +324,8 @@ stq_status stq_prefill(stq_state *s, int L, const float *d_q, const float *d_k, 
                        const float *d_alpha, const float *d_beta, float *d_o, float *d_S_out, uint64_t seed,
                        uint32_t step, void *stream);
 
-/* The same prefill in chunkwise form on the tensor cores (GDN states: a
- * scalar gate per token and page).  The prompt runs in chunks of 128 tokens;
+/* The same prefill in chunkwise form on the tensor cores.  The prompt runs
+ * in chunks of 128 tokens;
  * per chunk, with gam_i the product of the chunk's gates up to token i, the
  * chunk's deltas E are the triangular solve (I + A) E = R,
  *     A_ij = beta_i (gam_i / gam_j) (k_i . k_j)  (j < i),
@@ -342,9 +342,11 @@ stq_status stq_prefill(stq_state *s, int L, const float *d_q, const float *d_k, 
  * operands (fp32 = tf32 part + remainder, three products), the solve on the
  * CUDA cores; results agree with stq_prefill to fp32 rounding, not bit for
  * bit (the summation order differs), and the one requantization after the
- * last token is stq_prefill's.  Arguments, layouts and errors as
- * stq_prefill, plus UNSUPPORTED for gate_vector formats (KDA: use
- * stq_prefill).  One CTA per page (the whole shared memory and tensor
+ * last token is stq_prefill's.  Gate vectors (KDA): gam is per key channel
+ * and folded into the operands (k gam, q gam, k / gam); a chunk with a gate
+ * outside [0, 1] or a channel whose decay over the chunk falls below 2^-90
+ * runs token by token on the CUDA cores instead.  Arguments, layouts and
+ * errors as stq_prefill.  One CTA per page (the whole shared memory and tensor
  * memory of an SM); a bounded wait that ran out is reported by
  * stq_device_status. */
 stq_status stq_prefill_chunked(stq_state *s, int L, const float *d_q, const float *d_k, const float *d_v,
