@@ -151,12 +151,18 @@ def _check_chunked(name, w, fmt, perm, pages, qs, x, L):
           % (name, L, worst_o, worst_s, ties))
 
 
-def test_many_pages_per_cta():
-    """More pages than SMs: every CTA takes several pages in turn."""
+@pytest.mark.parametrize("name", ["int8row", "stepquant4_kda"])
+def test_many_pages_per_cta(name):
+    """More pages than SMs: every CTA takes several pages in turn (gate
+    vectors: some of them token by token, zero gates on every fifth page)."""
     sms = torch.cuda.get_device_properties(0).multi_processor_count
-    w, fmt, perm, pages, qs = _setup("int8row", (sms * 2) // 4 + 3, 4)
+    w, fmt, perm, pages, qs = _setup(name, (sms * 2) // 4 + 3, 4)
     L = 20
     x = _prompt(w, L)
+    if fmt.gate_vector:
+        a = x["alpha"].clone()
+        a.view(L, -1, 128)[4, ::5, :] = 0.0
+        x["alpha"] = a.contiguous()
     xd = {k: v.cuda() for k, v in x.items()}
     o = torch.empty(L, w.batch, w.heads, 128, device="cuda")
     B.stq_prefill_chunked(qs.state, xd["q"], xd["k"], xd["v"], xd["alpha"], xd["beta"], o, None, 0, 3)
@@ -193,8 +199,9 @@ def test_vector_gates_zero_and_vanishing():
     _check_chunked("stepquant4_kda", w, fmt, perm, pages, qs, x, L)
 
 
-def test_bounded_wait_times_out_and_writes_nothing():
-    w, fmt, perm, pages, qs = _setup("stepquant6", 4, 3)
+@pytest.mark.parametrize("name", ["stepquant6", "stepquant4_kda"])
+def test_bounded_wait_times_out_and_writes_nothing(name):
+    w, fmt, perm, pages, qs = _setup(name, 4, 3)
     L = 40
     x = _prompt(w, L)
     xd = {k: v.cuda() for k, v in x.items()}
