@@ -761,25 +761,29 @@ def main():
                                                "flops_per_head_token": fl}}
         # the chunkwise tensor-core form against the recurrent one: the
         # headline batch with a 512-token prompt, and one request x 32 heads
-        # with a 1,024-token prompt (32 pages: few CTAs for the recurrent form)
-        if not spec["gate_vector"]:
-            tf = chunked_flops_per_head_token()
-            tc_peak = tf32_peak()
-            for tag, wl, L, n in (("batch256_L512", w.resized(batch=min(w.batch, 256)), 512, 3),
-                                  ("one_request_L1024", w.resized(batch=1), 1024, 5)):
-                rr = run_prefill(wl, L, n, 2, rank, world)
-                rc = run_prefill(wl, L, n, 2, rank, world, chunked=True)
-                rate_r = R.aggregate_rate(wl.pages * L, world, rr["steps"], rr["ms"])
-                rate_c = R.aggregate_rate(wl.pages * L, world, rc["steps"], rc["ms"])
-                prefill["chunked_" + tag] = {
-                    "value": rate_c, "unit": "head-tokens/s", "prompt": L, "pages": wl.pages,
-                    "entry_point": "stq_prefill_chunked", "kernel": "stq::prefill_tc_kernel",
-                    "ms_per_prefill": rc["ms"] / rc["steps"],
-                    "recurrent_value": rate_r, "speedup_vs_recurrent": rate_c / rate_r,
-                    "roofline": {"bound": "tensor", "achieved": rate_c * tf / 1e12, "peak": tc_peak[0],
-                                 "unit": "TFLOP/s", "frac": rate_c * tf / 1e12 / tc_peak[0],
-                                 "peak_kind": tc_peak[1], "flops_per_head_token": tf,
-                                 "note": "fp32 products counted once; each runs as three tf32 MMAs"}}
+        # with a 1,024-token prompt (32 pages: few CTAs for the recurrent form);
+        # for a scalar-gate headline also one request of the KDA workload
+        tf = chunked_flops_per_head_token()
+        tc_peak = tf32_peak()
+        cases = [("batch256_L512", w.resized(batch=min(w.batch, 256)), 512, 3),
+                 ("one_request_L1024", w.resized(batch=1), 1024, 5)]
+        if not spec["gate_vector"]:   # the gate-vector form too
+            kda = [x for x in W.WORKLOADS if x.format["gate_vector"]][0]
+            cases.append(("kda_one_request_L1024", kda.resized(batch=1), 1024, 5))
+        for tag, wl, L, n in cases:
+            rr = run_prefill(wl, L, n, 2, rank, world)
+            rc = run_prefill(wl, L, n, 2, rank, world, chunked=True)
+            rate_r = R.aggregate_rate(wl.pages * L, world, rr["steps"], rr["ms"])
+            rate_c = R.aggregate_rate(wl.pages * L, world, rc["steps"], rc["ms"])
+            prefill["chunked_" + tag] = {
+                "workload": wl.name, "value": rate_c, "unit": "head-tokens/s", "prompt": L, "pages": wl.pages,
+                "entry_point": "stq_prefill_chunked", "kernel": "stq::prefill_tc_kernel",
+                "ms_per_prefill": rc["ms"] / rc["steps"],
+                "recurrent_value": rate_r, "speedup_vs_recurrent": rate_c / rate_r,
+                "roofline": {"bound": "tensor", "achieved": rate_c * tf / 1e12, "peak": tc_peak[0],
+                             "unit": "TFLOP/s", "frac": rate_c * tf / 1e12 / tc_peak[0],
+                             "peak_kind": tc_peak[1], "flops_per_head_token": tf,
+                             "note": "fp32 products counted once; each runs as three tf32 MMAs"}}
 
     lifetime = run_lifetime() if not args.only else None
 
