@@ -1,35 +1,39 @@
 // stq_prefill_tc.cu -- the chunkwise prefill on the fifth-generation tensor
 // cores (sm_100a, tcgen05): a prompt of L tokens through every page of a
-// GDN (scalar-gate) state, 128 tokens per chunk, one requantization after
-// the last token.
+// state, 128 tokens per chunk, one requantization after the last token.
 //
 // Per chunk of n <= 128 tokens from the state S0 (T = S / c units, key rows
 // in natural order), with gam_i = prod of the gates of tokens 0..i of the
-// chunk (the UT-transform form of the delta rule, "repeated prefill": DASC):
+// chunk (per key channel for gate vectors; the UT-transform form of the
+// delta rule, "repeated prefill": DASC):
 //   G  = K K^T,  A_ij = beta_i rho_ij G_ij  (j < i)
 //   E  = (I + A)^-1 R,  R_i = beta_i (v_i / c - gam_i (S0^T k_i))
 //   o_i = c (gam_i S0^T q_i + sum_{j<=i} rho_ij (q_i . k_j) E_j)
 //   S  <- gam_n S0 + sum_j rho_nj k_j E_j^T
-// where rho_ij = gam_i / gam_j is formed as the product of the gates of
-// tokens j + 1 .. i (defined for zero gates and vanishing decays).
+// with rho_ij = gam_i / gam_j.  Scalar gates take it as gam_i (1 / gam_j)
+// while every cumulative decay of the chunk lies in [2^-100, 2^100]
+// (otherwise a second launch forms it as the product of the gates of tokens
+// j + 1 .. i).  Gate vectors fold gam into the operands, G = (K Gam)(K /
+// Gam)^T and so on, while every gate lies in [0, 1] and each channel's
+// decay over the chunk is at least 2^-90 (otherwise that chunk runs token
+// by token on the CUDA cores).
 // The products run on the tensor cores in tf32 with each fp32 operand split
 // into a tf32 part and its remainder (three MMAs per product: hi hi, hi lo,
 // lo hi), which keeps fp32-level accuracy; the triangular solve runs on the
 // CUDA cores (thread v owns value column v of E).
 //
-// One CTA of 256 threads per page (persistent over pages; its 168 KB of
+// One CTA of 256 threads per page (persistent over pages; 170-216 KB of
 // shared memory and all 512 tensor-memory columns keep it alone on its SM).
 // Thread t of each 128-thread half owns row t of whatever a phase computes:
 // token t, value column t, or key channel t, which is also tensor-memory
 // lane t (warps w and w + 4 see the same 32 lanes); the two halves split the
 // row's columns between them.  The triangular solve runs on the first half.
-//   shared memory: six 16 KB operand tiles (128 rows x 32 fp32, 128-byte
-//   swizzled, K-major), reused as the solve's matrix A and as the page
-//   buffer; the state X = S^T (X[v][kappa], fp32, rows padded to 129
-//   floats); per-token scalars.
-//   tensor memory: G | Y^T = S0^T K^T | P = Q K^T | O^T (X Q^T, its column
-//   i then scaled by gam_i), then the
-//   state's increment in G's columns.
+//   shared memory: six (gate vectors: eight) 16 KB operand tiles (128 rows x
+//   32 fp32, 128-byte swizzled, K-major), reused as the solve's matrix A and
+//   as the page buffer; the state X = S^T (X[v][kappa], fp32, rows padded to
+//   129 floats); per-token scalars; (gate vectors) one slab's decays.
+//   tensor memory: G | Y^T | P | O^T, then the state's increment in G's
+//   columns.
 #include "stq_rows.cuh"
 #include "stq_tc.cuh"
 
