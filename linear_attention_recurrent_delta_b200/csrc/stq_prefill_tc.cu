@@ -373,31 +373,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const DevForm
                 if constexpr (!GV) M.al[tid] = real ? A.alpha[row] : 1.f;
             }
             if constexpr (GV) {
-                // thread (kappa = t, hf) multiplies the gates of tokens 64 hf ..
-                // + 63 of key channel kappa; the decay to the chunk's end is the
-                // product of the halves.  The matrix form needs every cumulative
-                // decay in [2^-100, 2^100]: with every gate in [0, 1] and each
-                // channel's whole product at least 2^-90 (a margin for the other
-                // orders in which the kernel forms them) it is.
-                float g = 1.f;
-                bool in_range = true;
-#pragma unroll 16
-                for (int i = 64 * hf; i < 64 * hf + 64; ++i) {
-                    const float a = i < cn ? __ldg(A.alpha + ((size_t)(t0 + i) * n + p) * kD + t) : 1.f;
-                    in_range = in_range && a >= 0.f && a <= 1.f;   // a NaN fails too
-                    g = __fmul_rn(g, a);
-                }
-                M.red[0][hf][t] = g;
-                __syncthreads();
-                if (hf == 0) {
-                    const float gn = __fmul_rn(M.red[0][0][t], M.red[0][1][t]);
-                    M.gn[t] = gn;
-                    in_range = in_range && gn >= 0x1p-90f;
-                }
-                if (!__syncthreads_and(in_range)) {
-                    gv_tokens(t0, cn);   // this chunk token by token
-                    continue;
-                }
+                // (the decays are staged, and their range tested, per slab in
+                // phase A; a chunk out of range switches to gv_tokens there)
             } else {
                 __syncthreads();
                 if (tid == 0) {
@@ -416,6 +393,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const DevForm
                     break;
                 }
             }
+            bool gv_fallback = false;   // gate vectors: this chunk's decays left the range
             auto chunk_body = [&]() {
                 constexpr bool quot = QUOT;
                 if constexpr (GV) {
@@ -456,7 +434,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const DevForm
                 // gate vectors: the decays Gam[token][channel] of one slab's 32
                 // channels staged in Gs; warp s takes tokens 16 s .. + 15 of
                 // channel 32 ks + lane (segment products, then their prefixes)
-                auto stage_gam = [&](int ks) {
+                // Returns (CTA-wide) whether every gate lies in [0, 1] and every
+                // decay it formed in [2^-100, 2^100] (so 1 / Gam is finite and
+                // the decays to the chunk's end, products of gates, are at
+                // most 1); the last segment's warp records those decays.
+                auto stage_gam = [&](int ks) -> bool {
                     float av[16];
                     float pr = 1.f;
 #pragma unroll
@@ -469,15 +451,24 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const DevForm
                     __syncthreads();
                     float g = 1.f;
                     for (int s2 = 0; s2 < warp; ++s2) g = __fmul_rn(g, M.segp[s2][lane]);
+                    bool in_range = true;   // a NaN fails the test too
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
                         g = __fmul_rn(g, av[i]);
+                        in_range = in_range && av[i] >= 0.f && av[i] <= 1.f && decay_in_range(g);
                         Gs[(16 * warp + i) * kGsStride + lane] = g;
                     }
-                    __syncthreads();
+                    if (warp == kTcThreads / 32 - 1) M.gn[32 * ks + lane] = g;
+                    return __syncthreads_and(in_range) != 0;
                 };
                 load_kq(0);
-                if constexpr (GV) stage_gam(0);
+                bool gam_ok = true;
+                if constexpr (GV) {
+                    if (!stage_gam(0)) {
+                        gv_fallback = true;   // before any product of the chunk
+                        return;
+                    }
+                }
                 for (int ks = 0; ks < kD / 32; ++ks) {
                     if constexpr (GV) {
                         // row t of the K Gam, Q Gam, X and K / Gam slabs, columns 16 hf .. + 15
@@ -527,9 +518,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const DevForm
                     }
                     if (ks + 1 < kD / 32) load_kq(ks + 1);
                     if constexpr (GV) {
-                        if (ks + 1 < kD / 32) stage_gam(ks + 1);   // Gs is free: this slab's tiles are written
+                        if (ks + 1 < kD / 32) gam_ok = stage_gam(ks + 1);   // Gs is free: this slab's tiles are written
                     }
                     if (__syncthreads_or(!wait_mma())) { failed = true; break; }
+                    if (GV && !gam_ok) {
+                        gv_fallback = true;   // the products so far wrote only tensor memory
+                        return;
+                    }
                 }
                 if (failed) return;
 
@@ -886,6 +881,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const DevForm
                 tc::fence_after_sync();
             };
             chunk_body();
+            if (GV && gv_fallback && !failed) gv_tokens(t0, cn);   // this chunk token by token
         }
         if (failed) break;
         if (QUOT && leave) {
