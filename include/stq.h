@@ -344,8 +344,8 @@ stq_status stq_prefill(stq_state *s, int L, const float *d_q, const float *d_k, 
  * bit (the summation order differs), and the one requantization after the
  * last token is stq_prefill's.  Gate vectors (KDA): gam is per key channel
  * and folded into the operands (k gam, q gam, k / gam); a chunk with a gate
- * outside [0, 1] or a channel whose decay over the chunk falls below 2^-90
- * runs token by token on the CUDA cores instead.  Arguments, layouts and
+ * outside [0, 1] or a cumulative decay below 2^-100 runs token by token on
+ * the CUDA cores instead.  Arguments, layouts and
  * errors as stq_prefill.  One CTA per page (the whole shared memory and tensor
  * memory of an SM); a bounded wait that ran out is reported by
  * stq_device_status. */

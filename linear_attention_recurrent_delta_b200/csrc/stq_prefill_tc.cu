@@ -14,9 +14,9 @@
 // while every cumulative decay of the chunk lies in [2^-100, 2^100]
 // (otherwise a second launch forms it as the product of the gates of tokens
 // j + 1 .. i).  Gate vectors fold gam into the operands, G = (K Gam)(K /
-// Gam)^T and so on, while every gate lies in [0, 1] and each channel's
-// decay over the chunk is at least 2^-90 (otherwise that chunk runs token
-// by token on the CUDA cores).
+// Gam)^T and so on, while every gate lies in [0, 1] and every cumulative
+// decay in [2^-100, 1] (tested on the staged decays, slab by slab; a chunk
+// that fails runs token by token on the CUDA cores).
 // The products run on the tensor cores in tf32 with each fp32 operand split
 // into a tf32 part and its remainder (three MMAs per product: hi hi, hi lo,
 // lo hi), which keeps fp32-level accuracy; the triangular solve runs on the
