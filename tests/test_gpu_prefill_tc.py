@@ -220,3 +220,85 @@ def test_bounded_wait_times_out_and_writes_nothing(name):
                                    x["k"][:, b, h].numpy(), x["v"][:, b, h].numpy(), x["alpha"][:, b, h].numpy(),
                                    x["beta"][:, b, h].numpy(), 128)
     assert rel_l2(o_g[:, b, h], o64) <= 1e-5
+
+
+def _tc_sample_positions(n, seed):
+    """Pages to check in a full-size launch: every page when there are few,
+    else the ends, both sides of each wrap of the one-CTA-per-SM persistent
+    grid, and seeded random positions."""
+    if n <= 64:
+        return list(range(n))
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    pos = {0, 1, n - 2, n - 1}
+    for m in (1, 2, n // sms):
+        for d in (-1, 0):
+            if 0 <= m * sms + d < n:
+                pos.add(m * sms + d)
+    rng = np.random.default_rng(seed)
+    pos.update(int(x) for x in rng.integers(0, n, 10))
+    return sorted(pos)
+
+
+SMALL_BATCH = 4   # CPU-generated requests the sampled pages are drawn from
+
+
+@pytest.mark.parametrize("name,batch,L", [("damp", 256, 512), ("damp", 1, 1024), ("stepquant4_kda", 1, 1024)])
+def test_full_size_chunked_prefill_on_sampled_pages(name, batch, L):
+    """The benchmark's launch configurations of stq_prefill_chunked (256
+    requests x 32 heads x 512 tokens; one request x 32 heads x 1,024 tokens,
+    scalar gates and gate vectors), checked on sampled pages against the
+    fp64 chunk algebra.  The state is the GPU's quantization of a
+    device-generated fp32 state except at the sampled positions, which hold
+    oracle-made pages of a small CPU-generated batch with CPU-generated
+    prompts; the bar is the one above (o and final state within rel-L2
+    1e-5, the requantized page the requantization of the kernel's state)."""
+    w = [x for x in W.WORKLOADS if x.fmt == name and x.index > 0][0].resized(batch=batch)
+    H, n = w.heads, w.pages
+    fmt = O.format_from_spec(w.format)
+    S_small = W.initial_state(w, batch=SMALL_BATCH).numpy()
+    perm = O.rank_rows(fmt, S_small)
+    pos = _tc_sample_positions(n, w.seed + 5)
+    src = [(i % SMALL_BATCH, p % H) for i, p in enumerate(pos)]
+    pages = [O.quantize_page(fmt, S_small[b, h], perm[h]) for b, h in src]
+
+    qs = make_state(w)
+    qs.perm().copy_(torch.from_numpy(np.ascontiguousarray(perm, np.uint8)))
+    S_dev = W.initial_state(w, device="cuda")
+    B.stq_quantize_state(qs.state, S_dev)
+    del S_dev
+    torch.cuda.synchronize()
+    idx = torch.tensor(pos, dtype=torch.long, device="cuda")
+    qs.pages()[idx] = torch.from_numpy(np.stack([O.pack_page(fmt, pg) for pg in pages])).cuda()
+
+    xd = {k: torch.stack([W.step_inputs(w, l, device="cuda")[k] for l in range(L)]).contiguous()
+          for k in ("q", "k", "v", "alpha", "beta")}
+    xc = [W.step_inputs(w, l, batch=SMALL_BATCH) for l in range(L)]
+    for k in xd:
+        flat = xd[k].view(L, n, -1)
+        flat[:, idx] = torch.stack([torch.stack([xc[l][k][b, h].reshape(-1) for b, h in src])
+                                    for l in range(L)]).cuda()
+    seed = W.sr_seed(w)
+    o = torch.full((L, w.batch, H, 128), float("nan"), device="cuda")
+    S_out = torch.empty(w.batch, H, 128, 128, device="cuda")
+    B.stq_prefill_chunked(qs.state, xd["q"], xd["k"], xd["v"], xd["alpha"], xd["beta"], o, S_out, seed, 3)
+    assert B.stq_device_status(qs.state) == B.STQ_OK
+    got_o = o.view(L, n, 128)[:, idx].cpu().numpy()
+    got_S = S_out.view(n, 128, 128)[idx].cpu().numpy()
+    got_pages = qs.pages()[idx].cpu().numpy()
+    del xd, o, S_out
+    ties, worst_o, worst_s = 0, 0.0, 0.0
+    for i, (p, (b, h)) in enumerate(zip(pos, src)):
+        arr = {k: np.stack([xc[l][k][b, h].numpy() for l in range(L)]) for k in ("q", "k", "v", "alpha", "beta")}
+        o64, S64 = O.prefill_chunked_f64(fmt, pages[i], perm[h], arr["q"], arr["k"], arr["v"], arr["alpha"],
+                                         arr["beta"], 128)
+        eo, es = rel_l2(got_o[:, i], o64), rel_l2(got_S[i], S64)
+        worst_o, worst_s = max(worst_o, eo), max(worst_s, es)
+        assert eo <= 1e-5, ("o", p, eo)
+        assert es <= 1e-5, ("state", p, es)
+        pg = O.unpack_page(fmt, got_pages[i])
+        c = pages[i].c.astype(np.float64) if fmt.col_scales else np.ones(128)
+        T = got_S[i].astype(np.float64)[perm[h]] / c
+        assert np.array_equal(pg.c.view(np.uint32), pages[i].c.view(np.uint32))
+        ties += _check_requant(fmt, pg, T, seed, 3, p // H, p % H)
+    print("\n%s, %d x %d pages, L = %d, %d sampled: max o rel-L2 %.2e, max state rel-L2 %.2e, near-tie codes %d"
+          % (name, w.batch, H, L, len(pos), worst_o, worst_s, ties))
