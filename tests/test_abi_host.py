@@ -213,7 +213,8 @@ def test_window_step_checks_arguments(lib):
     lib.stq_state_free(h)
 
 
-def test_prefill_checks_arguments(lib):
+@pytest.mark.parametrize("entry", ["stq_prefill", "stq_prefill_chunked"])
+def test_prefill_checks_arguments(lib, entry):
     fmt = B.format_from_spec(W.FORMATS["stepquant4_kda"])
     st, h = _alloc(lib, fmt, 2, 3)
     assert st == B.STQ_OK
@@ -221,10 +222,11 @@ def test_prefill_checks_arguments(lib):
     base = 1 << 41
     q, k, v, a, b, o = (base + i * (1 << 26) for i in range(6))
     S = 1 << 45
+    fn = getattr(lib, entry)
 
     def call(L=4, q=q, a=a, o=o, S_out=None, state=h):
-        return lib.stq_prefill(state, L, P(q) if q else None, P(k), P(v), P(a), P(b), P(o),
-                               P(S_out) if S_out else None, 0, 0, None)
+        return fn(state, L, P(q) if q else None, P(k), P(v), P(a), P(b), P(o),
+                  P(S_out) if S_out else None, 0, 0, None)
 
     assert call(state=None) == B.STQ_ERR_INVALID_ARG
     assert call(q=0) == B.STQ_ERR_INVALID_ARG
@@ -236,6 +238,12 @@ def test_prefill_checks_arguments(lib):
     assert call(o=q + 256) == B.STQ_ERR_INVALID_ARG               # output overlaps an input
     assert call(o=FAKE + 512) == B.STQ_ERR_INVALID_ARG            # output overlaps the state
     assert call(S_out=o) == B.STQ_ERR_INVALID_ARG                 # the state output overlaps o
+    lib.stq_state_free(h)
+    # scalar gates: alpha needs 4-byte alignment
+    st, h = _alloc(lib, B.format_from_spec(W.FORMATS["int8row"]), 2, 3)
+    assert st == B.STQ_OK
+    assert call(a=a + 2, state=h) == B.STQ_ERR_MISALIGNED
+    assert call(L=-1, state=h) == B.STQ_ERR_INVALID_ARG
     lib.stq_state_free(h)
 
 
