@@ -332,9 +332,11 @@ def run_gpu(w, steps, warmup, rank, world, sample_clocks=True, e2e_steps=16, pag
     # end to end through the pipelined host-buffer entry point: every step's
     # H2D of its inputs from pinned memory, the step and the D2H of its o,
     # all inside the timed region; the copies of neighbouring steps overlap
-    # the step (stq_decode_steps_host).  4 distinct steps of inputs, passed
-    # e2e_steps / 4 times.
-    chunk = 4
+    # the step (stq_decode_steps_host).  8 distinct steps of inputs, passed
+    # e2e_steps / 8 times (a call's copies start after the work before it on
+    # the stream, the previous call's last copy-out included, so the
+    # pipeline refills once per call).
+    chunk = 8
     host = {k: torch.stack([x[k] for x in [W.step_inputs(wr, t) for t in range(chunk)]]).contiguous().pin_memory()
             for k in inputs[0]}
     del inputs
@@ -360,10 +362,44 @@ def run_gpu(w, steps, warmup, rank, world, sample_clocks=True, e2e_steps=16, pag
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
     e2e_steps = n_calls * chunk
     barrier(world)
-    del qs, host, io_buf
+    # the same inputs' host-to-device copies alone, from the same pinned
+    # buffers: the PCIe bound of the end-to-end rate
+    del io_buf
+    dst = {k: torch.empty(v[0].shape, dtype=v.dtype, device=dev) for k, v in host.items()}
+    for k in host:
+        dst[k].copy_(host[k][0], non_blocking=True)
+    torch.cuda.synchronize()
+    n_copy = 8
+    c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    c0.record(stream)
+    for r in range(n_copy):
+        for k in host:
+            dst[k].copy_(host[k][r % chunk], non_blocking=True)
+    c1.record(stream)
+    torch.cuda.synchronize()
+    h2d_ms = max_over_ranks(c0.elapsed_time(c1), world) / n_copy
+    # and with each step's o copied back at the same time on a second stream
+    # (both directions of the link busy, as in the pipelined steps)
+    o_dev = torch.empty(o_host[0].shape, dtype=o_host.dtype, device=dev)
+    side = torch.cuda.Stream(device=dev)
+    side.wait_stream(stream)
+    torch.cuda.synchronize()
+    c0.record(stream)
+    side.wait_event(c0)
+    for r in range(n_copy):
+        for k in host:
+            dst[k].copy_(host[k][r % chunk], non_blocking=True)
+        with torch.cuda.stream(side):
+            o_host[r % chunk].copy_(o_dev, non_blocking=True)
+    stream.wait_stream(side)
+    c1.record(stream)
+    torch.cuda.synchronize()
+    both_ms = max_over_ranks(c0.elapsed_time(c1), world) / n_copy
+    barrier(world)
+    del qs, host, dst, o_dev
     torch.cuda.empty_cache()
     return {"ms": ms_max, "clocks": clk, "reps": reps, "e2e_ms": e2e_ms, "h2d": h2d, "d2h": d2h,
-            "e2e_steps": e2e_steps}
+            "e2e_steps": e2e_steps, "h2d_copy_ms": h2d_ms, "copies_ms": both_ms}
 
 
 def run_window(w, window, steps, warmup, rank, world):
@@ -729,6 +765,9 @@ def main():
     bpp = roof["bytes_per_head_step"]
     peak, peak_kind = roof["peak"], roof["peak_kind"]
     e2e_value = R.aggregate_rate(w.pages, world, res["e2e_steps"], res["e2e_ms"])
+    # the rate the host-to-device copies alone allow (one step's inputs per copy)
+    pcie_value = R.aggregate_rate(w.pages, world, 1, res["h2d_copy_ms"])
+    copies_value = R.aggregate_rate(w.pages, world, 1, res["copies_ms"])
 
     paged = None
     if not args.only:
@@ -838,7 +877,16 @@ def main():
                          if cpu_v else None),
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"],
                 "steps": res["e2e_steps"], "entry_point": "stq_decode_steps_host",
-                "overlap": "copies of neighbouring steps overlap the step (two staging slots)"},
+                "overlap": "copies of neighbouring steps overlap the step (two staging slots)",
+                "h2d_copy": {"ms_per_step": res["h2d_copy_ms"],
+                             "gbs": res["h2d"] / (res["h2d_copy_ms"] / 1000.0) / 1e9,
+                             "bound_value": pcie_value, "frac": e2e_value / pcie_value,
+                             "note": "the step's input copies alone from the same pinned buffers, "
+                                     "timed by CUDA events: the PCIe bound of value"},
+                "copies_both_ways": {"ms_per_step": res["copies_ms"], "bound_value": copies_value,
+                                     "frac": e2e_value / copies_value,
+                                     "note": "the input copies with o copied back at the same time on a "
+                                             "second stream, no kernel"}},
         "gpu_launches": args.steps * world,   # one decode_kernel launch per step and rank (timed region)
         "clocks": res["clocks"],
         "other_workloads": others,
