@@ -565,6 +565,53 @@ def run_lifetime(samples=32, batch=64, reps=20):
             "heads": w.heads, "format": w.fmt, "bytes_read": nbytes}
 
 
+def run_quantizer(batch=256, reps=3, iters=4):
+    """The quantizer side on a stepquant6 state of `batch` requests (column
+    scales, so the joint fit has both scales to fit): device time per call of
+    stq_calibrate, stq_quantize_state, stq_quantize_state_fit (`iters`
+    rounds, impact weights = the mean q^2 of 8 steps' queries per head and
+    channel) and stq_dequantize_state, with the HBM rate of the bytes each
+    call must move (fp32 state 64 KiB per page, the packed page)."""
+    from linear_attention_recurrent_delta_b200 import binding as B
+    w = [x for x in W.WORKLOADS if x.fmt == "stepquant6" and x.index > 0][0].resized(batch=batch)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    qs = B.QuantizedState(w.format, w.batch, w.heads, device=dev)
+    S = W.initial_state(w, device=dev)
+    imp = torch.stack([W.step_inputs(w, t, device=dev)["q"] for t in range(8)]).square().mean(dim=(0, 1)).contiguous()
+    ws = torch.empty(max(B.stq_calibrate_workspace_bytes(qs.state), 8), dtype=torch.uint8, device=dev)
+    S_back = torch.empty_like(S)
+    stream = torch.cuda.current_stream()
+    calls = {
+        "stq_calibrate": lambda: B.stq_calibrate(qs.state, S, None, ws, stream),
+        "stq_quantize_state": lambda: B.stq_quantize_state(qs.state, S, stream),
+        "stq_quantize_state_fit": lambda: B.stq_quantize_state_fit(qs.state, S, imp, iters, stream),
+        "stq_dequantize_state": lambda: B.stq_dequantize_state(qs.state, S_back, stream),
+    }
+    state_b = 128 * 128 * 4
+    page_b = B.stq_page_bytes(B.format_from_spec(w.format))
+    moved = {"stq_calibrate": state_b, "stq_quantize_state": state_b + page_b,
+             "stq_quantize_state_fit": state_b + page_b, "stq_dequantize_state": page_b + state_b}
+    out = {"workload": w.name, "pages": w.pages, "fit_rounds": iters}
+    for name, fn in calls.items():
+        fn()
+        torch.cuda.synchronize()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record(stream)
+        for _ in range(reps):
+            fn()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        ms = ev0.elapsed_time(ev1) / reps
+        gbs = moved[name] * w.pages / (ms / 1000.0) / 1e9
+        out[name] = {"ms": ms, "bytes_per_page": moved[name], "hbm_gbs": gbs}
+    status = B.stq_device_status(qs.state)
+    if status != B.STQ_OK:
+        raise RuntimeError("device status: %s" % B.stq_status_string(status))
+    del qs, S, S_back, ws
+    torch.cuda.empty_cache()
+    return out
+
+
 class OracleSample:
     """The CPU oracle (single thread, as written) stepping a sample of the
     workload's pages: the first ``n_pages`` pages of a batch whose fp32 state
@@ -825,6 +872,7 @@ def main():
                              "note": "fp32 products counted once; each runs as three tf32 MMAs"}}
 
     lifetime = run_lifetime() if not args.only else None
+    quantizer = run_quantizer() if (not args.only and rank == 0) else None
 
     # every other workload of the metric, each with its own roofline, clock
     # record and (rank 0, one GPU) CPU baseline
@@ -891,6 +939,7 @@ def main():
         "clocks": res["clocks"],
         "other_workloads": others,
         "paged_step": paged,
+        "quantizer": quantizer,
         "lifetime_weights": ({"entry_point": "stq_lifetime_weights", "kernel": "stq::lifetime_kernel",
                               "note": "cold path, once per calibration; one thread per (head, channel)",
                               **lifetime} if lifetime else None),
