@@ -51,6 +51,7 @@ struct DecodeArgs {
 };
 
 constexpr int kMaxStages = 4;
+constexpr int kSlotThread = 32;   // paged step: the thread (warp 1) that fetches and resolves slots
 
 struct SmemFixed {
     // per warp, its 32 rows in slice order (row 4b + i = block b, row i):
@@ -66,8 +67,11 @@ struct SmemFixed {
     uint64_t full[kMaxStages];              // stage-full barriers
     uint64_t never;                         // a barrier nothing completes (test hook)
     int pg[kMaxStages];                     // paged step: page in each stage (-1: bad slot)
+    int slot[kMaxStages];                   // paged step: the request's slot in each stage
     int bad[2];                             // paged step, per page parity: the page's slot was bad
-    int pf_slot;                            // paged step: slot of the next refill's item (async copy)
+    int pf_slot;                            // paged step: slot of a later refill's item (async copy)
+    int pf_b, pf_h;                         // paged step: that item's input row and head
+    int next_pg[2], next_slot[2];           // paged step, per page parity: the refill item's page, slot
 };
 
 constexpr size_t kFixedBytes = (sizeof(SmemFixed) + 127) / 128 * 128;
@@ -105,11 +109,11 @@ __device__ __forceinline__ int item_slot(const DecodeArgs &A, int p) {
     return __ldg(A.slots + p / A.heads);
 }
 
-// Start copying the slot of work item p into *dst (4-byte async copy; no
-// register holds it while it is in flight); cp_async_wait() before reading.
-__device__ __forceinline__ void prefetch_slot(const DecodeArgs &A, int p, int *dst) {
+// Start copying the slot of input row `row` into *dst (4-byte async copy;
+// no register holds it while it is in flight); cp_async_wait() before reading.
+__device__ __forceinline__ void prefetch_slot(const DecodeArgs &A, int row, int *dst) {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n\tcp.async.commit_group;"
-                 :: "r"(smem_u32(dst)), "l"(A.slots + p / A.heads) : "memory");
+                 :: "r"(smem_u32(dst)), "l"(A.slots + row) : "memory");
 }
 
 __device__ __forceinline__ void cp_async_wait() {
@@ -176,13 +180,24 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
     const int n = A.n_pages;
     const int NS = A.n_stages;
     if constexpr (SLOTS) {
-        // lanes of warp 0 look up the first stages' pages in parallel
+        // lanes of warp 0 look up the first stages' pages in parallel; warp
+        // 1 starts fetching the slot of the first refill's item
         if (tid < NS) {
             const int p = (int)blockIdx.x + tid * stride;
             if (p < n) {
-                const int pg = slot_page(A, p, item_slot(A, p));
+                const int sl = item_slot(A, p);
+                const int pg = slot_page(A, p, sl);
                 S.pg[tid] = pg;
+                S.slot[tid] = sl;
                 if (pg < 0) atomicOr(A.status, kStatusBadSlot);
+            }
+        }
+        if (tid == kSlotThread) {
+            const int p = (int)blockIdx.x + NS * stride;
+            if (p < n) {
+                S.pf_b = p / A.heads;
+                S.pf_h = p % A.heads;
+                prefetch_slot(A, S.pf_b, &S.pf_slot);
             }
         }
         __syncwarp();
@@ -195,10 +210,6 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
                 if constexpr (SLOTS) pg = S.pg[i];
                 issue_stage<SLOTS>(F, A, stages + i * A.stage_bytes, p, &S.full[i], pg);
             }
-        }
-        if constexpr (SLOTS) {
-            const int p = (int)blockIdx.x + NS * stride;
-            if (p < n) prefetch_slot(A, p, &S.pf_slot);
         }
     }
     // (request, head) of a page is carried along: p advances by `stride`,
@@ -341,8 +352,8 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
                         mbar_wait_bounded(&S.full[j % NS], (uint32_t)((j / NS) & 1), A.wait_limit_ns);
                 }
                 bulk_wait<0>();
-                if constexpr (SLOTS) cp_async_wait();   // no copy outlives the CTA
             }
+            if (SLOTS && tid == kSlotThread) cp_async_wait();   // no copy outlives the CTA
             __syncthreads();
             return;
         }
@@ -362,15 +373,39 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
                 const int pr = (int)blockIdx.x + j * stride;
                 if (pr < n) {
                     int pg = pr;
-                    if constexpr (SLOTS) {   // the slot of item pr was loaded a page ago
-                        cp_async_wait();
-                        pg = slot_page(A, pr, S.pf_slot);
+                    if constexpr (SLOTS) {   // looked up by the slot thread a page ago
+                        pg = S.next_pg[it & 1];
                         S.pg[j % NS] = pg;
-                        if (pg < 0) atomicOr(A.status, kStatusBadSlot);
-                        if (pr + stride < n) prefetch_slot(A, pr + stride, &S.pf_slot);
+                        S.slot[j % NS] = S.next_slot[it & 1];
                     }
                     fence_proxy_async_smem();
                     issue_stage<SLOTS>(F, A, stages + (j % NS) * A.stage_bytes, pr, &S.full[j % NS], pg);
+                }
+            }
+        }
+        if constexpr (SLOTS) {
+            // the slot thread (off the copy thread's path) looks up the page
+            // of the item the next page's refill loads, from the slot fetched
+            // a page ago, and starts fetching the one after it
+            if (tid == kSlotThread && (kEarly || it >= 1)) {
+                const int j = kEarly ? it + NS : it - 1 + NS;
+                const int pr = (int)blockIdx.x + j * stride;
+                if (pr < n) {
+                    // item pr is (row pf_b, head pf_h); the next one is
+                    // `stride` further: (stride / H, stride % H) with a carry
+                    cp_async_wait();
+                    const int sl = S.pf_slot, rb = S.pf_b, rh = S.pf_h;
+                    const int pg = (sl >= 0 && sl < A.n_slots) ? sl * H + rh : -1;
+                    S.next_pg[(it + 1) & 1] = pg;
+                    S.next_slot[(it + 1) & 1] = sl;
+                    if (pg < 0) atomicOr(A.status, kStatusBadSlot);
+                    if (pr + stride < n) {
+                        int nb = rb + sb, nh = rh + sh;
+                        if (nh >= H) { nh -= H; ++nb; }
+                        S.pf_b = nb;
+                        S.pf_h = nh;
+                        prefetch_slot(A, nb, &S.pf_slot);
+                    }
                 }
             }
         }
@@ -425,12 +460,10 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
                 const int pr = (int)blockIdx.x + j * stride;
             if (pr < n) {
                 int pg = pr;
-                if constexpr (SLOTS) {   // the slot of item pr was loaded a page ago
-                    cp_async_wait();
-                    pg = slot_page(A, pr, S.pf_slot);
+                if constexpr (SLOTS) {   // looked up by the slot thread a page ago
+                    pg = S.next_pg[it & 1];
                     S.pg[j % NS] = pg;
-                    if (pg < 0) atomicOr(A.status, kStatusBadSlot);
-                    if (pr + stride < n) prefetch_slot(A, pr + stride, &S.pf_slot);
+                    S.slot[j % NS] = S.next_slot[it & 1];
                 }
                 fence_proxy_async_smem();
                 issue_stage<SLOTS>(F, A, stages + (j % NS) * A.stage_bytes, pr, &S.full[j % NS], pg);
@@ -463,7 +496,7 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
         // S7 + S8, into the stage
         SrCtx sr;
         sr.k0 = A.seed_lo; sr.k1 = A.seed_hi; sr.step = A.step;
-        if constexpr (SLOTS) sr.b = (uint32_t)(S.pg[st] / H);   // the request's slot in the state
+        if constexpr (SLOTS) sr.b = (uint32_t)S.slot[st];   // the request's slot in the state
         else sr.b = (uint32_t)pb;
         sr.h = (uint32_t)ph;
         static_for<0, kBlocks>([&](auto bc) {
@@ -498,10 +531,8 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
         if (warp == kWarps - 1)
             write_o(S.red_o[(it - 1) & 1], A, p_prev, lane, S.cpg[(it - 1) & 1], col_scales, SLOTS && S.bad[(it - 1) & 1]);
     }
-    if (tid == 0) {
-        bulk_wait<0>();
-        if constexpr (SLOTS) cp_async_wait();   // no copy outlives the CTA
-    }
+    if (tid == 0) bulk_wait<0>();
+    if (SLOTS && tid == kSlotThread) cp_async_wait();   // no copy outlives the CTA
 }
 
 static int decode_stages(size_t stride, int ctas_per_sm) {
