@@ -15,7 +15,7 @@ import oracle as O
 from linear_attention_recurrent_delta_b200 import binding as B
 from linear_attention_recurrent_delta_b200 import workloads as W
 
-from parity_util import download, make_state, oracle_quantize, upload
+from parity_util import download, make_state, oracle_quantize, oracle_step, upload
 
 pytestmark = pytest.mark.gpu
 
@@ -123,3 +123,43 @@ def test_request_copy_out_and_back_restores_it():
     qs.view[off:off + nbytes].copy_(saved)          # a plain device copy restores request 4
     got = download(qs)
     assert np.array_equal(got[4 * HEADS:5 * HEADS], pages[4 * HEADS:5 * HEADS])
+
+
+@pytest.mark.parametrize("name", ["stepquant6", "int8row", "stepquant4_kda", "damp"])
+def test_many_pages_per_cta_with_a_bad_slot(name):
+    """More work than the persistent grid holds at once (800 requests x 4
+    heads: every CTA refills its ring several times, so the slots of later
+    items are resolved inside the page loop), a random permutation of the
+    slots, and one row near the end naming a slot outside the state.  The
+    oracle steps every page with its row's inputs in slot order; the pages
+    of the slot the bad row displaced stay as they were."""
+    base = [w for w in W.WORKLOADS if w.fmt == name and w.index > 0][0]
+    w = base.resized(batch=800, heads=4, steps=2)
+    H = w.heads
+    S = W.initial_state(w).numpy()
+    fmt, perm, pages = oracle_quantize(w, S)
+    qs = make_state(w)
+    upload(qs, perm, pages)
+    rng = np.random.default_rng(5)
+    table = rng.permutation(w.batch).astype(np.int32)
+    bad_row = 700                      # item 2,800: past the first ring fill of every CTA
+    dropped = int(table[bad_row])
+    table[bad_row] = w.batch + 17
+    x = W.step_inputs(w, 0)
+    seed = W.sr_seed(w)
+    xd = {k: v.cuda() for k, v in x.items()}
+    o = torch.empty(w.batch, H, 128, device="cuda")
+    B.stq_decode_step_slots(qs.state, torch.from_numpy(table).cuda(), xd["q"], xd["k"], xd["v"], xd["alpha"],
+                            xd["beta"], o, seed=seed, step=1)
+    assert B.stq_device_status(qs.state, clear=True) == B.STQ_ERR_INVALID_ARG
+    good = np.array([i for i in range(w.batch) if i != bad_row])
+    xs = {k: torch.zeros_like(v) for k, v in x.items()}
+    for k in x:
+        xs[k][torch.from_numpy(table[good]).long()] = x[k][torch.from_numpy(good)]
+    expect, o_ref = oracle_step(fmt, w, w.batch, H, pages, perm, xs, seed, 1)
+    expect[dropped * H:(dropped + 1) * H] = pages[dropped * H:(dropped + 1) * H]
+    got = download(qs)
+    o = o.cpu().numpy()
+    assert np.isnan(o[bad_row]).all()
+    assert np.array_equal(o[good], o_ref.reshape(w.batch, H, 128)[table[good]])
+    assert np.array_equal(got, expect)
