@@ -499,6 +499,7 @@ decode_kernel(const DevFormat F, const DecodeArgs A) {
         if constexpr (SLOTS) sr.b = (uint32_t)S.slot[st];   // the request's slot in the state
         else sr.b = (uint32_t)pb;
         sr.h = (uint32_t)ph;
+        if constexpr (SR) sr.fix();
         static_for<0, kBlocks>([&](auto bc) {
             constexpr int b = decltype(bc)::value;
             const float4 i4 = *reinterpret_cast<const float4 *>(&S.inv[warp][4 * b]);

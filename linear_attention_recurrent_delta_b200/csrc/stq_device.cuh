@@ -246,17 +246,30 @@ __device__ __forceinline__ uint32_t low_bytes(float y0, float y1, float y2, floa
 // pcg4d (Jarzynski and Olano, "Hash Functions for GPU Rendering", JCGT 9(3),
 // 2020): a linear congruential step on each word, each word plus the product
 // of two others, a 16-bit xorshift of every word, the products once more.
-// Input: the counter (c.x, c.y) and (c.z, c.w) xor the 64-bit seed (k0, k1).
-__device__ __forceinline__ uint4 sr_hash4(uint4 c, uint32_t k0, uint32_t k1) {
-    uint32_t x = c.x, y = c.y, z = c.z ^ k0, w = c.w ^ k1;
-    x = x * 1664525u + 1013904223u;
-    y = y * 1664525u + 1013904223u;
-    z = z * 1664525u + 1013904223u;
-    w = w * 1664525u + 1013904223u;
-    x += y * w;
-    y += z * x;
-    z += x * y;
-    w += y * z;
+// Input: the counter (x, step, request, head), the last two words xor the
+// 64-bit seed (k0, k1).  Within a page only x changes, so the terms the
+// other three words fix -- their congruential step and the product y w of
+// the first mixing round -- are formed once per page (sr_fix) and each hash
+// starts from x alone (sr_hash4_fixed): the same operations modulo 2^32,
+// the constant terms added first.
+struct SrFixed {
+    uint32_t y1, z1, w1, cx;
+};
+
+__device__ __forceinline__ SrFixed sr_fix(uint32_t y, uint32_t z, uint32_t w, uint32_t k0, uint32_t k1) {
+    SrFixed f;
+    f.y1 = y * 1664525u + 1013904223u;
+    f.z1 = (z ^ k0) * 1664525u + 1013904223u;
+    f.w1 = (w ^ k1) * 1664525u + 1013904223u;
+    f.cx = 1013904223u + f.y1 * f.w1;
+    return f;
+}
+
+__device__ __forceinline__ uint4 sr_hash4_fixed(uint32_t x0, const SrFixed &f) {
+    uint32_t x = x0 * 1664525u + f.cx;
+    uint32_t y = f.y1 + f.z1 * x;
+    uint32_t z = f.z1 + x * y;
+    uint32_t w = f.w1 + y * z;
     x ^= x >> 16;
     y ^= y >> 16;
     z ^= z >> 16;

@@ -322,6 +322,7 @@ __global__ void __launch_bounds__(kThreads, 3) prefill_kernel(const DevFormat F,
         sr.k0 = A.seed_lo; sr.k1 = A.seed_hi; sr.step = A.step;
         sr.b = (uint32_t)pb;
         sr.h = (uint32_t)ph;
+        if constexpr (SR) sr.fix();
         static_for<0, kBlocks>([&](auto bc) {
             constexpr int b = decltype(bc)::value;
             const float4 i4 = *reinterpret_cast<const float4 *>(&S.inv[warp][4 * b]);

@@ -912,6 +912,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const DevForm
         sr.k0 = A.seed_lo; sr.k1 = A.seed_hi; sr.step = A.step;
         sr.b = (uint32_t)pb;
         sr.h = (uint32_t)ph;
+        if constexpr (SR) sr.fix();
         auto finish_half = [&](auto hc) {
             constexpr int H = decltype(hc)::value;
             Tile T;

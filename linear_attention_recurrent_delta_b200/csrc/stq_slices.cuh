@@ -266,6 +266,8 @@ __device__ __forceinline__ void dequant_slice(const uint8_t *blk, int w, int lan
 // ---- S7 + S8 on slice w of block B, in place in the stage
 struct SrCtx {
     uint32_t k0, k1, step, b, h;
+    SrFixed f;   // the hash's terms fixed by (step, b, h) and the seed: set by fix()
+    __device__ __forceinline__ void fix() { f = sr_fix(step, b, h, k0, k1); }
 };
 
 template <int W, int B, bool SR>
@@ -297,8 +299,7 @@ __device__ __forceinline__ void requant_slice(uint8_t *blk, int w, int lane, con
             float2 y0, y1, y2, y3;
             if constexpr (SR) {
                 const uint32_t s = 16u * B + 4u * (uint32_t)w + (uint32_t)i;   // stored row, even
-                const uint4 h = sr_hash4(make_uint4((s >> 1) * 32u + (uint32_t)lane, sr.step, sr.b, sr.h),
-                                              sr.k0, sr.k1);
+                const uint4 h = sr_hash4_fixed((s >> 1) * 32u + (uint32_t)lane, sr.f);
                 y0 = __fadd2_rd(__ffma2_rd(T[B][i][0], i0, sr_offset_pair(h.x)), Mf2);
                 y1 = __fadd2_rd(__ffma2_rd(T[B][i][1], i0, sr_offset_pair(h.y)), Mf2);
                 y2 = __fadd2_rd(__ffma2_rd(T[B][i + 1][0], i1, sr_offset_pair(h.z)), Mf2);
