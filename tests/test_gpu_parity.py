@@ -379,3 +379,38 @@ def test_pipelined_host_steps_equal_device_steps(n):
     for t in range(n):
         assert torch.equal(ho[t], o_dev[t]), t
     assert torch.equal(qa.pages(), qb.pages())
+
+
+def test_pipelined_host_calls_back_to_back():
+    """Two stq_decode_steps_host calls of three steps each on one staging
+    buffer, with no host synchronization between them (the second call's
+    first copies may only start once the first call's steps no longer need
+    the slots): the o and pages of six device steps."""
+    w = _small("damp", batch=8, heads=6, steps=6)
+    S = W.initial_state(w).numpy()
+    fmt, perm, pages = oracle_quantize(w, S)
+    qa, qb = make_state(w), make_state(w)
+    upload(qa, perm, pages)
+    upload(qb, perm, pages)
+    xs = [W.step_inputs(w, t) for t in range(6)]
+    o_dev = []
+    for t, x in enumerate(xs):
+        xd = {k: v.cuda() for k, v in x.items()}
+        o_dev.append(qa.step(xd["q"], xd["k"], xd["v"], xd["alpha"], xd["beta"], seed=9, step=t).cpu())
+    io_bytes = 2 * B.stq_decode_io_bytes(qb.state)
+    io_raw = torch.empty(io_bytes + 256, dtype=torch.uint8, device="cuda")
+    off = (-io_raw.data_ptr()) % 256
+    io = io_raw[off:off + io_bytes]
+    hos = []
+    for c in range(2):
+        part = xs[3 * c:3 * c + 3]
+        host = {k: torch.stack([x[k] for x in part]).contiguous().pin_memory() for k in part[0]}
+        ho = torch.full((3, 8, 6, 128), float("nan")).pin_memory()
+        B.stq_decode_steps_host(qb.state, host["q"], host["k"], host["v"], host["alpha"], host["beta"], ho, io,
+                                seed=9, step=3 * c)
+        hos.append((host, ho))      # the host buffers stay alive until the stream is done
+    torch.cuda.synchronize()
+    assert B.stq_device_status(qb.state) == B.STQ_OK
+    for t in range(6):
+        assert torch.equal(hos[t // 3][1][t % 3], o_dev[t]), t
+    assert torch.equal(qa.pages(), qb.pages())
