@@ -163,3 +163,34 @@ def test_many_pages_per_cta_with_a_bad_slot(name):
     assert np.isnan(o[bad_row]).all()
     assert np.array_equal(o[good], o_ref.reshape(w.batch, H, 128)[table[good]])
     assert np.array_equal(got, expect)
+
+
+@pytest.mark.parametrize("stochastic", [False, True])
+def test_runtime_format(stochastic, monkeypatch):
+    """A format outside the four compiled-in ones (block widths read at run
+    time) through the slot table, many pages per CTA."""
+    name = "slots_runtime_%d" % stochastic
+    spec = {"groups": [(32, "int", 7), (16, "fp16", 0), (48, "int", 5), (32, "int", 2)], "col_scales": True,
+            "gate_vector": True, "stochastic": stochastic}
+    monkeypatch.setitem(W.FORMATS, name, spec)
+    kda = [w for w in W.WORKLOADS if w.fmt == "stepquant4_kda" and w.index > 0][0]
+    w = W.Workload(kda.index, name, name, 400, 4, 2, kda.gate_mu, kda.gate_sigma, kda.seed + 13)
+    H = w.heads
+    S = W.initial_state(w).numpy()
+    fmt, perm, pages = oracle_quantize(w, S)
+    qs = make_state(w)
+    upload(qs, perm, pages)
+    table = np.random.default_rng(8).permutation(w.batch).astype(np.int32)
+    x = W.step_inputs(w, 0)
+    seed = W.sr_seed(w)
+    xd = {k: v.cuda() for k, v in x.items()}
+    o = torch.empty(w.batch, H, 128, device="cuda")
+    B.stq_decode_step_slots(qs.state, torch.from_numpy(table).cuda(), xd["q"], xd["k"], xd["v"], xd["alpha"],
+                            xd["beta"], o, seed=seed, step=2)
+    assert B.stq_device_status(qs.state) == B.STQ_OK
+    xs = {k: torch.zeros_like(v) for k, v in x.items()}
+    for k in x:
+        xs[k][torch.from_numpy(table).long()] = x[k]
+    expect, o_ref = oracle_step(fmt, w, w.batch, H, pages, perm, xs, seed, 2)
+    assert np.array_equal(o.cpu().numpy(), o_ref.reshape(w.batch, H, 128)[table])
+    assert np.array_equal(download(qs), expect)
